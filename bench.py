@@ -1,0 +1,541 @@
+"""Benchmark of the KV-cache format conversions on B200.
+
+Headline workload (one JSON line on rank 0): the contiguous FP8 partial-window
+workload -- K and V FP16 caches [4, 4096, 8, 128] (N(0,1) with 1% +-U(20,60000)
+outliers and 0.1% subnormals), window offset 1024, width 2048.  One step is
+fp16_to_fp8(K), fp16_to_fp8(V), fp8_to_fp16(K), fp8_to_fp16(V) through the C
+ABI on resident device buffers.  The metric is algorithmic GB/s (bytes read +
+bytes written: 3 bytes per element per conversion), with L2 flushed between
+steps (a 256 MiB memset outside the per-step CUDA events).
+
+Extra keys:
+  roofline      the dominant kernel's achieved GB/s (algorithmic bytes per
+                launch / mean CUDA-event duration) against the measured HBM
+                copy peak in MEASURED_PEAKS.json;
+  cpu_baseline  the CPU oracle (single-threaded C++) timed on this host on the
+                same step;
+  e2e           the same metric through the public Python API with pinned host
+                buffers: host->device copy of the window, the four conversions,
+                device->host copy of the decoded window, all inside the events;
+  per_op        every other conversion on its own workload (contiguous Q4/Q6,
+                paged Q4 decode / prefill, the model-sized paged Q6 layers), each
+                as GB/s and fraction of the HBM peak (--per-op, on by default).
+
+Multi-GPU (torchrun, one rank per GPU): every rank converts its own shard of
+sequences (weak scaling, no collective on the data path); the step time is the
+max over ranks.  ``--impl reference`` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+HEADLINE = dict(workload="fp8_window_contiguous", shape=(4, 4096, 8, 128), offset=1024, width=2048)
+FLUSH_BYTES = 256 << 20
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+
+BYTES_PER_ELEM = {"fp8": 3.0, 4: 2.0 + 0.5 + 2.0 / 32, 6: 2.0 + 0.75 + 2.0 / 32}
+
+
+# ------------------------------------------------------------- host logic ----
+
+def shard_range(total: int, rank: int, world: int):
+    """Contiguous share [lo, hi) of `total` units for `rank` of `world` (sizes differ by <= 1)."""
+    base, rem = divmod(total, world)
+    lo = rank * base + min(rank, rem)
+    return lo, lo + base + (1 if rank < rem else 0)
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank float over the process group (identity without one)."""
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def hbm_peak():
+    try:
+        with open(PEAKS_PATH) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.marks = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self):
+        self.marks.append(time.time())
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for t, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((t, float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        lo, hi = (self.marks[0], self.marks[-1]) if len(self.marks) >= 2 else (rows[0][0], rows[-1][0])
+        inside = [r for r in rows if lo <= r[0] <= hi] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in inside for n, v in zip(names, r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": reasons, "samples": len(inside)}
+
+
+# ---------------------------------------------------------- GPU workloads ----
+
+class Fp8Step:
+    """Headline step on one rank: FP8 encode + decode of the K and V windows."""
+
+    def __init__(self, kvq, dev, batch, seed_shift=0):
+        B, S, H, D = HEADLINE["shape"]
+        shape = (batch, S, H, D)
+        k, v = workloads.fp8_window(seed=workloads.SEED_BASE + 2 + seed_shift, shape=shape, device=dev)
+        self.kvq, self.batch = kvq, batch
+        self.k, self.v = k, v
+        self.k8 = torch.zeros(shape, dtype=torch.uint8, device=dev)
+        self.v8 = torch.zeros_like(self.k8)
+        self.ky = torch.zeros_like(k)
+        self.vy = torch.zeros_like(v)
+        self.off, self.w = HEADLINE["offset"], HEADLINE["width"]
+        self.elems_per_tensor = batch * self.w * H * D
+        self.launch_bytes = BYTES_PER_ELEM["fp8"] * self.elems_per_tensor
+        self.bytes_per_step = 4 * self.launch_bytes
+        self.launches_per_step = 4
+
+    def run(self, ev=None):
+        kvq, b, o, w = self.kvq, self.batch, self.off, self.w
+        kvq.fp16_to_fp8(self.k, self.k8, b, o, w)
+        if ev is not None:
+            ev[0].record()
+        kvq.fp16_to_fp8(self.v, self.v8, b, o, w)
+        if ev is not None:
+            ev[1].record()
+        kvq.fp8_to_fp16(self.k8, self.ky, b, o, w)
+        if ev is not None:
+            ev[2].record()
+        kvq.fp8_to_fp16(self.v8, self.vy, b, o, w)
+
+
+def time_device(fn, steps, warmup, flush, sampler=None, n_marks=0):
+    """Per-step CUDA-event times (ms) of fn(ev) with an L2 flush before each step."""
+    for _ in range(warmup):
+        flush.zero_()
+        fn(None)
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    mids = [[torch.cuda.Event(enable_timing=True) for _ in range(n_marks)] for _ in range(steps)]
+    _barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.mark()
+    for i in range(steps):
+        flush.zero_()
+        starts[i].record()
+        fn(mids[i] if n_marks else None)
+        ends[i].record()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.mark()
+    _barrier()
+    per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    segs = []
+    for i in range(steps):
+        pts = [starts[i]] + mids[i] + [ends[i]]
+        segs.append([a.elapsed_time(b) for a, b in zip(pts[:-1], pts[1:])])
+    return per_step, segs
+
+
+def _barrier():
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def e2e_fp8(kvq, step: Fp8Step, steps, warmup, dev):
+    """Same step through the public API from pinned host buffers: H2D of the K/V windows,
+    the four conversions, D2H of the decoded windows, all inside the CUDA events."""
+    B, S, H, D = step.k.shape
+    o, w = step.off, step.w
+    hk = step.k.cpu().pin_memory()
+    hv = step.v.cpu().pin_memory()
+    hy_k = torch.empty_like(hk).pin_memory()
+    hy_v = torch.empty_like(hv).pin_memory()
+
+    def once():
+        for b in range(B):
+            step.k[b, o:o + w].copy_(hk[b, o:o + w], non_blocking=True)
+            step.v[b, o:o + w].copy_(hv[b, o:o + w], non_blocking=True)
+        step.run()
+        for b in range(B):
+            hy_k[b, o:o + w].copy_(step.ky[b, o:o + w], non_blocking=True)
+            hy_v[b, o:o + w].copy_(step.vy[b, o:o + w], non_blocking=True)
+
+    for _ in range(warmup):
+        once()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        once()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    win_bytes = B * w * H * D * 2
+    return ms, 2 * win_bytes, 2 * win_bytes
+
+
+def per_op_measurements(kvq, dev, peak, steps, flush, include_model=True):
+    """Each remaining conversion on its own workload; mean CUDA-event time per launch."""
+    out = []
+
+    def record(name, config, nbytes, fn, n=steps):
+        per, _ = time_device(lambda ev: fn(), n, 3, flush)
+        ms = statistics.mean(per)
+        out.append({"op": name, "config": config, "bytes": int(nbytes), "us": round(ms * 1e3, 2),
+                    "gbs": round(nbytes / ms / 1e6, 1), "frac": round(nbytes / ms / 1e6 / peak, 3)})
+
+    # contiguous Q4 / Q6, channel outliers [16, 8192, 8, 128]
+    k, v = workloads.channel_outliers(device=dev)
+    B, S, H, D = k.shape
+    n = 2 * k.numel()
+    ky, vy = torch.empty_like(k), torch.empty_like(v)
+    for wb in (4, 6):
+        cs, ss = kvq.q_shapes(tuple(k.shape), wb)
+        kc = torch.empty(cs, dtype=torch.uint8, device=dev)
+        vc = torch.empty_like(kc)
+        ks = torch.empty(ss, dtype=torch.float16, device=dev)
+        vs = torch.empty_like(ks)
+        cfg = f"contiguous [16,8192,8,128] K+V wbits={wb}"
+        record(f"fp16_to_q_kv/q{wb}", cfg, BYTES_PER_ELEM[wb] * n,
+               lambda: kvq.fp16_to_q_kv(k, kc, ks, v, vc, vs, B, 0, S, 0, None, None, wb))
+        record(f"q_to_fp16_kv/q{wb}", cfg, BYTES_PER_ELEM[wb] * n,
+               lambda: kvq.q_to_fp16_kv(kc, ky, ks, vc, vy, vs, B, 0, S, 0, None, None, wb))
+        del kc, vc, ks, vs
+    # FP8 alone on the big tensor
+    k8 = torch.empty(k.shape, dtype=torch.uint8, device=dev)
+    record("fp16_to_fp8", "contiguous [16,8192,8,128] K", 3.0 * k.numel(),
+           lambda: kvq.fp16_to_fp8(k, k8, B, 0, S))
+    record("fp8_to_fp16", "contiguous [16,8192,8,128] K", 3.0 * k.numel(),
+           lambda: kvq.fp8_to_fp16(k8, ky, B, 0, S))
+    del k, v, ky, vy, k8
+    torch.cuda.empty_cache()
+
+    # paged Q4 decode / prefill on the 2048-page pool
+    pool = workloads.paged_pool(device=dev)
+    P, ps, H, D = pool.k.shape
+    cs, ss = kvq.q_shapes(tuple(pool.k.shape), 4)
+    kc = torch.zeros(cs, dtype=torch.uint8, device=dev)
+    vc = torch.zeros_like(kc)
+    ks = torch.zeros(ss, dtype=torch.float16, device=dev)
+    vs = torch.zeros_like(ks)
+    lens = pool.cache_seqlens.cpu()
+    for phase, off, w in (("decode", 0, 1), ("prefill", -512, 512)):
+        npos = sum(max(0, int(L) + off + w) - max(0, int(L) + off) for L in lens)
+        nb = BYTES_PER_ELEM[4] * 2 * npos * H * D
+        cfg = f"paged 2048x256x8x128 pool, 32 seqs, {phase} width={w}"
+        record(f"fp16_to_q_kv/q4/{phase}", cfg, nb,
+               lambda: kvq.fp16_to_q_kv(pool.k, kc, ks, pool.v, vc, vs, 32, off, w, ps,
+                                        pool.cache_seqlens, pool.block_table, 4))
+        record(f"q_to_fp16_kv/q4/{phase}", cfg, nb,
+               lambda: kvq.q_to_fp16_kv(kc, pool.k, ks, vc, pool.v, vs, 32, off, w, ps,
+                                        pool.cache_seqlens, pool.block_table, 4))
+    del pool, kc, vc, ks, vs
+    torch.cuda.empty_cache()
+
+    if include_model:
+        out.extend(model_layers(kvq, dev, peak, max(3, steps // 10), flush))
+    return out
+
+
+def model_layers(kvq, dev, peak, steps, flush, layers=32):
+    """32 layers x K/V of 8 x 32768 x 8 x 128 FP16 in 256-position pages (~48 GB resident):
+    full-window q_to_fp16_kv over all layers, then fp16_to_q_kv over all layers."""
+    L = []
+    for i in range(layers):
+        pool = workloads.model_layer(i, device=dev)
+        cs, ss = kvq.q_shapes(tuple(pool.k.shape), 6)
+        kc = torch.empty(cs, dtype=torch.uint8, device=dev)
+        vc = torch.empty_like(kc)
+        ks = torch.empty(ss, dtype=torch.float16, device=dev)
+        vs = torch.empty_like(ks)
+        kvq.fp16_to_q_kv(pool.k, kc, ks, pool.v, vc, vs, 8, -32768, 32768, 256, pool.cache_seqlens,
+                         pool.block_table, 6)  # setup, untimed
+        L.append((pool, kc, vc, ks, vs))
+    torch.cuda.synchronize()
+    n = 2 * L[0][0].k.numel() * layers
+    nb = BYTES_PER_ELEM[6] * n
+
+    def deq():
+        for pool, kc, vc, ks, vs in L:
+            kvq.q_to_fp16_kv(kc, pool.k, ks, vc, pool.v, vs, 8, -32768, 32768, 256, pool.cache_seqlens,
+                             pool.block_table, 6)
+
+    def qnt():
+        for pool, kc, vc, ks, vs in L:
+            kvq.fp16_to_q_kv(pool.k, kc, ks, pool.v, vc, vs, 8, -32768, 32768, 256, pool.cache_seqlens,
+                             pool.block_table, 6)
+
+    res = []
+    cfg = "paged Q6, 32 layers x K/V 8x32768x8x128, page 256, shuffled block_table"
+    for name, fn in (("q_to_fp16_kv/q6/model32", deq), ("fp16_to_q_kv/q6/model32", qnt)):
+        per, _ = time_device(lambda ev: fn(), steps, 2, flush)
+        ms = statistics.mean(per)
+        res.append({"op": name, "config": cfg, "bytes": int(nb), "us": round(ms * 1e3, 1),
+                    "gbs": round(nb / ms / 1e6, 1), "frac": round(nb / ms / 1e6 / peak, 3)})
+    del L
+    torch.cuda.empty_cache()
+    return res
+
+
+# -------------------------------------------------------------- CPU oracle ----
+
+def oracle_step_sample(batch=4, max_seconds=12.0, min_reps=1):
+    """Time the CPU oracle on the headline step (all four conversions of the full window),
+    repeating until about max_seconds.  Returns (GB/s, seconds per step, reps, description)."""
+    import numpy as np
+
+    import oracle
+
+    B, S, H, D = HEADLINE["shape"]
+    k, v = workloads.fp8_window(shape=(batch, S, H, D))
+    kn = k.view(torch.int16).numpy().view(np.uint16)
+    vn = v.view(torch.int16).numpy().view(np.uint16)
+    k8 = np.zeros(kn.shape, np.uint8)
+    v8 = np.zeros(vn.shape, np.uint8)
+    ky = np.zeros(kn.shape, np.uint16)
+    vy = np.zeros(vn.shape, np.uint16)
+    o, w = HEADLINE["offset"], HEADLINE["width"]
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.fp16_to_fp8(kn, k8, batch, o, w)
+        oracle.fp16_to_fp8(vn, v8, batch, o, w)
+        oracle.fp8_to_fp16(k8, ky, batch, o, w)
+        oracle.fp8_to_fp16(v8, vy, batch, o, w)
+        reps += 1
+        if reps >= min_reps and time.perf_counter() - t0 >= max_seconds:
+            break
+    dt = (time.perf_counter() - t0) / reps
+    nbytes = 4 * BYTES_PER_ELEM["fp8"] * batch * w * H * D
+    desc = f"{reps} full step(s): FP8 encode+decode of K and V, batch {batch}, window {o}..{o + w}"
+    return nbytes / dt / 1e9, dt, reps, desc
+
+
+# ------------------------------------------------------------------- main ----
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-per-op", action="store_true", help="skip the per-op table")
+    ap.add_argument("--no-model", action="store_true", help="skip the 32-layer model-sized rows")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        return run_reference(args)
+
+    import datetime
+
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    import kv_cache_quantization_fp16_b200 as kvq
+
+    peak, peak_kind = hbm_peak()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    sampler = ClockSampler(local_rank).start() if rank == 0 else None
+
+    # each rank converts its own 4 sequences: a global batch of 4 * world (weak scaling)
+    batch = HEADLINE["shape"][0]
+    step = Fp8Step(kvq, dev, batch, seed_shift=rank)
+    per_step, segs = time_device(step.run, args.steps, args.warmup, flush, sampler, n_marks=3)
+    ms_local = statistics.mean(per_step)
+    ms = max_over_ranks(ms_local, dev)
+    names = ["fp16_to_fp8(K)", "fp16_to_fp8(V)", "fp8_to_fp16(K)", "fp8_to_fp16(V)"]
+    seg_ms = [statistics.mean(s[i] for s in segs) for i in range(4)]
+    enc_ms = (seg_ms[0] + seg_ms[1]) / 2
+    dec_ms = (seg_ms[2] + seg_ms[3]) / 2
+    dom = ("fp16_to_fp8", enc_ms) if enc_ms >= dec_ms else ("fp8_to_fp16", dec_ms)
+    achieved = step.launch_bytes / dom[1] / 1e6
+
+    e2e_ms, h2d, d2h = e2e_fp8(kvq, step, max(10, args.steps // 10), 3, dev)
+    e2e_ms = max_over_ranks(e2e_ms, dev)
+
+    per_op = []
+    if rank == 0 and not args.no_per_op:
+        del flush
+        flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        per_op = per_op_measurements(kvq, dev, peak, max(20, args.steps // 5), flush,
+                                     include_model=not args.no_model)
+    if sampler:
+        sampler.stop()
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    cpu = None
+    if not args.no_cpu_baseline:
+        gbs, dt, reps, desc = oracle_step_sample()
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": desc, "seconds_per_step": round(dt, 3)}
+
+    total_bytes = world * step.bytes_per_step
+    value = total_bytes / ms / 1e6
+    line = {
+        "metric": "KV-cache convert GB/s (read+write), FP8 E5M2 encode+decode of K and V",
+        "value": round(value, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16->u8->f16",
+        "data": "synthetic (seeded N(0,1) with 1% outliers and 0.1% subnormals, drawn on device)",
+        "config": {"workload": HEADLINE["workload"], "shape": list(HEADLINE["shape"]),
+                   "global_batch": batch * world, "offset": HEADLINE["offset"], "width": HEADLINE["width"],
+                   "ops": names, "l2": "flushed between steps (256 MiB memset outside the per-step events)",
+                   "parallelism": f"replicas x{world}, each rank its own 4 sequences"},
+        "roofline": {"bound": "hbm", "kernel": dom[0], "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 3), "peak_kind": peak_kind,
+                     "bytes_per_launch": int(step.launch_bytes), "us_per_launch": round(dom[1] * 1e3, 2),
+                     "traffic": None},
+        "per_kernel_us": {n: round(t * 1e3, 2) for n, t in zip(names, seg_ms)},
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(world * step.bytes_per_step / e2e_ms / 1e6, 2), "unit": "GB/s",
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": step.launches_per_step * args.steps,
+        "clocks": sampler.summary() if sampler else None,
+        "per_op": per_op,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_reference(args):
+    """The CPU oracle as the reference arm: each step = the headline step on batch 1 (one of the
+    four sequences), single-threaded, on this host."""
+    import numpy as np
+
+    import oracle
+
+    B, S, H, D = HEADLINE["shape"]
+    o, w = HEADLINE["offset"], HEADLINE["width"]
+    k, v = workloads.fp8_window(shape=(1, S, H, D))
+    kn = k.view(torch.int16).numpy().view(np.uint16)
+    vn = v.view(torch.int16).numpy().view(np.uint16)
+    k8, v8 = np.zeros(kn.shape, np.uint8), np.zeros(vn.shape, np.uint8)
+    ky, vy = np.zeros(kn.shape, np.uint16), np.zeros(vn.shape, np.uint16)
+
+    def once():
+        oracle.fp16_to_fp8(kn, k8, 1, o, w)
+        oracle.fp16_to_fp8(vn, v8, 1, o, w)
+        oracle.fp8_to_fp16(k8, ky, 1, o, w)
+        oracle.fp8_to_fp16(v8, vy, 1, o, w)
+
+    for _ in range(args.warmup):
+        once()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        once()
+    dt = (time.perf_counter() - t0) / args.steps
+    nbytes = 4 * BYTES_PER_ELEM["fp8"] * w * H * D
+    value = nbytes / dt / 1e9
+    sample = f"batch 1 of 4 per step (window {o}..{o + w}, K and V, encode + decode)"
+    line = {
+        "impl": "reference",
+        "metric": "KV-cache convert GB/s (read+write), FP8 E5M2 encode+decode of K and V",
+        "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16->u8->f16",
+        "data": "synthetic (seeded, same recipe as the GPU arm)",
+        "config": {"workload": HEADLINE["workload"], "shape": list(HEADLINE["shape"]),
+                   "global_batch": 1, "offset": o, "width": w},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,159 @@
+/*
+ * kvq.h -- C ABI of the B200 (sm_100a) KV-cache format conversion library,
+ * libkvq.so.
+ *
+ * The four conversions are the ones the page "Implementation: Turboderp org
+ * Exllamav2 Ext Cache" defines (sections Description, Signature and I/O
+ * Contract): fp16_to_fp8, fp8_to_fp16, fp16_to_q_kv and q_to_fp16_kv.  Each
+ * entry point keeps the page's argument order (in / out / scales pointers,
+ * batch_size, offset, width, page_size, cache_seqlens, block_table, wbits),
+ * replaces each torch tensor by a raw device pointer plus the shape the tensor
+ * carried (kvq_cache_desc), and takes the CUDA stream explicitly instead of
+ * using "the current stream".
+ *
+ * Numerics (fixed by this library, since the page leaves them open):
+ *   FP8   E5M2 = the upper byte of binary16 after rounding to 2 fraction bits,
+ *         round to nearest, ties to even; no saturation (|x| >= 61440 -> Inf);
+ *         any NaN -> sign | 0x7E.  Decoding is exact: half bits = byte << 8.
+ *   Q4/Q6 symmetric absmax over 32 consecutive head_dim elements.
+ *         maxq = 2^(wbits-1) - 1, z = 2^(wbits-1).
+ *         scale s = RN16(fl32(absmax / maxq)) stored as FP16;
+ *         code    = clamp(rint(fl32(x / s)) + z, 0, 2^wbits - 1), ties to even,
+ *                   and every code = z with s = +0 when s rounds to +0;
+ *         dequant = RN16((code - z) * s).
+ *         The codes of one head row form a little-endian bit stream: code j
+ *         occupies bits [wbits*j, wbits*j + wbits) of the row's bytes (Q4: two
+ *         codes per byte, even element in the low nibble; Q6: 16 codes per
+ *         three 32-bit little-endian words).
+ *   Results are bit-exact with these definitions; there is no tolerance.
+ *
+ * Layouts (row-major; all pointers are device memory on the current device):
+ *   FP16 cache   [dim0, dim1, kv_heads, head_dim]                 binary16
+ *   FP8 cache    [dim0, dim1, kv_heads, head_dim]                 uint8
+ *   Q codes      [dim0, dim1, kv_heads, head_dim * wbits / 8]     uint8
+ *   Q scales     [dim0, dim1, kv_heads, head_dim / 32]            binary16
+ *   Contiguous:  dim0 = allocated sequences, dim1 = max positions (seq).
+ *   Paged:       dim0 = pages in the pool, dim1 = page_size positions.
+ *   cache_seqlens [batch_size] int32; block_table [batch_size,
+ *   block_table_stride] int32 (entries that no window reaches may be -1).
+ *
+ * Windows:
+ *   Contiguous: for every sequence b < batch_size, positions
+ *               [offset, offset + width).
+ *   Paged:      for every sequence i < batch_size, logical positions
+ *               [max(0, cache_seqlens[i] + offset), cache_seqlens[i] + offset + width);
+ *               logical position p is row p % page_size of physical page
+ *               block_table[i][p / page_size].  FP16 and Q tensors share the
+ *               same page geometry and block table.
+ *   Nothing outside the window is read or written.
+ *
+ * Ownership: every buffer belongs to the caller and must stay valid until the
+ *   work enqueued on `stream` has finished.  The library allocates nothing.
+ *   Inputs and outputs must not overlap.  All calls are asynchronous: they
+ *   validate the arguments on the host, enqueue kernels on `stream` (a
+ *   cudaStream_t; NULL = the legacy default stream) and return.
+ *
+ * Errors: arguments are checked on the host before anything is enqueued; a
+ *   failed check returns a kvq_status and enqueues nothing.  Launch failures
+ *   return KVQ_ERR_CUDA.  Problems only the device can see (a block_table entry
+ *   outside [0, dim0), or a logical page index >= block_table_stride) skip the
+ *   affected positions and record a code in a per-device error word that
+ *   kvq_poll_device_error() reads.  No kernel traps and no exception crosses
+ *   the ABI.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kvq_status {
+  KVQ_OK = 0,
+  KVQ_ERR_NULL = 1,    /* a required pointer is NULL */
+  KVQ_ERR_SHAPE = 2,   /* bad dims: negative, head_dim not a multiple of 8 (FP8) or 32 (Q) */
+  KVQ_ERR_WBITS = 3,   /* wbits is not 4 or 6 */
+  KVQ_ERR_RANGE = 4,   /* window or batch outside the cache, page_size != dim1 */
+  KVQ_ERR_ALIGN = 5,   /* a buffer is not 16-byte aligned */
+  KVQ_ERR_CUDA = 6,    /* the CUDA runtime reported an error */
+  KVQ_ERR_DEVICE = 7   /* the device recorded bad paging metadata (kvq_poll_device_error) */
+} kvq_status;
+
+/* Device-side error codes stored in the error word. */
+enum {
+  KVQ_DEV_OK = 0,
+  KVQ_DEV_BAD_PAGE = 1,       /* block_table entry outside [0, dim0) */
+  KVQ_DEV_BAD_PAGE_INDEX = 2  /* logical page index >= block_table_stride */
+};
+
+/* The shape the torch tensor carried in the original extension. */
+typedef struct kvq_cache_desc {
+  int32_t dim0;               /* contiguous: allocated sequences; paged: pages in the pool */
+  int32_t dim1;               /* contiguous: max positions per sequence; paged: page_size */
+  int32_t kv_heads;           /* H */
+  int32_t head_dim;           /* D */
+  int32_t block_table_stride; /* paged: columns of block_table; contiguous: ignored */
+} kvq_cache_desc;
+
+/* fp16_to_fp8 (Description; Signature): encode the FP16 cache `in` into the
+ * E5M2 cache `out` (same shape) over the contiguous window.  head_dim must be
+ * a multiple of 8.  `in` and `out` 16-byte aligned. */
+KVQ_API kvq_status kvq_fp16_to_fp8(const void* in, void* out, const kvq_cache_desc* desc,
+                           int batch_size, int offset, int width, void* stream);
+
+/* fp8_to_fp16 (Description; Signature): decode the E5M2 cache `in` into the
+ * FP16 cache `out` over the same kind of window. */
+KVQ_API kvq_status kvq_fp8_to_fp16(const void* in, void* out, const kvq_cache_desc* desc,
+                           int batch_size, int offset, int width, void* stream);
+
+/* fp16_to_q_kv (Description; Signature; I/O Contract): quantize the FP16 K
+ * and V caches to wbits-bit codes and FP16 scales in one launch.  page_size
+ * == 0 selects contiguous mode (cache_seqlens, block_table ignored and may be
+ * NULL); page_size > 0 selects paged mode (page_size == desc->dim1,
+ * cache_seqlens and block_table required).  head_dim must be a multiple of
+ * 32 (the scale block, the page's Q_CACHE_BLOCKSIZE_Q alignment).  wbits is
+ * 4 or 6.  All six cache pointers 16-byte aligned. */
+KVQ_API kvq_status kvq_fp16_to_q_kv(const void* k_in, void* k_out, void* k_scales,
+                            const void* v_in, void* v_out, void* v_scales,
+                            const kvq_cache_desc* desc, int batch_size, int offset, int width,
+                            int page_size, const int32_t* cache_seqlens,
+                            const int32_t* block_table, int wbits, void* stream);
+
+/* q_to_fp16_kv (Description; Signature): dequantize K and V codes + scales
+ * back into the FP16 caches, same modes and checks as kvq_fp16_to_q_kv. */
+KVQ_API kvq_status kvq_q_to_fp16_kv(const void* k_in, void* k_out, const void* k_scales,
+                            const void* v_in, void* v_out, const void* v_scales,
+                            const kvq_cache_desc* desc, int batch_size, int offset, int width,
+                            int page_size, const int32_t* cache_seqlens,
+                            const int32_t* block_table, int wbits, void* stream);
+
+/* Human-readable name of a status (static storage; never NULL). */
+KVQ_API const char* kvq_status_string(kvq_status status);
+
+/* Waits for `stream`, then reads and clears the current device's error word.
+ * *code_out receives the KVQ_DEV_* code (0 when none).  Returns KVQ_ERR_DEVICE
+ * when the word was set, KVQ_OK when not, KVQ_ERR_CUDA on a runtime error. */
+KVQ_API kvq_status kvq_poll_device_error(int32_t* code_out, void* stream);
+
+/* Self-check (no counterpart on the page): compares, on the device, the
+ * kernels' fast code rounding (reciprocal, one FMA correction step, rounding
+ * by magic-number addition) with IEEE binary32 division followed by rint and
+ * the clamp, for every finite binary16 x and every positive finite binary16
+ * scale s (2^31 pairs).  `mismatches` is a caller-owned device pointer to one
+ * unsigned 64-bit counter; it is zeroed and then receives the number of
+ * pairs whose codes differ (0 expected).  Asynchronous on `stream`. */
+KVQ_API kvq_status kvq_selfcheck_code_rounding(int wbits, unsigned long long* mismatches, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

@@ -1,0 +1,211 @@
+"""B200-native KV-cache format conversion (FP16 <-> FP8 E5M2, FP16 <-> Q4 / Q6).
+
+Thin Python binding over ``libkvq.so`` (C ABI in ``include/kvq.h``).  It only
+marshals arguments: it checks dtypes, devices, shapes and contiguity the way
+the original extension's host wrappers did (page "Implementation: Turboderp
+org Exllamav2 Ext Cache", Description: input kHalf / output kUInt8, scales
+kHalf, cache_seqlens and block_table kInt), makes the tensors' device current
+and passes torch's current stream.  Every conversion runs in the library's
+CUDA kernels; there is no fallback of any kind.  If ``libkvq.so`` is missing,
+importing this package raises ``ImportError``.
+
+Names and argument order follow the page's Signature section::
+
+    fp16_to_fp8(in_tensor, out_tensor, batch_size, offset, width)
+    fp8_to_fp16(in_tensor, out_tensor, batch_size, offset, width)
+    fp16_to_q_kv(k_in, k_out, k_scales, v_in, v_out, v_scales,
+                 batch_size, offset, width, page_size, cache_seqlens, block_table, wbits)
+    q_to_fp16_kv(k_in, k_out, k_scales, v_in, v_out, v_scales,
+                 batch_size, offset, width, page_size, cache_seqlens, block_table, wbits)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["fp16_to_fp8", "fp8_to_fp16", "fp16_to_q_kv", "q_to_fp16_kv", "poll_device_error",
+           "selfcheck_code_rounding", "q_shapes", "KVQError", "LIB_PATH", "library"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvq.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python __graft_entry__.py` "
+                      "or kv_cache_quantization_fp16_b200/_build.py (nvcc, sm_100a)")
+
+
+class _Desc(ctypes.Structure):
+    _fields_ = [("dim0", ctypes.c_int32), ("dim1", ctypes.c_int32), ("kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("block_table_stride", ctypes.c_int32)]
+
+
+_STATUS = {0: "ok", 1: "null pointer", 2: "bad shape", 3: "wbits must be 4 or 6",
+           4: "window, batch or page geometry out of range", 5: "buffer not 16-byte aligned",
+           6: "CUDA runtime error", 7: "device recorded bad paging metadata"}
+
+
+class KVQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: kvq status {status} ({_STATUS.get(status, 'unknown')})")
+
+
+def _load() -> ctypes.CDLL:
+    L = ctypes.CDLL(LIB_PATH)
+    vp, I = ctypes.c_void_p, ctypes.c_int
+    dp = ctypes.POINTER(_Desc)
+    L.kvq_fp16_to_fp8.argtypes = [vp, vp, dp, I, I, I, vp]
+    L.kvq_fp8_to_fp16.argtypes = [vp, vp, dp, I, I, I, vp]
+    L.kvq_fp16_to_q_kv.argtypes = [vp, vp, vp, vp, vp, vp, dp, I, I, I, I, vp, vp, I, vp]
+    L.kvq_q_to_fp16_kv.argtypes = [vp, vp, vp, vp, vp, vp, dp, I, I, I, I, vp, vp, I, vp]
+    L.kvq_status_string.argtypes = [I]
+    L.kvq_status_string.restype = ctypes.c_char_p
+    L.kvq_poll_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), vp]
+    L.kvq_selfcheck_code_rounding.argtypes = [I, vp, vp]
+    for f in ("kvq_fp16_to_fp8", "kvq_fp8_to_fp16", "kvq_fp16_to_q_kv", "kvq_q_to_fp16_kv",
+              "kvq_poll_device_error", "kvq_selfcheck_code_rounding"):
+        getattr(L, f).restype = I
+    return L
+
+
+_lib = _load()
+
+
+def library() -> ctypes.CDLL:
+    return _lib
+
+
+def _check(st: int, where: str) -> None:
+    if st != 0:
+        raise KVQError(st, where)
+
+
+def _require(cond: bool, msg: str) -> None:
+    if not cond:
+        raise ValueError(msg)
+
+
+def _cuda4(t: torch.Tensor, dtype, name: str) -> None:
+    _require(isinstance(t, torch.Tensor), f"{name} must be a tensor")
+    _require(t.dtype == dtype, f"{name} must be {dtype}, got {t.dtype}")
+    _require(t.is_cuda, f"{name} must be a CUDA tensor")
+    _require(t.dim() == 4, f"{name} must be 4-D, got shape {tuple(t.shape)}")
+    _require(t.is_contiguous(), f"{name} must be contiguous")
+
+
+def _stream(dev: torch.device) -> int:
+    return torch.cuda.current_stream(dev).cuda_stream
+
+
+def q_shapes(shape, wbits: int):
+    """Shapes of the code and scale tensors for an FP16 cache of shape [d0, d1, H, D]."""
+    d0, d1, H, D = shape
+    return (d0, d1, H, D * wbits // 8), (d0, d1, H, D // 32)
+
+
+def _fp8(fn, in_tensor, out_tensor, batch_size, offset, width, in_dtype, out_dtype, where):
+    _cuda4(in_tensor, in_dtype, "in_tensor")
+    _cuda4(out_tensor, out_dtype, "out_tensor")
+    _require(in_tensor.shape == out_tensor.shape, "in_tensor and out_tensor must have the same shape")
+    _require(in_tensor.device == out_tensor.device, "tensors must be on one device")
+    d0, d1, H, D = in_tensor.shape
+    desc = _Desc(d0, d1, H, D, 0)
+    with torch.cuda.device(in_tensor.device):
+        st = fn(in_tensor.data_ptr(), out_tensor.data_ptr(), ctypes.byref(desc), int(batch_size),
+                int(offset), int(width), _stream(in_tensor.device))
+    _check(st, where)
+
+
+def fp16_to_fp8(in_tensor: torch.Tensor, out_tensor: torch.Tensor, batch_size: int, offset: int,
+                width: int) -> None:
+    """Encode the FP16 cache window into E5M2 bytes (out_tensor: uint8, same shape)."""
+    _fp8(_lib.kvq_fp16_to_fp8, in_tensor, out_tensor, batch_size, offset, width, torch.float16,
+         torch.uint8, "fp16_to_fp8")
+
+
+def fp8_to_fp16(in_tensor: torch.Tensor, out_tensor: torch.Tensor, batch_size: int, offset: int,
+                width: int) -> None:
+    """Decode the E5M2 cache window back into FP16 (out_tensor: float16, same shape)."""
+    _fp8(_lib.kvq_fp8_to_fp16, in_tensor, out_tensor, batch_size, offset, width, torch.uint8,
+         torch.float16, "fp8_to_fp16")
+
+
+def _q(fn, fp16_is_input, k_in, k_out, k_scales, v_in, v_out, v_scales, batch_size, offset, width,
+       page_size, cache_seqlens, block_table, wbits, where):
+    k16, kq = (k_in, k_out) if fp16_is_input else (k_out, k_in)
+    v16, vq = (v_in, v_out) if fp16_is_input else (v_out, v_in)
+    for t, n in ((k16, "FP16 K"), (v16, "FP16 V")):
+        _cuda4(t, torch.float16, n)
+    for t, n in ((kq, "K codes"), (vq, "V codes")):
+        _cuda4(t, torch.uint8, n)
+    for t, n in ((k_scales, "k_scales"), (v_scales, "v_scales")):
+        _cuda4(t, torch.float16, n)
+    _require(k16.shape == v16.shape, "K and V caches must have the same shape")
+    _require(wbits in (4, 6), f"wbits must be 4 or 6, got {wbits}")
+    _require(k16.shape[3] % 32 == 0, "head_dim must be a multiple of 32")
+    cshape, sshape = q_shapes(tuple(k16.shape), wbits)
+    for t, n in ((kq, "K codes"), (vq, "V codes")):
+        _require(tuple(t.shape) == cshape, f"{n} must have shape {cshape}, got {tuple(t.shape)}")
+    for t, n in ((k_scales, "k_scales"), (v_scales, "v_scales")):
+        _require(tuple(t.shape) == sshape, f"{n} must have shape {sshape}, got {tuple(t.shape)}")
+    dev = k16.device
+    for t in (kq, v16, vq, k_scales, v_scales):
+        _require(t.device == dev, "tensors must be on one device")
+    stride = 0
+    sl_ptr = bt_ptr = None
+    if page_size:
+        _require(cache_seqlens is not None and block_table is not None,
+                 "paged mode needs cache_seqlens and block_table")
+        _require(cache_seqlens.dtype == torch.int32 and block_table.dtype == torch.int32,
+                 "cache_seqlens and block_table must be int32")
+        _require(cache_seqlens.device == dev and block_table.device == dev, "tensors must be on one device")
+        _require(block_table.dim() == 2 and block_table.is_contiguous() and cache_seqlens.is_contiguous(),
+                 "block_table must be a contiguous [batch, max_pages] tensor")
+        _require(cache_seqlens.numel() >= batch_size and block_table.shape[0] >= batch_size,
+                 "cache_seqlens / block_table have fewer rows than batch_size")
+        stride = block_table.shape[1]
+        sl_ptr, bt_ptr = cache_seqlens.data_ptr(), block_table.data_ptr()
+    d0, d1, H, D = k16.shape
+    desc = _Desc(d0, d1, H, D, stride)
+    with torch.cuda.device(dev):
+        st = fn(k_in.data_ptr(), k_out.data_ptr(), k_scales.data_ptr(), v_in.data_ptr(), v_out.data_ptr(),
+                v_scales.data_ptr(), ctypes.byref(desc), int(batch_size), int(offset), int(width),
+                int(page_size), sl_ptr, bt_ptr, int(wbits), _stream(dev))
+    _check(st, where)
+
+
+def fp16_to_q_kv(k_in, k_out, k_scales, v_in, v_out, v_scales, batch_size, offset, width,
+                 page_size=0, cache_seqlens=None, block_table=None, wbits=4) -> None:
+    """Quantize the K and V FP16 cache windows to wbits-bit codes + FP16 scales (one launch)."""
+    _q(_lib.kvq_fp16_to_q_kv, True, k_in, k_out, k_scales, v_in, v_out, v_scales, batch_size, offset,
+       width, page_size, cache_seqlens, block_table, wbits, "fp16_to_q_kv")
+
+
+def q_to_fp16_kv(k_in, k_out, k_scales, v_in, v_out, v_scales, batch_size, offset, width,
+                 page_size=0, cache_seqlens=None, block_table=None, wbits=4) -> None:
+    """Dequantize the K and V code windows back into the FP16 caches (one launch)."""
+    _q(_lib.kvq_q_to_fp16_kv, False, k_in, k_out, k_scales, v_in, v_out, v_scales, batch_size, offset,
+       width, page_size, cache_seqlens, block_table, wbits, "q_to_fp16_kv")
+
+
+def poll_device_error(device=None) -> int:
+    """Synchronize the current stream and return (and clear) the device error code (0 = none)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    code = ctypes.c_int32(0)
+    with torch.cuda.device(dev):
+        st = _lib.kvq_poll_device_error(ctypes.byref(code), _stream(dev))
+    if st not in (0, 7):
+        raise KVQError(st, "poll_device_error")
+    return int(code.value)
+
+
+def selfcheck_code_rounding(wbits: int, device=None) -> int:
+    """Number of (x, s) binary16 pairs where the kernels' fast code rounding differs from
+    IEEE division + rint + clamp (0 expected)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    out = torch.zeros(1, dtype=torch.int64, device=dev)
+    with torch.cuda.device(dev):
+        st = _lib.kvq_selfcheck_code_rounding(int(wbits), out.data_ptr(), _stream(dev))
+    _check(st, "selfcheck_code_rounding")
+    return int(out.item())

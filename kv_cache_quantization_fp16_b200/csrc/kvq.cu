@@ -1,0 +1,486 @@
+// kvq.cu -- sm_100a kernels and the C ABI (include/kvq.h) of libkvq.so.
+//
+// KV-cache format conversions from the page "Implementation: Turboderp org
+// Exllamav2 Ext Cache": fp16_to_fp8 / fp8_to_fp16 (Description, Signature)
+// and fp16_to_q_kv / q_to_fp16_kv (Description, Signature, I/O Contract), in
+// contiguous and paged mode.
+//
+// Work decomposition.  A window of one sequence is a run of positions; every
+// position is H * D contiguous elements in the FP16 cache (and proportionally
+// many bytes in the FP8 / code / scale tensors).  The run is cut into tiles of
+// `tile_pos` positions; in paged mode tiles are aligned to multiples of
+// tile_pos in logical position space and tile_pos divides page_size, so a tile
+// never straddles a page.  One CTA converts one tile: thread 0 resolves the
+// tile (window clipping, the block_table lookup) once and stages the physical
+// row in shared memory, then all threads stream the tile's elements as a flat
+// array, 8 elements (16 bytes of FP16) per thread per step, with kUnroll
+// independent 16-byte loads in flight per thread.  Grid: x = tiles, y =
+// sequences, z = K / V (the fused K+V launch).
+//
+// This is a streaming, HBM-bound path: no tensor cores, no shared-memory
+// staging of the data, no collectives.
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kvq.h"
+#include "codec.cuh"
+
+namespace kvq {
+
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;
+constexpr int kBlockElems = 32;  // Q scale block along head_dim
+
+// Per-device error word for problems only the device can see.
+__device__ int g_device_error;
+
+__device__ __forceinline__ void record_error(int code) { atomicCAS(&g_device_error, 0, code); }
+
+struct Geometry {
+  int dim0, dim1;
+  long long hd;  // kv_heads * head_dim: elements per position
+  int bt_stride;
+  int batch, offset, width, page_size;
+  int tile_pos;
+  const int32_t* seqlens;
+  const int32_t* block_table;
+};
+
+// Tile `tile_x` of sequence `seq`: first physical row and number of positions,
+// or false when the tile is empty or its page is invalid.
+__device__ bool resolve_tile(const Geometry& g, int seq, int tile_x, long long& row0, int& nrows) {
+  if (g.page_size == 0) {
+    const long long p0 = static_cast<long long>(g.offset) + static_cast<long long>(tile_x) * g.tile_pos;
+    const long long p1 = min(static_cast<long long>(g.offset) + g.width, p0 + g.tile_pos);
+    if (p0 >= p1) return false;
+    row0 = static_cast<long long>(seq) * g.dim1 + p0;
+    nrows = static_cast<int>(p1 - p0);
+    return true;
+  }
+  const long long start = static_cast<long long>(g.seqlens[seq]) + g.offset;
+  const long long lo = start < 0 ? 0 : start;
+  const long long hi = start + g.width;
+  if (lo >= hi) return false;
+  const long long t0 = (lo / g.tile_pos) * g.tile_pos + static_cast<long long>(tile_x) * g.tile_pos;
+  const long long p0 = max(lo, t0);
+  const long long p1 = min(hi, t0 + g.tile_pos);
+  if (p0 >= p1) return false;
+  const long long lp = p0 / g.page_size;
+  if (lp >= g.bt_stride) {
+    record_error(KVQ_DEV_BAD_PAGE_INDEX);
+    return false;
+  }
+  const int page = g.block_table[static_cast<long long>(seq) * g.bt_stride + lp];
+  if (page < 0 || page >= g.dim0) {
+    record_error(KVQ_DEV_BAD_PAGE);
+    return false;
+  }
+  row0 = static_cast<long long>(page) * g.page_size + p0 % g.page_size;
+  nrows = static_cast<int>(p1 - p0);
+  return true;
+}
+
+struct Params {
+  Geometry g;
+  const void* in[2];
+  void* out[2];
+  void* scales[2];  // Q encode: written; Q decode: read
+};
+
+// ---------------------------------------------------------------------------
+// Per-tile bodies
+// ---------------------------------------------------------------------------
+
+struct Fp8Encode {
+  __device__ static void tile(const Params& p, int kv, long long row0, int nrows) {
+    const long long e0 = row0 * p.g.hd;
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __half*>(p.in[kv]) + e0);
+    uint2* dst = reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.out[kv]) + e0);
+    const int nvec = static_cast<int>(nrows * p.g.hd / 8);
+    for (int base = 0; base < nvec; base += kThreads * kUnroll) {
+      uint4 x[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int v = base + u * kThreads + threadIdx.x;
+        if (v < nvec) x[u] = __ldg(src + v);
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int v = base + u * kThreads + threadIdx.x;
+        if (v < nvec) dst[v] = e5m2_encode_v8(x[u]);
+      }
+    }
+  }
+};
+
+struct Fp8Decode {
+  __device__ static void tile(const Params& p, int kv, long long row0, int nrows) {
+    const long long e0 = row0 * p.g.hd;
+    const uint2* src = reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(p.in[kv]) + e0);
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__half*>(p.out[kv]) + e0);
+    const int nvec = static_cast<int>(nrows * p.g.hd / 8);
+    for (int base = 0; base < nvec; base += kThreads * kUnroll) {
+      uint2 x[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int v = base + u * kThreads + threadIdx.x;
+        if (v < nvec) x[u] = __ldg(src + v);
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int v = base + u * kThreads + threadIdx.x;
+        if (v < nvec) dst[v] = e5m2_decode_v8(x[u]);
+      }
+    }
+  }
+};
+
+// Q encode: a quad of lanes (4 x 8 elements) holds one 32-element block.
+template <int B>
+struct QEncode {
+  __device__ static void tile(const Params& p, int kv, long long row0, int nrows) {
+    const long long e0 = row0 * p.g.hd;
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __half*>(p.in[kv]) + e0);
+    uint8_t* codes = static_cast<uint8_t*>(p.out[kv]) + e0 * B / 8;
+    __half* scales = static_cast<__half*>(p.scales[kv]) + e0 / kBlockElems;
+    const int nvec = static_cast<int>(nrows * p.g.hd / 8);  // multiple of 4
+    for (int base = 0; base < nvec; base += kThreads * kUnroll) {
+      uint4 x[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int v = base + u * kThreads + threadIdx.x;
+        x[u] = make_uint4(0, 0, 0, 0);
+        if (v < nvec) x[u] = __ldg(src + v);
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int v = base + u * kThreads + threadIdx.x;
+        uint32_t m = absmax_bits_v8(x[u]);
+        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+        if (v >= nvec) continue;  // whole quads are in or out (nvec % 4 == 0)
+        const __half s16 = block_scale<B>(m);
+        const BlockScale bs = make_block_scale(s16);
+        uint32_t c[8];
+        quant_v8<B>(x[u], bs, c);
+        if (B == 4) {
+          reinterpret_cast<uint32_t*>(codes)[v] = pack_q4(c);
+        } else {
+          uint32_t lo, hi;
+          pack_q6(c, lo, hi);
+          uint8_t* dst = codes + static_cast<long long>(v) * 6;
+          if ((v & 1) == 0) {  // 4-byte aligned start
+            *reinterpret_cast<uint32_t*>(dst) = lo;
+            *reinterpret_cast<uint16_t*>(dst + 4) = static_cast<uint16_t>(hi);
+          } else {             // 2-byte aligned start, 4-byte aligned at +2
+            *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(lo);
+            *reinterpret_cast<uint32_t*>(dst + 2) = (lo >> 16) | (hi << 16);
+          }
+        }
+        if ((threadIdx.x & 3) == 0) scales[v >> 2] = s16;
+      }
+    }
+  }
+};
+
+template <int B>
+struct QDecode {
+  __device__ static void tile(const Params& p, int kv, long long row0, int nrows) {
+    const long long e0 = row0 * p.g.hd;
+    const uint8_t* codes = static_cast<const uint8_t*>(p.in[kv]) + e0 * B / 8;
+    const __half* scales = static_cast<const __half*>(p.scales[kv]) + e0 / kBlockElems;
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__half*>(p.out[kv]) + e0);
+    const int nvec = static_cast<int>(nrows * p.g.hd / 8);
+    for (int base = 0; base < nvec; base += kThreads * kUnroll) {
+      uint32_t lo[kUnroll], hi[kUnroll];
+      __half s[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int v = base + u * kThreads + threadIdx.x;
+        lo[u] = hi[u] = 0;
+        s[u] = __ushort_as_half(0);
+        if (v < nvec) {
+          if (B == 4) {
+            lo[u] = __ldg(reinterpret_cast<const uint32_t*>(codes) + v);
+          } else {
+            const uint8_t* src = codes + static_cast<long long>(v) * 6;
+            if ((v & 1) == 0) {
+              lo[u] = __ldg(reinterpret_cast<const uint32_t*>(src));
+              hi[u] = __ldg(reinterpret_cast<const uint16_t*>(src + 4));
+            } else {
+              const uint32_t a = __ldg(reinterpret_cast<const uint16_t*>(src));
+              const uint32_t b = __ldg(reinterpret_cast<const uint32_t*>(src + 2));
+              lo[u] = a | (b << 16);
+              hi[u] = b >> 16;
+            }
+          }
+          s[u] = __ldg(scales + (v >> 2));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int v = base + u * kThreads + threadIdx.x;
+        if (v >= nvec) continue;
+        const __half2 s2 = __halves2half2(s[u], s[u]);
+        dst[v] = (B == 4) ? dequant_q4_v8(lo[u], s2) : dequant_q6_v8(lo[u], hi[u], s2);
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// The kernel: one tile per CTA; the tile is resolved once and staged in smem.
+// ---------------------------------------------------------------------------
+
+template <class Op>
+__global__ void __launch_bounds__(kThreads) convert_kernel(const __grid_constant__ Params p) {
+  __shared__ long long s_row0;
+  __shared__ int s_nrows;
+  const int kv = blockIdx.z;
+  for (int seq = blockIdx.y; seq < p.g.batch; seq += gridDim.y) {
+    if (threadIdx.x == 0) {
+      long long r = -1;
+      int n = 0;
+      if (!resolve_tile(p.g, seq, blockIdx.x, r, n)) r = -1;
+      s_row0 = r;
+      s_nrows = n;
+    }
+    __syncthreads();
+    const long long row0 = s_row0;
+    const int nrows = s_nrows;
+    __syncthreads();
+    if (row0 >= 0) Op::tile(p, kv, row0, nrows);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Self-check of the fast code rounding against IEEE division.
+// ---------------------------------------------------------------------------
+
+template <int B>
+__global__ void selfcheck_rounding_kernel(unsigned long long* mismatches) {
+  // blockIdx.x + gridDim.x * blockIdx.y enumerates s bit patterns 1..0x7BFF;
+  // threads enumerate x over all 65536 bit patterns, skipping Inf / NaN.
+  const uint32_t s_bits = 1 + blockIdx.x;
+  const __half s16 = __ushort_as_half(static_cast<unsigned short>(s_bits));
+  const BlockScale bs = make_block_scale(s16);
+  unsigned long long bad = 0;
+  for (uint32_t xb = threadIdx.x; xb < 65536u; xb += blockDim.x) {
+    if (((xb >> 10) & 0x1F) == 0x1F) continue;
+    const float x = __half2float(__ushort_as_half(static_cast<unsigned short>(xb)));
+    const uint32_t fast = quant_code_bits<B>(x, bs) & ((1u << B) - 1);
+    const uint32_t ref = quant_code_ieee<B>(x, bs.s);
+    bad += (fast != ref);
+  }
+  if (bad) atomicAdd(mismatches, bad);
+}
+
+}  // namespace kvq
+
+// ===========================================================================
+// Host side: validation, tiling and launch.
+// ===========================================================================
+
+namespace {
+
+using namespace kvq;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+kvq_status check_desc(const kvq_cache_desc* d, int mult) {
+  if (!d) return KVQ_ERR_NULL;
+  if (d->dim0 < 1 || d->dim1 < 1 || d->kv_heads < 1 || d->head_dim < 1) return KVQ_ERR_SHAPE;
+  if (d->head_dim % mult) return KVQ_ERR_SHAPE;
+  if (static_cast<long long>(d->kv_heads) * d->head_dim > (1LL << 30)) return KVQ_ERR_SHAPE;
+  return KVQ_OK;
+}
+
+int floor_pow2(long long x) {
+  int r = 1;
+  while (static_cast<long long>(r) * 2 <= x && r < (1 << 30)) r *= 2;
+  return r;
+}
+
+int gcd_int(int a, int b) {
+  while (b) {
+    const int t = a % b;
+    a = b;
+    b = t;
+  }
+  return a;
+}
+
+// Positions per tile: about kThreads * kUnroll * 8 elements, a power of two,
+// and a divisor of page_size in paged mode.
+int pick_tile_pos(long long hd, int page_size) {
+  const long long target = static_cast<long long>(kThreads) * kUnroll * 8;
+  int t = floor_pow2(target / hd > 0 ? target / hd : 1);
+  if (page_size > 0) t = gcd_int(t, page_size);
+  return t;
+}
+
+kvq_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+template <class Op>
+kvq_status launch(const Params& p, int nkv, void* stream) {
+  const int paged = p.g.page_size > 0;
+  const long long tiles = (static_cast<long long>(p.g.width) + p.g.tile_pos - 1) / p.g.tile_pos + paged;
+  if (tiles > 0x7FFFFFFFLL) return KVQ_ERR_RANGE;
+  dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(p.g.batch < 65535 ? p.g.batch : 65535),
+            static_cast<unsigned>(nkv));
+  convert_kernel<Op><<<grid, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return launch_status();
+}
+
+Geometry make_geometry(const kvq_cache_desc* d, int batch, int offset, int width, int page_size,
+                       const int32_t* seqlens, const int32_t* block_table) {
+  Geometry g;
+  g.dim0 = d->dim0;
+  g.dim1 = d->dim1;
+  g.hd = static_cast<long long>(d->kv_heads) * d->head_dim;
+  g.bt_stride = d->block_table_stride;
+  g.batch = batch;
+  g.offset = offset;
+  g.width = width;
+  g.page_size = page_size;
+  g.tile_pos = pick_tile_pos(g.hd, page_size);
+  g.seqlens = seqlens;
+  g.block_table = block_table;
+  return g;
+}
+
+kvq_status check_contiguous_window(const kvq_cache_desc* d, int batch, int offset, int width) {
+  if (batch < 0 || width < 0 || offset < 0) return KVQ_ERR_RANGE;
+  if (batch > d->dim0) return KVQ_ERR_RANGE;
+  if (static_cast<long long>(offset) + width > d->dim1) return KVQ_ERR_RANGE;
+  return KVQ_OK;
+}
+
+kvq_status fp8_common(const void* in, void* out, const kvq_cache_desc* d, int batch, int offset,
+                      int width, void* stream, bool encode) {
+  if (!in || !out) return KVQ_ERR_NULL;
+  kvq_status st = check_desc(d, 8);
+  if (st != KVQ_OK) return st;
+  if (!aligned16(in) || !aligned16(out)) return KVQ_ERR_ALIGN;
+  st = check_contiguous_window(d, batch, offset, width);
+  if (st != KVQ_OK) return st;
+  if (batch == 0 || width == 0) return KVQ_OK;
+  Params p{};
+  p.g = make_geometry(d, batch, offset, width, 0, nullptr, nullptr);
+  p.in[0] = in;
+  p.out[0] = out;
+  return encode ? launch<Fp8Encode>(p, 1, stream) : launch<Fp8Decode>(p, 1, stream);
+}
+
+kvq_status q_common(const void* k_in, void* k_out, void* k_scales, const void* v_in, void* v_out,
+                    void* v_scales, const kvq_cache_desc* d, int batch, int offset, int width,
+                    int page_size, const int32_t* seqlens, const int32_t* block_table, int wbits,
+                    void* stream, bool encode) {
+  if (!k_in || !k_out || !k_scales || !v_in || !v_out || !v_scales) return KVQ_ERR_NULL;
+  kvq_status st = check_desc(d, kBlockElems);
+  if (st != KVQ_OK) return st;
+  if (wbits != 4 && wbits != 6) return KVQ_ERR_WBITS;
+  const void* ptrs[6] = {k_in, k_out, k_scales, v_in, v_out, v_scales};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return KVQ_ERR_ALIGN;
+  if (page_size < 0) return KVQ_ERR_RANGE;
+  if (page_size == 0) {
+    st = check_contiguous_window(d, batch, offset, width);
+    if (st != KVQ_OK) return st;
+  } else {
+    if (!seqlens || !block_table) return KVQ_ERR_NULL;
+    if (page_size != d->dim1 || batch < 0 || width < 0) return KVQ_ERR_RANGE;
+    if (d->block_table_stride < 1) return KVQ_ERR_RANGE;
+    if ((reinterpret_cast<uintptr_t>(seqlens) | reinterpret_cast<uintptr_t>(block_table)) & 3u)
+      return KVQ_ERR_ALIGN;
+  }
+  if (batch == 0 || width == 0) return KVQ_OK;
+  Params p{};
+  p.g = make_geometry(d, batch, offset, width, page_size, seqlens, block_table);
+  p.in[0] = k_in;
+  p.in[1] = v_in;
+  p.out[0] = k_out;
+  p.out[1] = v_out;
+  p.scales[0] = k_scales;
+  p.scales[1] = v_scales;
+  if (encode) return wbits == 4 ? launch<QEncode<4>>(p, 2, stream) : launch<QEncode<6>>(p, 2, stream);
+  return wbits == 4 ? launch<QDecode<4>>(p, 2, stream) : launch<QDecode<6>>(p, 2, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_fp16_to_fp8(const void* in, void* out, const kvq_cache_desc* desc, int batch_size,
+                           int offset, int width, void* stream) {
+  return fp8_common(in, out, desc, batch_size, offset, width, stream, true);
+}
+
+kvq_status kvq_fp8_to_fp16(const void* in, void* out, const kvq_cache_desc* desc, int batch_size,
+                           int offset, int width, void* stream) {
+  return fp8_common(in, out, desc, batch_size, offset, width, stream, false);
+}
+
+kvq_status kvq_fp16_to_q_kv(const void* k_in, void* k_out, void* k_scales, const void* v_in,
+                            void* v_out, void* v_scales, const kvq_cache_desc* desc, int batch_size,
+                            int offset, int width, int page_size, const int32_t* cache_seqlens,
+                            const int32_t* block_table, int wbits, void* stream) {
+  return q_common(k_in, k_out, k_scales, v_in, v_out, v_scales, desc, batch_size, offset, width,
+                  page_size, cache_seqlens, block_table, wbits, stream, true);
+}
+
+kvq_status kvq_q_to_fp16_kv(const void* k_in, void* k_out, const void* k_scales, const void* v_in,
+                            void* v_out, const void* v_scales, const kvq_cache_desc* desc,
+                            int batch_size, int offset, int width, int page_size,
+                            const int32_t* cache_seqlens, const int32_t* block_table, int wbits,
+                            void* stream) {
+  return q_common(k_in, k_out, const_cast<void*>(k_scales), v_in, v_out, const_cast<void*>(v_scales),
+                  desc, batch_size, offset, width, page_size, cache_seqlens, block_table, wbits,
+                  stream, false);
+}
+
+const char* kvq_status_string(kvq_status s) {
+  switch (s) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_NULL: return "null pointer";
+    case KVQ_ERR_SHAPE: return "bad shape";
+    case KVQ_ERR_WBITS: return "wbits must be 4 or 6";
+    case KVQ_ERR_RANGE: return "window, batch or page geometry out of range";
+    case KVQ_ERR_ALIGN: return "buffer not 16-byte aligned";
+    case KVQ_ERR_CUDA: return "CUDA runtime error";
+    case KVQ_ERR_DEVICE: return "device recorded bad paging metadata";
+  }
+  return "unknown status";
+}
+
+kvq_status kvq_poll_device_error(int32_t* code_out, void* stream) {
+  if (!code_out) return KVQ_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int h = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbolAsync(&h, kvq::g_device_error, sizeof(int), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return KVQ_ERR_CUDA;
+  if (cudaMemcpyToSymbolAsync(kvq::g_device_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return KVQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return KVQ_ERR_CUDA;
+  *code_out = h;
+  return h ? KVQ_ERR_DEVICE : KVQ_OK;
+}
+
+kvq_status kvq_selfcheck_code_rounding(int wbits, unsigned long long* mismatches, void* stream) {
+  if (!mismatches) return KVQ_ERR_NULL;
+  if (wbits != 4 && wbits != 6) return KVQ_ERR_WBITS;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(mismatches, 0, sizeof(unsigned long long), s) != cudaSuccess) return KVQ_ERR_CUDA;
+  if (wbits == 4)
+    kvq::selfcheck_rounding_kernel<4><<<0x7BFF, 256, 0, s>>>(mismatches);
+  else
+    kvq::selfcheck_rounding_kernel<6><<<0x7BFF, 256, 0, s>>>(mismatches);
+  return launch_status();
+}
+
+}  // extern "C"

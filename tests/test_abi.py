@@ -1,0 +1,119 @@
+"""Host-side checks of the C ABI (no GPU needed): libkvq.so loads, exports every
+function include/kvq.h declares, and rejects bad arguments before touching the
+device.  Pointers passed here are never dereferenced: every call is expected to
+fail validation (or be a no-op) on the host."""
+from __future__ import annotations
+
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def kvq():
+    from kv_cache_quantization_fp16_b200 import _build
+
+    _build.build()
+    import kv_cache_quantization_fp16_b200 as m
+
+    return m
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"KVQ_API\s+[\w\s\*]+?\b(kvq_\w+)\s*\(", text):
+            names.add(m.group(1))
+    return names
+
+
+def test_header_declares_the_four_conversions():
+    names = _declared_functions()
+    for n in ("kvq_fp16_to_fp8", "kvq_fp8_to_fp16", "kvq_fp16_to_q_kv", "kvq_q_to_fp16_kv",
+              "kvq_status_string", "kvq_poll_device_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(kvq):
+    lib = ctypes.CDLL(kvq.LIB_PATH)
+    for n in _declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(kvq):
+    L = kvq.library()
+    for s in range(8):
+        assert L.kvq_status_string(s)
+    assert L.kvq_status_string(99) == b"unknown status"
+
+
+def _desc(kvq, d0=2, d1=16, H=2, D=64, stride=0):
+    return kvq._Desc(d0, d1, H, D, stride)
+
+
+FAKE = 0x7F0000000000  # 16-byte aligned, never dereferenced
+
+
+def test_fp8_validation(kvq):
+    L = kvq.library()
+    d = _desc(kvq)
+    by = ctypes.byref
+    assert L.kvq_fp16_to_fp8(None, FAKE, by(d), 2, 0, 16, None) == 1
+    assert L.kvq_fp16_to_fp8(FAKE, FAKE, None, 2, 0, 16, None) == 1
+    assert L.kvq_fp16_to_fp8(FAKE + 8, FAKE, by(d), 2, 0, 16, None) == 5
+    assert L.kvq_fp8_to_fp16(FAKE, FAKE, by(d), 3, 0, 16, None) == 4   # batch > dim0
+    assert L.kvq_fp8_to_fp16(FAKE, FAKE, by(d), 2, 8, 9, None) == 4    # window past the end
+    assert L.kvq_fp8_to_fp16(FAKE, FAKE, by(d), 2, -1, 2, None) == 4   # negative offset
+    assert L.kvq_fp8_to_fp16(FAKE, FAKE, by(_desc(kvq, D=12)), 2, 0, 1, None) == 2
+    assert L.kvq_fp8_to_fp16(FAKE, FAKE, by(_desc(kvq, H=0)), 2, 0, 1, None) == 2
+    # empty windows are accepted and enqueue nothing
+    assert L.kvq_fp16_to_fp8(FAKE, FAKE, by(d), 2, 3, 0, None) == 0
+    assert L.kvq_fp16_to_fp8(FAKE, FAKE, by(d), 0, 0, 16, None) == 0
+
+
+def test_q_validation(kvq):
+    L = kvq.library()
+    d = _desc(kvq)
+    by = ctypes.byref
+    P = [FAKE] * 6
+    assert L.kvq_fp16_to_q_kv(*P, by(d), 2, 0, 16, 0, None, None, 5, None) == 3
+    assert L.kvq_fp16_to_q_kv(*P, by(d), 2, 0, 16, 0, None, None, 8, None) == 3
+    assert L.kvq_q_to_fp16_kv(*P, by(_desc(kvq, D=48)), 2, 0, 16, 0, None, None, 4, None) == 2
+    assert L.kvq_fp16_to_q_kv(*P[:5], None, by(d), 2, 0, 16, 0, None, None, 4, None) == 1
+    assert L.kvq_fp16_to_q_kv(*P[:3], FAKE + 4, *P[4:], by(d), 2, 0, 16, 0, None, None, 4, None) == 5
+    assert L.kvq_fp16_to_q_kv(*P, by(d), 2, 10, 7, 0, None, None, 4, None) == 4
+    # paged: needs seqlens + block_table, page_size == dim1, stride >= 1
+    dp = _desc(kvq, d0=10, d1=16, stride=4)
+    assert L.kvq_fp16_to_q_kv(*P, by(dp), 2, 0, 16, 16, None, FAKE, 4, None) == 1
+    assert L.kvq_fp16_to_q_kv(*P, by(dp), 2, 0, 16, 8, FAKE, FAKE, 4, None) == 4
+    assert L.kvq_fp16_to_q_kv(*P, by(_desc(kvq, d0=10, d1=16, stride=0)), 2, 0, 16, 16, FAKE, FAKE, 4,
+                              None) == 4
+    assert L.kvq_fp16_to_q_kv(*P, by(dp), 2, 0, 16, 16, FAKE + 2, FAKE, 4, None) == 5
+    assert L.kvq_fp16_to_q_kv(*P, by(dp), 2, 0, 16, -1, FAKE, FAKE, 4, None) == 4
+    # paged offsets may be negative (windows end at cache_seqlens); empty is a no-op
+    assert L.kvq_fp16_to_q_kv(*P, by(dp), 2, -5, 0, 16, FAKE, FAKE, 4, None) == 0
+    assert L.kvq_q_to_fp16_kv(*P, by(dp), 0, -5, 5, 16, FAKE, FAKE, 6, None) == 0
+
+
+def test_selfcheck_validation(kvq):
+    L = kvq.library()
+    assert L.kvq_selfcheck_code_rounding(4, None, None) == 1
+    assert L.kvq_selfcheck_code_rounding(5, FAKE, None) == 3
+    assert L.kvq_poll_device_error(None, None) == 1
+
+
+def test_python_binding_checks_dtypes(kvq):
+    import torch
+
+    k = torch.zeros(1, 4, 1, 32, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        kvq.fp16_to_fp8(k, torch.zeros(1, 4, 1, 32, dtype=torch.uint8), 1, 0, 4)  # CPU tensors
+    with pytest.raises(ValueError):
+        kvq.fp16_to_fp8(k.float(), k, 1, 0, 4)

@@ -6,7 +6,8 @@ outliers and 0.1% subnormals), window offset 1024, width 2048.  One step is
 fp16_to_fp8(K), fp16_to_fp8(V), fp8_to_fp16(K), fp8_to_fp16(V) through the C
 ABI on resident device buffers.  The metric is algorithmic GB/s (bytes read +
 bytes written: 3 bytes per element per conversion), with L2 flushed between
-steps (a 256 MiB memset outside the per-step CUDA events).
+steps (a 256 MiB write then a 256 MiB read, outside the per-step CUDA events,
+so no dirty flush lines are written back inside a timed kernel).
 
 Extra keys:
   roofline      the dominant kernel's achieved GB/s (algorithmic bytes per
@@ -140,6 +141,20 @@ class ClockSampler:
 
 # ---------------------------------------------------------- GPU workloads ----
 
+class L2Flush:
+    """Evict L2 between timed steps without leaving dirty lines behind: write a buffer
+    twice the size of L2, then read another one, so the lines the next step evicts
+    are clean and no write-back of the flush lands inside its timing."""
+
+    def __init__(self, dev, nbytes=FLUSH_BYTES):
+        self.w = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(nbytes // 4, dtype=torch.int32, device=dev)
+
+    def __call__(self):
+        self.w.zero_()
+        self.sink = torch.amax(self.r)
+
+
 class Fp8Step:
     """Headline step on one rank: FP8 encode + decode of the K and V windows."""
 
@@ -160,6 +175,7 @@ class Fp8Step:
         self.launches_per_step = 4
 
     def run(self, ev=None):
+        """The four conversions; `ev` (3 events) marks the boundaries between them."""
         kvq, b, o, w = self.kvq, self.batch, self.off, self.w
         kvq.fp16_to_fp8(self.k, self.k8, b, o, w)
         if ev is not None:
@@ -173,33 +189,54 @@ class Fp8Step:
         kvq.fp8_to_fp16(self.v8, self.vy, b, o, w)
 
 
-def time_device(fn, steps, warmup, flush, sampler=None, n_marks=0):
-    """Per-step CUDA-event times (ms) of fn(ev) with an L2 flush before each step."""
-    for _ in range(warmup):
-        flush.zero_()
+def capture(fn, n_marks=0):
+    """Capture fn(marks) in a CUDA graph (after one eager warm-up on a side stream), so
+    a step replays its launches back to back without host launch gaps.  `marks` are
+    external events recorded between the launches, readable after each replay."""
+    marks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_marks)]
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
         fn(None)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn(marks if n_marks else None)
+    torch.cuda.synchronize()
+    return g, marks
+
+
+def time_device(fn, steps, warmup, flush, sampler=None, n_marks=0):
+    """Per-step CUDA-event times (ms) of the captured fn, with an L2 flush (outside the
+    events) before each step.  With marks, also the per-launch segments of every step."""
+    g, marks = capture(fn, n_marks)
+    for _ in range(warmup):
+        flush()
+        g.replay()
     torch.cuda.synchronize()
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    mids = [[torch.cuda.Event(enable_timing=True) for _ in range(n_marks)] for _ in range(steps)]
+    segs = []
     _barrier()
     torch.cuda.synchronize()
     if sampler:
         sampler.mark()
     for i in range(steps):
-        flush.zero_()
+        flush()
         starts[i].record()
-        fn(mids[i] if n_marks else None)
+        g.replay()
         ends[i].record()
+        if n_marks:
+            ends[i].synchronize()
+            pts = [starts[i]] + marks + [ends[i]]
+            segs.append([a.elapsed_time(b) for a, b in zip(pts[:-1], pts[1:])])
     torch.cuda.synchronize()
     if sampler:
         sampler.mark()
     _barrier()
     per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    segs = []
-    for i in range(steps):
-        pts = [starts[i]] + mids[i] + [ends[i]]
-        segs.append([a.elapsed_time(b) for a, b in zip(pts[:-1], pts[1:])])
+    del g
     return per_step, segs
 
 
@@ -346,6 +383,70 @@ def model_layers(kvq, dev, peak, steps, flush, layers=32):
     return res
 
 
+# ------------------------------------------------------ single-op cases ----
+
+CASES = ("fp8enc", "fp8dec", "q4enc", "q4dec", "q6enc", "q6dec", "paged_prefill_q4enc", "paged_prefill_q4dec",
+         "paged_decode_q4enc", "model_layer_q6enc", "model_layer_q6dec")
+
+
+def run_case(kvq, dev, name, batch, steps, warmup, peak):
+    """One conversion on one workload, `steps` timed launches (for quick sweeps and ncu).
+    Contiguous cases use the channel-outlier recipe at [batch, 8192, 8, 128] (batch 4:
+    268 MB of FP16 K+V, above the L2 size); paged cases the 2048-page pool; model cases
+    one 1024-page layer."""
+    flush = L2Flush(dev)
+    if name.startswith("fp8") or name[:2] in ("q4", "q6"):
+        k, v = workloads.channel_outliers(shape=(batch, 8192, 8, 128), device=dev)
+        B, S = k.shape[:2]
+        if name.startswith("fp8"):
+            k8 = torch.zeros(k.shape, dtype=torch.uint8, device=dev)
+            y = torch.empty_like(k)
+            kvq.fp16_to_fp8(k, k8, B, 0, S)
+            nb = 3.0 * k.numel()
+            fn = (lambda: kvq.fp16_to_fp8(k, k8, B, 0, S)) if name == "fp8enc" else \
+                 (lambda: kvq.fp8_to_fp16(k8, y, B, 0, S))
+        else:
+            wb = int(name[1])
+            cs, ss = kvq.q_shapes(tuple(k.shape), wb)
+            kc, vc = (torch.zeros(cs, dtype=torch.uint8, device=dev) for _ in range(2))
+            ks, vs = (torch.zeros(ss, dtype=torch.float16, device=dev) for _ in range(2))
+            ky, vy = torch.empty_like(k), torch.empty_like(v)
+            kvq.fp16_to_q_kv(k, kc, ks, v, vc, vs, B, 0, S, 0, None, None, wb)
+            nb = BYTES_PER_ELEM[wb] * 2 * k.numel()
+            fn = (lambda: kvq.fp16_to_q_kv(k, kc, ks, v, vc, vs, B, 0, S, 0, None, None, wb)) \
+                if name.endswith("enc") else (lambda: kvq.q_to_fp16_kv(kc, ky, ks, vc, vy, vs, B, 0, S, 0, None,
+                                                                        None, wb))
+    elif name.startswith("paged"):
+        pool = workloads.paged_pool(device=dev)
+        P, ps, H, D = pool.k.shape
+        off, w = (0, 1) if "decode" in name else (-512, 512)
+        cs, ss = kvq.q_shapes(tuple(pool.k.shape), 4)
+        kc, vc = (torch.zeros(cs, dtype=torch.uint8, device=dev) for _ in range(2))
+        ks, vs = (torch.zeros(ss, dtype=torch.float16, device=dev) for _ in range(2))
+        lens = pool.cache_seqlens.cpu()
+        npos = sum(max(0, int(L) + off + w) - max(0, int(L) + off) for L in lens)
+        nb = BYTES_PER_ELEM[4] * 2 * npos * H * D
+        args = (32, off, w, ps, pool.cache_seqlens, pool.block_table, 4)
+        kvq.fp16_to_q_kv(pool.k, kc, ks, pool.v, vc, vs, *args)
+        fn = (lambda: kvq.fp16_to_q_kv(pool.k, kc, ks, pool.v, vc, vs, *args)) if name.endswith("enc") else \
+             (lambda: kvq.q_to_fp16_kv(kc, pool.k, ks, vc, pool.v, vs, *args))
+    else:
+        pool = workloads.model_layer(0, device=dev)
+        cs, ss = kvq.q_shapes(tuple(pool.k.shape), 6)
+        kc, vc = (torch.zeros(cs, dtype=torch.uint8, device=dev) for _ in range(2))
+        ks, vs = (torch.zeros(ss, dtype=torch.float16, device=dev) for _ in range(2))
+        args = (8, -32768, 32768, 256, pool.cache_seqlens, pool.block_table, 6)
+        kvq.fp16_to_q_kv(pool.k, kc, ks, pool.v, vc, vs, *args)
+        nb = BYTES_PER_ELEM[6] * 2 * pool.k.numel()
+        fn = (lambda: kvq.fp16_to_q_kv(pool.k, kc, ks, pool.v, vc, vs, *args)) if name.endswith("enc") else \
+             (lambda: kvq.q_to_fp16_kv(kc, pool.k, ks, vc, pool.v, vs, *args))
+    per, _ = time_device(lambda ev: fn(), steps, warmup, flush)
+    ms = statistics.mean(per)
+    return {"case": name, "batch": batch, "bytes": int(nb), "us": round(ms * 1e3, 2),
+            "us_min": round(min(per) * 1e3, 2), "gbs": round(nb / ms / 1e6, 1),
+            "frac": round(nb / ms / 1e6 / peak, 3)}
+
+
 # -------------------------------------------------------------- CPU oracle ----
 
 def oracle_step_sample(batch=4, max_seconds=12.0, min_reps=1):
@@ -390,6 +491,9 @@ def main():
     ap.add_argument("--no-per-op", action="store_true", help="skip the per-op table")
     ap.add_argument("--no-model", action="store_true", help="skip the 32-layer model-sized rows")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", choices=CASES, action="append",
+                    help="time only these single conversions (for sweeps and ncu); no headline line")
+    ap.add_argument("--case-batch", type=int, default=4)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -415,7 +519,11 @@ def main():
     import kv_cache_quantization_fp16_b200 as kvq
 
     peak, peak_kind = hbm_peak()
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    if args.case:
+        for c in args.case:
+            print(json.dumps(run_case(kvq, dev, c, args.case_batch, args.steps, args.warmup, peak)), flush=True)
+        return 0
+    flush = L2Flush(dev)
     sampler = ClockSampler(local_rank).start() if rank == 0 else None
 
     # each rank converts its own 4 sequences: a global batch of 4 * world (weak scaling)
@@ -436,8 +544,6 @@ def main():
 
     per_op = []
     if rank == 0 and not args.no_per_op:
-        del flush
-        flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
         per_op = per_op_measurements(kvq, dev, peak, max(20, args.steps // 5), flush,
                                      include_model=not args.no_model)
     if sampler:
@@ -472,7 +578,7 @@ def main():
         "data": "synthetic (seeded N(0,1) with 1% outliers and 0.1% subnormals, drawn on device)",
         "config": {"workload": HEADLINE["workload"], "shape": list(HEADLINE["shape"]),
                    "global_batch": batch * world, "offset": HEADLINE["offset"], "width": HEADLINE["width"],
-                   "ops": names, "l2": "flushed between steps (256 MiB memset outside the per-step events)",
+                   "ops": names, "launch": "CUDA graph of the 4 conversions, replayed once per step", "l2": "flushed between steps (256 MiB write + 256 MiB read, outside the per-step events)",
                    "parallelism": f"replicas x{world}, each rank its own 4 sequences"},
         "roofline": {"bound": "hbm", "kernel": dom[0], "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 3), "peak_kind": peak_kind,

@@ -93,6 +93,7 @@ struct Params {
 // ---------------------------------------------------------------------------
 
 struct Fp8Encode {
+  static constexpr int kElemsPerTile = kThreads * kUnroll * 8;
   __device__ static void tile(const Params& p, int kv, long long row0, int nrows) {
     const long long e0 = row0 * p.g.hd;
     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __half*>(p.in[kv]) + e0);
@@ -115,6 +116,7 @@ struct Fp8Encode {
 };
 
 struct Fp8Decode {
+  static constexpr int kElemsPerTile = kThreads * kUnroll * 8;
   __device__ static void tile(const Params& p, int kv, long long row0, int nrows) {
     const long long e0 = row0 * p.g.hd;
     const uint2* src = reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(p.in[kv]) + e0);
@@ -136,49 +138,51 @@ struct Fp8Decode {
   }
 };
 
-// Q encode: a quad of lanes (4 x 8 elements) holds one 32-element block.
+// Q encode: one thread owns whole 32-element blocks (4 x 16-byte loads), so
+// the absmax needs no shuffles, the scale and reciprocal are computed once per
+// block, and the packed codes leave as one 16-byte (Q4) or three 8-byte (Q6)
+// stores.  Two blocks per thread are loaded before either is encoded.
 template <int B>
 struct QEncode {
+  static constexpr int kUnrollBlocks = 2;
+  static constexpr int kElemsPerTile = kThreads * kBlockElems * kUnrollBlocks;
+
   __device__ static void tile(const Params& p, int kv, long long row0, int nrows) {
     const long long e0 = row0 * p.g.hd;
     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __half*>(p.in[kv]) + e0);
     uint8_t* codes = static_cast<uint8_t*>(p.out[kv]) + e0 * B / 8;
     __half* scales = static_cast<__half*>(p.scales[kv]) + e0 / kBlockElems;
-    const int nvec = static_cast<int>(nrows * p.g.hd / 8);  // multiple of 4
-    for (int base = 0; base < nvec; base += kThreads * kUnroll) {
-      uint4 x[kUnroll];
+    const int nblk = static_cast<int>(nrows * p.g.hd / kBlockElems);
+    for (int base = 0; base < nblk; base += kThreads * kUnrollBlocks) {
+      uint4 x[kUnrollBlocks][4];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int v = base + u * kThreads + threadIdx.x;
-        x[u] = make_uint4(0, 0, 0, 0);
-        if (v < nvec) x[u] = __ldg(src + v);
+      for (int u = 0; u < kUnrollBlocks; ++u) {
+        const int b = base + u * kThreads + threadIdx.x;
+        if (b < nblk) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) x[u][k] = __ldg(src + static_cast<long long>(b) * 4 + k);
+        }
       }
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int v = base + u * kThreads + threadIdx.x;
-        uint32_t m = absmax_bits_v8(x[u]);
-        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-        if (v >= nvec) continue;  // whole quads are in or out (nvec % 4 == 0)
-        const __half s16 = block_scale<B>(m);
+      for (int u = 0; u < kUnrollBlocks; ++u) {
+        const int b = base + u * kThreads + threadIdx.x;
+        if (b >= nblk) continue;
+        const __half s16 = block_scale<B>(absmax_bits_block(x[u]));
         const BlockScale bs = make_block_scale(s16);
-        uint32_t c[8];
-        quant_v8<B>(x[u], bs, c);
+        uint32_t w[B];
+        if (__half_as_ushort(s16) < 0x0400u)
+          encode_block_words<B, true>(x[u], bs, w);
+        else
+          encode_block_words<B, false>(x[u], bs, w);
         if (B == 4) {
-          reinterpret_cast<uint32_t*>(codes)[v] = pack_q4(c);
+          reinterpret_cast<uint4*>(codes)[b] = make_uint4(w[0], w[1], w[2 % B], w[3 % B]);
         } else {
-          uint32_t lo, hi;
-          pack_q6(c, lo, hi);
-          uint8_t* dst = codes + static_cast<long long>(v) * 6;
-          if ((v & 1) == 0) {  // 4-byte aligned start
-            *reinterpret_cast<uint32_t*>(dst) = lo;
-            *reinterpret_cast<uint16_t*>(dst + 4) = static_cast<uint16_t>(hi);
-          } else {             // 2-byte aligned start, 4-byte aligned at +2
-            *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(lo);
-            *reinterpret_cast<uint32_t*>(dst + 2) = (lo >> 16) | (hi << 16);
-          }
+          uint2* dst = reinterpret_cast<uint2*>(codes + static_cast<long long>(b) * 24);
+          dst[0] = make_uint2(w[0], w[1]);
+          dst[1] = make_uint2(w[2 % B], w[3 % B]);
+          dst[2] = make_uint2(w[4 % B], w[5 % B]);
         }
-        if ((threadIdx.x & 3) == 0) scales[v >> 2] = s16;
+        scales[b] = s16;
       }
     }
   }
@@ -186,6 +190,7 @@ struct QEncode {
 
 template <int B>
 struct QDecode {
+  static constexpr int kElemsPerTile = kThreads * kUnroll * 8;
   __device__ static void tile(const Params& p, int kv, long long row0, int nrows) {
     const long long e0 = row0 * p.g.hd;
     const uint8_t* codes = static_cast<const uint8_t*>(p.in[kv]) + e0 * B / 8;
@@ -204,16 +209,14 @@ struct QDecode {
           if (B == 4) {
             lo[u] = __ldg(reinterpret_cast<const uint32_t*>(codes) + v);
           } else {
-            const uint8_t* src = codes + static_cast<long long>(v) * 6;
-            if ((v & 1) == 0) {
-              lo[u] = __ldg(reinterpret_cast<const uint32_t*>(src));
-              hi[u] = __ldg(reinterpret_cast<const uint16_t*>(src + 4));
-            } else {
-              const uint32_t a = __ldg(reinterpret_cast<const uint16_t*>(src));
-              const uint32_t b = __ldg(reinterpret_cast<const uint32_t*>(src + 2));
-              lo[u] = a | (b << 16);
-              hi[u] = b >> 16;
-            }
+            // lane pair = one 12-byte group; the even lane needs words 0-1, the
+            // odd lane words 1-2 (bits 48..95 of the group)
+            const uint32_t* grp = reinterpret_cast<const uint32_t*>(codes + static_cast<long long>(v >> 1) * 12);
+            const uint32_t sh = (v & 1) * 16;
+            const uint32_t a = __ldg(grp + (v & 1));
+            const uint32_t b = __ldg(grp + (v & 1) + 1);
+            lo[u] = __funnelshift_r(a, b, sh);
+            hi[u] = (b >> sh) & 0xFFFFu;
           }
           s[u] = __ldg(scales + (v >> 2));
         }
@@ -260,18 +263,30 @@ __global__ void __launch_bounds__(kThreads) convert_kernel(const __grid_constant
 
 template <int B>
 __global__ void selfcheck_rounding_kernel(unsigned long long* mismatches) {
-  // blockIdx.x + gridDim.x * blockIdx.y enumerates s bit patterns 1..0x7BFF;
-  // threads enumerate x over all 65536 bit patterns, skipping Inf / NaN.
+  // blockIdx.x enumerates s bit patterns 1..0x7BFF; threads enumerate x over
+  // all 65536 bit patterns, skipping Inf / NaN.  Both forms the kernels use
+  // are checked: the clamped one for every pair, the unclamped one (used when
+  // the scale is normal) for every pair a block can produce.  A block gets the
+  // scale s only if absmax / maxq rounds to s, so its elements satisfy
+  // |x| <= maxq * (s + ulp(s) / 2).
   const uint32_t s_bits = 1 + blockIdx.x;
   const __half s16 = __ushort_as_half(static_cast<unsigned short>(s_bits));
   const BlockScale bs = make_block_scale(s16);
+  const bool normal = s_bits >= 0x0400u;
+  const int e_field = static_cast<int>(s_bits >> 10);  // binary16 exponent field, 1..30 when normal
+  const float half_ulp = normal ? __int_as_float((e_field - 26 + 127) << 23) : 0.0f;
+  const float reach = QParams<B>::maxq * (bs.s + half_ulp);  // exact: <= 17 significant bits
   unsigned long long bad = 0;
   for (uint32_t xb = threadIdx.x; xb < 65536u; xb += blockDim.x) {
     if (((xb >> 10) & 0x1F) == 0x1F) continue;
     const float x = __half2float(__ushort_as_half(static_cast<unsigned short>(xb)));
-    const uint32_t fast = quant_code_bits<B>(x, bs) & ((1u << B) - 1);
     const uint32_t ref = quant_code_ieee<B>(x, bs.s);
-    bad += (fast != ref);
+    const uint32_t clamped = quant_code_bits<B, true>(x, bs) & ((1u << B) - 1);
+    bad += (clamped != ref);
+    if (normal && fabsf(x) <= reach) {
+      const uint32_t plain = quant_code_bits<B, false>(x, bs) & ((1u << B) - 1);
+      bad += (plain != ref);
+    }
   }
   if (bad) atomicAdd(mismatches, bad);
 }
@@ -311,10 +326,9 @@ int gcd_int(int a, int b) {
   return a;
 }
 
-// Positions per tile: about kThreads * kUnroll * 8 elements, a power of two,
-// and a divisor of page_size in paged mode.
-int pick_tile_pos(long long hd, int page_size) {
-  const long long target = static_cast<long long>(kThreads) * kUnroll * 8;
+// Positions per tile: about `target` elements, a power of two, and a divisor
+// of page_size in paged mode.
+int pick_tile_pos(long long hd, int page_size, long long target) {
   int t = floor_pow2(target / hd > 0 ? target / hd : 1);
   if (page_size > 0) t = gcd_int(t, page_size);
   return t;
@@ -326,7 +340,8 @@ kvq_status launch_status() {
 }
 
 template <class Op>
-kvq_status launch(const Params& p, int nkv, void* stream) {
+kvq_status launch(Params p, int nkv, void* stream) {
+  p.g.tile_pos = pick_tile_pos(p.g.hd, p.g.page_size, Op::kElemsPerTile);
   const int paged = p.g.page_size > 0;
   const long long tiles = (static_cast<long long>(p.g.width) + p.g.tile_pos - 1) / p.g.tile_pos + paged;
   if (tiles > 0x7FFFFFFFLL) return KVQ_ERR_RANGE;
@@ -347,7 +362,7 @@ Geometry make_geometry(const kvq_cache_desc* d, int batch, int offset, int width
   g.offset = offset;
   g.width = width;
   g.page_size = page_size;
-  g.tile_pos = pick_tile_pos(g.hd, page_size);
+  g.tile_pos = 1;  // set per kernel by launch()
   g.seqlens = seqlens;
   g.block_table = block_table;
   return g;

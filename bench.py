@@ -81,6 +81,35 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.txt")
+
+
+def kernel_source_digest() -> str:
+    """sha256 over the CUDA sources, to tell whether recorded ncu counters are current."""
+    import glob
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "kv_cache_quantization_fp16_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes (read + write) per launch of `kernel` on the headline workload from the
+    committed ncu summary, or None when the kernels changed since it was captured."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) == 3 and not line.startswith("#") and parts[0] == kernel:
+                    return int(parts[1]) if parts[2] == kernel_source_digest() else None
+    except OSError:
+        pass
+    return None
+
+
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons while running."""
 
@@ -385,7 +414,7 @@ def model_layers(kvq, dev, peak, steps, flush, layers=32):
 
 # ------------------------------------------------------ single-op cases ----
 
-CASES = ("fp8enc", "fp8dec", "q4enc", "q4dec", "q6enc", "q6dec", "paged_prefill_q4enc", "paged_prefill_q4dec",
+CASES = ("headline_fp8enc", "headline_fp8dec", "fp8enc", "fp8dec", "q4enc", "q4dec", "q6enc", "q6dec", "paged_prefill_q4enc", "paged_prefill_q4dec",
          "paged_decode_q4enc", "model_layer_q6enc", "model_layer_q6dec")
 
 
@@ -395,7 +424,17 @@ def run_case(kvq, dev, name, batch, steps, warmup, peak):
     268 MB of FP16 K+V, above the L2 size); paged cases the 2048-page pool; model cases
     one 1024-page layer."""
     flush = L2Flush(dev)
-    if name.startswith("fp8") or name[:2] in ("q4", "q6"):
+    if name.startswith("headline"):
+        B, S, H, D = HEADLINE["shape"]
+        o, w = HEADLINE["offset"], HEADLINE["width"]
+        k, _ = workloads.fp8_window(shape=(B, S, H, D), device=dev)
+        k8 = torch.zeros(k.shape, dtype=torch.uint8, device=dev)
+        y = torch.empty_like(k)
+        kvq.fp16_to_fp8(k, k8, B, o, w)
+        nb = 3.0 * B * w * H * D
+        fn = (lambda: kvq.fp16_to_fp8(k, k8, B, o, w)) if name.endswith("enc") else \
+             (lambda: kvq.fp8_to_fp16(k8, y, B, o, w))
+    elif name.startswith("fp8") or name[:2] in ("q4", "q6"):
         k, v = workloads.channel_outliers(shape=(batch, 8192, 8, 128), device=dev)
         B, S = k.shape[:2]
         if name.startswith("fp8"):
@@ -529,15 +568,24 @@ def main():
     # each rank converts its own 4 sequences: a global batch of 4 * world (weak scaling)
     batch = HEADLINE["shape"][0]
     step = Fp8Step(kvq, dev, batch, seed_shift=rank)
-    per_step, segs = time_device(step.run, args.steps, args.warmup, flush, sampler, n_marks=3)
+    # timed region: the step graph replayed as it is (no event nodes inside it)
+    per_step, _ = time_device(step.run, args.steps, args.warmup, flush, sampler)
     ms_local = statistics.mean(per_step)
     ms = max_over_ranks(ms_local, dev)
+    # per-launch durations: the same graph with events between its launches
+    _, segs = time_device(step.run, max(50, args.steps // 10), 3, flush, None, n_marks=3)
     names = ["fp16_to_fp8(K)", "fp16_to_fp8(V)", "fp8_to_fp16(K)", "fp8_to_fp16(V)"]
     seg_ms = [statistics.mean(s[i] for s in segs) for i in range(4)]
-    enc_ms = (seg_ms[0] + seg_ms[1]) / 2
-    dec_ms = (seg_ms[2] + seg_ms[3]) / 2
-    dom = ("fp16_to_fp8", enc_ms) if enc_ms >= dec_ms else ("fp8_to_fp16", dec_ms)
+    # Event nodes between launches cost time of their own, so each launch's duration
+    # inside the timed (unmarked) step is the step time split in the proportions of
+    # the marked segments.
+    share = [t / sum(seg_ms) for t in seg_ms]
+    launch_ms = [ms_local * f for f in share]
+    enc_ms = (launch_ms[0] + launch_ms[1]) / 2
+    dec_ms = (launch_ms[2] + launch_ms[3]) / 2
+    dom = ("fp16_to_fp8", enc_ms, 0) if enc_ms >= dec_ms else ("fp8_to_fp16", dec_ms, 2)
     achieved = step.launch_bytes / dom[1] / 1e6
+    dom_isolated_ms = (seg_ms[dom[2]] + seg_ms[dom[2] + 1]) / 2
 
     e2e_ms, h2d, d2h = e2e_fp8(kvq, step, max(10, args.steps // 10), 3, dev)
     e2e_ms = max_over_ranks(e2e_ms, dev)
@@ -583,8 +631,11 @@ def main():
         "roofline": {"bound": "hbm", "kernel": dom[0], "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 3), "peak_kind": peak_kind,
                      "bytes_per_launch": int(step.launch_bytes), "us_per_launch": round(dom[1] * 1e3, 2),
-                     "traffic": None},
-        "per_kernel_us": {n: round(t * 1e3, 2) for n, t in zip(names, seg_ms)},
+                     "duration": "timed step x this launch's share of the event-marked step",
+                     "us_per_launch_marked": round(dom_isolated_ms * 1e3, 2),
+                     "traffic": recorded_traffic(dom[0])},
+        "per_kernel_us": {n: round(t * 1e3, 2) for n, t in zip(names, launch_ms)},
+        "per_kernel_us_marked": {n: round(t * 1e3, 2) for n, t in zip(names, seg_ms)},
         "cpu_baseline": cpu,
         "e2e": {"value": round(world * step.bytes_per_step / e2e_ms / 1e6, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

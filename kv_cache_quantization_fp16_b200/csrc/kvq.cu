@@ -13,8 +13,8 @@
 // never straddles a page.  One CTA converts one tile: thread 0 resolves the
 // tile (window clipping, the block_table lookup) once and stages the physical
 // row in shared memory, then all threads stream the tile's elements as a flat
-// array, 8 elements (16 bytes of FP16) per thread per step, with kUnroll
-// independent 16-byte loads in flight per thread.  Grid: x = tiles, y =
+// array; each op fixes its CTA size and how many independent loads every
+// thread has in flight (see the per-op structs).  Grid: x = tiles, y =
 // sequences, z = K / V (the fused K+V launch).
 //
 // This is a streaming, HBM-bound path: no tensor cores, no shared-memory
@@ -28,8 +28,6 @@
 
 namespace kvq {
 
-constexpr int kThreads = 256;
-constexpr int kUnroll = 4;
 constexpr int kBlockElems = 32;  // Q scale block along head_dim
 
 // Per-device error word for problems only the device can see.
@@ -47,18 +45,27 @@ struct Geometry {
   const int32_t* block_table;
 };
 
-// Tile `tile_x` of sequence `seq`: first physical row and number of positions,
-// or false when the tile is empty or its page is invalid.
-__device__ bool resolve_tile(const Geometry& g, int seq, int tile_x, long long& row0, int& nrows) {
-  if (g.page_size == 0) {
-    const long long p0 = static_cast<long long>(g.offset) + static_cast<long long>(tile_x) * g.tile_pos;
-    const long long p1 = min(static_cast<long long>(g.offset) + g.width, p0 + g.tile_pos);
-    if (p0 >= p1) return false;
-    row0 = static_cast<long long>(seq) * g.dim1 + p0;
-    nrows = static_cast<int>(p1 - p0);
-    return true;
-  }
-  const long long start = static_cast<long long>(g.seqlens[seq]) + g.offset;
+// Tile `tile_x` of sequence `seq` in contiguous mode: first row and number of
+// positions, or false when the tile lies past the end of the window.
+__device__ __forceinline__ bool contiguous_tile(const Geometry& g, int seq, int tile_x, long long& row0,
+                                                int& nrows) {
+  const long long p0 = static_cast<long long>(g.offset) + static_cast<long long>(tile_x) * g.tile_pos;
+  const long long p1 = min(static_cast<long long>(g.offset) + g.width, p0 + g.tile_pos);
+  if (p0 >= p1) return false;
+  row0 = static_cast<long long>(seq) * g.dim1 + p0;
+  nrows = static_cast<int>(p1 - p0);
+  return true;
+}
+
+// Paged mode: the window of sequence `seq` is [max(0, seqlen + offset),
+// seqlen + offset + width) in logical positions; tile `tile_x` is the x-th
+// tile_pos-aligned run of it (tile_pos divides page_size, so the run lies in
+// one page).  `bt_row` is the sequence's block-table row staged in shared
+// memory (or null: read it from global memory).  Bad metadata is recorded by
+// the thread with `report` set and the tile is skipped.
+__device__ __forceinline__ bool paged_tile(const Geometry& g, int seq, int tile_x, int seqlen,
+                                           const int* bt_row, bool report, long long& row0, int& nrows) {
+  const long long start = static_cast<long long>(seqlen) + g.offset;
   const long long lo = start < 0 ? 0 : start;
   const long long hi = start + g.width;
   if (lo >= hi) return false;
@@ -68,12 +75,12 @@ __device__ bool resolve_tile(const Geometry& g, int seq, int tile_x, long long& 
   if (p0 >= p1) return false;
   const long long lp = p0 / g.page_size;
   if (lp >= g.bt_stride) {
-    record_error(KVQ_DEV_BAD_PAGE_INDEX);
+    if (report) record_error(KVQ_DEV_BAD_PAGE_INDEX);
     return false;
   }
-  const int page = g.block_table[static_cast<long long>(seq) * g.bt_stride + lp];
+  const int page = bt_row ? bt_row[lp] : g.block_table[static_cast<long long>(seq) * g.bt_stride + lp];
   if (page < 0 || page >= g.dim0) {
-    record_error(KVQ_DEV_BAD_PAGE);
+    if (report) record_error(KVQ_DEV_BAD_PAGE);
     return false;
   }
   row0 = static_cast<long long>(page) * g.page_size + p0 % g.page_size;
@@ -92,8 +99,14 @@ struct Params {
 // Per-tile bodies
 // ---------------------------------------------------------------------------
 
+// FP8: 128-thread CTAs with 8 independent 16-byte loads (or 8-byte loads for
+// decode) per thread, so a whole tile is requested at once and enough CTAs
+// stay resident (up to 16 per SM) for small windows to run in one wave.
 struct Fp8Encode {
+  static constexpr int kThreads = 128;
+  static constexpr int kUnroll = 8;
   static constexpr int kElemsPerTile = kThreads * kUnroll * 8;
+  static constexpr int kMinBlocksPerSM = 8;
   __device__ static void tile(const Params& p, int kv, long long row0, int nrows) {
     const long long e0 = row0 * p.g.hd;
     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __half*>(p.in[kv]) + e0);
@@ -116,7 +129,10 @@ struct Fp8Encode {
 };
 
 struct Fp8Decode {
+  static constexpr int kThreads = 128;
+  static constexpr int kUnroll = 8;
   static constexpr int kElemsPerTile = kThreads * kUnroll * 8;
+  static constexpr int kMinBlocksPerSM = 8;
   __device__ static void tile(const Params& p, int kv, long long row0, int nrows) {
     const long long e0 = row0 * p.g.hd;
     const uint2* src = reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(p.in[kv]) + e0);
@@ -144,8 +160,10 @@ struct Fp8Decode {
 // stores.  Two blocks per thread are loaded before either is encoded.
 template <int B>
 struct QEncode {
+  static constexpr int kThreads = 256;
   static constexpr int kUnrollBlocks = 2;
   static constexpr int kElemsPerTile = kThreads * kBlockElems * kUnrollBlocks;
+  static constexpr int kMinBlocksPerSM = 4;
 
   __device__ static void tile(const Params& p, int kv, long long row0, int nrows) {
     const long long e0 = row0 * p.g.hd;
@@ -190,7 +208,10 @@ struct QEncode {
 
 template <int B>
 struct QDecode {
+  static constexpr int kThreads = 256;
+  static constexpr int kUnroll = 4;
   static constexpr int kElemsPerTile = kThreads * kUnroll * 8;
+  static constexpr int kMinBlocksPerSM = 5;
   __device__ static void tile(const Params& p, int kv, long long row0, int nrows) {
     const long long e0 = row0 * p.g.hd;
     const uint8_t* codes = static_cast<const uint8_t*>(p.in[kv]) + e0 * B / 8;
@@ -237,23 +258,34 @@ struct QDecode {
 // ---------------------------------------------------------------------------
 
 template <class Op>
-__global__ void __launch_bounds__(kThreads) convert_kernel(const __grid_constant__ Params p) {
-  __shared__ long long s_row0;
-  __shared__ int s_nrows;
+__global__ void __launch_bounds__(Op::kThreads, Op::kMinBlocksPerSM) convert_kernel(const __grid_constant__ Params p) {
+  // Programmatic dependent launch: this grid may be launched while the
+  // previous kernel on the stream is still running; wait for it to finish (and
+  // its writes to become visible) before touching global memory, and let the
+  // next kernel start launching as soon as every CTA of this grid has started.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ int s_bt[Op::kThreads];
+  __shared__ int s_seqlen;
   const int kv = blockIdx.z;
   for (int seq = blockIdx.y; seq < p.g.batch; seq += gridDim.y) {
-    if (threadIdx.x == 0) {
-      long long r = -1;
-      int n = 0;
-      if (!resolve_tile(p.g, seq, blockIdx.x, r, n)) r = -1;
-      s_row0 = r;
-      s_nrows = n;
+    long long row0 = 0;
+    int nrows = 0;
+    bool ok;
+    if (p.g.page_size == 0) {
+      ok = contiguous_tile(p.g, seq, blockIdx.x, row0, nrows);
+    } else {
+      // Stage the sequence's block-table row (when it fits) together with its
+      // length, so the page lookup costs one memory round trip, not two.
+      const bool staged = p.g.bt_stride <= Op::kThreads;
+      if (staged && static_cast<int>(threadIdx.x) < p.g.bt_stride)
+        s_bt[threadIdx.x] = p.g.block_table[static_cast<long long>(seq) * p.g.bt_stride + threadIdx.x];
+      if (threadIdx.x == 0) s_seqlen = p.g.seqlens[seq];
+      __syncthreads();
+      ok = paged_tile(p.g, seq, blockIdx.x, s_seqlen, staged ? s_bt : nullptr, threadIdx.x == 0, row0, nrows);
+      __syncthreads();  // s_bt and s_seqlen are rewritten for the next sequence
     }
-    __syncthreads();
-    const long long row0 = s_row0;
-    const int nrows = s_nrows;
-    __syncthreads();
-    if (row0 >= 0) Op::tile(p, kv, row0, nrows);
+    if (ok) Op::tile(p, kv, row0, nrows);
   }
 }
 
@@ -345,9 +377,21 @@ kvq_status launch(Params p, int nkv, void* stream) {
   const int paged = p.g.page_size > 0;
   const long long tiles = (static_cast<long long>(p.g.width) + p.g.tile_pos - 1) / p.g.tile_pos + paged;
   if (tiles > 0x7FFFFFFFLL) return KVQ_ERR_RANGE;
-  dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(p.g.batch < 65535 ? p.g.batch : 65535),
-            static_cast<unsigned>(nkv));
-  convert_kernel<Op><<<grid, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(p.g.batch < 65535 ? p.g.batch : 65535),
+                     static_cast<unsigned>(nkv));
+  cfg.blockDim = dim3(Op::kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, convert_kernel<Op>, p) != cudaSuccess) {
+    cudaGetLastError();
+    return KVQ_ERR_CUDA;
+  }
   return launch_status();
 }
 

@@ -333,3 +333,14 @@ def test_runs_on_a_side_stream(kvq, oracle_mod, dev):
     s = torch.cuda.Stream(dev)
     with torch.cuda.stream(s):
         run_q(kvq, oracle_mod, k, v, 6, 2, 0, 64, dev)
+
+
+@pytest.mark.parametrize("wbits", [4, 6])
+def test_paged_wide_block_table(kvq, oracle_mod, dev, wbits):
+    """A block table wider than a CTA (300 pages per sequence) takes the unstaged lookup."""
+    ps, H, D, batch = 2, 1, 32, 2
+    lens = torch.tensor([599, 433], dtype=torch.int32)
+    lens, bt = workloads.paged_tables(9, batch, 599, 610, ps, lens=lens)
+    assert bt.shape[1] == 300
+    k, v = workloads.small(shape=(610, ps, H, D))
+    run_q(kvq, oracle_mod, k, v, wbits, batch, -500, 501, dev, page_size=ps, seqlens=lens, bt=bt)

@@ -533,6 +533,8 @@ def main():
     ap.add_argument("--case", choices=CASES, action="append",
                     help="time only these single conversions (for sweeps and ncu); no headline line")
     ap.add_argument("--case-batch", type=int, default=4)
+    ap.add_argument("--engine", choices=["auto", "ldg", "bulk"], default="auto",
+                    help="load engine of the conversion kernels (plain loads or TMA bulk copies)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -558,6 +560,7 @@ def main():
     import kv_cache_quantization_fp16_b200 as kvq
 
     peak, peak_kind = hbm_peak()
+    kvq.set_engine(args.engine)
     if args.case:
         for c in args.case:
             print(json.dumps(run_case(kvq, dev, c, args.case_batch, args.steps, args.warmup, peak)), flush=True)

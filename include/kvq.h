@@ -91,7 +91,18 @@ typedef enum kvq_status {
 enum {
   KVQ_DEV_OK = 0,
   KVQ_DEV_BAD_PAGE = 1,       /* block_table entry outside [0, dim0) */
-  KVQ_DEV_BAD_PAGE_INDEX = 2  /* logical page index >= block_table_stride */
+  KVQ_DEV_BAD_PAGE_INDEX = 2, /* logical page index >= block_table_stride */
+  KVQ_DEV_TIMEOUT = 3         /* a bulk-engine pipeline wait ran past its limit (1 s) */
+};
+
+/* Load engines (kvq_set_engine).  Both give bit-identical results. */
+enum {
+  KVQ_ENGINE_AUTO = 0, /* per operation, the engine measured faster on B200 (default) */
+  KVQ_ENGINE_LDG = 1,  /* one tile per CTA, 16-byte global loads issued up front */
+  KVQ_ENGINE_BULK = 2  /* persistent CTAs, TMA bulk copies (cp.async.bulk, no multicast)
+                          into a 4-stage shared-memory ring, one producer warp and eight
+                          consumer warps; used when one position of the input stream is a
+                          multiple of 16 bytes, otherwise the LDG engine runs */
 };
 
 /* The shape the torch tensor carried in the original extension. */
@@ -142,6 +153,13 @@ KVQ_API const char* kvq_status_string(kvq_status status);
  * *code_out receives the KVQ_DEV_* code (0 when none).  Returns KVQ_ERR_DEVICE
  * when the word was set, KVQ_OK when not, KVQ_ERR_CUDA on a runtime error. */
 KVQ_API kvq_status kvq_poll_device_error(int32_t* code_out, void* stream);
+
+/* Select the load engine for all later calls in this process (any thread).
+ * Returns KVQ_ERR_RANGE for an unknown value.  Host-only; no device work. */
+KVQ_API kvq_status kvq_set_engine(int engine);
+
+/* The engine currently selected (a KVQ_ENGINE_* value). */
+KVQ_API int kvq_get_engine(void);
 
 /* Self-check (no counterpart on the page): compares, on the device, the
  * kernels' fast code rounding (reciprocal, one FMA correction step, rounding

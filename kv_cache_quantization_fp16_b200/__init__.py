@@ -26,7 +26,10 @@ import os
 import torch
 
 __all__ = ["fp16_to_fp8", "fp8_to_fp16", "fp16_to_q_kv", "q_to_fp16_kv", "poll_device_error",
-           "selfcheck_code_rounding", "q_shapes", "KVQError", "LIB_PATH", "library"]
+           "selfcheck_code_rounding", "q_shapes", "set_engine", "get_engine", "engine", "KVQError",
+           "LIB_PATH", "library"]
+
+ENGINES = {"auto": 0, "ldg": 1, "bulk": 2}
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvq.so")
 
@@ -63,8 +66,11 @@ def _load() -> ctypes.CDLL:
     L.kvq_status_string.restype = ctypes.c_char_p
     L.kvq_poll_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), vp]
     L.kvq_selfcheck_code_rounding.argtypes = [I, vp, vp]
+    L.kvq_set_engine.argtypes = [I]
+    L.kvq_get_engine.argtypes = []
+    L.kvq_get_engine.restype = I
     for f in ("kvq_fp16_to_fp8", "kvq_fp8_to_fp16", "kvq_fp16_to_q_kv", "kvq_q_to_fp16_kv",
-              "kvq_poll_device_error", "kvq_selfcheck_code_rounding"):
+              "kvq_poll_device_error", "kvq_selfcheck_code_rounding", "kvq_set_engine"):
         getattr(L, f).restype = I
     return L
 
@@ -209,3 +215,31 @@ def selfcheck_code_rounding(wbits: int, device=None) -> int:
         st = _lib.kvq_selfcheck_code_rounding(int(wbits), out.data_ptr(), _stream(dev))
     _check(st, "selfcheck_code_rounding")
     return int(out.item())
+
+
+def set_engine(name: str) -> None:
+    """Select the load engine for all later conversions: "auto" (default: the engine
+    measured faster for each operation), "ldg" (plain 16-byte loads, one tile per CTA)
+    or "bulk" (TMA bulk copies into a shared-memory pipeline)."""
+    _check(_lib.kvq_set_engine(ENGINES[name]), "set_engine")
+
+
+def get_engine() -> str:
+    code = _lib.kvq_get_engine()
+    return {v: k for k, v in ENGINES.items()}[code]
+
+
+class engine:
+    """Context manager: ``with engine("bulk"): ...`` selects an engine temporarily."""
+
+    def __init__(self, name: str):
+        self.name = name
+
+    def __enter__(self):
+        self.prev = get_engine()
+        set_engine(self.name)
+        return self
+
+    def __exit__(self, *exc):
+        set_engine(self.prev)
+        return False

@@ -1,4 +1,5 @@
-// kvq.cu -- sm_100a kernels and the C ABI (include/kvq.h) of libkvq.so.
+// kvq.cu -- the C ABI (include/kvq.h) of libkvq.so: host-side validation,
+// tiling and launch of the sm_100a conversion kernels.
 //
 // KV-cache format conversions from the page "Implementation: Turboderp org
 // Exllamav2 Ext Cache": fp16_to_fp8 / fp8_to_fp16 (Description, Signature)
@@ -10,284 +11,26 @@
 // many bytes in the FP8 / code / scale tensors).  The run is cut into tiles of
 // `tile_pos` positions; in paged mode tiles are aligned to multiples of
 // tile_pos in logical position space and tile_pos divides page_size, so a tile
-// never straddles a page.  One CTA converts one tile: thread 0 resolves the
-// tile (window clipping, the block_table lookup) once and stages the physical
-// row in shared memory, then all threads stream the tile's elements as a flat
-// array; each op fixes its CTA size and how many independent loads every
-// thread has in flight (see the per-op structs).  Grid: x = tiles, y =
-// sequences, z = K / V (the fused K+V launch).
+// never straddles a page.  Two load engines convert tiles (ldg_engine.cuh:
+// one tile per CTA from plain global loads; bulk_engine.cuh: persistent CTAs
+// fed by TMA bulk copies through shared memory); both share the per-tile
+// bodies in ops.cuh and the arithmetic in codec.cuh.
 //
-// This is a streaming, HBM-bound path: no tensor cores, no shared-memory
-// staging of the data, no collectives.
+// This is a streaming, HBM-bound path: no tensor cores, no collectives.
 
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/kvq.h"
+#include "bulk_engine.cuh"
 #include "codec.cuh"
+#include "ldg_engine.cuh"
+#include "ops.cuh"
+#include "tiles.cuh"
 
 namespace kvq {
-
-constexpr int kBlockElems = 32;  // Q scale block along head_dim
-
-// Per-device error word for problems only the device can see.
-__device__ int g_device_error;
-
-__device__ __forceinline__ void record_error(int code) { atomicCAS(&g_device_error, 0, code); }
-
-struct Geometry {
-  int dim0, dim1;
-  long long hd;  // kv_heads * head_dim: elements per position
-  int bt_stride;
-  int batch, offset, width, page_size;
-  int tile_pos;
-  const int32_t* seqlens;
-  const int32_t* block_table;
-};
-
-// Tile `tile_x` of sequence `seq` in contiguous mode: first row and number of
-// positions, or false when the tile lies past the end of the window.
-__device__ __forceinline__ bool contiguous_tile(const Geometry& g, int seq, int tile_x, long long& row0,
-                                                int& nrows) {
-  const long long p0 = static_cast<long long>(g.offset) + static_cast<long long>(tile_x) * g.tile_pos;
-  const long long p1 = min(static_cast<long long>(g.offset) + g.width, p0 + g.tile_pos);
-  if (p0 >= p1) return false;
-  row0 = static_cast<long long>(seq) * g.dim1 + p0;
-  nrows = static_cast<int>(p1 - p0);
-  return true;
-}
-
-// Paged mode: the window of sequence `seq` is [max(0, seqlen + offset),
-// seqlen + offset + width) in logical positions; tile `tile_x` is the x-th
-// tile_pos-aligned run of it (tile_pos divides page_size, so the run lies in
-// one page).  `bt_row` is the sequence's block-table row staged in shared
-// memory (or null: read it from global memory).  Bad metadata is recorded by
-// the thread with `report` set and the tile is skipped.
-__device__ __forceinline__ bool paged_tile(const Geometry& g, int seq, int tile_x, int seqlen,
-                                           const int* bt_row, bool report, long long& row0, int& nrows) {
-  const long long start = static_cast<long long>(seqlen) + g.offset;
-  const long long lo = start < 0 ? 0 : start;
-  const long long hi = start + g.width;
-  if (lo >= hi) return false;
-  const long long t0 = (lo / g.tile_pos) * g.tile_pos + static_cast<long long>(tile_x) * g.tile_pos;
-  const long long p0 = max(lo, t0);
-  const long long p1 = min(hi, t0 + g.tile_pos);
-  if (p0 >= p1) return false;
-  const long long lp = p0 / g.page_size;
-  if (lp >= g.bt_stride) {
-    if (report) record_error(KVQ_DEV_BAD_PAGE_INDEX);
-    return false;
-  }
-  const int page = bt_row ? bt_row[lp] : g.block_table[static_cast<long long>(seq) * g.bt_stride + lp];
-  if (page < 0 || page >= g.dim0) {
-    if (report) record_error(KVQ_DEV_BAD_PAGE);
-    return false;
-  }
-  row0 = static_cast<long long>(page) * g.page_size + p0 % g.page_size;
-  nrows = static_cast<int>(p1 - p0);
-  return true;
-}
-
-struct Params {
-  Geometry g;
-  const void* in[2];
-  void* out[2];
-  void* scales[2];  // Q encode: written; Q decode: read
-};
-
-// ---------------------------------------------------------------------------
-// Per-tile bodies
-// ---------------------------------------------------------------------------
-
-// FP8: 128-thread CTAs with 8 independent 16-byte loads (or 8-byte loads for
-// decode) per thread, so a whole tile is requested at once and enough CTAs
-// stay resident (up to 16 per SM) for small windows to run in one wave.
-struct Fp8Encode {
-  static constexpr int kThreads = 128;
-  static constexpr int kUnroll = 8;
-  static constexpr int kElemsPerTile = kThreads * kUnroll * 8;
-  static constexpr int kMinBlocksPerSM = 8;
-  __device__ static void tile(const Params& p, int kv, long long row0, int nrows) {
-    const long long e0 = row0 * p.g.hd;
-    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __half*>(p.in[kv]) + e0);
-    uint2* dst = reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.out[kv]) + e0);
-    const int nvec = static_cast<int>(nrows * p.g.hd / 8);
-    for (int base = 0; base < nvec; base += kThreads * kUnroll) {
-      uint4 x[kUnroll];
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int v = base + u * kThreads + threadIdx.x;
-        if (v < nvec) x[u] = __ldg(src + v);
-      }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int v = base + u * kThreads + threadIdx.x;
-        if (v < nvec) dst[v] = e5m2_encode_v8(x[u]);
-      }
-    }
-  }
-};
-
-struct Fp8Decode {
-  static constexpr int kThreads = 128;
-  static constexpr int kUnroll = 8;
-  static constexpr int kElemsPerTile = kThreads * kUnroll * 8;
-  static constexpr int kMinBlocksPerSM = 8;
-  __device__ static void tile(const Params& p, int kv, long long row0, int nrows) {
-    const long long e0 = row0 * p.g.hd;
-    const uint2* src = reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(p.in[kv]) + e0);
-    uint4* dst = reinterpret_cast<uint4*>(static_cast<__half*>(p.out[kv]) + e0);
-    const int nvec = static_cast<int>(nrows * p.g.hd / 8);
-    for (int base = 0; base < nvec; base += kThreads * kUnroll) {
-      uint2 x[kUnroll];
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int v = base + u * kThreads + threadIdx.x;
-        if (v < nvec) x[u] = __ldg(src + v);
-      }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int v = base + u * kThreads + threadIdx.x;
-        if (v < nvec) dst[v] = e5m2_decode_v8(x[u]);
-      }
-    }
-  }
-};
-
-// Q encode: one thread owns whole 32-element blocks (4 x 16-byte loads), so
-// the absmax needs no shuffles, the scale and reciprocal are computed once per
-// block, and the packed codes leave as one 16-byte (Q4) or three 8-byte (Q6)
-// stores.  Two blocks per thread are loaded before either is encoded.
-template <int B>
-struct QEncode {
-  static constexpr int kThreads = 256;
-  static constexpr int kUnrollBlocks = 2;
-  static constexpr int kElemsPerTile = kThreads * kBlockElems * kUnrollBlocks;
-  static constexpr int kMinBlocksPerSM = 4;
-
-  __device__ static void tile(const Params& p, int kv, long long row0, int nrows) {
-    const long long e0 = row0 * p.g.hd;
-    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __half*>(p.in[kv]) + e0);
-    uint8_t* codes = static_cast<uint8_t*>(p.out[kv]) + e0 * B / 8;
-    __half* scales = static_cast<__half*>(p.scales[kv]) + e0 / kBlockElems;
-    const int nblk = static_cast<int>(nrows * p.g.hd / kBlockElems);
-    for (int base = 0; base < nblk; base += kThreads * kUnrollBlocks) {
-      uint4 x[kUnrollBlocks][4];
-#pragma unroll
-      for (int u = 0; u < kUnrollBlocks; ++u) {
-        const int b = base + u * kThreads + threadIdx.x;
-        if (b < nblk) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) x[u][k] = __ldg(src + static_cast<long long>(b) * 4 + k);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kUnrollBlocks; ++u) {
-        const int b = base + u * kThreads + threadIdx.x;
-        if (b >= nblk) continue;
-        const __half s16 = block_scale<B>(absmax_bits_block(x[u]));
-        const BlockScale bs = make_block_scale(s16);
-        uint32_t w[B];
-        if (__half_as_ushort(s16) < 0x0400u)
-          encode_block_words<B, true>(x[u], bs, w);
-        else
-          encode_block_words<B, false>(x[u], bs, w);
-        if (B == 4) {
-          reinterpret_cast<uint4*>(codes)[b] = make_uint4(w[0], w[1], w[2 % B], w[3 % B]);
-        } else {
-          uint2* dst = reinterpret_cast<uint2*>(codes + static_cast<long long>(b) * 24);
-          dst[0] = make_uint2(w[0], w[1]);
-          dst[1] = make_uint2(w[2 % B], w[3 % B]);
-          dst[2] = make_uint2(w[4 % B], w[5 % B]);
-        }
-        scales[b] = s16;
-      }
-    }
-  }
-};
-
-template <int B>
-struct QDecode {
-  static constexpr int kThreads = 256;
-  static constexpr int kUnroll = 4;
-  static constexpr int kElemsPerTile = kThreads * kUnroll * 8;
-  static constexpr int kMinBlocksPerSM = 5;
-  __device__ static void tile(const Params& p, int kv, long long row0, int nrows) {
-    const long long e0 = row0 * p.g.hd;
-    const uint8_t* codes = static_cast<const uint8_t*>(p.in[kv]) + e0 * B / 8;
-    const __half* scales = static_cast<const __half*>(p.scales[kv]) + e0 / kBlockElems;
-    uint4* dst = reinterpret_cast<uint4*>(static_cast<__half*>(p.out[kv]) + e0);
-    const int nvec = static_cast<int>(nrows * p.g.hd / 8);
-    for (int base = 0; base < nvec; base += kThreads * kUnroll) {
-      uint32_t lo[kUnroll], hi[kUnroll];
-      __half s[kUnroll];
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int v = base + u * kThreads + threadIdx.x;
-        lo[u] = hi[u] = 0;
-        s[u] = __ushort_as_half(0);
-        if (v < nvec) {
-          if (B == 4) {
-            lo[u] = __ldg(reinterpret_cast<const uint32_t*>(codes) + v);
-          } else {
-            // lane pair = one 12-byte group; the even lane needs words 0-1, the
-            // odd lane words 1-2 (bits 48..95 of the group)
-            const uint32_t* grp = reinterpret_cast<const uint32_t*>(codes + static_cast<long long>(v >> 1) * 12);
-            const uint32_t sh = (v & 1) * 16;
-            const uint32_t a = __ldg(grp + (v & 1));
-            const uint32_t b = __ldg(grp + (v & 1) + 1);
-            lo[u] = __funnelshift_r(a, b, sh);
-            hi[u] = (b >> sh) & 0xFFFFu;
-          }
-          s[u] = __ldg(scales + (v >> 2));
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int v = base + u * kThreads + threadIdx.x;
-        if (v >= nvec) continue;
-        const __half2 s2 = __halves2half2(s[u], s[u]);
-        dst[v] = (B == 4) ? dequant_q4_v8(lo[u], s2) : dequant_q6_v8(lo[u], hi[u], s2);
-      }
-    }
-  }
-};
-
-// ---------------------------------------------------------------------------
-// The kernel: one tile per CTA; the tile is resolved once and staged in smem.
-// ---------------------------------------------------------------------------
-
-template <class Op>
-__global__ void __launch_bounds__(Op::kThreads, Op::kMinBlocksPerSM) convert_kernel(const __grid_constant__ Params p) {
-  // Programmatic dependent launch: this grid may be launched while the
-  // previous kernel on the stream is still running; wait for it to finish (and
-  // its writes to become visible) before touching global memory, and let the
-  // next kernel start launching as soon as every CTA of this grid has started.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  __shared__ int s_bt[Op::kThreads];
-  __shared__ int s_seqlen;
-  const int kv = blockIdx.z;
-  for (int seq = blockIdx.y; seq < p.g.batch; seq += gridDim.y) {
-    long long row0 = 0;
-    int nrows = 0;
-    bool ok;
-    if (p.g.page_size == 0) {
-      ok = contiguous_tile(p.g, seq, blockIdx.x, row0, nrows);
-    } else {
-      // Stage the sequence's block-table row (when it fits) together with its
-      // length, so the page lookup costs one memory round trip, not two.
-      const bool staged = p.g.bt_stride <= Op::kThreads;
-      if (staged && static_cast<int>(threadIdx.x) < p.g.bt_stride)
-        s_bt[threadIdx.x] = p.g.block_table[static_cast<long long>(seq) * p.g.bt_stride + threadIdx.x];
-      if (threadIdx.x == 0) s_seqlen = p.g.seqlens[seq];
-      __syncthreads();
-      ok = paged_tile(p.g, seq, blockIdx.x, s_seqlen, staged ? s_bt : nullptr, threadIdx.x == 0, row0, nrows);
-      __syncthreads();  // s_bt and s_seqlen are rewritten for the next sequence
-    }
-    if (ok) Op::tile(p, kv, row0, nrows);
-  }
-}
 
 // ---------------------------------------------------------------------------
 // Self-check of the fast code rounding against IEEE division.
@@ -371,28 +114,107 @@ kvq_status launch_status() {
   return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
+// Engine chosen by kvq_set_engine (process-wide).
+std::atomic<int> g_engine{KVQ_ENGINE_AUTO};
+
+// What KVQ_ENGINE_AUTO runs: the engine measured faster on B200.  Plain
+// loads win every contiguous conversion and the short paged windows (their
+// CTAs resolve a tile with arithmetic only, or few tiles exist); the bulk
+// pipeline wins long paged dequantize sweeps, where its producer warp
+// resolves block-table pages ahead of the consumers instead of every CTA
+// waiting on its own lookup before its first data load.
 template <class Op>
-kvq_status launch(Params p, int nkv, void* stream) {
-  p.g.tile_pos = pick_tile_pos(p.g.hd, p.g.page_size, Op::kElemsPerTile);
-  const int paged = p.g.page_size > 0;
-  const long long tiles = (static_cast<long long>(p.g.width) + p.g.tile_pos - 1) / p.g.tile_pos + paged;
-  if (tiles > 0x7FFFFFFFLL) return KVQ_ERR_RANGE;
+struct AutoEngine {
+  static int pick(const Params&) { return KVQ_ENGINE_LDG; }
+};
+template <int B>
+struct AutoEngine<QDecode<B>> {
+  static int pick(const Params& p) {
+    return (p.g.page_size > 0 && p.g.width >= 4096) ? KVQ_ENGINE_BULK : KVQ_ENGINE_LDG;
+  }
+};
+
+// Launch with programmatic stream serialization (the kernels wait on the
+// previous grid themselves).
+template <class Kernel, class... Args>
+kvq_status launch_pdl(Kernel kernel, dim3 grid, int threads, int smem, void* stream, Args... args) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(p.g.batch < 65535 ? p.g.batch : 65535),
-                     static_cast<unsigned>(nkv));
-  cfg.blockDim = dim3(Op::kThreads);
-  cfg.dynamicSmemBytes = 0;
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = static_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, convert_kernel<Op>, p) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess) {
     cudaGetLastError();
     return KVQ_ERR_CUDA;
   }
   return launch_status();
+}
+
+template <class Op>
+kvq_status launch_ldg(Params p, int nkv, void* stream) {
+  p.g.tile_pos = pick_tile_pos(p.g.hd, p.g.page_size, ldg_tile_elems<Op>());
+  const int paged = p.g.page_size > 0;
+  const long long tiles = (static_cast<long long>(p.g.width) + p.g.tile_pos - 1) / p.g.tile_pos + paged;
+  if (tiles > 0x7FFFFFFFLL) return KVQ_ERR_RANGE;
+  const dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(p.g.batch < 65535 ? p.g.batch : 65535),
+                  static_cast<unsigned>(nkv));
+  return launch_pdl(convert_kernel<Op>, grid, LdgCfg<Op>::kThreads, 0, stream, p);
+}
+
+// The bulk engine needs every tile of the input stream 16-byte aligned and a
+// multiple of 16 bytes (one position's bytes a multiple of 16), and one tile
+// to fit a shared-memory stage.
+template <class Op>
+bool bulk_eligible(const Params& p) {
+  const long long pos_bytes = p.g.hd * Op::kInNum / Op::kInDen;
+  if (pos_bytes % 16 != 0) return false;
+  const int tp = pick_tile_pos(p.g.hd, p.g.page_size, kBulkTileElems);
+  return static_cast<long long>(tp) * pos_bytes <= kBulkStageBytes;
+}
+
+// Persistent grid: as many CTAs as fit on the device at once (cached per
+// device), never more than there are tiles.
+template <class Op>
+kvq_status launch_bulk(Params p, int nkv, void* stream) {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<int> ctas_per_device[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVQ_ERR_CUDA;
+  int ctas = ctas_per_device[dev].load();
+  if (ctas == 0) {
+    int sms = 0, per_sm = 0;
+    if (cudaFuncSetAttribute(bulk_kernel<Op>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBulkSmemBytes) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bulk_kernel<Op>, kBulkThreads, kBulkSmemBytes) !=
+            cudaSuccess) {
+      cudaGetLastError();
+      return KVQ_ERR_CUDA;
+    }
+    ctas = sms * (per_sm > 0 ? per_sm : 1);
+    ctas_per_device[dev].store(ctas);
+  }
+  p.g.tile_pos = pick_tile_pos(p.g.hd, p.g.page_size, kBulkTileElems);
+  const int paged = p.g.page_size > 0;
+  const long long tiles_x = (static_cast<long long>(p.g.width) + p.g.tile_pos - 1) / p.g.tile_pos + paged;
+  const long long total = tiles_x * p.g.batch * nkv;
+  if (tiles_x > 0x7FFFFFFFLL) return KVQ_ERR_RANGE;
+  const unsigned grid = static_cast<unsigned>(total < ctas ? total : ctas);
+  return launch_pdl(bulk_kernel<Op>, dim3(grid), kBulkThreads, kBulkSmemBytes, stream, p,
+                    static_cast<int>(tiles_x), nkv);
+}
+
+template <class Op>
+kvq_status launch(const Params& p, int nkv, void* stream) {
+  int engine = g_engine.load(std::memory_order_relaxed);
+  if (engine == KVQ_ENGINE_AUTO) engine = AutoEngine<Op>::pick(p);
+  if (engine == KVQ_ENGINE_BULK && bulk_eligible<Op>(p)) return launch_bulk<Op>(p, nkv, stream);
+  return launch_ldg<Op>(p, nkv, stream);
 }
 
 Geometry make_geometry(const kvq_cache_desc* d, int batch, int offset, int width, int page_size,
@@ -406,7 +228,7 @@ Geometry make_geometry(const kvq_cache_desc* d, int batch, int offset, int width
   g.offset = offset;
   g.width = width;
   g.page_size = page_size;
-  g.tile_pos = 1;  // set per kernel by launch()
+  g.tile_pos = 1;  // set per kernel at launch
   g.seqlens = seqlens;
   g.block_table = block_table;
   return g;
@@ -529,6 +351,14 @@ kvq_status kvq_poll_device_error(int32_t* code_out, void* stream) {
   *code_out = h;
   return h ? KVQ_ERR_DEVICE : KVQ_OK;
 }
+
+kvq_status kvq_set_engine(int engine) {
+  if (engine != KVQ_ENGINE_AUTO && engine != KVQ_ENGINE_LDG && engine != KVQ_ENGINE_BULK) return KVQ_ERR_RANGE;
+  g_engine.store(engine);
+  return KVQ_OK;
+}
+
+int kvq_get_engine(void) { return g_engine.load(); }
 
 kvq_status kvq_selfcheck_code_rounding(int wbits, unsigned long long* mismatches, void* stream) {
   if (!mismatches) return KVQ_ERR_NULL;

@@ -1,0 +1,120 @@
+"""Both load engines (plain loads and TMA bulk copies) against the CPU oracle, and
+against each other, bit for bit: contiguous and paged windows, FP8 and Q4/Q6,
+ragged tails, shapes where the bulk engine is not applicable (it then runs the
+plain-load engine), and the empty-window no-op."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from test_gpu_parity import run_fp8, run_q, u8, u16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kvq():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import kv_cache_quantization_fp16_b200 as m
+
+    return m
+
+
+@pytest.fixture(scope="module")
+def dev(kvq):
+    return torch.device("cuda:0")
+
+
+@pytest.fixture(params=["ldg", "bulk"])
+def eng(request, kvq):
+    with kvq.engine(request.param):
+        yield request.param
+
+
+def test_engine_switch(kvq):
+    assert kvq.get_engine() == "auto"
+    with kvq.engine("bulk"):
+        assert kvq.get_engine() == "bulk"
+    assert kvq.get_engine() == "auto"
+    assert kvq.library().kvq_set_engine(7) == 4  # KVQ_ERR_RANGE
+    assert kvq.get_engine() == "auto"
+
+
+def test_fp8_window(kvq, oracle_mod, dev, eng):
+    k, _ = workloads.fp8_window(shape=(4, 1024, 8, 128))
+    run_fp8(kvq, oracle_mod, k, 4, 100, 801, dev)
+
+
+@pytest.mark.parametrize("wbits", [4, 6])
+def test_q_contiguous(kvq, oracle_mod, dev, eng, wbits):
+    k, v = workloads.channel_outliers(shape=(2, 512, 8, 128))
+    run_q(kvq, oracle_mod, k, v, wbits, 2, 3, 500, dev)
+
+
+@pytest.mark.parametrize("wbits", [4, 6])
+def test_q_paged(kvq, oracle_mod, dev, eng, wbits):
+    pool = workloads.paged_pool(num_pages=160, batch=6, max_len=1500, heads=4, head_dim=64)
+    for offset, width in ((0, 1), (-300, 300), (-1500, 1501)):
+        run_q(kvq, oracle_mod, pool.k, pool.v, wbits, 6, offset, width, dev, page_size=256,
+              seqlens=pool.cache_seqlens, bt=pool.block_table)
+
+
+@pytest.mark.parametrize("shape", [(2, 40, 1, 32), (3, 17, 3, 96), (2, 5, 32, 512)])
+def test_ragged_and_fallback_shapes(kvq, oracle_mod, dev, eng, shape):
+    """H*D = 32 or 288 make one position of the Q6 / FP8 streams not a multiple of 16 bytes
+    (the bulk engine falls back); H*D = 16384 exceeds a bulk stage (falls back too)."""
+    k, v = workloads.channel_outliers(shape=shape)
+    for wbits in (4, 6):
+        run_q(kvq, oracle_mod, k, v, wbits, shape[0], 1, shape[1] - 2, dev)
+    run_fp8(kvq, oracle_mod, k, shape[0], 0, shape[1], dev)
+
+
+def test_engines_agree_at_scale(kvq, dev):
+    """Full-size channel-outlier Q4/Q6 both directions: both engines write identical bytes."""
+    k, v = workloads.channel_outliers(shape=(4, 8192, 8, 128), device=dev)
+    B, S = k.shape[:2]
+    for wbits in (4, 6):
+        outs = []
+        for name in ("ldg", "bulk"):
+            with kvq.engine(name):
+                cs, ss = kvq.q_shapes(tuple(k.shape), wbits)
+                kc = torch.zeros(cs, dtype=torch.uint8, device=dev)
+                vc = torch.zeros_like(kc)
+                ks = torch.zeros(ss, dtype=torch.float16, device=dev)
+                vs = torch.zeros_like(ks)
+                kvq.fp16_to_q_kv(k, kc, ks, v, vc, vs, B, 0, S, 0, None, None, wbits)
+                ky, vy = torch.zeros_like(k), torch.zeros_like(v)
+                kvq.q_to_fp16_kv(kc, ky, ks, vc, vy, vs, B, 0, S, 0, None, None, wbits)
+                f8 = torch.zeros(k.shape, dtype=torch.uint8, device=dev)
+                kvq.fp16_to_fp8(k, f8, B, 0, S)
+                fy = torch.zeros_like(k)
+                kvq.fp8_to_fp16(f8, fy, B, 0, S)
+                torch.cuda.synchronize()
+                outs.append((kc, vc, ks.view(torch.int16), vs.view(torch.int16), ky.view(torch.int16),
+                             vy.view(torch.int16), f8, fy.view(torch.int16)))
+        for a, b in zip(*outs):
+            assert torch.equal(a, b)
+    assert kvq.poll_device_error() == 0
+
+
+def test_bulk_bad_block_table_reports(kvq, oracle_mod, dev):
+    ps, H, D, npages = 8, 2, 64, 6
+    k, v = workloads.small(shape=(npages, ps, H, D))
+    bt = torch.tensor([[0, 7], [1, -1]], dtype=torch.int32)
+    lens = torch.tensor([4, 6], dtype=torch.int32)
+    cs, ss = kvq.q_shapes(tuple(k.shape), 4)
+    kd, vd = k.to(dev), v.to(dev)
+    kc, vc = torch.full(cs, 0xA5, dtype=torch.uint8, device=dev), torch.full(cs, 0xA5, dtype=torch.uint8,
+                                                                              device=dev)
+    ks, vs = torch.zeros(ss, dtype=torch.float16, device=dev), torch.zeros(ss, dtype=torch.float16, device=dev)
+    assert kvq.poll_device_error() == 0
+    with kvq.engine("bulk"):
+        kvq.fp16_to_q_kv(kd, kc, ks, vd, vc, vs, 2, 0, 8, ps, lens.to(dev), bt.to(dev), 4)
+    assert kvq.poll_device_error() in (1, 2)
+    rc = np.full(cs, 0xA5, np.uint8)
+    rs = np.zeros(ss, np.uint16)
+    oracle_mod.fp16_to_q_kv(u16(k), rc, rs, u16(v), rc.copy(), rs.copy(), 2, 0, 8, ps, lens.numpy(), bt.numpy(), 4)
+    assert np.array_equal(u8(kc), rc)

@@ -164,8 +164,8 @@ KVQ_API int kvq_get_engine(void);
 /* Self-check (no counterpart on the page): compares, on the device, the
  * kernels' fast code rounding (reciprocal, one FMA correction step, rounding
  * by magic-number addition) with IEEE binary32 division followed by rint and
- * the clamp, for every finite binary16 x and every positive finite binary16
- * scale s (2^31 pairs).  `mismatches` is a caller-owned device pointer to one
+ * the clamp, for every finite binary16 x and every binary16 scale s in
+ * [+0, 65504] (about 2^31 pairs).  `mismatches` is a caller-owned device pointer to one
  * unsigned 64-bit counter; it is zeroed and then receives the number of
  * pairs whose codes differ (0 expected).  Asynchronous on `stream`. */
 KVQ_API kvq_status kvq_selfcheck_code_rounding(int wbits, unsigned long long* mismatches, void* stream);

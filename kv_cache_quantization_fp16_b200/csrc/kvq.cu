@@ -38,13 +38,15 @@ namespace kvq {
 
 template <int B>
 __global__ void selfcheck_rounding_kernel(unsigned long long* mismatches) {
-  // blockIdx.x enumerates s bit patterns 1..0x7BFF; threads enumerate x over
-  // all 65536 bit patterns, skipping Inf / NaN.  Both forms the kernels use
-  // are checked: the clamped one for every pair, the unclamped one (used when
-  // the scale is normal) for every pair a block can produce.  A block gets the
-  // scale s only if absmax / maxq rounds to s, so its elements satisfy
-  // |x| <= maxq * (s + ulp(s) / 2).
-  const uint32_t s_bits = 1 + blockIdx.x;
+  // blockIdx.x enumerates the scale bit patterns 0..0x7BFF (+0 and every
+  // positive finite binary16); threads enumerate x over all 65536 bit patterns,
+  // skipping Inf / NaN.  Both forms the kernels use are checked: the clamped
+  // one for every pair, the unclamped one (used unless the scale is a nonzero
+  // subnormal) for every pair a block can produce.  A block gets the scale s
+  // only if absmax / maxq rounds to s, so its elements satisfy
+  // |x| <= maxq * (s + ulp(s) / 2); s = +0 comes with x = +-0 only, but the
+  // unclamped form is checked there for every finite x.
+  const uint32_t s_bits = blockIdx.x;
   const __half s16 = __ushort_as_half(static_cast<unsigned short>(s_bits));
   const BlockScale bs = make_block_scale(s16);
   const bool normal = s_bits >= 0x0400u;
@@ -58,7 +60,7 @@ __global__ void selfcheck_rounding_kernel(unsigned long long* mismatches) {
     const uint32_t ref = quant_code_ieee<B>(x, bs.s);
     const uint32_t clamped = quant_code_bits<B, true>(x, bs) & ((1u << B) - 1);
     bad += (clamped != ref);
-    if (normal && fabsf(x) <= reach) {
+    if (s_bits == 0 || (normal && fabsf(x) <= reach)) {
       const uint32_t plain = quant_code_bits<B, false>(x, bs) & ((1u << B) - 1);
       bad += (plain != ref);
     }
@@ -366,9 +368,9 @@ kvq_status kvq_selfcheck_code_rounding(int wbits, unsigned long long* mismatches
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(mismatches, 0, sizeof(unsigned long long), s) != cudaSuccess) return KVQ_ERR_CUDA;
   if (wbits == 4)
-    kvq::selfcheck_rounding_kernel<4><<<0x7BFF, 256, 0, s>>>(mismatches);
+    kvq::selfcheck_rounding_kernel<4><<<0x7C00, 256, 0, s>>>(mismatches);
   else
-    kvq::selfcheck_rounding_kernel<6><<<0x7BFF, 256, 0, s>>>(mismatches);
+    kvq::selfcheck_rounding_kernel<6><<<0x7C00, 256, 0, s>>>(mismatches);
   return launch_status();
 }
 

@@ -109,7 +109,10 @@ struct QEncode {
         const __half s16 = block_scale<B>(absmax_bits_block(x[u]));
         const BlockScale bs = make_block_scale(s16);
         uint32_t w[B];
-        if (__half_as_ushort(s16) < 0x0400u)
+        // Only a nonzero subnormal scale needs the clamp; a zero scale (all-zero
+        // block) gives rh = rl = 0, hence code z, on the unclamped path too, so
+        // zero blocks do not split a warp across both paths.
+        if (__half_as_ushort(s16) - 1u < 0x03FFu)
           encode_block_words<B, true>(x[u], bs, w);
         else
           encode_block_words<B, false>(x[u], bs, w);

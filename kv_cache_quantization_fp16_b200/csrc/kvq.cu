@@ -119,21 +119,13 @@ kvq_status launch_status() {
 // Engine chosen by kvq_set_engine (process-wide).
 std::atomic<int> g_engine{KVQ_ENGINE_AUTO};
 
-// What KVQ_ENGINE_AUTO runs: the engine measured faster on B200.  Plain
-// loads win every contiguous conversion and the short paged windows (their
-// CTAs resolve a tile with arithmetic only, or few tiles exist); the bulk
-// pipeline wins long paged dequantize sweeps, where its producer warp
-// resolves block-table pages ahead of the consumers instead of every CTA
-// waiting on its own lookup before its first data load.
+// What KVQ_ENGINE_AUTO runs: the engine measured faster on B200 for each
+// operation.  With four-round paged tiles the plain-load engine wins every
+// conversion measured (contiguous and paged, quantize and dequantize), so
+// AUTO is the plain-load engine throughout; the bulk engine stays available.
 template <class Op>
 struct AutoEngine {
   static int pick(const Params&) { return KVQ_ENGINE_LDG; }
-};
-template <int B>
-struct AutoEngine<QDecode<B>> {
-  static int pick(const Params& p) {
-    return (p.g.page_size > 0 && p.g.width >= 4096) ? KVQ_ENGINE_BULK : KVQ_ENGINE_LDG;
-  }
 };
 
 // Launch with programmatic stream serialization (the kernels wait on the
@@ -159,7 +151,10 @@ kvq_status launch_pdl(Kernel kernel, dim3 grid, int threads, int smem, void* str
 
 template <class Op>
 kvq_status launch_ldg(Params p, int nkv, void* stream) {
-  p.g.tile_pos = pick_tile_pos(p.g.hd, p.g.page_size, ldg_tile_elems<Op>());
+  // Paged tiles are four CTA rounds long: each CTA pays one block-table lookup
+  // before its first data load, and a longer tile amortizes it.
+  const long long target = static_cast<long long>(ldg_tile_elems<Op>()) * (p.g.page_size > 0 ? 4 : 1);
+  p.g.tile_pos = pick_tile_pos(p.g.hd, p.g.page_size, target);
   const int paged = p.g.page_size > 0;
   const long long tiles = (static_cast<long long>(p.g.width) + p.g.tile_pos - 1) / p.g.tile_pos + paged;
   if (tiles > 0x7FFFFFFFLL) return KVQ_ERR_RANGE;

@@ -236,9 +236,11 @@ def capture(fn, n_marks=0):
     return g, marks
 
 
-def time_device(fn, steps, warmup, flush, sampler=None, n_marks=0):
+def time_device(fn, steps, warmup, flush, sampler=None, n_marks=0, collective=True):
     """Per-step CUDA-event times (ms) of the captured fn, with an L2 flush (outside the
-    events) before each step.  With marks, also the per-launch segments of every step."""
+    events) before each step.  With marks, also the per-launch segments of every step.
+    `collective`: bracket the timed region with a barrier over all ranks (every rank must
+    then make the same call); False for rank-local measurements."""
     g, marks = capture(fn, n_marks)
     for _ in range(warmup):
         flush()
@@ -247,7 +249,8 @@ def time_device(fn, steps, warmup, flush, sampler=None, n_marks=0):
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     segs = []
-    _barrier()
+    if collective:
+        _barrier()
     torch.cuda.synchronize()
     if sampler:
         sampler.mark()
@@ -263,7 +266,8 @@ def time_device(fn, steps, warmup, flush, sampler=None, n_marks=0):
     torch.cuda.synchronize()
     if sampler:
         sampler.mark()
-    _barrier()
+    if collective:
+        _barrier()
     per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     del g
     return per_step, segs
@@ -314,7 +318,7 @@ def per_op_measurements(kvq, dev, peak, steps, flush, include_model=True):
     out = []
 
     def record(name, config, nbytes, fn, n=steps):
-        per, _ = time_device(lambda ev: fn(), n, 3, flush)
+        per, _ = time_device(lambda ev: fn(), n, 3, flush, collective=False)
         ms = statistics.mean(per)
         out.append({"op": name, "config": config, "bytes": int(nbytes), "us": round(ms * 1e3, 2),
                     "gbs": round(nbytes / ms / 1e6, 1), "frac": round(nbytes / ms / 1e6 / peak, 3)})
@@ -403,7 +407,7 @@ def model_layers(kvq, dev, peak, steps, flush, layers=32):
     res = []
     cfg = "paged Q6, 32 layers x K/V 8x32768x8x128, page 256, shuffled block_table"
     for name, fn in (("q_to_fp16_kv/q6/model32", deq), ("fp16_to_q_kv/q6/model32", qnt)):
-        per, _ = time_device(lambda ev: fn(), steps, 2, flush)
+        per, _ = time_device(lambda ev: fn(), steps, 2, flush, collective=False)
         ms = statistics.mean(per)
         res.append({"op": name, "config": cfg, "bytes": int(nb), "us": round(ms * 1e3, 1),
                     "gbs": round(nb / ms / 1e6, 1), "frac": round(nb / ms / 1e6 / peak, 3)})
@@ -479,7 +483,7 @@ def run_case(kvq, dev, name, batch, steps, warmup, peak):
         nb = BYTES_PER_ELEM[6] * 2 * pool.k.numel()
         fn = (lambda: kvq.fp16_to_q_kv(pool.k, kc, ks, pool.v, vc, vs, *args)) if name.endswith("enc") else \
              (lambda: kvq.q_to_fp16_kv(kc, pool.k, ks, vc, pool.v, vs, *args))
-    per, _ = time_device(lambda ev: fn(), steps, warmup, flush)
+    per, _ = time_device(lambda ev: fn(), steps, warmup, flush, collective=False)
     ms = statistics.mean(per)
     return {"case": name, "batch": batch, "bytes": int(nb), "us": round(ms * 1e3, 2),
             "us_min": round(min(per) * 1e3, 2), "gbs": round(nb / ms / 1e6, 1),
@@ -594,7 +598,7 @@ def main():
     e2e_ms = max_over_ranks(e2e_ms, dev)
 
     per_op = []
-    if rank == 0 and not args.no_per_op:
+    if world == 1 and not args.no_per_op:
         per_op = per_op_measurements(kvq, dev, peak, max(20, args.steps // 5), flush,
                                      include_model=not args.no_model)
     if sampler:

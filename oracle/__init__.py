@@ -47,11 +47,14 @@ def lib() -> ctypes.CDLL:
         L.kvqref_unpack_row.argtypes = [u8p, I, I, u8p]
         L.kvqref_fp16_to_fp8.argtypes = [u16p, u8p] + [I] * 7
         L.kvqref_fp8_to_fp16.argtypes = [u8p, u16p] + [I] * 7
+        L.kvqref_fp16_to_fp8_kv.argtypes = [u16p, u8p, u16p, u8p] + [I] * 8 + [i32p, i32p, I]
+        L.kvqref_fp8_to_fp16_kv.argtypes = [u8p, u16p, u8p, u16p] + [I] * 8 + [i32p, i32p, I]
         L.kvqref_fp16_to_q_kv.argtypes = [u16p, u8p, u16p, u16p, u8p, u16p] + [I] * 8 + [i32p, i32p, I, I]
         L.kvqref_q_to_fp16_kv.argtypes = [u8p, u16p, u16p, u8p, u16p, u16p] + [I] * 8 + [i32p, i32p, I, I]
         for name in ("kvqref_quantize_row", "kvqref_dequantize_row", "kvqref_pack_row",
                      "kvqref_unpack_row", "kvqref_fp16_to_fp8", "kvqref_fp8_to_fp16",
-                     "kvqref_fp16_to_q_kv", "kvqref_q_to_fp16_kv"):
+                     "kvqref_fp16_to_q_kv", "kvqref_q_to_fp16_kv", "kvqref_fp16_to_fp8_kv",
+                     "kvqref_fp8_to_fp16_kv"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -161,6 +164,33 @@ def _page_args(page_size, cache_seqlens, block_table):
         stride = bt.shape[1] if bt.ndim == 2 else 0
         return sl, bt, stride
     return None, None, 0
+
+
+def fp16_to_fp8_kv(k_in, k_out, v_in, v_out, batch_size, offset, width, page_size=0, cache_seqlens=None,
+                   block_table=None) -> int:
+    """E5M2-encode K and V (float16/uint16 [d0, d1, H, D]) into uint8 caches, contiguous or paged."""
+    d0, d1, H, D = k_in.shape
+    sl, bt, stride = _page_args(page_size, cache_seqlens, block_table)
+    for a in (k_out, v_out):
+        assert a.flags["C_CONTIGUOUS"] and a.dtype == np.uint8
+    return lib().kvqref_fp16_to_fp8_kv(
+        _p(np.ascontiguousarray(_bits(k_in)), ctypes.c_uint16), _p(k_out, ctypes.c_uint8),
+        _p(np.ascontiguousarray(_bits(v_in)), ctypes.c_uint16), _p(v_out, ctypes.c_uint8),
+        d0, d1, H, D, batch_size, offset, width, page_size, _p(sl, ctypes.c_int32), _p(bt, ctypes.c_int32), stride)
+
+
+def fp8_to_fp16_kv(k_in, k_out, v_in, v_out, batch_size, offset, width, page_size=0, cache_seqlens=None,
+                   block_table=None) -> int:
+    """Decode K and V E5M2 caches (uint8 [d0, d1, H, D]) into FP16 caches, contiguous or paged."""
+    d0, d1, H, D = k_in.shape
+    sl, bt, stride = _page_args(page_size, cache_seqlens, block_table)
+    ko, vo = _bits(k_out), _bits(v_out)
+    for a in (ko, vo):
+        assert a.flags["C_CONTIGUOUS"]
+    return lib().kvqref_fp8_to_fp16_kv(
+        _p(np.ascontiguousarray(k_in, np.uint8), ctypes.c_uint8), _p(ko, ctypes.c_uint16),
+        _p(np.ascontiguousarray(v_in, np.uint8), ctypes.c_uint8), _p(vo, ctypes.c_uint16),
+        d0, d1, H, D, batch_size, offset, width, page_size, _p(sl, ctypes.c_int32), _p(bt, ctypes.c_int32), stride)
 
 
 def fp16_to_q_kv(k_in, k_out, k_scales, v_in, v_out, v_scales, batch_size, offset, width,

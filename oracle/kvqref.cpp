@@ -315,6 +315,43 @@ int kvqref_fp8_to_fp16(const uint8_t* in, uint16_t* out, int dim0, int dim1, int
   });
 }
 
+// FP8 applied to K and V over one window description (contiguous or paged);
+// the page's fp16_to_fp8 / fp8_to_fp16 per element, with the window and page
+// rules of fp16_to_q_kv.
+int kvqref_fp16_to_fp8_kv(const uint16_t* k_in, uint8_t* k_out, const uint16_t* v_in, uint8_t* v_out,
+                          int dim0, int dim1, int heads, int head_dim,
+                          int batch_size, int offset, int width,
+                          int page_size, const int32_t* cache_seqlens,
+                          const int32_t* block_table, int bt_stride) {
+  if (heads < 0 || head_dim < 0) return KVQREF_BAD_ARG;
+  const Window w{dim0, dim1, batch_size, offset, width, page_size, bt_stride, cache_seqlens, block_table};
+  if (!window_args_ok(w)) return KVQREF_BAD_ARG;
+  const long row_elems = static_cast<long>(heads) * head_dim;
+  auto one = [&](const uint16_t* in, uint8_t* out, long row) {
+    for (long e = 0; e < row_elems; ++e) out[row * row_elems + e] = e5m2_encode(in[row * row_elems + e]);
+  };
+  const int st_k = for_each_row(w, [&](long row) { one(k_in, k_out, row); });
+  const int st_v = for_each_row(w, [&](long row) { one(v_in, v_out, row); });
+  return st_k != KVQREF_OK ? st_k : st_v;
+}
+
+int kvqref_fp8_to_fp16_kv(const uint8_t* k_in, uint16_t* k_out, const uint8_t* v_in, uint16_t* v_out,
+                          int dim0, int dim1, int heads, int head_dim,
+                          int batch_size, int offset, int width,
+                          int page_size, const int32_t* cache_seqlens,
+                          const int32_t* block_table, int bt_stride) {
+  if (heads < 0 || head_dim < 0) return KVQREF_BAD_ARG;
+  const Window w{dim0, dim1, batch_size, offset, width, page_size, bt_stride, cache_seqlens, block_table};
+  if (!window_args_ok(w)) return KVQREF_BAD_ARG;
+  const long row_elems = static_cast<long>(heads) * head_dim;
+  auto one = [&](const uint8_t* in, uint16_t* out, long row) {
+    for (long e = 0; e < row_elems; ++e) out[row * row_elems + e] = e5m2_decode(in[row * row_elems + e]);
+  };
+  const int st_k = for_each_row(w, [&](long row) { one(k_in, k_out, row); });
+  const int st_v = for_each_row(w, [&](long row) { one(v_in, v_out, row); });
+  return st_k != KVQREF_OK ? st_k : st_v;
+}
+
 // Description, fp16_to_q_kv: K and V are each quantized per head row.
 int kvqref_fp16_to_q_kv(const uint16_t* k_in, uint8_t* k_out, uint16_t* k_scales,
                         const uint16_t* v_in, uint8_t* v_out, uint16_t* v_scales,

@@ -90,6 +90,20 @@ int kvqref_fp8_to_fp16(const uint8_t* in, uint16_t* out,
                        int dim0, int dim1, int heads, int head_dim,
                        int batch_size, int offset, int width);
 
+/* FP8 for K and V together, contiguous (page_size == 0) or paged (page_size
+ * > 0, same window and page rules as the Q functions below). */
+int kvqref_fp16_to_fp8_kv(const uint16_t* k_in, uint8_t* k_out, const uint16_t* v_in, uint8_t* v_out,
+                          int dim0, int dim1, int heads, int head_dim,
+                          int batch_size, int offset, int width,
+                          int page_size, const int32_t* cache_seqlens,
+                          const int32_t* block_table, int bt_stride);
+
+int kvqref_fp8_to_fp16_kv(const uint8_t* k_in, uint16_t* k_out, const uint8_t* v_in, uint16_t* v_out,
+                          int dim0, int dim1, int heads, int head_dim,
+                          int batch_size, int offset, int width,
+                          int page_size, const int32_t* cache_seqlens,
+                          const int32_t* block_table, int bt_stride);
+
 /* page_size == 0: contiguous (cache_seqlens / block_table ignored).
  * page_size  > 0: paged; dim1 must equal page_size and block_table is
  *                 [batch_size, bt_stride] int32. */

@@ -193,3 +193,53 @@ def test_numpy_restatement_agrees(oracle_mod, wbits):
         assert np.array_equal(ks.reshape(-1), s16.view(np.uint16))
         got = np.stack([oracle_mod.unpack_row(r, D, wbits) for r in kc.reshape(-1, D * wbits // 8)])
         assert np.array_equal(got.reshape(-1, 32), codes)
+
+
+def test_fp8_kv_contiguous_matches_single_tensor(oracle_mod):
+    k, v = workloads.fp8_window(shape=(3, 64, 2, 64))
+    k, v = _np16(k), _np16(v)
+    k8, v8 = np.full(k.shape, SENT8, np.uint8), np.full(v.shape, SENT8, np.uint8)
+    assert oracle_mod.fp16_to_fp8_kv(k, k8, v, v8, 2, 7, 40) == oracle_mod.OK
+    r8 = np.full(k.shape, SENT8, np.uint8)
+    assert oracle_mod.fp16_to_fp8(k, r8, 2, 7, 40) == oracle_mod.OK
+    assert np.array_equal(k8, r8)
+    r8v = np.full(v.shape, SENT8, np.uint8)
+    assert oracle_mod.fp16_to_fp8(v, r8v, 2, 7, 40) == oracle_mod.OK
+    assert np.array_equal(v8, r8v)
+    ky, vy = np.full(k.shape, SENT16, np.uint16), np.full(v.shape, SENT16, np.uint16)
+    assert oracle_mod.fp8_to_fp16_kv(k8, ky, v8, vy, 2, 7, 40) == oracle_mod.OK
+    ry = np.full(k.shape, SENT16, np.uint16)
+    assert oracle_mod.fp8_to_fp16(k8, ry, 2, 7, 40) == oracle_mod.OK
+    assert np.array_equal(ky, ry)
+
+
+@pytest.mark.parametrize("offset,width", [(0, 1), (-40, 40), (-1000, 17)])
+def test_fp8_kv_paged_identity_and_rows(oracle_mod, offset, width):
+    # identity block table: paged == contiguous
+    B, S, H, D, ps = 3, 96, 2, 32, 32
+    k, v = workloads.fp8_window(shape=(B, S, H, D))
+    k, v = _np16(k), _np16(v)
+    bt = workloads.identity_block_table(B, S, ps).numpy()
+    pages = (B * S // ps, ps, H, D)
+    c_k = np.full(k.shape, SENT8, np.uint8)
+    c_v = np.full(v.shape, SENT8, np.uint8)
+    assert oracle_mod.fp16_to_fp8_kv(k, c_k, v, c_v, B, 20, 50) == oracle_mod.OK
+    p_k = np.full(pages, SENT8, np.uint8)
+    p_v = np.full(pages, SENT8, np.uint8)
+    assert oracle_mod.fp16_to_fp8_kv(k.reshape(pages), p_k, v.reshape(pages), p_v, B, 20, 50, ps,
+                                     np.zeros(B, np.int32), bt) == oracle_mod.OK
+    assert np.array_equal(c_k.reshape(-1), p_k.reshape(-1)) and np.array_equal(c_v.reshape(-1), p_v.reshape(-1))
+    # shuffled pool: exactly the window rows are written
+    ps, npages, batch = 16, 40, 5
+    lens, bt = workloads.paged_tables(3, batch, 60, npages, ps)
+    lens, bt = lens.numpy(), bt.numpy()
+    k, v = workloads.fp8_window(shape=(npages, ps, H, D))
+    k, v = _np16(k), _np16(v)
+    ko, vo = np.full(k.shape, SENT8, np.uint8), np.full(v.shape, SENT8, np.uint8)
+    assert oracle_mod.fp16_to_fp8_kv(k, ko, v, vo, batch, offset, width, ps, lens, bt) == oracle_mod.OK
+    rows = _expected_rows_paged(lens, bt, ps, batch, offset, width)
+    flat = ko.reshape(npages * ps, -1)
+    assert {r for r in range(npages * ps) if np.any(flat[r] != SENT8)} == rows
+    for r in rows:  # each written row is the element-wise E5M2 encoding
+        src = k.reshape(npages * ps, -1)[r]
+        assert np.array_equal(flat[r], [oracle_mod.e5m2_encode(int(h)) for h in src])

@@ -3,8 +3,9 @@
 Headline workload (one JSON line on rank 0): the contiguous FP8 partial-window
 workload -- K and V FP16 caches [4, 4096, 8, 128] (N(0,1) with 1% +-U(20,60000)
 outliers and 0.1% subnormals), window offset 1024, width 2048.  One step is
-fp16_to_fp8(K), fp16_to_fp8(V), fp8_to_fp16(K), fp8_to_fp16(V) through the C
-ABI on resident device buffers.  The metric is algorithmic GB/s (bytes read +
+fp16_to_fp8 of K and V, then fp8_to_fp16 of K and V, through the C ABI's fused
+K+V calls (one launch per direction) on resident device buffers; the same step
+through the single-tensor calls (4 launches) is reported in per_op.  The metric is algorithmic GB/s (bytes read +
 bytes written: 3 bytes per element per conversion), with L2 flushed between
 steps (a 256 MiB write then a 256 MiB read, outside the per-step CUDA events,
 so no dirty flush lines are written back inside a timed kernel).
@@ -185,7 +186,8 @@ class L2Flush:
 
 
 class Fp8Step:
-    """Headline step on one rank: FP8 encode + decode of the K and V windows."""
+    """Headline step on one rank: FP8 encode then decode of the K and V windows, through
+    the fused K+V calls (one launch per direction)."""
 
     def __init__(self, kvq, dev, batch, seed_shift=0):
         B, S, H, D = HEADLINE["shape"]
@@ -199,23 +201,18 @@ class Fp8Step:
         self.vy = torch.zeros_like(v)
         self.off, self.w = HEADLINE["offset"], HEADLINE["width"]
         self.elems_per_tensor = batch * self.w * H * D
-        self.launch_bytes = BYTES_PER_ELEM["fp8"] * self.elems_per_tensor
-        self.bytes_per_step = 4 * self.launch_bytes
-        self.launches_per_step = 4
+        self.launch_bytes = BYTES_PER_ELEM["fp8"] * 2 * self.elems_per_tensor  # K and V
+        self.bytes_per_step = 2 * self.launch_bytes
+        self.launches_per_step = 2
+        self.names = ["fp16_to_fp8_kv", "fp8_to_fp16_kv"]
 
     def run(self, ev=None):
-        """The four conversions; `ev` (3 events) marks the boundaries between them."""
+        """The two conversions; `ev` (1 event) marks the boundary between them."""
         kvq, b, o, w = self.kvq, self.batch, self.off, self.w
-        kvq.fp16_to_fp8(self.k, self.k8, b, o, w)
+        kvq.fp16_to_fp8_kv(self.k, self.k8, self.v, self.v8, b, o, w)
         if ev is not None:
             ev[0].record()
-        kvq.fp16_to_fp8(self.v, self.v8, b, o, w)
-        if ev is not None:
-            ev[1].record()
-        kvq.fp8_to_fp16(self.k8, self.ky, b, o, w)
-        if ev is not None:
-            ev[2].record()
-        kvq.fp8_to_fp16(self.v8, self.vy, b, o, w)
+        kvq.fp8_to_fp16_kv(self.k8, self.ky, self.v8, self.vy, b, o, w)
 
 
 def capture(fn, n_marks=0):
@@ -323,6 +320,22 @@ def per_op_measurements(kvq, dev, peak, steps, flush, include_model=True):
         out.append({"op": name, "config": config, "bytes": int(nbytes), "us": round(ms * 1e3, 2),
                     "gbs": round(nbytes / ms / 1e6, 1), "frac": round(nbytes / ms / 1e6 / peak, 3)})
 
+    # the headline step through the page's single-tensor calls (4 launches instead of 2)
+    B, S, H, D = HEADLINE["shape"]
+    o, w = HEADLINE["offset"], HEADLINE["width"]
+    hk, hv = workloads.fp8_window(shape=(B, S, H, D), device=dev)
+    hk8, hv8 = torch.zeros(hk.shape, dtype=torch.uint8, device=dev), torch.zeros(hv.shape, dtype=torch.uint8, device=dev)
+    hky, hvy = torch.empty_like(hk), torch.empty_like(hv)
+
+    def per_tensor_step():
+        kvq.fp16_to_fp8(hk, hk8, B, o, w)
+        kvq.fp16_to_fp8(hv, hv8, B, o, w)
+        kvq.fp8_to_fp16(hk8, hky, B, o, w)
+        kvq.fp8_to_fp16(hv8, hvy, B, o, w)
+    record("fp8_step_single_tensor_calls", "headline window, fp16_to_fp8(K), (V), fp8_to_fp16(K), (V): 4 launches",
+           4 * BYTES_PER_ELEM["fp8"] * B * w * H * D, per_tensor_step)
+    del hk, hv, hk8, hv8, hky, hvy
+
     # contiguous Q4 / Q6, channel outliers [16, 8192, 8, 128]
     k, v = workloads.channel_outliers(device=dev)
     B, S, H, D = k.shape
@@ -358,8 +371,18 @@ def per_op_measurements(kvq, dev, peak, steps, flush, include_model=True):
     ks = torch.zeros(ss, dtype=torch.float16, device=dev)
     vs = torch.zeros_like(ks)
     lens = pool.cache_seqlens.cpu()
+    k8p, v8p = torch.zeros(pool.k.shape, dtype=torch.uint8, device=dev), torch.zeros(pool.k.shape, dtype=torch.uint8,
+                                                                                    device=dev)
     for phase, off, w in (("decode", 0, 1), ("prefill", -512, 512)):
         npos = sum(max(0, int(L) + off + w) - max(0, int(L) + off) for L in lens)
+        nb8 = BYTES_PER_ELEM["fp8"] * 2 * npos * H * D
+        cfg8 = f"paged 2048x256x8x128 pool, 32 seqs, {phase} width={w}, K+V"
+        record(f"fp16_to_fp8_kv/{phase}", cfg8, nb8,
+               lambda: kvq.fp16_to_fp8_kv(pool.k, k8p, pool.v, v8p, 32, off, w, ps, pool.cache_seqlens,
+                                          pool.block_table))
+        record(f"fp8_to_fp16_kv/{phase}", cfg8, nb8,
+               lambda: kvq.fp8_to_fp16_kv(k8p, pool.k, v8p, pool.v, 32, off, w, ps, pool.cache_seqlens,
+                                          pool.block_table))
         nb = BYTES_PER_ELEM[4] * 2 * npos * H * D
         cfg = f"paged 2048x256x8x128 pool, 32 seqs, {phase} width={w}"
         record(f"fp16_to_q_kv/q4/{phase}", cfg, nb,
@@ -368,7 +391,7 @@ def per_op_measurements(kvq, dev, peak, steps, flush, include_model=True):
         record(f"q_to_fp16_kv/q4/{phase}", cfg, nb,
                lambda: kvq.q_to_fp16_kv(kc, pool.k, ks, vc, pool.v, vs, 32, off, w, ps,
                                         pool.cache_seqlens, pool.block_table, 4))
-    del pool, kc, vc, ks, vs
+    del pool, kc, vc, ks, vs, k8p, v8p
     torch.cuda.empty_cache()
 
     if include_model:
@@ -418,7 +441,7 @@ def model_layers(kvq, dev, peak, steps, flush, layers=32):
 
 # ------------------------------------------------------ single-op cases ----
 
-CASES = ("headline_fp8enc", "headline_fp8dec", "fp8enc", "fp8dec", "q4enc", "q4dec", "q6enc", "q6dec", "paged_prefill_q4enc", "paged_prefill_q4dec",
+CASES = ("headline_fp8enc_kv", "headline_fp8dec_kv", "headline_fp8enc", "headline_fp8dec", "fp8enc", "fp8dec", "q4enc", "q4dec", "q6enc", "q6dec", "paged_prefill_q4enc", "paged_prefill_q4dec",
          "paged_decode_q4enc", "model_layer_q6enc", "model_layer_q6dec")
 
 
@@ -428,7 +451,17 @@ def run_case(kvq, dev, name, batch, steps, warmup, peak):
     268 MB of FP16 K+V, above the L2 size); paged cases the 2048-page pool; model cases
     one 1024-page layer."""
     flush = L2Flush(dev)
-    if name.startswith("headline"):
+    if name.startswith("headline") and name.endswith("_kv"):
+        B, S, H, D = HEADLINE["shape"]
+        o, w = HEADLINE["offset"], HEADLINE["width"]
+        k, v = workloads.fp8_window(shape=(B, S, H, D), device=dev)
+        k8, v8 = torch.zeros(k.shape, dtype=torch.uint8, device=dev), torch.zeros(v.shape, dtype=torch.uint8, device=dev)
+        ky, vy = torch.empty_like(k), torch.empty_like(v)
+        kvq.fp16_to_fp8_kv(k, k8, v, v8, B, o, w)
+        nb = 3.0 * 2 * B * w * H * D
+        fn = (lambda: kvq.fp16_to_fp8_kv(k, k8, v, v8, B, o, w)) if "enc" in name else \
+             (lambda: kvq.fp8_to_fp16_kv(k8, ky, v8, vy, B, o, w))
+    elif name.startswith("headline"):
         B, S, H, D = HEADLINE["shape"]
         o, w = HEADLINE["offset"], HEADLINE["width"]
         k, _ = workloads.fp8_window(shape=(B, S, H, D), device=dev)
@@ -510,10 +543,8 @@ def oracle_step_sample(batch=4, max_seconds=12.0, min_reps=1):
     o, w = HEADLINE["offset"], HEADLINE["width"]
     reps, t0 = 0, time.perf_counter()
     while True:
-        oracle.fp16_to_fp8(kn, k8, batch, o, w)
-        oracle.fp16_to_fp8(vn, v8, batch, o, w)
-        oracle.fp8_to_fp16(k8, ky, batch, o, w)
-        oracle.fp8_to_fp16(v8, vy, batch, o, w)
+        oracle.fp16_to_fp8_kv(kn, k8, vn, v8, batch, o, w)
+        oracle.fp8_to_fp16_kv(k8, ky, v8, vy, batch, o, w)
         reps += 1
         if reps >= min_reps and time.perf_counter() - t0 >= max_seconds:
             break
@@ -580,19 +611,18 @@ def main():
     ms_local = statistics.mean(per_step)
     ms = max_over_ranks(ms_local, dev)
     # per-launch durations: the same graph with events between its launches
-    _, segs = time_device(step.run, max(50, args.steps // 10), 3, flush, None, n_marks=3)
-    names = ["fp16_to_fp8(K)", "fp16_to_fp8(V)", "fp8_to_fp16(K)", "fp8_to_fp16(V)"]
-    seg_ms = [statistics.mean(s[i] for s in segs) for i in range(4)]
+    _, segs = time_device(step.run, max(50, args.steps // 10), 3, flush, None, n_marks=1)
+    names = step.names
+    seg_ms = [statistics.mean(s[i] for s in segs) for i in range(2)]
     # Event nodes between launches cost time of their own, so each launch's duration
     # inside the timed (unmarked) step is the step time split in the proportions of
     # the marked segments.
     share = [t / sum(seg_ms) for t in seg_ms]
     launch_ms = [ms_local * f for f in share]
-    enc_ms = (launch_ms[0] + launch_ms[1]) / 2
-    dec_ms = (launch_ms[2] + launch_ms[3]) / 2
-    dom = ("fp16_to_fp8", enc_ms, 0) if enc_ms >= dec_ms else ("fp8_to_fp16", dec_ms, 2)
+    dom_i = 0 if launch_ms[0] >= launch_ms[1] else 1
+    dom = (names[dom_i], launch_ms[dom_i])
     achieved = step.launch_bytes / dom[1] / 1e6
-    dom_isolated_ms = (seg_ms[dom[2]] + seg_ms[dom[2] + 1]) / 2
+    dom_isolated_ms = seg_ms[dom_i]
 
     e2e_ms, h2d, d2h = e2e_fp8(kvq, step, max(10, args.steps // 10), 3, dev)
     e2e_ms = max_over_ranks(e2e_ms, dev)
@@ -633,7 +663,8 @@ def main():
         "data": "synthetic (seeded N(0,1) with 1% outliers and 0.1% subnormals, drawn on device)",
         "config": {"workload": HEADLINE["workload"], "shape": list(HEADLINE["shape"]),
                    "global_batch": batch * world, "offset": HEADLINE["offset"], "width": HEADLINE["width"],
-                   "ops": names, "launch": "CUDA graph of the 4 conversions, replayed once per step", "l2": "flushed between steps (256 MiB write + 256 MiB read, outside the per-step events)",
+                   "ops": ["fp16_to_fp8 of K and V (one fused launch)", "fp8_to_fp16 of K and V (one fused launch)"],
+                   "launch": "CUDA graph of the 2 fused K+V conversions, replayed once per step", "l2": "flushed between steps (256 MiB write + 256 MiB read, outside the per-step events)",
                    "parallelism": f"replicas x{world}, each rank its own 4 sequences"},
         "roofline": {"bound": "hbm", "kernel": dom[0], "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 3), "peak_kind": peak_kind,
@@ -670,10 +701,8 @@ def run_reference(args):
     ky, vy = np.zeros(kn.shape, np.uint16), np.zeros(vn.shape, np.uint16)
 
     def once():
-        oracle.fp16_to_fp8(kn, k8, 1, o, w)
-        oracle.fp16_to_fp8(vn, v8, 1, o, w)
-        oracle.fp8_to_fp16(k8, ky, 1, o, w)
-        oracle.fp8_to_fp16(v8, vy, 1, o, w)
+        oracle.fp16_to_fp8_kv(kn, k8, vn, v8, 1, o, w)
+        oracle.fp8_to_fp16_kv(k8, ky, v8, vy, 1, o, w)
 
     for _ in range(args.warmup):
         once()

@@ -125,6 +125,24 @@ KVQ_API kvq_status kvq_fp16_to_fp8(const void* in, void* out, const kvq_cache_de
 KVQ_API kvq_status kvq_fp8_to_fp16(const void* in, void* out, const kvq_cache_desc* desc,
                            int batch_size, int offset, int width, void* stream);
 
+/* FP8 for K and V in one launch, contiguous or paged.  No counterpart on the
+ * page: it extends fp16_to_fp8 (Description; Signature) to both caches and to
+ * the paged layout, with exactly the window, page, alignment and error rules
+ * of kvq_fp16_to_q_kv (page_size == 0: contiguous, cache_seqlens /
+ * block_table ignored; page_size > 0: paged, page_size == desc->dim1).
+ * head_dim must be a multiple of 8.  All four cache pointers 16-byte
+ * aligned. */
+KVQ_API kvq_status kvq_fp16_to_fp8_kv(const void* k_in, void* k_out, const void* v_in, void* v_out,
+                                      const kvq_cache_desc* desc, int batch_size, int offset, int width,
+                                      int page_size, const int32_t* cache_seqlens,
+                                      const int32_t* block_table, void* stream);
+
+/* The reverse of kvq_fp16_to_fp8_kv (extends fp8_to_fp16 the same way). */
+KVQ_API kvq_status kvq_fp8_to_fp16_kv(const void* k_in, void* k_out, const void* v_in, void* v_out,
+                                      const kvq_cache_desc* desc, int batch_size, int offset, int width,
+                                      int page_size, const int32_t* cache_seqlens,
+                                      const int32_t* block_table, void* stream);
+
 /* fp16_to_q_kv (Description; Signature; I/O Contract): quantize the FP16 K
  * and V caches to wbits-bit codes and FP16 scales in one launch.  page_size
  * == 0 selects contiguous mode (cache_seqlens, block_table ignored and may be

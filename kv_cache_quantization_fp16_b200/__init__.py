@@ -25,7 +25,7 @@ import os
 
 import torch
 
-__all__ = ["fp16_to_fp8", "fp8_to_fp16", "fp16_to_q_kv", "q_to_fp16_kv", "poll_device_error",
+__all__ = ["fp16_to_fp8", "fp8_to_fp16", "fp16_to_fp8_kv", "fp8_to_fp16_kv", "fp16_to_q_kv", "q_to_fp16_kv", "poll_device_error",
            "selfcheck_code_rounding", "q_shapes", "set_engine", "get_engine", "engine", "KVQError",
            "LIB_PATH", "library"]
 
@@ -60,6 +60,8 @@ def _load() -> ctypes.CDLL:
     dp = ctypes.POINTER(_Desc)
     L.kvq_fp16_to_fp8.argtypes = [vp, vp, dp, I, I, I, vp]
     L.kvq_fp8_to_fp16.argtypes = [vp, vp, dp, I, I, I, vp]
+    L.kvq_fp16_to_fp8_kv.argtypes = [vp, vp, vp, vp, dp, I, I, I, I, vp, vp, vp]
+    L.kvq_fp8_to_fp16_kv.argtypes = [vp, vp, vp, vp, dp, I, I, I, I, vp, vp, vp]
     L.kvq_fp16_to_q_kv.argtypes = [vp, vp, vp, vp, vp, vp, dp, I, I, I, I, vp, vp, I, vp]
     L.kvq_q_to_fp16_kv.argtypes = [vp, vp, vp, vp, vp, vp, dp, I, I, I, I, vp, vp, I, vp]
     L.kvq_status_string.argtypes = [I]
@@ -69,7 +71,8 @@ def _load() -> ctypes.CDLL:
     L.kvq_set_engine.argtypes = [I]
     L.kvq_get_engine.argtypes = []
     L.kvq_get_engine.restype = I
-    for f in ("kvq_fp16_to_fp8", "kvq_fp8_to_fp16", "kvq_fp16_to_q_kv", "kvq_q_to_fp16_kv",
+    for f in ("kvq_fp16_to_fp8", "kvq_fp8_to_fp16", "kvq_fp16_to_fp8_kv", "kvq_fp8_to_fp16_kv",
+              "kvq_fp16_to_q_kv", "kvq_q_to_fp16_kv",
               "kvq_poll_device_error", "kvq_selfcheck_code_rounding", "kvq_set_engine"):
         getattr(L, f).restype = I
     return L
@@ -137,6 +140,56 @@ def fp8_to_fp16(in_tensor: torch.Tensor, out_tensor: torch.Tensor, batch_size: i
          torch.float16, "fp8_to_fp16")
 
 
+def _paging(page_size, cache_seqlens, block_table, batch_size, dev):
+    """Checks of the paged-mode metadata (kInt tensors on the caches' device)."""
+    if not page_size:
+        return 0, None, None
+    _require(cache_seqlens is not None and block_table is not None,
+             "paged mode needs cache_seqlens and block_table")
+    _require(cache_seqlens.dtype == torch.int32 and block_table.dtype == torch.int32,
+             "cache_seqlens and block_table must be int32")
+    _require(cache_seqlens.device == dev and block_table.device == dev, "tensors must be on one device")
+    _require(block_table.dim() == 2 and block_table.is_contiguous() and cache_seqlens.is_contiguous(),
+             "block_table must be a contiguous [batch, max_pages] tensor")
+    _require(cache_seqlens.numel() >= batch_size and block_table.shape[0] >= batch_size,
+             "cache_seqlens / block_table have fewer rows than batch_size")
+    return block_table.shape[1], cache_seqlens.data_ptr(), block_table.data_ptr()
+
+
+def _fp8_kv(fn, k_in, k_out, v_in, v_out, batch_size, offset, width, page_size, cache_seqlens, block_table,
+            in_dtype, out_dtype, where):
+    for t, n in ((k_in, "k_in"), (v_in, "v_in")):
+        _cuda4(t, in_dtype, n)
+    for t, n in ((k_out, "k_out"), (v_out, "v_out")):
+        _cuda4(t, out_dtype, n)
+    _require(k_in.shape == k_out.shape == v_in.shape == v_out.shape, "K and V caches must share one shape")
+    dev = k_in.device
+    for t in (k_out, v_in, v_out):
+        _require(t.device == dev, "tensors must be on one device")
+    stride, sl_ptr, bt_ptr = _paging(page_size, cache_seqlens, block_table, batch_size, dev)
+    d0, d1, H, D = k_in.shape
+    desc = _Desc(d0, d1, H, D, stride)
+    with torch.cuda.device(dev):
+        st = fn(k_in.data_ptr(), k_out.data_ptr(), v_in.data_ptr(), v_out.data_ptr(), ctypes.byref(desc),
+                int(batch_size), int(offset), int(width), int(page_size), sl_ptr, bt_ptr, _stream(dev))
+    _check(st, where)
+
+
+def fp16_to_fp8_kv(k_in, k_out, v_in, v_out, batch_size, offset, width, page_size=0, cache_seqlens=None,
+                   block_table=None) -> None:
+    """E5M2-encode the K and V FP16 cache windows in one launch, contiguous or paged
+    (an extension of fp16_to_fp8 with the window and page rules of fp16_to_q_kv)."""
+    _fp8_kv(_lib.kvq_fp16_to_fp8_kv, k_in, k_out, v_in, v_out, batch_size, offset, width, page_size,
+            cache_seqlens, block_table, torch.float16, torch.uint8, "fp16_to_fp8_kv")
+
+
+def fp8_to_fp16_kv(k_in, k_out, v_in, v_out, batch_size, offset, width, page_size=0, cache_seqlens=None,
+                   block_table=None) -> None:
+    """Decode the K and V E5M2 cache windows into FP16 in one launch, contiguous or paged."""
+    _fp8_kv(_lib.kvq_fp8_to_fp16_kv, k_in, k_out, v_in, v_out, batch_size, offset, width, page_size,
+            cache_seqlens, block_table, torch.uint8, torch.float16, "fp8_to_fp16_kv")
+
+
 def _q(fn, fp16_is_input, k_in, k_out, k_scales, v_in, v_out, v_scales, batch_size, offset, width,
        page_size, cache_seqlens, block_table, wbits, where):
     k16, kq = (k_in, k_out) if fp16_is_input else (k_out, k_in)
@@ -158,20 +211,7 @@ def _q(fn, fp16_is_input, k_in, k_out, k_scales, v_in, v_out, v_scales, batch_si
     dev = k16.device
     for t in (kq, v16, vq, k_scales, v_scales):
         _require(t.device == dev, "tensors must be on one device")
-    stride = 0
-    sl_ptr = bt_ptr = None
-    if page_size:
-        _require(cache_seqlens is not None and block_table is not None,
-                 "paged mode needs cache_seqlens and block_table")
-        _require(cache_seqlens.dtype == torch.int32 and block_table.dtype == torch.int32,
-                 "cache_seqlens and block_table must be int32")
-        _require(cache_seqlens.device == dev and block_table.device == dev, "tensors must be on one device")
-        _require(block_table.dim() == 2 and block_table.is_contiguous() and cache_seqlens.is_contiguous(),
-                 "block_table must be a contiguous [batch, max_pages] tensor")
-        _require(cache_seqlens.numel() >= batch_size and block_table.shape[0] >= batch_size,
-                 "cache_seqlens / block_table have fewer rows than batch_size")
-        stride = block_table.shape[1]
-        sl_ptr, bt_ptr = cache_seqlens.data_ptr(), block_table.data_ptr()
+    stride, sl_ptr, bt_ptr = _paging(page_size, cache_seqlens, block_table, batch_size, dev)
     d0, d1, H, D = k16.shape
     desc = _Desc(d0, d1, H, D, stride)
     with torch.cuda.device(dev):

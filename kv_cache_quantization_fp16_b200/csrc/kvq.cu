@@ -254,6 +254,39 @@ kvq_status fp8_common(const void* in, void* out, const kvq_cache_desc* d, int ba
   return encode ? launch<Fp8Encode>(p, 1, stream) : launch<Fp8Decode>(p, 1, stream);
 }
 
+// Window / page checks shared by the K+V conversions.
+kvq_status check_kv_window(const kvq_cache_desc* d, int batch, int offset, int width, int page_size,
+                           const int32_t* seqlens, const int32_t* block_table) {
+  if (page_size < 0) return KVQ_ERR_RANGE;
+  if (page_size == 0) return check_contiguous_window(d, batch, offset, width);
+  if (!seqlens || !block_table) return KVQ_ERR_NULL;
+  if (page_size != d->dim1 || batch < 0 || width < 0) return KVQ_ERR_RANGE;
+  if (d->block_table_stride < 1) return KVQ_ERR_RANGE;
+  if ((reinterpret_cast<uintptr_t>(seqlens) | reinterpret_cast<uintptr_t>(block_table)) & 3u) return KVQ_ERR_ALIGN;
+  return KVQ_OK;
+}
+
+kvq_status fp8_kv_common(const void* k_in, void* k_out, const void* v_in, void* v_out, const kvq_cache_desc* d,
+                         int batch, int offset, int width, int page_size, const int32_t* seqlens,
+                         const int32_t* block_table, void* stream, bool encode) {
+  if (!k_in || !k_out || !v_in || !v_out) return KVQ_ERR_NULL;
+  kvq_status st = check_desc(d, 8);
+  if (st != KVQ_OK) return st;
+  const void* ptrs[4] = {k_in, k_out, v_in, v_out};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return KVQ_ERR_ALIGN;
+  st = check_kv_window(d, batch, offset, width, page_size, seqlens, block_table);
+  if (st != KVQ_OK) return st;
+  if (batch == 0 || width == 0) return KVQ_OK;
+  Params p{};
+  p.g = make_geometry(d, batch, offset, width, page_size, seqlens, block_table);
+  p.in[0] = k_in;
+  p.in[1] = v_in;
+  p.out[0] = k_out;
+  p.out[1] = v_out;
+  return encode ? launch<Fp8Encode>(p, 2, stream) : launch<Fp8Decode>(p, 2, stream);
+}
+
 kvq_status q_common(const void* k_in, void* k_out, void* k_scales, const void* v_in, void* v_out,
                     void* v_scales, const kvq_cache_desc* d, int batch, int offset, int width,
                     int page_size, const int32_t* seqlens, const int32_t* block_table, int wbits,
@@ -265,17 +298,8 @@ kvq_status q_common(const void* k_in, void* k_out, void* k_scales, const void* v
   const void* ptrs[6] = {k_in, k_out, k_scales, v_in, v_out, v_scales};
   for (const void* q : ptrs)
     if (!aligned16(q)) return KVQ_ERR_ALIGN;
-  if (page_size < 0) return KVQ_ERR_RANGE;
-  if (page_size == 0) {
-    st = check_contiguous_window(d, batch, offset, width);
-    if (st != KVQ_OK) return st;
-  } else {
-    if (!seqlens || !block_table) return KVQ_ERR_NULL;
-    if (page_size != d->dim1 || batch < 0 || width < 0) return KVQ_ERR_RANGE;
-    if (d->block_table_stride < 1) return KVQ_ERR_RANGE;
-    if ((reinterpret_cast<uintptr_t>(seqlens) | reinterpret_cast<uintptr_t>(block_table)) & 3u)
-      return KVQ_ERR_ALIGN;
-  }
+  st = check_kv_window(d, batch, offset, width, page_size, seqlens, block_table);
+  if (st != KVQ_OK) return st;
   if (batch == 0 || width == 0) return KVQ_OK;
   Params p{};
   p.g = make_geometry(d, batch, offset, width, page_size, seqlens, block_table);
@@ -301,6 +325,22 @@ kvq_status kvq_fp16_to_fp8(const void* in, void* out, const kvq_cache_desc* desc
 kvq_status kvq_fp8_to_fp16(const void* in, void* out, const kvq_cache_desc* desc, int batch_size,
                            int offset, int width, void* stream) {
   return fp8_common(in, out, desc, batch_size, offset, width, stream, false);
+}
+
+kvq_status kvq_fp16_to_fp8_kv(const void* k_in, void* k_out, const void* v_in, void* v_out,
+                              const kvq_cache_desc* desc, int batch_size, int offset, int width,
+                              int page_size, const int32_t* cache_seqlens, const int32_t* block_table,
+                              void* stream) {
+  return fp8_kv_common(k_in, k_out, v_in, v_out, desc, batch_size, offset, width, page_size, cache_seqlens,
+                       block_table, stream, true);
+}
+
+kvq_status kvq_fp8_to_fp16_kv(const void* k_in, void* k_out, const void* v_in, void* v_out,
+                              const kvq_cache_desc* desc, int batch_size, int offset, int width,
+                              int page_size, const int32_t* cache_seqlens, const int32_t* block_table,
+                              void* stream) {
+  return fp8_kv_common(k_in, k_out, v_in, v_out, desc, batch_size, offset, width, page_size, cache_seqlens,
+                       block_table, stream, false);
 }
 
 kvq_status kvq_fp16_to_q_kv(const void* k_in, void* k_out, void* k_scales, const void* v_in,

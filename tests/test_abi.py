@@ -117,3 +117,19 @@ def test_python_binding_checks_dtypes(kvq):
         kvq.fp16_to_fp8(k, torch.zeros(1, 4, 1, 32, dtype=torch.uint8), 1, 0, 4)  # CPU tensors
     with pytest.raises(ValueError):
         kvq.fp16_to_fp8(k.float(), k, 1, 0, 4)
+
+
+def test_fp8_kv_validation(kvq):
+    L = kvq.library()
+    by = ctypes.byref
+    d = _desc(kvq)
+    P = [FAKE] * 4
+    assert L.kvq_fp16_to_fp8_kv(None, *P[1:], by(d), 2, 0, 16, 0, None, None, None) == 1
+    assert L.kvq_fp16_to_fp8_kv(*P, by(_desc(kvq, D=12)), 2, 0, 16, 0, None, None, None) == 2
+    assert L.kvq_fp16_to_fp8_kv(*P, by(d), 3, 0, 16, 0, None, None, None) == 4
+    assert L.kvq_fp8_to_fp16_kv(FAKE + 8, *P[1:], by(d), 2, 0, 16, 0, None, None, None) == 5
+    dp = _desc(kvq, d0=10, d1=16, stride=4)
+    assert L.kvq_fp16_to_fp8_kv(*P, by(dp), 2, 0, 16, 16, None, FAKE, None) == 1
+    assert L.kvq_fp16_to_fp8_kv(*P, by(dp), 2, 0, 16, 8, FAKE, FAKE, None) == 4
+    assert L.kvq_fp8_to_fp16_kv(*P, by(dp), 2, -3, 0, 16, FAKE, FAKE, None) == 0   # empty window
+    assert L.kvq_set_engine(9) == 4 and L.kvq_get_engine() == 0

@@ -118,3 +118,61 @@ def test_bulk_bad_block_table_reports(kvq, oracle_mod, dev):
     rs = np.zeros(ss, np.uint16)
     oracle_mod.fp16_to_q_kv(u16(k), rc, rs, u16(v), rc.copy(), rs.copy(), 2, 0, 8, ps, lens.numpy(), bt.numpy(), 4)
     assert np.array_equal(u8(kc), rc)
+
+
+def run_fp8_kv(kvq, oracle_mod, k, v, batch, offset, width, dev, page_size=0, seqlens=None, bt=None):
+    """Fused K+V FP8 encode then decode on the GPU and in the oracle, sentinel-filled buffers."""
+    kd, vd = k.to(dev), v.to(dev)
+    k8 = torch.full(k.shape, 0xA5, dtype=torch.uint8, device=dev)
+    v8 = torch.full(k.shape, 0xA5, dtype=torch.uint8, device=dev)
+    sl = seqlens.to(dev) if seqlens is not None else None
+    btd = bt.to(dev) if bt is not None else None
+    kvq.fp16_to_fp8_kv(kd, k8, vd, v8, batch, offset, width, page_size, sl, btd)
+    ky = torch.full(k.shape, 0xA5A5 - 65536, dtype=torch.int16, device=dev).view(torch.float16)
+    vy = ky.clone()
+    kvq.fp8_to_fp16_kv(k8, ky, v8, vy, batch, offset, width, page_size, sl, btd)
+    assert kvq.poll_device_error() == 0
+    rk8, rv8 = np.full(k.shape, 0xA5, np.uint8), np.full(k.shape, 0xA5, np.uint8)
+    sln = seqlens.numpy() if seqlens is not None else None
+    btn = bt.numpy() if bt is not None else None
+    assert oracle_mod.fp16_to_fp8_kv(u16(k), rk8, u16(v), rv8, batch, offset, width, page_size, sln, btn) == 0
+    rky, rvy = np.full(k.shape, 0xA5A5, np.uint16), np.full(k.shape, 0xA5A5, np.uint16)
+    assert oracle_mod.fp8_to_fp16_kv(rk8, rky, rv8, rvy, batch, offset, width, page_size, sln, btn) == 0
+    assert np.array_equal(u8(k8), rk8) and np.array_equal(u8(v8), rv8)
+    assert np.array_equal(u16(ky), rky) and np.array_equal(u16(vy), rvy)
+
+
+def test_fp8_kv_contiguous_window(kvq, oracle_mod, dev, eng):
+    k, v = workloads.fp8_window(shape=(4, 1024, 8, 128))
+    run_fp8_kv(kvq, oracle_mod, k, v, 4, 100, 801, dev)
+
+
+def test_fp8_kv_paged(kvq, oracle_mod, dev, eng):
+    pool = workloads.paged_pool(num_pages=160, batch=6, max_len=1500, heads=4, head_dim=64)
+    for offset, width in ((0, 1), (-300, 300), (-1500, 1501)):
+        run_fp8_kv(kvq, oracle_mod, pool.k, pool.v, 6, offset, width, dev, page_size=256,
+                   seqlens=pool.cache_seqlens, bt=pool.block_table)
+
+
+@pytest.mark.parametrize("ps", [16, 7])
+def test_fp8_kv_paged_identity_equals_contiguous(kvq, oracle_mod, dev, eng, ps):
+    B, H, D = 3, 2, 24
+    S = ps * 6
+    k, v = workloads.fp8_window(shape=(B, S, H, D))
+    bt = workloads.identity_block_table(B, S, ps)
+    run_fp8_kv(kvq, oracle_mod, k, v, B, 5, S - 9, dev)
+    pages = (B * S // ps, ps, H, D)
+    run_fp8_kv(kvq, oracle_mod, k.reshape(pages), v.reshape(pages), B, 5, S - 9, dev, page_size=ps,
+               seqlens=torch.zeros(B, dtype=torch.int32), bt=bt)
+
+
+def test_fp8_kv_bad_block_table(kvq, dev, eng):
+    ps, H, D, npages = 8, 1, 32, 6
+    k, v = workloads.small(shape=(npages, ps, H, D))
+    bt = torch.tensor([[0, 7], [1, -1]], dtype=torch.int32, device=dev)
+    lens = torch.tensor([4, 6], dtype=torch.int32, device=dev)
+    kd, vd = k.to(dev), v.to(dev)
+    k8, v8 = torch.zeros(k.shape, dtype=torch.uint8, device=dev), torch.zeros(k.shape, dtype=torch.uint8, device=dev)
+    assert kvq.poll_device_error() == 0
+    kvq.fp16_to_fp8_kv(kd, k8, vd, v8, 2, 0, 8, ps, lens, bt)
+    assert kvq.poll_device_error() in (1, 2)

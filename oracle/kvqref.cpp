@@ -112,13 +112,15 @@ uint16_t e5m2_decode(uint8_t b) {
 }
 
 // ---------------------------------------------------------------------------
-// Q4 / Q6 codec (I/O Contract: k_scales / v_scales are "per-block
-// quantization scale factors", kHalf; wbits is 4 or 6).
+// Q4 / Q6 / Q8 codec (I/O Contract: k_scales / v_scales are "per-block
+// quantization scale factors", kHalf; wbits is 4 or 6 there, and the page's
+// Usage section also names a Q8 cache class, so 8 is accepted with the same
+// rules: maxq 127, zero point 128, one byte per code).
 // ---------------------------------------------------------------------------
 
 constexpr int kBlock = 32;  // elements per scale block along head_dim
 
-bool valid_wbits(int wbits) { return wbits == 4 || wbits == 6; }
+bool valid_wbits(int wbits) { return wbits == 4 || wbits == 6 || wbits == 8; }
 int maxq_of(int wbits) { return (1 << (wbits - 1)) - 1; }
 int zero_of(int wbits) { return 1 << (wbits - 1); }
 

@@ -19,7 +19,8 @@
  *              nearest, ties to even, IEEE overflow to +-Inf (no
  *              saturation), NaN -> quiet NaN (sign | 0x7E).  Decoding is
  *              exact (every E5M2 value is a binary16 value).
- *   Q4 / Q6  = symmetric absmax over 32-element blocks along head_dim.
+ *   Q4/Q6/Q8 = symmetric absmax over 32-element blocks along head_dim
+ *              (wbits 4, 6 or 8).
  *              maxq = 2^(b-1) - 1, zero point z = 2^(b-1).
  *              s    = RN16( fl32( absmax / maxq ) )      (stored as FP16)
  *              code = clamp( rint( fl32( x / s ) ) + z, 0, 2^b - 1 ),

@@ -134,7 +134,7 @@ def test_e5m2_worked_values(oracle_mod, h, byte, dec):
 
 # ------------------------------------------------------------------- scale ----
 
-@pytest.mark.parametrize("wbits", [4, 6])
+@pytest.mark.parametrize("wbits", [4, 6, 8])
 def test_block_scale_exhaustive_exact(oracle_mod, wbits):
     """s = RN16(fl32(a / maxq)) equals the binary16 nearest to the exact quotient for
     every finite absmax a (so the binary32 intermediate never double-rounds)."""
@@ -182,7 +182,7 @@ def _test_blocks(seed):
     for _ in range(200):  # subnormal magnitudes: scale is subnormal or zero
         bits = rng.integers(0, 64, 32).astype(np.uint16) | np.where(rng.random(32) < 0.5, 0x8000, 0).astype(np.uint16)
         blocks.append(bits.view(np.float16))
-    for wb in (4, 6):  # exact ties: absmax maxq * 2^k, members (k+0.5) * 2^k
+    for wb in (4, 6, 8):  # exact ties: absmax maxq * 2^k, members (k+0.5) * 2^k
         maxq = (1 << (wb - 1)) - 1
         for _ in range(100):
             e = float(2.0 ** rng.integers(-8, 8))
@@ -194,7 +194,7 @@ def _test_blocks(seed):
     return blocks
 
 
-@pytest.mark.parametrize("wbits", [4, 6])
+@pytest.mark.parametrize("wbits", [4, 6, 8])
 def test_quantize_codes_exact(oracle_mod, wbits):
     for blk in _test_blocks(11 + wbits):
         bits = blk.view(np.uint16)
@@ -204,7 +204,7 @@ def test_quantize_codes_exact(oracle_mod, wbits):
         assert codes.tolist() == ref_codes, (blk, codes, ref_codes)
 
 
-@pytest.mark.parametrize("wbits", [4, 6])
+@pytest.mark.parametrize("wbits", [4, 6, 8])
 def test_dequantize_exact(oracle_mod, wbits):
     rng = np.random.default_rng(5 + wbits)
     for blk in _test_blocks(21 + wbits)[:400]:
@@ -216,9 +216,9 @@ def test_dequantize_exact(oracle_mod, wbits):
     z = 1 << (wbits - 1)
     for _ in range(200):
         s_bits = int(rng.integers(0, 0x7C00))
-        codes = np.arange(1 << wbits, dtype=np.uint8)
-        codes = np.resize(codes, 64)
-        scales = np.array([s_bits, s_bits], np.uint16)
+        n = max(64, 1 << wbits)
+        codes = np.resize(np.arange(1 << wbits, dtype=np.uint8), n)
+        scales = np.full(n // 32, s_bits, np.uint16)
         y = oracle_mod.dequantize_row(codes, scales, wbits)
         with np.errstate(over="ignore"):
             ref = (codes.astype(np.float16) - np.float16(z)) * scales.view(np.float16)[0]
@@ -228,7 +228,7 @@ def test_dequantize_exact(oracle_mod, wbits):
 
 # ----------------------------------------------------------------- packing ----
 
-@pytest.mark.parametrize("wbits", [4, 6])
+@pytest.mark.parametrize("wbits", [4, 6, 8])
 def test_pack_bitstream(oracle_mod, wbits):
     rng = np.random.default_rng(wbits)
     for n in (32, 64, 128, 256):

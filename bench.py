@@ -51,7 +51,7 @@ FLUSH_BYTES = 256 << 20
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 
-BYTES_PER_ELEM = {"fp8": 3.0, 4: 2.0 + 0.5 + 2.0 / 32, 6: 2.0 + 0.75 + 2.0 / 32}
+BYTES_PER_ELEM = {"fp8": 3.0, 4: 2.0 + 0.5 + 2.0 / 32, 6: 2.0 + 0.75 + 2.0 / 32, 8: 2.0 + 1.0 + 2.0 / 32}
 
 
 # ------------------------------------------------------------- host logic ----
@@ -341,7 +341,7 @@ def per_op_measurements(kvq, dev, peak, steps, flush, include_model=True):
     B, S, H, D = k.shape
     n = 2 * k.numel()
     ky, vy = torch.empty_like(k), torch.empty_like(v)
-    for wb in (4, 6):
+    for wb in (4, 6, 8):
         cs, ss = kvq.q_shapes(tuple(k.shape), wb)
         kc = torch.empty(cs, dtype=torch.uint8, device=dev)
         vc = torch.empty_like(kc)
@@ -441,7 +441,8 @@ def model_layers(kvq, dev, peak, steps, flush, layers=32):
 
 # ------------------------------------------------------ single-op cases ----
 
-CASES = ("headline_fp8enc_kv", "headline_fp8dec_kv", "headline_fp8enc", "headline_fp8dec", "fp8enc", "fp8dec", "q4enc", "q4dec", "q6enc", "q6dec", "paged_prefill_q4enc", "paged_prefill_q4dec",
+CASES = ("headline_fp8enc_kv", "headline_fp8dec_kv", "headline_fp8enc", "headline_fp8dec", "fp8enc", "fp8dec", "q4enc",
+         "q4dec", "q6enc", "q6dec", "q8enc", "q8dec", "paged_prefill_q4enc", "paged_prefill_q4dec",
          "paged_decode_q4enc", "model_layer_q6enc", "model_layer_q6dec")
 
 
@@ -471,7 +472,7 @@ def run_case(kvq, dev, name, batch, steps, warmup, peak):
         nb = 3.0 * B * w * H * D
         fn = (lambda: kvq.fp16_to_fp8(k, k8, B, o, w)) if name.endswith("enc") else \
              (lambda: kvq.fp8_to_fp16(k8, y, B, o, w))
-    elif name.startswith("fp8") or name[:2] in ("q4", "q6"):
+    elif name.startswith("fp8") or name[:2] in ("q4", "q6", "q8"):
         k, v = workloads.channel_outliers(shape=(batch, 8192, 8, 128), device=dev)
         B, S = k.shape[:2]
         if name.startswith("fp8"):

@@ -15,7 +15,9 @@
  *   FP8   E5M2 = the upper byte of binary16 after rounding to 2 fraction bits,
  *         round to nearest, ties to even; no saturation (|x| >= 61440 -> Inf);
  *         any NaN -> sign | 0x7E.  Decoding is exact: half bits = byte << 8.
- *   Q4/Q6 symmetric absmax over 32 consecutive head_dim elements.
+ *   Q4/Q6/Q8 symmetric absmax over 32 consecutive head_dim elements
+ *         (wbits 4 or 6 as the page's I/O Contract gives; 8 as its Usage
+ *         section's Q8 cache class implies, same rules).
  *         maxq = 2^(wbits-1) - 1, z = 2^(wbits-1).
  *         scale s = RN16(fl32(absmax / maxq)) stored as FP16;
  *         code    = clamp(rint(fl32(x / s)) + z, 0, 2^wbits - 1), ties to even,
@@ -24,7 +26,7 @@
  *         The codes of one head row form a little-endian bit stream: code j
  *         occupies bits [wbits*j, wbits*j + wbits) of the row's bytes (Q4: two
  *         codes per byte, even element in the low nibble; Q6: 16 codes per
- *         three 32-bit little-endian words).
+ *         three 32-bit little-endian words; Q8: one byte per code).
  *   Results are bit-exact with these definitions; there is no tolerance.
  *
  * Layouts (row-major; all pointers are device memory on the current device):
@@ -80,7 +82,7 @@ typedef enum kvq_status {
   KVQ_OK = 0,
   KVQ_ERR_NULL = 1,    /* a required pointer is NULL */
   KVQ_ERR_SHAPE = 2,   /* bad dims: negative, head_dim not a multiple of 8 (FP8) or 32 (Q) */
-  KVQ_ERR_WBITS = 3,   /* wbits is not 4 or 6 */
+  KVQ_ERR_WBITS = 3,   /* wbits is not 4, 6 or 8 */
   KVQ_ERR_RANGE = 4,   /* window or batch outside the cache, page_size != dim1 */
   KVQ_ERR_ALIGN = 5,   /* a buffer is not 16-byte aligned */
   KVQ_ERR_CUDA = 6,    /* the CUDA runtime reported an error */
@@ -149,7 +151,7 @@ KVQ_API kvq_status kvq_fp8_to_fp16_kv(const void* k_in, void* k_out, const void*
  * NULL); page_size > 0 selects paged mode (page_size == desc->dim1,
  * cache_seqlens and block_table required).  head_dim must be a multiple of
  * 32 (the scale block, the page's Q_CACHE_BLOCKSIZE_Q alignment).  wbits is
- * 4 or 6.  All six cache pointers 16-byte aligned. */
+ * 4, 6 or 8.  All six cache pointers 16-byte aligned. */
 KVQ_API kvq_status kvq_fp16_to_q_kv(const void* k_in, void* k_out, void* k_scales,
                             const void* v_in, void* v_out, void* v_scales,
                             const kvq_cache_desc* desc, int batch_size, int offset, int width,

@@ -43,7 +43,7 @@ class _Desc(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("block_table_stride", ctypes.c_int32)]
 
 
-_STATUS = {0: "ok", 1: "null pointer", 2: "bad shape", 3: "wbits must be 4 or 6",
+_STATUS = {0: "ok", 1: "null pointer", 2: "bad shape", 3: "wbits must be 4, 6 or 8",
            4: "window, batch or page geometry out of range", 5: "buffer not 16-byte aligned",
            6: "CUDA runtime error", 7: "device recorded bad paging metadata"}
 
@@ -201,7 +201,7 @@ def _q(fn, fp16_is_input, k_in, k_out, k_scales, v_in, v_out, v_scales, batch_si
     for t, n in ((k_scales, "k_scales"), (v_scales, "v_scales")):
         _cuda4(t, torch.float16, n)
     _require(k16.shape == v16.shape, "K and V caches must have the same shape")
-    _require(wbits in (4, 6), f"wbits must be 4 or 6, got {wbits}")
+    _require(wbits in (4, 6, 8), f"wbits must be 4, 6 or 8, got {wbits}")
     _require(k16.shape[3] % 32 == 0, "head_dim must be a multiple of 32")
     cshape, sshape = q_shapes(tuple(k16.shape), wbits)
     for t, n in ((kq, "K codes"), (vq, "V codes")):

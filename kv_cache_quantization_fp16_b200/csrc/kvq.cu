@@ -294,7 +294,7 @@ kvq_status q_common(const void* k_in, void* k_out, void* k_scales, const void* v
   if (!k_in || !k_out || !k_scales || !v_in || !v_out || !v_scales) return KVQ_ERR_NULL;
   kvq_status st = check_desc(d, kBlockElems);
   if (st != KVQ_OK) return st;
-  if (wbits != 4 && wbits != 6) return KVQ_ERR_WBITS;
+  if (wbits != 4 && wbits != 6 && wbits != 8) return KVQ_ERR_WBITS;
   const void* ptrs[6] = {k_in, k_out, k_scales, v_in, v_out, v_scales};
   for (const void* q : ptrs)
     if (!aligned16(q)) return KVQ_ERR_ALIGN;
@@ -309,8 +309,14 @@ kvq_status q_common(const void* k_in, void* k_out, void* k_scales, const void* v
   p.out[1] = v_out;
   p.scales[0] = k_scales;
   p.scales[1] = v_scales;
-  if (encode) return wbits == 4 ? launch<QEncode<4>>(p, 2, stream) : launch<QEncode<6>>(p, 2, stream);
-  return wbits == 4 ? launch<QDecode<4>>(p, 2, stream) : launch<QDecode<6>>(p, 2, stream);
+  if (encode) {
+    if (wbits == 4) return launch<QEncode<4>>(p, 2, stream);
+    if (wbits == 6) return launch<QEncode<6>>(p, 2, stream);
+    return launch<QEncode<8>>(p, 2, stream);
+  }
+  if (wbits == 4) return launch<QDecode<4>>(p, 2, stream);
+  if (wbits == 6) return launch<QDecode<6>>(p, 2, stream);
+  return launch<QDecode<8>>(p, 2, stream);
 }
 
 }  // namespace
@@ -366,7 +372,7 @@ const char* kvq_status_string(kvq_status s) {
     case KVQ_OK: return "ok";
     case KVQ_ERR_NULL: return "null pointer";
     case KVQ_ERR_SHAPE: return "bad shape";
-    case KVQ_ERR_WBITS: return "wbits must be 4 or 6";
+    case KVQ_ERR_WBITS: return "wbits must be 4, 6 or 8";
     case KVQ_ERR_RANGE: return "window, batch or page geometry out of range";
     case KVQ_ERR_ALIGN: return "buffer not 16-byte aligned";
     case KVQ_ERR_CUDA: return "CUDA runtime error";
@@ -399,13 +405,15 @@ int kvq_get_engine(void) { return g_engine.load(); }
 
 kvq_status kvq_selfcheck_code_rounding(int wbits, unsigned long long* mismatches, void* stream) {
   if (!mismatches) return KVQ_ERR_NULL;
-  if (wbits != 4 && wbits != 6) return KVQ_ERR_WBITS;
+  if (wbits != 4 && wbits != 6 && wbits != 8) return KVQ_ERR_WBITS;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(mismatches, 0, sizeof(unsigned long long), s) != cudaSuccess) return KVQ_ERR_CUDA;
   if (wbits == 4)
     kvq::selfcheck_rounding_kernel<4><<<0x7C00, 256, 0, s>>>(mismatches);
-  else
+  else if (wbits == 6)
     kvq::selfcheck_rounding_kernel<6><<<0x7C00, 256, 0, s>>>(mismatches);
+  else
+    kvq::selfcheck_rounding_kernel<8><<<0x7C00, 256, 0, s>>>(mismatches);
   return launch_status();
 }
 

@@ -80,8 +80,8 @@ struct Fp8Decode {
 
 // Q encode: one thread owns whole 32-element blocks (4 x 16-byte loads), so
 // the absmax needs no shuffles, the scale and reciprocal are computed once per
-// block, and the packed codes leave as one 16-byte (Q4) or three 8-byte (Q6)
-// stores.  U blocks per thread are loaded before any is encoded.
+// block, and the packed codes leave as one 16-byte (Q4), three 8-byte (Q6) or
+// two 16-byte (Q8) stores.  U blocks per thread are loaded before any is encoded.
 template <int B>
 struct QEncode {
   static constexpr int kInNum = 2, kInDen = 1;
@@ -118,6 +118,10 @@ struct QEncode {
           encode_block_words<B, false>(x[u], bs, w);
         if (B == 4) {
           reinterpret_cast<uint4*>(codes)[b] = make_uint4(w[0], w[1], w[2 % B], w[3 % B]);
+        } else if (B == 8) {
+          uint4* dst = reinterpret_cast<uint4*>(codes + static_cast<long long>(b) * 32);
+          dst[0] = make_uint4(w[0], w[1], w[2 % B], w[3 % B]);
+          dst[1] = make_uint4(w[4 % B], w[5 % B], w[6 % B], w[7 % B]);
         } else {
           uint2* dst = reinterpret_cast<uint2*>(codes + static_cast<long long>(b) * 24);
           dst[0] = make_uint2(w[0], w[1]);
@@ -153,6 +157,10 @@ struct QDecode {
         if (v < nvec) {
           if (B == 4) {
             lo[u] = Src::load(reinterpret_cast<const uint32_t*>(codes) + v);
+          } else if (B == 8) {
+            const uint2 q = Src::load(reinterpret_cast<const uint2*>(codes) + v);
+            lo[u] = q.x;
+            hi[u] = q.y;
           } else {
             // lane pair = one 12-byte group; the even lane needs words 0-1, the
             // odd lane words 1-2 (bits 48..95 of the group)
@@ -171,7 +179,9 @@ struct QDecode {
         const int v = base + u * NT + tid;
         if (v >= nvec) continue;
         const __half2 s2 = __halves2half2(s[u], s[u]);
-        dst[v] = (B == 4) ? dequant_q4_v8(lo[u], s2) : dequant_q6_v8(lo[u], hi[u], s2);
+        dst[v] = (B == 4) ? dequant_q4_v8(lo[u], s2)
+                 : (B == 8) ? dequant_q8_v8(lo[u], hi[u], s2)
+                            : dequant_q6_v8(lo[u], hi[u], s2);
       }
     }
   }

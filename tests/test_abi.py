@@ -84,7 +84,7 @@ def test_q_validation(kvq):
     by = ctypes.byref
     P = [FAKE] * 6
     assert L.kvq_fp16_to_q_kv(*P, by(d), 2, 0, 16, 0, None, None, 5, None) == 3
-    assert L.kvq_fp16_to_q_kv(*P, by(d), 2, 0, 16, 0, None, None, 8, None) == 3
+    assert L.kvq_fp16_to_q_kv(*P, by(d), 2, 0, 16, 0, None, None, 7, None) == 3
     assert L.kvq_q_to_fp16_kv(*P, by(_desc(kvq, D=48)), 2, 0, 16, 0, None, None, 4, None) == 2
     assert L.kvq_fp16_to_q_kv(*P[:5], None, by(d), 2, 0, 16, 0, None, None, 4, None) == 1
     assert L.kvq_fp16_to_q_kv(*P[:3], FAKE + 4, *P[4:], by(d), 2, 0, 16, 0, None, None, 4, None) == 5

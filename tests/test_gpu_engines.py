@@ -48,13 +48,13 @@ def test_fp8_window(kvq, oracle_mod, dev, eng):
     run_fp8(kvq, oracle_mod, k, 4, 100, 801, dev)
 
 
-@pytest.mark.parametrize("wbits", [4, 6])
+@pytest.mark.parametrize("wbits", [4, 6, 8])
 def test_q_contiguous(kvq, oracle_mod, dev, eng, wbits):
     k, v = workloads.channel_outliers(shape=(2, 512, 8, 128))
     run_q(kvq, oracle_mod, k, v, wbits, 2, 3, 500, dev)
 
 
-@pytest.mark.parametrize("wbits", [4, 6])
+@pytest.mark.parametrize("wbits", [4, 6, 8])
 def test_q_paged(kvq, oracle_mod, dev, eng, wbits):
     pool = workloads.paged_pool(num_pages=160, batch=6, max_len=1500, heads=4, head_dim=64)
     for offset, width in ((0, 1), (-300, 300), (-1500, 1501)):
@@ -67,7 +67,7 @@ def test_ragged_and_fallback_shapes(kvq, oracle_mod, dev, eng, shape):
     """H*D = 32 or 288 make one position of the Q6 / FP8 streams not a multiple of 16 bytes
     (the bulk engine falls back); H*D = 16384 exceeds a bulk stage (falls back too)."""
     k, v = workloads.channel_outliers(shape=shape)
-    for wbits in (4, 6):
+    for wbits in (4, 6, 8):
         run_q(kvq, oracle_mod, k, v, wbits, shape[0], 1, shape[1] - 2, dev)
     run_fp8(kvq, oracle_mod, k, shape[0], 0, shape[1], dev)
 
@@ -76,7 +76,7 @@ def test_engines_agree_at_scale(kvq, dev):
     """Full-size channel-outlier Q4/Q6 both directions: both engines write identical bytes."""
     k, v = workloads.channel_outliers(shape=(4, 8192, 8, 128), device=dev)
     B, S = k.shape[:2]
-    for wbits in (4, 6):
+    for wbits in (4, 6, 8):
         outs = []
         for name in ("ldg", "bulk"):
             with kvq.engine(name):

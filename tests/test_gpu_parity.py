@@ -122,7 +122,7 @@ def test_fp8_decode_every_byte(kvq, oracle_mod, dev):
     assert np.array_equal(u16(out), ref)
 
 
-@pytest.mark.parametrize("wbits", [4, 6])
+@pytest.mark.parametrize("wbits", [4, 6, 8])
 def test_scale_every_absmax(kvq, oracle_mod, dev, wbits):
     """One block per finite binary16 absmax a (block = [a, -a/3, 0, ...] shuffled)."""
     n = 0x7C00
@@ -135,13 +135,13 @@ def test_scale_every_absmax(kvq, oracle_mod, dev, wbits):
     run_q(kvq, oracle_mod, x, x.flip(1).contiguous(), wbits, 1, 0, n, dev)
 
 
-@pytest.mark.parametrize("wbits", [4, 6])
+@pytest.mark.parametrize("wbits", [4, 6, 8])
 def test_code_rounding_selfcheck(kvq, dev, wbits):
     """The fast code rounding equals IEEE division + rint + clamp for all 2^31 (x, s) pairs."""
     assert kvq.selfcheck_code_rounding(wbits) == 0
 
 
-@pytest.mark.parametrize("wbits", [4, 6])
+@pytest.mark.parametrize("wbits", [4, 6, 8])
 def test_ties_and_subnormal_scales(kvq, oracle_mod, dev, wbits):
     rng = np.random.default_rng(100 + wbits)
     maxq = (1 << (wbits - 1)) - 1
@@ -175,7 +175,7 @@ def test_fp8_partial_window_full_size(kvq, oracle_mod, dev):
     run_fp8(kvq, oracle_mod, v, 4, 1024, 2048, dev)
 
 
-@pytest.mark.parametrize("wbits", [4, 6])
+@pytest.mark.parametrize("wbits", [4, 6, 8])
 def test_channel_outliers_reduced(kvq, oracle_mod, dev, wbits):
     """Channel-outlier K, N(0, 0.5) V, 2% zero blocks, at [2, 512, 8, 128] (every tile
     boundary and a ragged window), full comparison."""
@@ -184,7 +184,7 @@ def test_channel_outliers_reduced(kvq, oracle_mod, dev, wbits):
     run_q(kvq, oracle_mod, k, v, wbits, 2, 37, 301, dev)
 
 
-@pytest.mark.parametrize("wbits", [4, 6])
+@pytest.mark.parametrize("wbits", [4, 6, 8])
 def test_channel_outliers_full_size_sampled(kvq, oracle_mod, dev, wbits):
     """[16, 8192, 8, 128] on the device; 3000 sampled positions checked against the oracle
     one position at a time."""
@@ -222,7 +222,7 @@ def test_paged_decode_prefill_full_pool(kvq, oracle_mod, dev, phase):
           seqlens=pool.cache_seqlens, bt=pool.block_table)
 
 
-@pytest.mark.parametrize("wbits", [4, 6])
+@pytest.mark.parametrize("wbits", [4, 6, 8])
 def test_model_layer_paged_q6_sampled(kvq, oracle_mod, dev, wbits):
     """One 8 x 32768-position layer (1024 pages), full-window dequantize then quantize,
     sampled rows against the oracle; the round trip of a quantized cache is a fixed point."""
@@ -250,7 +250,7 @@ def test_model_layer_paged_q6_sampled(kvq, oracle_mod, dev, wbits):
 # -------------------------------------------------------------- edge cases ----
 
 @pytest.mark.parametrize("shape", [(2, 40, 1, 32), (3, 17, 3, 96), (1, 9, 5, 64), (2, 5, 32, 512)])
-@pytest.mark.parametrize("wbits", [4, 6])
+@pytest.mark.parametrize("wbits", [4, 6, 8])
 def test_ragged_shapes(kvq, oracle_mod, dev, shape, wbits):
     k, v = workloads.channel_outliers(shape=shape)
     B, S = shape[0], shape[1]
@@ -279,7 +279,7 @@ def test_empty_windows_write_nothing(kvq, dev):
 
 
 @pytest.mark.parametrize("ps", [16, 24, 7, 256])
-@pytest.mark.parametrize("wbits", [4, 6])
+@pytest.mark.parametrize("wbits", [4, 6, 8])
 def test_paged_identity_equals_contiguous(kvq, oracle_mod, dev, ps, wbits):
     B, H, D = 3, 2, 64
     S = ps * 6
@@ -300,7 +300,7 @@ def test_paged_windows_small_pool(kvq, oracle_mod, dev, offset, width):
     ps, H, D, npages, batch = 16, 2, 32, 40, 5
     lens, bt = workloads.paged_tables(3, batch, 60, npages, ps)
     k, v = workloads.small(shape=(npages, ps, H, D))
-    for wbits in (4, 6):
+    for wbits in (4, 6, 8):
         run_q(kvq, oracle_mod, k, v, wbits, batch, offset, width, dev, page_size=ps, seqlens=lens, bt=bt)
 
 
@@ -335,7 +335,7 @@ def test_runs_on_a_side_stream(kvq, oracle_mod, dev):
         run_q(kvq, oracle_mod, k, v, 6, 2, 0, 64, dev)
 
 
-@pytest.mark.parametrize("wbits", [4, 6])
+@pytest.mark.parametrize("wbits", [4, 6, 8])
 def test_paged_wide_block_table(kvq, oracle_mod, dev, wbits):
     """A block table wider than a CTA (300 pages per sequence) takes the unstaged lookup."""
     ps, H, D, batch = 2, 1, 32, 2

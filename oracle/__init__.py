@@ -51,6 +51,10 @@ def lib() -> ctypes.CDLL:
         L.kvqref_fp8_to_fp16_kv.argtypes = [u8p, u16p, u8p, u16p] + [I] * 8 + [i32p, i32p, I]
         L.kvqref_fp16_to_q_kv.argtypes = [u16p, u8p, u16p, u16p, u8p, u16p] + [I] * 8 + [i32p, i32p, I, I]
         L.kvqref_q_to_fp16_kv.argtypes = [u8p, u16p, u16p, u8p, u16p, u16p] + [I] * 8 + [i32p, i32p, I, I]
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        LL = ctypes.c_longlong
+        L.kvqref_count_match.argtypes = [i64p, LL, i64p, LL, LL]
+        L.kvqref_count_match.restype = LL
         for name in ("kvqref_quantize_row", "kvqref_dequantize_row", "kvqref_pack_row",
                      "kvqref_unpack_row", "kvqref_fp16_to_fp8", "kvqref_fp8_to_fp16",
                      "kvqref_fp16_to_q_kv", "kvqref_q_to_fp16_kv", "kvqref_fp16_to_fp8_kv",
@@ -225,3 +229,10 @@ def q_to_fp16_kv(k_in, k_out, k_scales, v_in, v_out, v_scales, batch_size, offse
         _p(np.ascontiguousarray(_bits(v_scales)), ctypes.c_uint16),
         d0, d1, H, D, batch_size, offset, width, page_size,
         _p(sl, ctypes.c_int32), _p(bt, ctypes.c_int32), stride, wbits)
+
+
+def count_match(a: np.ndarray, b: np.ndarray, max_a: int) -> int:
+    """Common-prefix length of two int64 sequences, capped at max_a."""
+    a = np.ascontiguousarray(a, np.int64)
+    b = np.ascontiguousarray(b, np.int64)
+    return lib().kvqref_count_match(_p(a, ctypes.c_int64), a.size, _p(b, ctypes.c_int64), b.size, int(max_a))

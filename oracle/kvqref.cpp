@@ -406,4 +406,15 @@ int kvqref_q_to_fp16_kv(const uint8_t* k_in, uint16_t* k_out, const uint16_t* k_
   return st_k != KVQREF_OK ? st_k : st_v;
 }
 
+// Description, count_match: compare element by element from the start and
+// stop at the first difference, at the end of either sequence, or at max_a.
+long long kvqref_count_match(const int64_t* a, long long a_len, const int64_t* b, long long b_len,
+                             long long max_a) {
+  long long n = a_len < b_len ? a_len : b_len;
+  if (max_a < n) n = max_a;
+  long long i = 0;
+  while (i < n && a[i] == b[i]) ++i;
+  return i < 0 ? 0 : i;
+}
+
 }  // extern "C"

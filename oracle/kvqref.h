@@ -122,6 +122,11 @@ int kvqref_q_to_fp16_kv(const uint8_t* k_in, uint16_t* k_out, const uint16_t* k_
                         int page_size, const int32_t* cache_seqlens,
                         const int32_t* block_table, int bt_stride, int wbits);
 
+/* count_match (Description; I/O Contract): length of the common prefix of two
+ * 64-bit element sequences, looking at no more than max_a elements. */
+long long kvqref_count_match(const int64_t* a, long long a_len, const int64_t* b, long long b_len,
+                             long long max_a);
+
 #ifdef __cplusplus
 }
 #endif

@@ -166,6 +166,14 @@ KVQ_API kvq_status kvq_q_to_fp16_kv(const void* k_in, void* k_out, const void* k
                             int page_size, const int32_t* cache_seqlens,
                             const int32_t* block_table, int wbits, void* stream);
 
+/* count_match (Description; I/O Contract): the number of leading elements on
+ * which the 64-bit sequences a[0..a_len) and b[0..b_len) agree, comparing no
+ * more than max_a elements (max_a <= 0 gives 0).  Host function: a and b are
+ * host pointers, read only; nothing is enqueued on any device.  Returns -1
+ * when a pointer is NULL and there is something to compare. */
+KVQ_API long long kvq_count_match(const int64_t* a, long long a_len, const int64_t* b, long long b_len,
+                                  long long max_a);
+
 /* Human-readable name of a status (static storage; never NULL). */
 KVQ_API const char* kvq_status_string(kvq_status status);
 

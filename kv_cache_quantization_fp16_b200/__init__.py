@@ -26,7 +26,7 @@ import os
 import torch
 
 __all__ = ["fp16_to_fp8", "fp8_to_fp16", "fp16_to_fp8_kv", "fp8_to_fp16_kv", "fp16_to_q_kv", "q_to_fp16_kv", "poll_device_error",
-           "selfcheck_code_rounding", "q_shapes", "set_engine", "get_engine", "engine", "KVQError",
+           "selfcheck_code_rounding", "count_match", "q_shapes", "set_engine", "get_engine", "engine", "KVQError",
            "LIB_PATH", "library"]
 
 ENGINES = {"auto": 0, "ldg": 1, "bulk": 2}
@@ -68,6 +68,9 @@ def _load() -> ctypes.CDLL:
     L.kvq_status_string.restype = ctypes.c_char_p
     L.kvq_poll_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), vp]
     L.kvq_selfcheck_code_rounding.argtypes = [I, vp, vp]
+    LL = ctypes.c_longlong
+    L.kvq_count_match.argtypes = [vp, LL, vp, LL, LL]
+    L.kvq_count_match.restype = LL
     L.kvq_set_engine.argtypes = [I]
     L.kvq_get_engine.argtypes = []
     L.kvq_get_engine.restype = I
@@ -283,3 +286,18 @@ class engine:
     def __exit__(self, *exc):
         set_engine(self.prev)
         return False
+
+
+def count_match(a: torch.Tensor, b: torch.Tensor, max_a: int) -> int:
+    """Length of the matching prefix of two 1-D int64 CPU tensors (e.g. token ids),
+    comparing at most max_a elements (page Description: count_match)."""
+    for t, n in ((a, "a"), (b, "b")):
+        _require(isinstance(t, torch.Tensor) and t.dtype == torch.int64 and t.dim() == 1,
+                 f"{n} must be a 1-D int64 tensor")
+        _require(t.device.type == "cpu", f"{n} must be a CPU tensor")
+    a, b = a.contiguous(), b.contiguous()
+    n = _lib.kvq_count_match(a.data_ptr() if a.numel() else None, a.numel(),
+                             b.data_ptr() if b.numel() else None, b.numel(), int(max_a))
+    if n < 0:
+        raise KVQError(1, "count_match")
+    return int(n)

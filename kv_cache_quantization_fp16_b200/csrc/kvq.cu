@@ -395,6 +395,16 @@ kvq_status kvq_poll_device_error(int32_t* code_out, void* stream) {
   return h ? KVQ_ERR_DEVICE : KVQ_OK;
 }
 
+long long kvq_count_match(const int64_t* a, long long a_len, const int64_t* b, long long b_len, long long max_a) {
+  long long n = a_len < b_len ? a_len : b_len;
+  if (max_a < n) n = max_a;
+  if (n <= 0) return 0;
+  if (!a || !b) return -1;
+  long long i = 0;
+  while (i < n && a[i] == b[i]) ++i;
+  return i;
+}
+
 kvq_status kvq_set_engine(int engine) {
   if (engine != KVQ_ENGINE_AUTO && engine != KVQ_ENGINE_LDG && engine != KVQ_ENGINE_BULK) return KVQ_ERR_RANGE;
   g_engine.store(engine);

@@ -51,6 +51,10 @@ def lib() -> ctypes.CDLL:
         L.kvqref_fp8_to_fp16_kv.argtypes = [u8p, u16p, u8p, u16p] + [I] * 8 + [i32p, i32p, I]
         L.kvqref_fp16_to_q_kv.argtypes = [u16p, u8p, u16p, u16p, u8p, u16p] + [I] * 8 + [i32p, i32p, I, I]
         L.kvqref_q_to_fp16_kv.argtypes = [u8p, u16p, u16p, u8p, u16p, u16p] + [I] * 8 + [i32p, i32p, I, I]
+        f64p = ctypes.POINTER(ctypes.c_double)
+        L.kvqref_decode_attention_q.argtypes = [u16p, u8p, u16p, u8p, u16p, u16p, f64p] + [I] * 7 + \
+            [i32p, i32p, I, I, ctypes.c_double]
+        L.kvqref_decode_attention_q.restype = ctypes.c_int
         i64p = ctypes.POINTER(ctypes.c_int64)
         LL = ctypes.c_longlong
         L.kvqref_count_match.argtypes = [i64p, LL, i64p, LL, LL]
@@ -236,3 +240,28 @@ def count_match(a: np.ndarray, b: np.ndarray, max_a: int) -> int:
     a = np.ascontiguousarray(a, np.int64)
     b = np.ascontiguousarray(b, np.int64)
     return lib().kvqref_count_match(_p(a, ctypes.c_int64), a.size, _p(b, ctypes.c_int64), b.size, int(max_a))
+
+
+def decode_attention_q(q, k_codes, k_scales, v_codes, v_scales, batch_size, n_heads, page_size,
+                       cache_seqlens, block_table, wbits, softmax_scale, head_dim):
+    """fp64 decode attention over the dequantized cache.  q: [batch, n_heads, D] float16/uint16;
+    codes [d0, d1, H, D*wbits/8] uint8; scales [d0, d1, H, D/32].  Returns (status, out uint16
+    [batch, n_heads, D], exact float64 [batch, n_heads, D])."""
+    d0, d1, H, _ = k_codes.shape
+    qb = np.ascontiguousarray(_bits(q))
+    out = np.zeros((batch_size, n_heads, head_dim), np.uint16)
+    ex = np.zeros((batch_size, n_heads, head_dim), np.float64)
+    sl = np.ascontiguousarray(cache_seqlens, np.int32)
+    if page_size:
+        bt = np.ascontiguousarray(block_table, np.int32)
+        stride = bt.shape[1]
+    else:
+        bt, stride = None, 0
+    st = lib().kvqref_decode_attention_q(
+        _p(qb, ctypes.c_uint16), _p(np.ascontiguousarray(k_codes, np.uint8), ctypes.c_uint8),
+        _p(np.ascontiguousarray(_bits(k_scales)), ctypes.c_uint16),
+        _p(np.ascontiguousarray(v_codes, np.uint8), ctypes.c_uint8),
+        _p(np.ascontiguousarray(_bits(v_scales)), ctypes.c_uint16), _p(out, ctypes.c_uint16),
+        _p(ex, ctypes.c_double), d0, d1, H, head_dim, batch_size, n_heads, page_size,
+        _p(sl, ctypes.c_int32), _p(bt, ctypes.c_int32), stride, wbits, float(softmax_scale))
+    return st, out, ex

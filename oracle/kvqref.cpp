@@ -406,6 +406,82 @@ int kvqref_q_to_fp16_kv(const uint8_t* k_in, uint16_t* k_out, const uint16_t* k_
   return st_k != KVQREF_OK ? st_k : st_v;
 }
 
+// Usage ("convert KV tensors during the attention forward pass"): attention of
+// one new query per sequence over the dequantized cache, in double precision,
+// one position at a time.
+int kvqref_decode_attention_q(const uint16_t* q, const uint8_t* k_codes, const uint16_t* k_scales,
+                              const uint8_t* v_codes, const uint16_t* v_scales, uint16_t* out,
+                              double* out_exact, int dim0, int dim1, int heads, int head_dim,
+                              int batch_size, int n_heads, int page_size, const int32_t* cache_seqlens,
+                              const int32_t* block_table, int bt_stride, int wbits, double softmax_scale) {
+  if (!valid_wbits(wbits) || heads <= 0 || head_dim <= 0 || head_dim % kBlock || head_dim > 65536) return KVQREF_BAD_ARG;
+  if (n_heads <= 0 || n_heads % heads || batch_size < 0 || dim0 < 0 || dim1 < 0 || !cache_seqlens) return KVQREF_BAD_ARG;
+  if (page_size < 0 || (page_size > 0 && (dim1 != page_size || !block_table))) return KVQREF_BAD_ARG;
+  if (page_size == 0 && batch_size > dim0) return KVQREF_BAD_ARG;
+  const int group = n_heads / heads;
+  const long code_bytes = static_cast<long>(head_dim) * wbits / 8;
+  const long nscales = head_dim / kBlock;
+  int status = KVQREF_OK;
+  uint8_t codes[65536];
+  uint16_t deq[65536];
+  for (int i = 0; i < batch_size; ++i) {
+    const long L = cache_seqlens[i] < 0 ? 0 : cache_seqlens[i];
+    if (page_size == 0 && L > dim1) return KVQREF_BAD_ARG;
+    for (int h = 0; h < n_heads; ++h) {
+      const int kvh = h / group;
+      const uint16_t* qh = q + (static_cast<long>(i) * n_heads + h) * head_dim;
+      // pass 1: scores
+      double* s = new double[L > 0 ? L : 1];
+      long n_valid = 0;
+      long* rows = new long[L > 0 ? L : 1];
+      for (long p = 0; p < L; ++p) {
+        long row;
+        if (page_size == 0) {
+          row = static_cast<long>(i) * dim1 + p;
+        } else {
+          const long lp = p / page_size;
+          const int32_t page = lp < bt_stride ? block_table[static_cast<long>(i) * bt_stride + lp] : -1;
+          if (lp >= bt_stride || page < 0 || page >= dim0) {
+            status = KVQREF_BAD_PAGE;
+            continue;
+          }
+          row = static_cast<long>(page) * page_size + p % page_size;
+        }
+        const long hr = row * heads + kvh;
+        unpack_row(k_codes + hr * code_bytes, head_dim, wbits, codes);
+        dequantize_row(codes, k_scales + hr * nscales, head_dim, wbits, deq);
+        double dot = 0.0;
+        for (int d = 0; d < head_dim; ++d) dot += half_to_double(qh[d]) * half_to_double(deq[d]);
+        s[n_valid] = softmax_scale * dot;
+        rows[n_valid] = hr;
+        ++n_valid;
+      }
+      double m = -INFINITY;
+      for (long j = 0; j < n_valid; ++j) m = s[j] > m ? s[j] : m;
+      double denom = 0.0;
+      for (long j = 0; j < n_valid; ++j) denom += std::exp(s[j] - m);
+      // pass 2: weighted values
+      double* acc = new double[head_dim];
+      for (int d = 0; d < head_dim; ++d) acc[d] = 0.0;
+      for (long j = 0; j < n_valid; ++j) {
+        const double w = std::exp(s[j] - m) / denom;
+        unpack_row(v_codes + rows[j] * code_bytes, head_dim, wbits, codes);
+        dequantize_row(codes, v_scales + rows[j] * nscales, head_dim, wbits, deq);
+        for (int d = 0; d < head_dim; ++d) acc[d] += w * half_to_double(deq[d]);
+      }
+      uint16_t* oh = out + (static_cast<long>(i) * n_heads + h) * head_dim;
+      for (int d = 0; d < head_dim; ++d) {
+        oh[d] = double_to_half(acc[d]);
+        if (out_exact) out_exact[(static_cast<long>(i) * n_heads + h) * head_dim + d] = acc[d];
+      }
+      delete[] acc;
+      delete[] rows;
+      delete[] s;
+    }
+  }
+  return status;
+}
+
 // Description, count_match: compare element by element from the start and
 // stop at the first difference, at the end of either sequence, or at max_a.
 long long kvqref_count_match(const int64_t* a, long long a_len, const int64_t* b, long long b_len,

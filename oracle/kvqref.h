@@ -122,6 +122,22 @@ int kvqref_q_to_fp16_kv(const uint8_t* k_in, uint16_t* k_out, const uint16_t* k_
                         int page_size, const int32_t* cache_seqlens,
                         const int32_t* block_table, int bt_stride, int wbits);
 
+/* Decode attention over a quantized cache: for every sequence i < batch_size
+ * and query head h < n_heads (GQA: kv head h / (n_heads / heads)), attend the
+ * single query q[i, h, :] to logical positions [0, cache_seqlens[i]) of the
+ * cache, whose keys and values are the dequantized codes (exactly what
+ * kvqref_q_to_fp16_kv produces).  In double precision:
+ *   s_p = softmax_scale * sum_d q_d * k_{p,d};  w_p = exp(s_p - max_p s_p);
+ *   o = sum_p w_p * v_p / sum_p w_p;   out = RN16(o)   (0 when the window is empty).
+ * q, out: [batch_size, n_heads, head_dim] binary16.  out_exact (optional,
+ * may be NULL) receives o before rounding.  Paged / contiguous addressing as
+ * in kvqref_q_to_fp16_kv.  Returns KVQREF_BAD_ARG / KVQREF_BAD_PAGE like it. */
+int kvqref_decode_attention_q(const uint16_t* q, const uint8_t* k_codes, const uint16_t* k_scales,
+                              const uint8_t* v_codes, const uint16_t* v_scales, uint16_t* out,
+                              double* out_exact, int dim0, int dim1, int heads, int head_dim,
+                              int batch_size, int n_heads, int page_size, const int32_t* cache_seqlens,
+                              const int32_t* block_table, int bt_stride, int wbits, double softmax_scale);
+
 /* count_match (Description; I/O Contract): length of the common prefix of two
  * 64-bit element sequences, looking at no more than max_a elements. */
 long long kvqref_count_match(const int64_t* a, long long a_len, const int64_t* b, long long b_len,

@@ -66,6 +66,7 @@
 #ifndef KVQ_H
 #define KVQ_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #if defined(__GNUC__)
@@ -165,6 +166,41 @@ KVQ_API kvq_status kvq_q_to_fp16_kv(const void* k_in, void* k_out, const void* k
                             const kvq_cache_desc* desc, int batch_size, int offset, int width,
                             int page_size, const int32_t* cache_seqlens,
                             const int32_t* block_table, int wbits, void* stream);
+
+/* Decode attention over a quantized KV cache (the conversions' consumer: the
+ * page's Usage section converts the cache "during the attention forward
+ * pass"; this reads the Q4/Q6/Q8 codes directly, so no FP16 cache is written).
+ * For every sequence i < batch_size and query head h < n_heads (GQA: kv head
+ * h / (n_heads / kv_heads)), the query q[i, h, :] attends to logical
+ * positions [0, cache_seqlens[i]) of the cache, keys and values being
+ * exactly what kvq_q_to_fp16_kv would produce:
+ *   out[i, h, :] = sum_p softmax_p(softmax_scale * q . k_p) * v_p   (binary16),
+ * 0 for an empty window.  Arithmetic: fp16 products with fp32 accumulation
+ * (tensor cores), base-2 online softmax in fp32; tests bound the difference
+ * to the fp64 result by one binary16 ulp plus 2^-14 of the largest |v|.
+ *   q, out     [batch_size, n_heads, head_dim] binary16, 16-byte aligned
+ *   k/v codes  [dim0, dim1, kv_heads, head_dim * wbits / 8] uint8
+ *   k/v scales [dim0, dim1, kv_heads, head_dim / 32] binary16
+ *   page_size == 0: contiguous (dim1 = max positions, cache_seqlens[i] <=
+ *   dim1); page_size > 0: paged as in kvq_fp16_to_q_kv.  head_dim is 64, 128
+ *   or 256; n_heads / kv_heads <= 8; wbits 4, 6 or 8.
+ *   workspace: caller-owned device memory of at least
+ *   kvq_decode_attention_workspace_size(...) bytes (per-chunk partial
+ *   results), 16-byte aligned; its contents on entry do not matter.
+ * Two kernels are enqueued on `stream`.  A window longer than the cache, or
+ * paging metadata pointing outside it, skips those positions and sets the
+ * device error word. */
+KVQ_API kvq_status kvq_decode_attention_q(const void* q, const void* k_codes, const void* k_scales,
+                                          const void* v_codes, const void* v_scales, void* out,
+                                          const kvq_cache_desc* desc, int batch_size, int n_heads, int page_size,
+                                          const int32_t* cache_seqlens, const int32_t* block_table, int wbits,
+                                          float softmax_scale, void* workspace, size_t workspace_bytes,
+                                          void* stream);
+
+/* Workspace bytes kvq_decode_attention_q needs for this geometry (0 for bad
+ * arguments).  Host-only. */
+KVQ_API size_t kvq_decode_attention_workspace_size(const kvq_cache_desc* desc, int batch_size, int n_heads,
+                                                   int page_size);
 
 /* count_match (Description; I/O Contract): the number of leading elements on
  * which the 64-bit sequences a[0..a_len) and b[0..b_len) agree, comparing no

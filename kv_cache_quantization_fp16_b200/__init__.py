@@ -26,7 +26,7 @@ import os
 import torch
 
 __all__ = ["fp16_to_fp8", "fp8_to_fp16", "fp16_to_fp8_kv", "fp8_to_fp16_kv", "fp16_to_q_kv", "q_to_fp16_kv", "poll_device_error",
-           "selfcheck_code_rounding", "count_match", "q_shapes", "set_engine", "get_engine", "engine", "KVQError",
+           "selfcheck_code_rounding", "count_match", "decode_attention_q", "attention_workspace_bytes", "q_shapes", "set_engine", "get_engine", "engine", "KVQError",
            "LIB_PATH", "library"]
 
 ENGINES = {"auto": 0, "ldg": 1, "bulk": 2}
@@ -69,6 +69,11 @@ def _load() -> ctypes.CDLL:
     L.kvq_poll_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), vp]
     L.kvq_selfcheck_code_rounding.argtypes = [I, vp, vp]
     LL = ctypes.c_longlong
+    L.kvq_decode_attention_q.argtypes = [vp, vp, vp, vp, vp, vp, dp, I, I, I, vp, vp, I, ctypes.c_float, vp,
+                                         ctypes.c_size_t, vp]
+    L.kvq_decode_attention_q.restype = I
+    L.kvq_decode_attention_workspace_size.argtypes = [dp, I, I, I]
+    L.kvq_decode_attention_workspace_size.restype = ctypes.c_size_t
     L.kvq_count_match.argtypes = [vp, LL, vp, LL, LL]
     L.kvq_count_match.restype = LL
     L.kvq_set_engine.argtypes = [I]
@@ -301,3 +306,61 @@ def count_match(a: torch.Tensor, b: torch.Tensor, max_a: int) -> int:
     if n < 0:
         raise KVQError(1, "count_match")
     return int(n)
+
+
+def attention_workspace_bytes(cache_shape, batch_size: int, n_heads: int, page_size: int = 0,
+                              block_table_stride: int = 0) -> int:
+    """Workspace bytes decode_attention_q needs: cache_shape is the FP16 cache shape
+    [d0, d1, kv_heads, head_dim] the codes were made from."""
+    d0, d1, H, D = cache_shape
+    desc = _Desc(d0, d1, H, D, block_table_stride if page_size else 0)
+    return int(_lib.kvq_decode_attention_workspace_size(ctypes.byref(desc), int(batch_size), int(n_heads),
+                                                        int(page_size)))
+
+
+def decode_attention_q(q, k_codes, k_scales, v_codes, v_scales, out, batch_size, cache_seqlens, wbits,
+                       softmax_scale, page_size=0, block_table=None, workspace=None) -> None:
+    """Decode attention reading the quantized cache directly (no FP16 cache is written).
+
+    q, out: [batch, n_heads, head_dim] float16 CUDA tensors; codes / scales as written by
+    fp16_to_q_kv ([d0, d1, kv_heads, head_dim * wbits / 8] uint8, [d0, d1, kv_heads,
+    head_dim / 32] float16); cache_seqlens [batch] int32 (positions [0, len) are attended);
+    paged mode with page_size > 0 and block_table.  ``workspace`` is a CUDA uint8 tensor of at
+    least attention_workspace_bytes(...) bytes; when omitted one is allocated with torch."""
+    _require(isinstance(q, torch.Tensor) and q.dtype == torch.float16 and q.is_cuda and q.dim() == 3
+             and q.is_contiguous(), "q must be a contiguous [batch, n_heads, head_dim] float16 CUDA tensor")
+    _require(out.shape == q.shape and out.dtype == torch.float16 and out.is_contiguous() and out.device == q.device,
+             "out must match q")
+    for t, n in ((k_codes, "k_codes"), (v_codes, "v_codes")):
+        _cuda4(t, torch.uint8, n)
+    for t, n in ((k_scales, "k_scales"), (v_scales, "v_scales")):
+        _cuda4(t, torch.float16, n)
+    _require(wbits in (4, 6, 8), f"wbits must be 4, 6 or 8, got {wbits}")
+    D = q.shape[2]
+    cshape, sshape = q_shapes((*k_codes.shape[:3], D), wbits)
+    for t, n in ((k_codes, "k_codes"), (v_codes, "v_codes")):
+        _require(tuple(t.shape) == cshape, f"{n} must have shape {cshape}, got {tuple(t.shape)}")
+    for t, n in ((k_scales, "k_scales"), (v_scales, "v_scales")):
+        _require(tuple(t.shape) == sshape, f"{n} must have shape {sshape}, got {tuple(t.shape)}")
+    dev = q.device
+    for t in (k_codes, k_scales, v_codes, v_scales):
+        _require(t.device == dev, "tensors must be on one device")
+    _require(cache_seqlens is not None and cache_seqlens.dtype == torch.int32 and cache_seqlens.device == dev
+             and cache_seqlens.is_contiguous() and cache_seqlens.numel() >= batch_size,
+             "cache_seqlens must be a contiguous int32 tensor on the caches' device with batch_size entries")
+    stride, _, bt_ptr = _paging(page_size, cache_seqlens, block_table, batch_size, dev)
+    d0, d1, H, _ = k_codes.shape
+    desc = _Desc(d0, d1, H, D, stride)
+    n_heads = q.shape[1]
+    need = int(_lib.kvq_decode_attention_workspace_size(ctypes.byref(desc), int(batch_size), int(n_heads),
+                                                        int(page_size)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _require(workspace.is_cuda and workspace.device == dev and workspace.numel() >= need,
+             f"workspace must hold at least {need} bytes on the caches' device")
+    with torch.cuda.device(dev):
+        st = _lib.kvq_decode_attention_q(q.data_ptr(), k_codes.data_ptr(), k_scales.data_ptr(), v_codes.data_ptr(),
+                                         v_scales.data_ptr(), out.data_ptr(), ctypes.byref(desc), int(batch_size),
+                                         int(n_heads), int(page_size), cache_seqlens.data_ptr(), bt_ptr, int(wbits),
+                                         float(softmax_scale), workspace.data_ptr(), workspace.numel(), _stream(dev))
+    _check(st, "decode_attention_q")

@@ -24,6 +24,7 @@
 #include <atomic>
 
 #include "../../include/kvq.h"
+#include "attention.cuh"
 #include "bulk_engine.cuh"
 #include "codec.cuh"
 #include "ldg_engine.cuh"
@@ -393,6 +394,100 @@ kvq_status kvq_poll_device_error(int32_t* code_out, void* stream) {
   if (cudaStreamSynchronize(s) != cudaSuccess) return KVQ_ERR_CUDA;
   *code_out = h;
   return h ? KVQ_ERR_DEVICE : KVQ_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+// Chunks of kAttnChunk positions a sequence can have: the longest window the
+// cache geometry allows.
+long long attn_max_chunks(const kvq_cache_desc* d, int page_size) {
+  const long long max_len = page_size > 0 ? static_cast<long long>(d->block_table_stride) * page_size
+                                          : static_cast<long long>(d->dim1);
+  return (max_len + kvq::kAttnChunk - 1) / kvq::kAttnChunk;
+}
+
+template <int B, int D>
+kvq_status launch_attention(const kvq::AttnParams& a, void* stream) {
+  kvq_status st = launch_pdl(kvq::attn_partial_kernel<B, D>, dim3(a.max_chunks, a.kv_heads, a.batch),
+                             kvq::kAttnThreads, 0, stream, a);
+  if (st != KVQ_OK) return st;
+  return launch_pdl(kvq::attn_combine_kernel<D>, dim3(a.n_heads, a.batch), D, 0, stream, a);
+}
+
+template <int B>
+kvq_status launch_attention_b(const kvq::AttnParams& a, int head_dim, void* stream) {
+  if (head_dim == 64) return launch_attention<B, 64>(a, stream);
+  if (head_dim == 128) return launch_attention<B, 128>(a, stream);
+  return launch_attention<B, 256>(a, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kvq_decode_attention_workspace_size(const kvq_cache_desc* desc, int batch_size, int n_heads,
+                                           int page_size) {
+  if (!desc || batch_size < 0 || n_heads < 0 || page_size < 0) return 0;
+  return static_cast<size_t>(batch_size) * n_heads * attn_max_chunks(desc, page_size) * (desc->head_dim + 2) *
+         sizeof(float);
+}
+
+kvq_status kvq_decode_attention_q(const void* q, const void* k_codes, const void* k_scales, const void* v_codes,
+                                  const void* v_scales, void* out, const kvq_cache_desc* desc, int batch_size,
+                                  int n_heads, int page_size, const int32_t* cache_seqlens,
+                                  const int32_t* block_table, int wbits, float softmax_scale, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  if (!q || !k_codes || !k_scales || !v_codes || !v_scales || !out || !desc || !cache_seqlens) return KVQ_ERR_NULL;
+  if (wbits != 4 && wbits != 6 && wbits != 8) return KVQ_ERR_WBITS;
+  kvq_status st = check_desc(desc, 32);
+  if (st != KVQ_OK) return st;
+  const int D = desc->head_dim;
+  if (D != 64 && D != 128 && D != 256) return KVQ_ERR_SHAPE;
+  if (n_heads < 1 || n_heads % desc->kv_heads || n_heads / desc->kv_heads > kvq::kAttnMaxGroup) return KVQ_ERR_SHAPE;
+  if (batch_size < 0 || batch_size > 65535 || desc->kv_heads > 65535 || n_heads > 0x7FFFFFFF) return KVQ_ERR_RANGE;
+  if (page_size < 0) return KVQ_ERR_RANGE;
+  if (page_size == 0) {
+    if (batch_size > desc->dim0) return KVQ_ERR_RANGE;
+  } else {
+    if (!block_table) return KVQ_ERR_NULL;
+    if (page_size != desc->dim1 || desc->block_table_stride < 1) return KVQ_ERR_RANGE;
+  }
+  const void* ptrs[7] = {q, k_codes, k_scales, v_codes, v_scales, out, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return KVQ_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(cache_seqlens) | reinterpret_cast<uintptr_t>(block_table)) & 3u)
+    return KVQ_ERR_ALIGN;
+  if (batch_size == 0) return KVQ_OK;
+  const long long max_chunks = attn_max_chunks(desc, page_size);
+  if (max_chunks < 1 || max_chunks > 0x7FFFFFFFLL) return KVQ_ERR_RANGE;
+  if (!workspace) return KVQ_ERR_NULL;
+  if (workspace_bytes < kvq_decode_attention_workspace_size(desc, batch_size, n_heads, page_size))
+    return KVQ_ERR_RANGE;
+  kvq::AttnParams a{};
+  a.q = static_cast<const __half*>(q);
+  a.k_codes = static_cast<const uint8_t*>(k_codes);
+  a.k_scales = static_cast<const __half*>(k_scales);
+  a.v_codes = static_cast<const uint8_t*>(v_codes);
+  a.v_scales = static_cast<const __half*>(v_scales);
+  a.out = static_cast<__half*>(out);
+  a.ws = static_cast<float*>(workspace);
+  a.seqlens = cache_seqlens;
+  a.block_table = block_table;
+  a.dim0 = desc->dim0;
+  a.dim1 = desc->dim1;
+  a.kv_heads = desc->kv_heads;
+  a.batch = batch_size;
+  a.n_heads = n_heads;
+  a.group = n_heads / desc->kv_heads;
+  a.page_size = page_size;
+  a.bt_stride = desc->block_table_stride;
+  a.max_chunks = static_cast<int>(max_chunks);
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  if (wbits == 4) return launch_attention_b<4>(a, D, stream);
+  if (wbits == 6) return launch_attention_b<6>(a, D, stream);
+  return launch_attention_b<8>(a, D, stream);
 }
 
 long long kvq_count_match(const int64_t* a, long long a_len, const int64_t* b, long long b_len, long long max_a) {

@@ -133,3 +133,32 @@ def test_fp8_kv_validation(kvq):
     assert L.kvq_fp16_to_fp8_kv(*P, by(dp), 2, 0, 16, 8, FAKE, FAKE, None) == 4
     assert L.kvq_fp8_to_fp16_kv(*P, by(dp), 2, -3, 0, 16, FAKE, FAKE, None) == 0   # empty window
     assert L.kvq_set_engine(9) == 4 and L.kvq_get_engine() == 0
+
+
+def test_decode_attention_validation(kvq):
+    L = kvq.library()
+    by = ctypes.byref
+    d = _desc(kvq, d0=2, d1=16, H=2, D=64)
+    P = [FAKE] * 6  # q, k_codes, k_scales, v_codes, v_scales, out
+    ws = kvq.attention_workspace_bytes((2, 16, 2, 64), 2, 4)
+    assert ws == L.kvq_decode_attention_workspace_size(by(d), 2, 4, 0) > 0
+
+    def call(*args, desc=d, bs=2, nh=4, ps=0, lens=FAKE, bt=None, wbits=4, wsp=FAKE, wsb=ws):
+        return L.kvq_decode_attention_q(*(args or P), by(desc) if desc else None, bs, nh, ps, lens, bt, wbits,
+                                        ctypes.c_float(0.125), wsp, wsb, None)
+
+    assert call(None, *P[1:]) == 1
+    assert call(lens=None) == 1
+    assert call(wsp=None) == 1                          # workspace needed for a non-empty batch
+    assert call(wbits=5) == 3
+    assert call(desc=_desc(kvq, D=96)) == 2             # head_dim 64, 128 or 256
+    assert call(nh=3) == 2                              # query heads must split over the kv heads
+    assert call(nh=18) == 2                             # at most 8 query heads per kv head
+    assert call(bs=3) == 4                              # batch > dim0 (contiguous)
+    assert call(wsb=ws - 1) == 4                        # workspace too small
+    assert call(P[0] + 8, *P[1:]) == 5
+    assert call(lens=FAKE + 2) == 5
+    dp = _desc(kvq, d0=10, d1=16, H=2, D=64, stride=4)
+    assert call(desc=dp, ps=16) == 1                    # paged needs a block table
+    assert call(desc=dp, ps=8, bt=FAKE) == 4            # page_size must equal dim1
+    assert call(bs=0, wsp=None, wsb=0) == 0             # empty batch enqueues nothing

@@ -1,0 +1,150 @@
+"""Decode attention reading the quantized cache (the conversions' consumer) against
+the CPU oracle's fp64 attention over the dequantized cache.
+
+Tolerance, from the arithmetic: products q_d * k_d are exact (binary16 x
+binary16 in fp32), dot products and sums accumulate in fp32 (relative error a
+few 2^-24 per term), softmax weights carry ~22 bits (binary16 high part +
+binary16 residual) and exp2f is within 2 ulp; the fp32 result before the final
+RN16 is within ~1e-5 of the largest |v| of the exact value, so the binary16
+output is within one binary16 ulp of the exact value plus 2^-14 max|v|
+(a margin for cancellation when the result is near 0).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kvq():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import kv_cache_quantization_fp16_b200 as m
+
+    return m
+
+
+@pytest.fixture(scope="module")
+def dev(kvq):
+    return torch.device("cuda:0")
+
+
+def u16(t):
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def quantize_on_gpu(kvq, k, v, wbits, dev):
+    cs, ss = kvq.q_shapes(tuple(k.shape), wbits)
+    kc = torch.zeros(cs, dtype=torch.uint8, device=dev)
+    vc = torch.zeros_like(kc)
+    ks = torch.zeros(ss, dtype=torch.float16, device=dev)
+    vs = torch.zeros_like(ks)
+    d0, d1 = k.shape[:2]
+    kvq.fp16_to_q_kv(k.to(dev), kc, ks, v.to(dev), vc, vs, d0, 0, d1, 0, None, None, wbits)
+    return kc, ks, vc, vs
+
+
+def check(kvq, oracle_mod, q, kc, ks, vc, vs, lens, wbits, scale, dev, page_size=0, bt=None, heads_subset=None):
+    B, NH, D = q.shape
+    out = torch.full((B, NH, D), float("nan"), dtype=torch.float16, device=dev)
+    ws = torch.full((kvq.attention_workspace_bytes((*kc.shape[:3], D), B, NH, page_size,
+                                                   bt.shape[1] if bt is not None else 0),), 0xFF,
+                    dtype=torch.uint8, device=dev)
+    kvq.decode_attention_q(q.to(dev), kc, ks, vc, vs, out, B, lens.to(dev), wbits, scale, page_size,
+                           bt.to(dev) if bt is not None else None, workspace=ws)
+    assert kvq.poll_device_error() == 0
+    st, ref, ex = oracle_mod.decode_attention_q(u16(q), kc.cpu().numpy(), u16(ks), vc.cpu().numpy(), u16(vs), B, NH,
+                                                page_size, lens.numpy(), bt.numpy() if bt is not None else None,
+                                                wbits, scale, D)
+    assert st == oracle_mod.OK
+    got = out.float().cpu().numpy().astype(np.float64)
+    assert not np.isnan(got).any()
+    # dequantized |v| bound for the absolute margin
+    vmax = float(ks.float().abs().max().cpu()) * ((1 << (wbits - 1)))
+    tol = np.spacing(np.maximum(np.abs(ex), 2.0 ** -14).astype(np.float16)).astype(np.float64) + 2.0 ** -14 * vmax
+    err = np.abs(got - ex)
+    bad = np.nonzero(err > tol)
+    assert bad[0].size == 0, f"{bad[0].size} outputs off, worst {err.max():.3g} (tol there {tol[bad][0]:.3g})"
+    exact16 = (ref == u16(out))
+    return err.max(), float(exact16.mean())
+
+
+@pytest.mark.parametrize("wbits", [4, 6, 8])
+@pytest.mark.parametrize("D,H,NH", [(128, 2, 8), (64, 4, 4), (256, 1, 8), (128, 1, 2)])
+def test_contiguous(kvq, oracle_mod, dev, wbits, D, H, NH):
+    B, S = 3, 600
+    k, v = workloads.channel_outliers(shape=(B, S, H, D))
+    kc, ks, vc, vs = quantize_on_gpu(kvq, k, v, wbits, dev)
+    q = torch.randn(B, NH, D).half()
+    lens = torch.tensor([600, 37, 257], dtype=torch.int32)
+    err, same = check(kvq, oracle_mod, q, kc, ks, vc, vs, lens, wbits, 1.0 / math.sqrt(D), dev)
+    assert same > 0.9  # nearly every output is the correctly rounded fp64 result
+
+
+@pytest.mark.parametrize("wbits", [4, 6, 8])
+@pytest.mark.parametrize("ps", [256, 16, 7])
+def test_paged(kvq, oracle_mod, dev, wbits, ps):
+    pool = workloads.paged_pool(num_pages=4000 // ps + 40, page_size=ps, heads=2, head_dim=128, batch=5,
+                                max_len=700)
+    kc, ks, vc, vs = quantize_on_gpu(kvq, pool.k, pool.v, wbits, dev)
+    q = torch.randn(5, 8, 128).half()
+    lens = pool.cache_seqlens.clone()
+    lens[0] = 0
+    lens[1] = 1
+    check(kvq, oracle_mod, q, kc, ks, vc, vs, lens, wbits, 0.088, dev, page_size=ps, bt=pool.block_table)
+
+
+def test_sharp_and_flat_softmax(kvq, oracle_mod, dev):
+    """Large scores (one-hot) and zero scores (mean) exercise the online max / rescale."""
+    B, S, H, D, NH = 2, 900, 1, 128, 4
+    k, v = workloads.normal_kv((B, S, H, D), 11)
+    kc, ks, vc, vs = quantize_on_gpu(kvq, k, v, 6, dev)
+    lens = torch.tensor([900, 513], dtype=torch.int32)
+    q = torch.randn(B, NH, D).half() * 4
+    check(kvq, oracle_mod, q, kc, ks, vc, vs, lens, 6, 2.0, dev)
+    check(kvq, oracle_mod, torch.zeros(B, NH, D).half(), kc, ks, vc, vs, lens, 6, 1.0, dev)
+
+
+@pytest.mark.parametrize("wbits", [4, 6])
+def test_paged_pool_full_size_sampled(kvq, oracle_mod, dev, wbits):
+    """The 2048-page pool (32 sequences, lengths up to 16384, 8 kv heads, 32 query heads),
+    checked against the oracle on 6 sequences (all heads)."""
+    pool = workloads.paged_pool(device=dev)
+    kc, ks, vc, vs = quantize_on_gpu(kvq, pool.k, pool.v, wbits, dev)
+    NH, D = 32, 128
+    q = torch.randn(32, NH, D, generator=torch.Generator().manual_seed(7)).half()
+    out = torch.empty(32, NH, D, dtype=torch.float16, device=dev)
+    kvq.decode_attention_q(q.to(dev), kc, ks, vc, vs, out, 32, pool.cache_seqlens, wbits, 1.0 / math.sqrt(D), 256,
+                           pool.block_table)
+    assert kvq.poll_device_error() == 0
+    pick = [0, 5, 11, 17, 23, 31]
+    lens = pool.cache_seqlens.cpu()[pick].contiguous()
+    bt = pool.block_table.cpu()[pick].contiguous()
+    st, ref, ex = oracle_mod.decode_attention_q(u16(q[pick]), kc.cpu().numpy(), u16(ks), vc.cpu().numpy(), u16(vs),
+                                                len(pick), NH, 256, lens.numpy(), bt.numpy(), wbits,
+                                                1.0 / math.sqrt(D), D)
+    assert st == oracle_mod.OK
+    got = out[pick].float().cpu().numpy().astype(np.float64)
+    vmax = float(ks.float().abs().max().cpu()) * (1 << (wbits - 1))
+    tol = np.spacing(np.maximum(np.abs(ex), 2.0 ** -14).astype(np.float16)).astype(np.float64) + 2.0 ** -14 * vmax
+    assert np.all(np.abs(got - ex) <= tol)
+
+
+def test_bad_paging_reported(kvq, dev):
+    ps, H, D = 16, 1, 64
+    k, v = workloads.small(shape=(4, ps, H, D))
+    kc, ks, vc, vs = quantize_on_gpu(kvq, k, v, 4, dev)
+    bt = torch.tensor([[0, 9]], dtype=torch.int32, device=dev)  # page 9 is outside the 4-page pool
+    lens = torch.tensor([30], dtype=torch.int32, device=dev)
+    out = torch.empty(1, 2, D, dtype=torch.float16, device=dev)
+    assert kvq.poll_device_error() == 0
+    kvq.decode_attention_q(torch.randn(1, 2, D).half().to(dev), kc, ks, vc, vs, out, 1, lens, 4, 0.1, ps, bt)
+    assert kvq.poll_device_error() != 0
+    assert not torch.isnan(out.float()).any()

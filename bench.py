@@ -31,6 +31,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -391,12 +392,58 @@ def per_op_measurements(kvq, dev, peak, steps, flush, include_model=True):
         record(f"q_to_fp16_kv/q4/{phase}", cfg, nb,
                lambda: kvq.q_to_fp16_kv(kc, pool.k, ks, vc, pool.v, vs, 32, off, w, ps,
                                         pool.cache_seqlens, pool.block_table, 4))
-    del pool, kc, vc, ks, vs, k8p, v8p
+    del kc, vc, ks, vs, k8p, v8p
+    torch.cuda.empty_cache()
+
+    # decode attention straight from the quantized pool: 32 sequences, 32 query heads
+    # (4 per kv head), one new token each, every cached position attended
+    for wb in (4, 6, 8):
+        fn, nb = attention_setup(kvq, dev, pool, wb)
+        record(f"decode_attention_q/q{wb}/paged",
+               f"paged 2048x256x8x128 pool, 32 seqs, 32 query heads, wbits={wb}", nb, fn)
+        del fn
+        torch.cuda.empty_cache()
+    del pool
     torch.cuda.empty_cache()
 
     if include_model:
         out.extend(model_layers(kvq, dev, peak, max(3, steps // 10), flush))
     return out
+
+
+ATTN_QUERY_HEADS = 32
+
+
+def attention_bytes(lens, kv_heads, head_dim, wbits, n_heads=ATTN_QUERY_HEADS):
+    """Algorithmic bytes of one decode_attention_q launch: the K and V codes and scales
+    of every attended position, the queries read and the outputs written."""
+    per_row = head_dim * wbits // 8 + 2 * (head_dim // 32)
+    npos = sum(int(L) for L in lens)
+    return 2 * npos * kv_heads * per_row + 2 * 2 * len(lens) * n_heads * head_dim
+
+
+def attention_setup(kvq, dev, pool, wbits, n_heads=ATTN_QUERY_HEADS):
+    """Quantize the whole pool (untimed) and return (launch, algorithmic bytes)."""
+    P, ps, H, D = pool.k.shape
+    batch = pool.cache_seqlens.numel()
+    cs, ss = kvq.q_shapes(tuple(pool.k.shape), wbits)
+    kc, vc = (torch.zeros(cs, dtype=torch.uint8, device=dev) for _ in range(2))
+    ks, vs = (torch.zeros(ss, dtype=torch.float16, device=dev) for _ in range(2))
+    full = pool.block_table.shape[1] * ps
+    kvq.fp16_to_q_kv(pool.k, kc, ks, pool.v, vc, vs, batch, -full, full, ps, pool.cache_seqlens, pool.block_table,
+                     wbits)
+    g = torch.Generator(device="cpu").manual_seed(workloads.SEED_BASE + 77)
+    q = torch.randn(batch, n_heads, D, generator=g).half().to(dev)
+    out = torch.empty_like(q)
+    ws = torch.empty(max(16, kvq.attention_workspace_bytes(tuple(pool.k.shape), batch, n_heads, ps,
+                                                           pool.block_table.shape[1])), dtype=torch.uint8, device=dev)
+    scale = 1.0 / math.sqrt(D)
+
+    def fn():
+        kvq.decode_attention_q(q, kc, ks, vc, vs, out, batch, pool.cache_seqlens, wbits, scale, ps, pool.block_table,
+                               ws)
+    fn()
+    return fn, attention_bytes(pool.cache_seqlens.cpu().tolist(), H, D, wbits, n_heads)
 
 
 def model_layers(kvq, dev, peak, steps, flush, layers=32):
@@ -443,7 +490,8 @@ def model_layers(kvq, dev, peak, steps, flush, layers=32):
 
 CASES = ("headline_fp8enc_kv", "headline_fp8dec_kv", "headline_fp8enc", "headline_fp8dec", "fp8enc", "fp8dec", "q4enc",
          "q4dec", "q6enc", "q6dec", "q8enc", "q8dec", "paged_prefill_q4enc", "paged_prefill_q4dec",
-         "paged_decode_q4enc", "model_layer_q6enc", "model_layer_q6dec")
+         "paged_decode_q4enc", "model_layer_q6enc", "model_layer_q6dec", "attn_paged_q4", "attn_paged_q6",
+         "attn_paged_q8")
 
 
 def run_case(kvq, dev, name, batch, steps, warmup, peak):
@@ -493,6 +541,9 @@ def run_case(kvq, dev, name, batch, steps, warmup, peak):
             fn = (lambda: kvq.fp16_to_q_kv(k, kc, ks, v, vc, vs, B, 0, S, 0, None, None, wb)) \
                 if name.endswith("enc") else (lambda: kvq.q_to_fp16_kv(kc, ky, ks, vc, vy, vs, B, 0, S, 0, None,
                                                                         None, wb))
+    elif name.startswith("attn_paged"):
+        pool = workloads.paged_pool(device=dev)
+        fn, nb = attention_setup(kvq, dev, pool, int(name[-1]))
     elif name.startswith("paged"):
         pool = workloads.paged_pool(device=dev)
         P, ps, H, D = pool.k.shape

@@ -8,8 +8,10 @@
 // q_to_fp16_kv writes (dequantized in registers with the same arithmetic).
 //
 // Split-K flash decoding.  Kernel 1 (attn_partial_kernel): one CTA per
-// (chunk of kAttnChunk positions, kv head, sequence), four warps; each warp
-// takes 16 positions at a time and
+// (chunk of positions, kv head, sequence), four warps.  The CTA first copies
+// its whole chunk of K and V codes and scales into shared memory with
+// cp.async (all copies in flight at once, so a CTA keeps tens of KB of
+// loads outstanding), then each warp takes 16 positions at a time and
 //   * dequantizes K for the 16 positions into mma.sync m16n8k16 A fragments
 //     (positions are the M dimension, the query heads of the group the N
 //     dimension, padded to 8), multiplies by the preloaded query fragments
@@ -32,7 +34,6 @@
 
 namespace kvq {
 
-constexpr int kAttnChunk = 256;  // positions per CTA
 constexpr int kAttnWarps = 4;
 constexpr int kAttnThreads = 32 * kAttnWarps;
 constexpr int kAttnMaxGroup = 8;  // query heads per kv head (one MMA N block)
@@ -48,6 +49,7 @@ struct AttnParams {
   const int32_t* seqlens;
   const int32_t* block_table;
   int dim0, dim1, kv_heads, batch, n_heads, group, page_size, bt_stride, max_chunks;
+  int chunk;  // positions per CTA (AttnTile<B, D>::kChunk)
   float scale_log2;  // softmax_scale * log2(e)
 };
 
@@ -64,28 +66,87 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Dequantize N consecutive elements [d, d + N) (d a multiple of 8) of one
-// head row into N / 2 half2 registers (element pairs (d + 2e, d + 2e + 1)).
+// Shared-memory staging of one CTA's chunk: K codes, V codes (rows padded
+// by 16 bytes so that the fragment reads of neighbouring rows fall in
+// different banks), K scales, V scales, then each position's cache row index.
+// Rows of up to 64 code bytes take 256-position chunks, longer rows 128.
+template <int B, int D>
+struct AttnTile {
+  static constexpr int kRowBytes = D * B / 8;
+  static constexpr int kStride = kRowBytes + 16;
+  static constexpr int kScales = D / 32;
+  static constexpr int kChunk = kRowBytes <= 64 ? 256 : 128;
+  static constexpr int kCodeBytes = kChunk * kStride;
+  static constexpr int kScaleBytes = kChunk * kScales * 2;
+  static constexpr int kStageBytes = 2 * (kCodeBytes + kScaleBytes);
+  static constexpr int kAccBytes = kAttnWarps * D * (kAttnMaxGroup + 1) * 4;  // merge area (aliases the stage)
+  static constexpr int kRowIdxOffset = kStageBytes > kAccBytes ? kStageBytes : kAccBytes;
+  static constexpr int kSmemBytes = kRowIdxOffset + kChunk * 8;
+};
+constexpr int kAttnMinChunk = 128;  // smallest chunk any (B, D) uses: sizes the workspace
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void cp_async_small(void* dst, const void* src) {
+  static_assert(N == 4 || N == 8 || N == 16, "cp.async sizes");
+  asm volatile("cp.async.ca.shared.global [%0], [%1], %2;\n" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src), "n"(N)
+               : "memory");
+}
+
+// Dequantize N consecutive elements [d, d + N) of one staged row (d a
+// multiple of N, N a multiple of 8) into N / 2 half2 registers (element
+// pairs (d + 2e, d + 2e + 1)).  Every 32-element block inside the span
+// starts at a multiple of 32, so 8-element unit u uses scale (d >> 5) + (u >> 2).
 template <int B, int N>
-__device__ __forceinline__ void dequant_range(const uint8_t* codes_row, const __half* scales_row, int d,
-                                              uint32_t out[N / 2]) {
+__device__ __forceinline__ void dequant_span(const uint8_t* row, const __half* srow, int d, uint32_t out[N / 2]) {
   static_assert(N % 8 == 0, "whole 8-element units");
+  constexpr int NB = N * B / 8;  // bytes of the span; the span starts at a multiple of NB
+  const uint8_t* p = row + d * B / 8;
+  uint32_t w[(NB + 3) / 4 + 1];
+  if constexpr (B == 6 && N == 8) {
+    // 6 bytes at a 2-byte offset: the two words of the 12-byte group half
+    const uint32_t* grp = reinterpret_cast<const uint32_t*>(row + (d >> 4) * 12);
+    const int half = (d >> 3) & 1;
+    const uint32_t a = grp[half], b = grp[half + 1];
+    w[0] = __funnelshift_r(a, b, 16 * half);
+    w[1] = (b >> (16 * half)) & 0xFFFFu;
+  } else if constexpr (NB % 16 == 0) {
+#pragma unroll
+    for (int v = 0; v < NB / 16; ++v) {
+      const uint4 x = reinterpret_cast<const uint4*>(p)[v];
+      w[4 * v] = x.x, w[4 * v + 1] = x.y, w[4 * v + 2] = x.z, w[4 * v + 3] = x.w;
+    }
+  } else if constexpr (NB % 8 == 0) {
+#pragma unroll
+    for (int v = 0; v < NB / 8; ++v) {
+      const uint2 x = reinterpret_cast<const uint2*>(p)[v];
+      w[2 * v] = x.x, w[2 * v + 1] = x.y;
+    }
+  } else {
+#pragma unroll
+    for (int v = 0; v < NB / 4; ++v) w[v] = reinterpret_cast<const uint32_t*>(p)[v];
+  }
 #pragma unroll
   for (int u = 0; u < N / 8; ++u) {
-    const int e = d + 8 * u;
-    const __half s = __ldg(scales_row + (e >> 5));
+    const __half s = srow[(d >> 5) + (u >> 2)];
     const __half2 s2 = __halves2half2(s, s);
     uint4 r;
-    if (B == 4) {
-      r = dequant_q4_v8(__ldg(reinterpret_cast<const uint32_t*>(codes_row + (e >> 1))), s2);
-    } else if (B == 8) {
-      const uint2 w = __ldg(reinterpret_cast<const uint2*>(codes_row + e));
-      r = dequant_q8_v8(w.x, w.y, s2);
+    if constexpr (B == 4) {
+      r = dequant_q4_v8(w[u], s2);
+    } else if constexpr (B == 8) {
+      r = dequant_q8_v8(w[2 * u], w[2 * u + 1], s2);
+    } else if constexpr (N == 8) {
+      r = dequant_q6_v8(w[0], w[1], s2);
     } else {
-      const uint32_t* grp = reinterpret_cast<const uint32_t*>(codes_row + (e >> 4) * 12);
-      const int half = (e >> 3) & 1;
-      const uint32_t a = __ldg(grp + half), b = __ldg(grp + half + 1);
-      r = dequant_q6_v8(__funnelshift_r(a, b, 16 * half), (b >> (16 * half)) & 0xFFFFu, s2);
+      const int q = u >> 1;  // 16-code group: words 3q .. 3q + 2
+      r = (u & 1) ? dequant_q6_v8(__funnelshift_r(w[3 * q + 1], w[3 * q + 2], 16), w[3 * q + 2] >> 16, s2)
+                  : dequant_q6_v8(w[3 * q], w[3 * q + 1] & 0xFFFFu, s2);
     }
     out[4 * u + 0] = r.x;
     out[4 * u + 1] = r.y;
@@ -94,8 +155,8 @@ __device__ __forceinline__ void dequant_range(const uint8_t* codes_row, const __
   }
 }
 
-// Physical row of logical position p of sequence `seq`, or -1 (recorded as a
-// device error when `report`) when the paging metadata points outside.
+// Physical row of logical position p of sequence `seq`, or -1 when the paging
+// metadata points outside the cache.
 __device__ __forceinline__ long long attn_row(const AttnParams& a, int seq, long long p, const int* bt_chunk,
                                               long long lp0) {
   if (a.page_size == 0) return static_cast<long long>(seq) * a.dim1 + p;
@@ -108,38 +169,45 @@ __device__ __forceinline__ long long attn_row(const AttnParams& a, int seq, long
 
 template <int B, int D>
 __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(const __grid_constant__ AttnParams a) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  constexpr int KS = D / 16;                    // k-steps of Q K^T, m-blocks of V^T P^T
-  constexpr int KN = D / 4;                     // K elements per lane per position
-  constexpr int VN = D / 8;                     // V elements per lane per position
-  constexpr long long code_bytes = D * B / 8;   // one head row
-  constexpr int nscales = D / 32;
-  constexpr int kMaxChunkPages = kAttnChunk + 1;
+  using T = AttnTile<B, D>;
+  constexpr int KS = D / 16;  // k-steps of Q K^T, m-blocks of V^T P^T
+  constexpr int KN = D / 4;   // K elements per lane per position
+  constexpr int VN = D / 8;   // V elements per lane per position
+  constexpr int C = T::kChunk;
 
-  __shared__ int s_bt[kMaxChunkPages];
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint8_t* const sk = smem;
+  uint8_t* const sv = smem + T::kCodeBytes;
+  __half* const sks = reinterpret_cast<__half*>(smem + 2 * T::kCodeBytes);
+  __half* const svs = sks + C * T::kScales;
+  long long* const s_hr = reinterpret_cast<long long*>(smem + T::kRowIdxOffset);
+  float(*const s_acc)[D][kAttnMaxGroup + 1] = reinterpret_cast<float(*)[D][kAttnMaxGroup + 1]>(smem);
+  __shared__ int s_bt[C + 1];
   __shared__ float s_p[kAttnWarps][16][kAttnMaxGroup + 1];
   __shared__ float s_m[kAttnWarps][kAttnMaxGroup];
   __shared__ float s_l[kAttnWarps][kAttnMaxGroup];
-  __shared__ float s_acc[kAttnWarps][D][kAttnMaxGroup + 1];
   __shared__ int s_bad;
 
   const int chunk = blockIdx.x, kvh = blockIdx.y, seq = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, j = lane & 3;
+
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0) s_bad = 0;
 
   long long L = a.seqlens[seq];
   if (L < 0) L = 0;
   const long long max_len = a.page_size == 0 ? static_cast<long long>(a.dim1)
-                                             : static_cast<long long>(a.max_chunks) * kAttnChunk;
+                                             : static_cast<long long>(a.max_chunks) * C;
   if (L > max_len) {  // longer than the cache (contiguous) or than the launched chunks (paged)
     if (threadIdx.x == 0 && chunk == 0 && kvh == 0) record_error(KVQ_DEV_BAD_PAGE_INDEX);
     L = max_len;
   }
-  const long long p0 = static_cast<long long>(chunk) * kAttnChunk;
+  const long long p0 = static_cast<long long>(chunk) * C;
   if (p0 >= L) return;  // the whole CTA leaves together
-  const long long p1 = min(L, p0 + kAttnChunk);
+  const long long p1 = min(L, p0 + C);
+  const int n = static_cast<int>(p1 - p0);
 
   // block-table entries of the chunk's logical pages, staged once
   long long lp0 = 0;
@@ -151,8 +219,46 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(const __grid
   }
   __syncthreads();
 
+  // cache row of every position of the chunk (-1: bad paging metadata, -2: past the window)
+  for (int i = threadIdx.x; i < C; i += kAttnThreads) {
+    long long hr = -2;
+    if (i < n) {
+      const long long row = attn_row(a, seq, p0 + i, s_bt, lp0);
+      if (row < 0) s_bad = 1;
+      hr = row < 0 ? -1 : row * a.kv_heads + kvh;
+    }
+    s_hr[i] = hr;
+  }
+  __syncthreads();
+
+  // issue every copy of the chunk; rows without data get zero scales, which
+  // dequantize whatever codes the buffer holds to zero
+  {
+    constexpr int P = T::kRowBytes / 16;
+    for (int t = threadIdx.x; t < C * P; t += kAttnThreads) {
+      const int i = t / P, part = t - i * P;
+      const long long hr = s_hr[i];
+      if (hr >= 0) {
+        const long long off = hr * T::kRowBytes + part * 16;
+        cp_async16(sk + i * T::kStride + part * 16, a.k_codes + off);
+        cp_async16(sv + i * T::kStride + part * 16, a.v_codes + off);
+      }
+    }
+    for (int i = threadIdx.x; i < C; i += kAttnThreads) {
+      const long long hr = s_hr[i];
+      if (hr >= 0) {
+        cp_async_small<T::kScales * 2>(sks + i * T::kScales, a.k_scales + hr * T::kScales);
+        cp_async_small<T::kScales * 2>(svs + i * T::kScales, a.v_scales + hr * T::kScales);
+      } else {
+#pragma unroll
+        for (int e = 0; e < T::kScales; ++e) sks[i * T::kScales + e] = svs[i * T::kScales + e] = __ushort_as_half(0);
+      }
+    }
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+  }
+
   // query fragments (B operand of Q K^T): head g of the group, this lane's
-  // permuted head_dim slice d = KN*j + 4s + {0..3}
+  // permuted head_dim slice d = KN*j + 4s + {0..3}; loaded while the copies fly
   uint32_t qf[KS][2];
   {
     const bool live = g < a.group;
@@ -164,6 +270,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(const __grid
       qf[s][1] = live ? __ldg(reinterpret_cast<const uint32_t*>(qrow + d0 + 2)) : 0u;
     }
   }
+  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+  __syncthreads();
 
   float m_run[2] = {-INFINITY, -INFINITY};  // heads 2j, 2j+1 (log2 domain)
   float l_run[2] = {0.0f, 0.0f};
@@ -171,23 +279,15 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(const __grid
 #pragma unroll
   for (int mb = 0; mb < KS; ++mb) acc[mb][0] = acc[mb][1] = acc[mb][2] = acc[mb][3] = 0.0f;
 
-  for (long long base = p0 + 16 * warp; base < p1; base += 16 * kAttnWarps) {
-    // ---- K: positions base + g and base + g + 8, elements [KN*j, KN*j + KN)
+  for (int t0 = 16 * warp; t0 < n; t0 += 16 * kAttnWarps) {
+    // ---- K: positions t0 + g and t0 + g + 8, elements [KN*j, KN*j + KN)
     uint32_t kd[2][KN / 2];
     bool kvalid[2];
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      const long long p = base + g + 8 * r;
-      const long long row = p < p1 ? attn_row(a, seq, p, s_bt, lp0) : -2;
-      kvalid[r] = row >= 0;
-      if (row == -1) s_bad = 1;
-      if (kvalid[r]) {
-        const long long hr = row * a.kv_heads + kvh;
-        dequant_range<B, KN>(a.k_codes + hr * code_bytes, a.k_scales + hr * nscales, KN * j, kd[r]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < KN / 2; ++e) kd[r][e] = 0u;
-      }
+      const int i = t0 + g + 8 * r;
+      kvalid[r] = s_hr[i] >= 0;
+      dequant_span<B, KN>(sk + i * T::kStride, sks + i * T::kScales, KN * j, kd[r]);
     }
     float sc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
@@ -217,10 +317,12 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(const __grid
       sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 16);
       l_run[h] = l_run[h] * alpha + sum;
       m_run[h] = m_new;
+      if (alpha != 1.0f) {
 #pragma unroll
-      for (int mb = 0; mb < KS; ++mb) {
-        acc[mb][h] *= alpha;
-        acc[mb][2 + h] *= alpha;
+        for (int mb = 0; mb < KS; ++mb) {
+          acc[mb][h] *= alpha;
+          acc[mb][2 + h] *= alpha;
+        }
       }
     }
 
@@ -238,19 +340,12 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(const __grid
     const float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
     const uint32_t bl0 = pack_half2(b0 - f0.x, b1 - f0.y), bl1 = pack_half2(b2 - f1.x, b3 - f1.y);
 
-    // ---- V: positions base + {2j, 2j+1, 2j+8, 2j+9}, elements [VN*g, VN*g + VN)
+    // ---- V: positions t0 + {2j, 2j+1, 2j+8, 2j+9}, elements [VN*g, VN*g + VN)
     uint32_t vd[4][VN / 2];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      const long long p = base + 2 * j + (r & 1) + 8 * (r >> 1);
-      const long long row = p < p1 ? attn_row(a, seq, p, s_bt, lp0) : -2;
-      if (row >= 0) {
-        const long long hr = row * a.kv_heads + kvh;
-        dequant_range<B, VN>(a.v_codes + hr * code_bytes, a.v_scales + hr * nscales, VN * g, vd[r]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < VN / 2; ++e) vd[r][e] = 0u;
-      }
+      const int i = t0 + 2 * j + (r & 1) + 8 * (r >> 1);
+      dequant_span<B, VN>(sv + i * T::kStride, svs + i * T::kScales, VN * g, vd[r]);
     }
 #pragma unroll
     for (int mb = 0; mb < KS; ++mb) {
@@ -263,7 +358,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(const __grid
   }
 
   // ---- merge the four warps: acc[mb] holds O^T[d][h] for d = VN*g + 2mb (c0, c1: heads 2j, 2j+1)
-  // and d + 1 (c2, c3)
+  // and d + 1 (c2, c3).  The merge area aliases the staged chunk.
+  __syncthreads();
   if (g == 0) {
     s_m[warp][2 * j] = m_run[0];
     s_m[warp][2 * j + 1] = m_run[1];
@@ -310,7 +406,7 @@ __global__ void __launch_bounds__(D) attn_combine_kernel(const __grid_constant__
   long long L = a.seqlens[seq];
   if (L < 0) L = 0;
   if (a.page_size == 0 && L > a.dim1) L = a.dim1;
-  long long nch = (L + kAttnChunk - 1) / kAttnChunk;
+  long long nch = (L + a.chunk - 1) / a.chunk;
   if (nch > a.max_chunks) nch = a.max_chunks;
   const float* ws = a.ws + (static_cast<long long>(seq) * a.n_heads + h) * a.max_chunks * (D + 2);
   float mstar = -INFINITY;

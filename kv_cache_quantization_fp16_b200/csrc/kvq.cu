@@ -400,27 +400,51 @@ kvq_status kvq_poll_device_error(int32_t* code_out, void* stream) {
 
 namespace {
 
-// Chunks of kAttnChunk positions a sequence can have: the longest window the
+// Chunks of `chunk` positions a sequence can have: the longest window the
 // cache geometry allows.
-long long attn_max_chunks(const kvq_cache_desc* d, int page_size) {
+long long attn_max_chunks(const kvq_cache_desc* d, int page_size, int chunk) {
   const long long max_len = page_size > 0 ? static_cast<long long>(d->block_table_stride) * page_size
                                           : static_cast<long long>(d->dim1);
-  return (max_len + kvq::kAttnChunk - 1) / kvq::kAttnChunk;
+  return (max_len + chunk - 1) / chunk;
+}
+
+// Dynamic shared memory opt-in, once per device for each (B, D) kernel
+// (static plus dynamic shared memory above 48 KB needs it).
+template <int B, int D>
+bool allow_attention_smem() {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<bool> done[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  if (done[dev].load()) return true;
+  if (cudaFuncSetAttribute(kvq::attn_partial_kernel<B, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kvq::AttnTile<B, D>::kSmemBytes) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  done[dev].store(true);
+  return true;
 }
 
 template <int B, int D>
-kvq_status launch_attention(const kvq::AttnParams& a, void* stream) {
+kvq_status launch_attention(kvq::AttnParams a, const kvq_cache_desc* desc, void* stream) {
+  using T = kvq::AttnTile<B, D>;
+  a.chunk = T::kChunk;
+  const long long max_chunks = attn_max_chunks(desc, a.page_size, T::kChunk);
+  if (max_chunks < 1 || max_chunks > 0x7FFFFFFFLL) return KVQ_ERR_RANGE;
+  a.max_chunks = static_cast<int>(max_chunks);
+  if (!allow_attention_smem<B, D>()) return KVQ_ERR_CUDA;
   kvq_status st = launch_pdl(kvq::attn_partial_kernel<B, D>, dim3(a.max_chunks, a.kv_heads, a.batch),
-                             kvq::kAttnThreads, 0, stream, a);
+                             kvq::kAttnThreads, T::kSmemBytes, stream, a);
   if (st != KVQ_OK) return st;
   return launch_pdl(kvq::attn_combine_kernel<D>, dim3(a.n_heads, a.batch), D, 0, stream, a);
 }
 
 template <int B>
-kvq_status launch_attention_b(const kvq::AttnParams& a, int head_dim, void* stream) {
-  if (head_dim == 64) return launch_attention<B, 64>(a, stream);
-  if (head_dim == 128) return launch_attention<B, 128>(a, stream);
-  return launch_attention<B, 256>(a, stream);
+kvq_status launch_attention_b(const kvq::AttnParams& a, const kvq_cache_desc* desc, void* stream) {
+  if (desc->head_dim == 64) return launch_attention<B, 64>(a, desc, stream);
+  if (desc->head_dim == 128) return launch_attention<B, 128>(a, desc, stream);
+  return launch_attention<B, 256>(a, desc, stream);
 }
 
 }  // namespace
@@ -430,8 +454,9 @@ extern "C" {
 size_t kvq_decode_attention_workspace_size(const kvq_cache_desc* desc, int batch_size, int n_heads,
                                            int page_size) {
   if (!desc || batch_size < 0 || n_heads < 0 || page_size < 0) return 0;
-  return static_cast<size_t>(batch_size) * n_heads * attn_max_chunks(desc, page_size) * (desc->head_dim + 2) *
-         sizeof(float);
+  // sized for the smallest chunk any wbits / head_dim uses
+  return static_cast<size_t>(batch_size) * n_heads * attn_max_chunks(desc, page_size, kvq::kAttnMinChunk) *
+         (desc->head_dim + 2) * sizeof(float);
 }
 
 kvq_status kvq_decode_attention_q(const void* q, const void* k_codes, const void* k_scales, const void* v_codes,
@@ -460,7 +485,7 @@ kvq_status kvq_decode_attention_q(const void* q, const void* k_codes, const void
   if ((reinterpret_cast<uintptr_t>(cache_seqlens) | reinterpret_cast<uintptr_t>(block_table)) & 3u)
     return KVQ_ERR_ALIGN;
   if (batch_size == 0) return KVQ_OK;
-  const long long max_chunks = attn_max_chunks(desc, page_size);
+  const long long max_chunks = attn_max_chunks(desc, page_size, kvq::kAttnMinChunk);
   if (max_chunks < 1 || max_chunks > 0x7FFFFFFFLL) return KVQ_ERR_RANGE;
   if (!workspace) return KVQ_ERR_NULL;
   if (workspace_bytes < kvq_decode_attention_workspace_size(desc, batch_size, n_heads, page_size))
@@ -483,11 +508,10 @@ kvq_status kvq_decode_attention_q(const void* q, const void* k_codes, const void
   a.group = n_heads / desc->kv_heads;
   a.page_size = page_size;
   a.bt_stride = desc->block_table_stride;
-  a.max_chunks = static_cast<int>(max_chunks);
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
-  if (wbits == 4) return launch_attention_b<4>(a, D, stream);
-  if (wbits == 6) return launch_attention_b<6>(a, D, stream);
-  return launch_attention_b<8>(a, D, stream);
+  if (wbits == 4) return launch_attention_b<4>(a, desc, stream);
+  if (wbits == 6) return launch_attention_b<6>(a, desc, stream);
+  return launch_attention_b<8>(a, desc, stream);
 }
 
 long long kvq_count_match(const int64_t* a, long long a_len, const int64_t* b, long long b_len, long long max_a) {

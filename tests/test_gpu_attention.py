@@ -67,7 +67,7 @@ def check(kvq, oracle_mod, q, kc, ks, vc, vs, lens, wbits, scale, dev, page_size
     got = out.float().cpu().numpy().astype(np.float64)
     assert not np.isnan(got).any()
     # dequantized |v| bound for the absolute margin
-    vmax = float(ks.float().abs().max().cpu()) * ((1 << (wbits - 1)))
+    vmax = float(vs.float().abs().max().cpu()) * ((1 << (wbits - 1)))
     tol = np.spacing(np.maximum(np.abs(ex), 2.0 ** -14).astype(np.float16)).astype(np.float64) + 2.0 ** -14 * vmax
     err = np.abs(got - ex)
     bad = np.nonzero(err > tol)

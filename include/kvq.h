@@ -202,6 +202,38 @@ KVQ_API kvq_status kvq_decode_attention_q(const void* q, const void* k_codes, co
 KVQ_API size_t kvq_decode_attention_workspace_size(const kvq_cache_desc* desc, int batch_size, int n_heads,
                                                    int page_size);
 
+/* Size of the scratch array kvq_decode_attention_q_noalloc uses (16 MiB per
+ * device). */
+#define KVQ_ATTENTION_SCRATCH_BYTES ((size_t)16 << 20)
+
+/* kvq_decode_attention_q without a caller workspace.  The pages have no
+ * counterpart: this is a convenience of this library for callers that cannot
+ * allocate device memory at the call site (a serving loop whose HBM belongs
+ * to its own KV-page pool, or a decode step that cannot afford the device
+ * synchronization cudaMalloc / cudaFree may cause).  The split-K workspace is
+ * a fixed array of KVQ_ATTENTION_SCRATCH_BYTES inside the library (one per
+ * device), so the call allocates nothing.
+ *   Arguments, layouts, results and errors are those of
+ *   kvq_decode_attention_q.  A geometry whose
+ *   kvq_decode_attention_workspace_size(...) exceeds
+ *   KVQ_ATTENTION_SCRATCH_BYTES returns KVQ_ERR_RANGE and enqueues nothing
+ *   (for example, batch 8 x 32 query heads x head_dim 128 with up to 8192
+ *   positions needs 8.5 MB and fits).
+ *   The first call on each device, made with that device current, looks up
+ *   the array's device address; make that first call before any stream
+ *   capture.  KVQ_ERR_CUDA if the lookup fails.
+ *   Every call on a device shares the one array and leaves its partial
+ *   results there; nothing in it has to start at zero, because each call
+ *   writes every entry it later reads.  Calls whose kernels overlap on the
+ *   GPU (other streams, other host threads) race on the array and must be
+ *   serialized by the caller. */
+KVQ_API kvq_status kvq_decode_attention_q_noalloc(const void* q, const void* k_codes, const void* k_scales,
+                                                  const void* v_codes, const void* v_scales, void* out,
+                                                  const kvq_cache_desc* desc, int batch_size, int n_heads,
+                                                  int page_size, const int32_t* cache_seqlens,
+                                                  const int32_t* block_table, int wbits, float softmax_scale,
+                                                  void* stream);
+
 /* count_match (Description; I/O Contract): the number of leading elements on
  * which the 64-bit sequences a[0..a_len) and b[0..b_len) agree, comparing no
  * more than max_a elements (max_a <= 0 gives 0).  Host function: a and b are

@@ -26,7 +26,8 @@ import os
 import torch
 
 __all__ = ["fp16_to_fp8", "fp8_to_fp16", "fp16_to_fp8_kv", "fp8_to_fp16_kv", "fp16_to_q_kv", "q_to_fp16_kv", "poll_device_error",
-           "selfcheck_code_rounding", "count_match", "decode_attention_q", "attention_workspace_bytes", "q_shapes", "set_engine", "get_engine", "engine", "KVQError",
+           "selfcheck_code_rounding", "count_match", "decode_attention_q", "decode_attention_q_noalloc",
+           "attention_workspace_bytes", "q_shapes", "set_engine", "get_engine", "engine", "KVQError",
            "LIB_PATH", "library"]
 
 ENGINES = {"auto": 0, "ldg": 1, "bulk": 2}
@@ -72,6 +73,9 @@ def _load() -> ctypes.CDLL:
     L.kvq_decode_attention_q.argtypes = [vp, vp, vp, vp, vp, vp, dp, I, I, I, vp, vp, I, ctypes.c_float, vp,
                                          ctypes.c_size_t, vp]
     L.kvq_decode_attention_q.restype = I
+    L.kvq_decode_attention_q_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, dp, I, I, I, vp, vp, I, ctypes.c_float,
+                                                 vp]
+    L.kvq_decode_attention_q_noalloc.restype = I
     L.kvq_decode_attention_workspace_size.argtypes = [dp, I, I, I]
     L.kvq_decode_attention_workspace_size.restype = ctypes.c_size_t
     L.kvq_count_match.argtypes = [vp, LL, vp, LL, LL]
@@ -364,3 +368,51 @@ def decode_attention_q(q, k_codes, k_scales, v_codes, v_scales, out, batch_size,
                                          int(n_heads), int(page_size), cache_seqlens.data_ptr(), bt_ptr, int(wbits),
                                          float(softmax_scale), workspace.data_ptr(), workspace.numel(), _stream(dev))
     _check(st, "decode_attention_q")
+
+
+ATTENTION_SCRATCH_BYTES = 16 << 20  # KVQ_ATTENTION_SCRATCH_BYTES
+
+
+def decode_attention_q_noalloc(q, k_codes, k_scales, v_codes, v_scales, out, batch_size, cache_seqlens, wbits,
+                               softmax_scale, page_size=0, block_table=None) -> None:
+    """decode_attention_q for callers that cannot allocate device memory at the call
+    site: the workspace is the library's own 16 MiB array (one per device), so nothing is
+    allocated, by torch or by CUDA.  Geometries needing more workspace than
+    ATTENTION_SCRATCH_BYTES are rejected.  Calls that overlap on the GPU share the array
+    and race; make the first call on a device before any stream capture."""
+    _require(isinstance(q, torch.Tensor) and q.dtype == torch.float16 and q.is_cuda and q.dim() == 3
+             and q.is_contiguous(), "q must be a contiguous [batch, n_heads, head_dim] float16 CUDA tensor")
+    _require(out.shape == q.shape and out.dtype == torch.float16 and out.is_contiguous() and out.device == q.device,
+             "out must match q")
+    for t, n in ((k_codes, "k_codes"), (v_codes, "v_codes")):
+        _cuda4(t, torch.uint8, n)
+    for t, n in ((k_scales, "k_scales"), (v_scales, "v_scales")):
+        _cuda4(t, torch.float16, n)
+    _require(wbits in (4, 6, 8), f"wbits must be 4, 6 or 8, got {wbits}")
+    D = q.shape[2]
+    cshape, sshape = q_shapes((*k_codes.shape[:3], D), wbits)
+    for t, n in ((k_codes, "k_codes"), (v_codes, "v_codes")):
+        _require(tuple(t.shape) == cshape, f"{n} must have shape {cshape}, got {tuple(t.shape)}")
+    for t, n in ((k_scales, "k_scales"), (v_scales, "v_scales")):
+        _require(tuple(t.shape) == sshape, f"{n} must have shape {sshape}, got {tuple(t.shape)}")
+    dev = q.device
+    for t in (k_codes, k_scales, v_codes, v_scales):
+        _require(t.device == dev, "tensors must be on one device")
+    _require(cache_seqlens is not None and cache_seqlens.dtype == torch.int32 and cache_seqlens.device == dev
+             and cache_seqlens.is_contiguous() and cache_seqlens.numel() >= batch_size,
+             "cache_seqlens must be a contiguous int32 tensor on the caches' device with batch_size entries")
+    stride, _, bt_ptr = _paging(page_size, cache_seqlens, block_table, batch_size, dev)
+    d0, d1, H, _ = k_codes.shape
+    desc = _Desc(d0, d1, H, D, stride)
+    n_heads = q.shape[1]
+    need = int(_lib.kvq_decode_attention_workspace_size(ctypes.byref(desc), int(batch_size), int(n_heads),
+                                                        int(page_size)))
+    _require(need <= ATTENTION_SCRATCH_BYTES,
+             f"this geometry needs {need} bytes of workspace, above the {ATTENTION_SCRATCH_BYTES}-byte scratch array")
+    with torch.cuda.device(dev):
+        st = _lib.kvq_decode_attention_q_noalloc(q.data_ptr(), k_codes.data_ptr(), k_scales.data_ptr(),
+                                                 v_codes.data_ptr(), v_scales.data_ptr(), out.data_ptr(),
+                                                 ctypes.byref(desc), int(batch_size), int(n_heads), int(page_size),
+                                                 cache_seqlens.data_ptr(), bt_ptr, int(wbits), float(softmax_scale),
+                                                 _stream(dev))
+    _check(st, "decode_attention_q_noalloc")

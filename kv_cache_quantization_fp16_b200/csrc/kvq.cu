@@ -547,3 +547,59 @@ kvq_status kvq_selfcheck_code_rounding(int wbits, unsigned long long* mismatches
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode attention with library-owned scratch.
+//
+// Some callers cannot allocate device memory where they call attention: a
+// serving loop whose HBM is all handed to its own KV-page pool up front has
+// no allocator to draw a workspace from, and cudaMalloc / cudaFree may
+// synchronize the device, which a per-token decode step on a busy stream
+// cannot afford.  This entry point takes its split-K workspace from a fixed
+// array compiled into the library instead, so it allocates nothing.
+
+static __device__ __align__(256) unsigned char g_attention_scratch[KVQ_ATTENTION_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kScratchMaxDevices = 64;
+std::atomic<void*> g_attention_scratch_ptr[kScratchMaxDevices];
+
+// Device address of this device's copy of the array, looked up on the first
+// call made with the device current.  Null on failure.
+void* attention_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kScratchMaxDevices) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  void* ptr = g_attention_scratch_ptr[dev].load();
+  if (ptr) return ptr;
+  if (cudaGetSymbolAddress(&ptr, g_attention_scratch) != cudaSuccess || !ptr) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  g_attention_scratch_ptr[dev].store(ptr);
+  return ptr;
+}
+
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_decode_attention_q_noalloc(const void* q, const void* k_codes, const void* k_scales,
+                                          const void* v_codes, const void* v_scales, void* out,
+                                          const kvq_cache_desc* desc, int batch_size, int n_heads, int page_size,
+                                          const int32_t* cache_seqlens, const int32_t* block_table, int wbits,
+                                          float softmax_scale, void* stream) {
+  if (!desc) return KVQ_ERR_NULL;
+  if (kvq_decode_attention_workspace_size(desc, batch_size, n_heads, page_size) > KVQ_ATTENTION_SCRATCH_BYTES)
+    return KVQ_ERR_RANGE;
+  void* scratch = attention_scratch();
+  if (!scratch) return KVQ_ERR_CUDA;
+  return kvq_decode_attention_q(q, k_codes, k_scales, v_codes, v_scales, out, desc, batch_size, n_heads,
+                                page_size, cache_seqlens, block_table, wbits, softmax_scale, scratch,
+                                KVQ_ATTENTION_SCRATCH_BYTES, stream);
+}
+
+}  // extern "C"

@@ -162,3 +162,14 @@ def test_decode_attention_validation(kvq):
     assert call(desc=dp, ps=16) == 1                    # paged needs a block table
     assert call(desc=dp, ps=8, bt=FAKE) == 4            # page_size must equal dim1
     assert call(bs=0, wsp=None, wsb=0) == 0             # empty batch enqueues nothing
+
+
+def test_decode_attention_noalloc_validation(kvq):
+    L = kvq.library()
+    by = ctypes.byref
+    P = [FAKE] * 6
+    big = _desc(kvq, d0=64, d1=1 << 20, H=8, D=128)
+    assert L.kvq_decode_attention_workspace_size(by(big), 64, 64, 0) > kvq.ATTENTION_SCRATCH_BYTES
+    assert L.kvq_decode_attention_q_noalloc(*P, None, 2, 4, 0, FAKE, None, 4, ctypes.c_float(1.0), None) == 1
+    # beyond the scratch array: rejected on the host, nothing enqueued
+    assert L.kvq_decode_attention_q_noalloc(*P, by(big), 64, 64, 0, FAKE, None, 4, ctypes.c_float(1.0), None) == 4

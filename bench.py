@@ -5,10 +5,17 @@ workload -- K and V FP16 caches [4, 4096, 8, 128] (N(0,1) with 1% +-U(20,60000)
 outliers and 0.1% subnormals), window offset 1024, width 2048.  One step is
 fp16_to_fp8 of K and V, then fp8_to_fp16 of K and V, through the C ABI's fused
 K+V calls (one launch per direction) on resident device buffers; the same step
-through the single-tensor calls (4 launches) is reported in per_op.  The metric is algorithmic GB/s (bytes read +
-bytes written: 3 bytes per element per conversion), with L2 flushed between
-steps (a 256 MiB write then a 256 MiB read, outside the per-step CUDA events,
-so no dirty flush lines are written back inside a timed kernel).
+through the single-tensor calls (4 launches) is reported in per_op.  The metric
+is algorithmic GB/s (bytes read + bytes written: 3 bytes per element per
+conversion).
+
+Timing.  `--steps` consecutive steps run back to back (replayed from CUDA
+graphs) between one pair of CUDA events.  The inputs are larger than L2: the
+step keeps 8 independent copies of the workload (about 1.3 GB) and step i
+converts copy i % 8, so every copy has been evicted by the other copies'
+traffic before it comes round again; L2 is flushed once before the timed
+steps.  The latency of one step on its own (L2 flushed before it, events
+around it) is reported beside it under `isolated`.
 
 Extra keys:
   roofline      the dominant kernel's achieved GB/s (algorithmic bytes per
@@ -129,7 +136,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             threading.Thread(target=self._read, daemon=True).start()
         except (OSError, ValueError):
             self.proc = None
@@ -186,20 +193,30 @@ class L2Flush:
         self.sink = torch.amax(self.r)
 
 
+STREAM_SETS = 8  # input sets a stream of steps rotates through (8 x ~168 MB, well above the 126 MB L2)
+
+
 class Fp8Step:
     """Headline step on one rank: FP8 encode then decode of the K and V windows, through
-    the fused K+V calls (one launch per direction)."""
+    the fused K+V calls (one launch per direction).  The step holds `sets` independent
+    copies of the workload; step i converts copy i % sets, so a stream of steps never
+    finds its inputs in L2 (every copy is evicted by the others' traffic before it
+    comes round again)."""
 
-    def __init__(self, kvq, dev, batch, seed_shift=0):
+    def __init__(self, kvq, dev, batch, seed_shift=0, sets=STREAM_SETS):
         B, S, H, D = HEADLINE["shape"]
         shape = (batch, S, H, D)
-        k, v = workloads.fp8_window(seed=workloads.SEED_BASE + 2 + seed_shift, shape=shape, device=dev)
         self.kvq, self.batch = kvq, batch
-        self.k, self.v = k, v
-        self.k8 = torch.zeros(shape, dtype=torch.uint8, device=dev)
-        self.v8 = torch.zeros_like(self.k8)
-        self.ky = torch.zeros_like(k)
-        self.vy = torch.zeros_like(v)
+        self.sets = []
+        for r in range(sets):
+            k, v = workloads.fp8_window(seed=workloads.SEED_BASE + 2 + seed_shift + 100 * r, shape=shape,
+                                        device=dev)
+            self.sets.append(dict(k=k, v=v, k8=torch.zeros(shape, dtype=torch.uint8, device=dev),
+                                  v8=torch.zeros(shape, dtype=torch.uint8, device=dev),
+                                  ky=torch.zeros_like(k), vy=torch.zeros_like(v)))
+        first = self.sets[0]
+        self.set_bytes = sum(t.numel() * t.element_size() for t in first.values())
+        self.k, self.v, self.k8, self.v8, self.ky, self.vy = (first[n] for n in ("k", "v", "k8", "v8", "ky", "vy"))
         self.off, self.w = HEADLINE["offset"], HEADLINE["width"]
         self.elems_per_tensor = batch * self.w * H * D
         self.launch_bytes = BYTES_PER_ELEM["fp8"] * 2 * self.elems_per_tensor  # K and V
@@ -207,13 +224,24 @@ class Fp8Step:
         self.launches_per_step = 2
         self.names = ["fp16_to_fp8_kv", "fp8_to_fp16_kv"]
 
-    def run(self, ev=None):
-        """The two conversions; `ev` (1 event) marks the boundary between them."""
+    def launch(self, j, i=0):
+        """Launch j (0: encode, 1: decode) of step i alone."""
+        t = self.sets[i % len(self.sets)]
         kvq, b, o, w = self.kvq, self.batch, self.off, self.w
-        kvq.fp16_to_fp8_kv(self.k, self.k8, self.v, self.v8, b, o, w)
+        if j == 0:
+            kvq.fp16_to_fp8_kv(t["k"], t["k8"], t["v"], t["v8"], b, o, w)
+        else:
+            kvq.fp8_to_fp16_kv(t["k8"], t["ky"], t["v8"], t["vy"], b, o, w)
+
+    def run(self, i=0, ev=None):
+        """Step i (input copy i % sets); `ev`, if given, is an event recorded between
+        the two conversions."""
+        t = self.sets[i % len(self.sets)]
+        kvq, b, o, w = self.kvq, self.batch, self.off, self.w
+        kvq.fp16_to_fp8_kv(t["k"], t["k8"], t["v"], t["v8"], b, o, w)
         if ev is not None:
-            ev[0].record()
-        kvq.fp8_to_fp16_kv(self.k8, self.ky, self.v8, self.vy, b, o, w)
+            ev.record()
+        kvq.fp8_to_fp16_kv(t["k8"], t["ky"], t["v8"], t["vy"], b, o, w)
 
 
 def capture(fn, n_marks=0):
@@ -278,6 +306,93 @@ def _barrier():
         dist.barrier()
 
 
+def _stream_graph(launch, n):
+    """CUDA graph of steps 0..n-1 of `launch(i)`, back to back."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(n):
+            launch(i)
+    return g
+
+
+def time_stream(launch, sets, steps, warmup, flush, sampler=None, collective=True):
+    """Mean device time (ms) per step of `steps` consecutive steps, timed by one pair of
+    CUDA events around all of them.  Step i is launch(i); it converts input copy i % sets,
+    so no step finds its inputs in L2 (sets = 1 for workloads larger than L2).  The steps
+    are replayed from a CUDA graph of `sets` steps (plus one of steps % sets), L2 is
+    flushed once before the timed region, and with `collective` a barrier over all ranks
+    brackets it."""
+    cur = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+    side.wait_stream(cur)
+    with torch.cuda.stream(side):  # eager first calls (library set-up) before capture
+        for i in range(sets):
+            launch(i)
+    cur.wait_stream(side)
+    torch.cuda.synchronize()
+    full = _stream_graph(launch, sets)
+    tails = {n: _stream_graph(launch, n) for n in {steps % sets, warmup % sets} if n}
+
+    def run(n):
+        for _ in range(n // sets):
+            full.replay()
+        if n % sets:
+            tails[n % sets].replay()
+
+    run(warmup)
+    flush()
+    torch.cuda.synchronize()
+    if collective:
+        _barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.mark()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    run(steps)
+    e.record()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.mark()
+    if collective:
+        _barrier()
+    ms = s.elapsed_time(e) / steps
+    del full, tails
+    return ms
+
+
+def stream_shares(step, sets, reps=20):
+    """Fraction of a stream step taken by each of its two launches: the same stream with an
+    event between every two launches (captured in the graph), averaged over `reps` replays.
+    Event nodes serialize the launches, so only the proportions are used."""
+    n = sets
+    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * n + 1)]
+    cur = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+    side.wait_stream(cur)
+    with torch.cuda.stream(side):
+        for i in range(n):
+            step.run(i)
+    cur.wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(n):
+            evs[2 * i].record()
+            step.run(i, evs[2 * i + 1])
+        evs[2 * n].record()
+    seg = [0.0, 0.0]
+    for _ in range(reps):
+        g.replay()
+        torch.cuda.synchronize()
+        for i in range(n):
+            seg[0] += evs[2 * i].elapsed_time(evs[2 * i + 1])
+            seg[1] += evs[2 * i + 1].elapsed_time(evs[2 * i + 2])
+    del g
+    tot = seg[0] + seg[1]
+    return [x / tot for x in seg], [x / (reps * n) for x in seg]
+
+
 def e2e_fp8(kvq, step: Fp8Step, steps, warmup, dev):
     """Same step through the public API from pinned host buffers: H2D of the K/V windows,
     the four conversions, D2H of the decoded windows, all inside the CUDA events."""
@@ -311,33 +426,40 @@ def e2e_fp8(kvq, step: Fp8Step, steps, warmup, dev):
     return ms, 2 * win_bytes, 2 * win_bytes
 
 
-def per_op_measurements(kvq, dev, peak, steps, flush, include_model=True):
-    """Each remaining conversion on its own workload; mean CUDA-event time per launch."""
+def per_op_measurements(kvq, dev, peak, steps, flush, step, include_model=True):
+    """Each remaining conversion on its own workload.  Throughput rows time `steps`
+    consecutive launches (time_stream) on inputs larger than L2: workloads above the L2
+    size as they are, smaller ones rotating through independent input copies.  Rows
+    whose launch moves under a megabyte (paged decode, width 1) report the latency of one
+    launch on its own instead (L2 flushed before it, CUDA events around it)."""
     out = []
 
-    def record(name, config, nbytes, fn, n=steps):
-        per, _ = time_device(lambda ev: fn(), n, 3, flush, collective=False)
-        ms = statistics.mean(per)
+    def record(name, config, nbytes, launch, sets=1, n=steps):
+        if nbytes >= 1 << 20:
+            ms, timing = time_stream(launch, sets, n, 3, flush, collective=False), "stream"
+            if sets > 1:
+                timing += f", {sets} rotating input copies"
+        else:
+            per, _ = time_device(lambda ev: launch(0), n, 3, flush, collective=False)
+            ms, timing = statistics.mean(per), "isolated launch, L2 flushed"
         out.append({"op": name, "config": config, "bytes": int(nbytes), "us": round(ms * 1e3, 2),
-                    "gbs": round(nbytes / ms / 1e6, 1), "frac": round(nbytes / ms / 1e6 / peak, 3)})
+                    "gbs": round(nbytes / ms / 1e6, 1), "frac": round(nbytes / ms / 1e6 / peak, 3),
+                    "timing": timing})
 
     # the headline step through the page's single-tensor calls (4 launches instead of 2)
     B, S, H, D = HEADLINE["shape"]
     o, w = HEADLINE["offset"], HEADLINE["width"]
-    hk, hv = workloads.fp8_window(shape=(B, S, H, D), device=dev)
-    hk8, hv8 = torch.zeros(hk.shape, dtype=torch.uint8, device=dev), torch.zeros(hv.shape, dtype=torch.uint8, device=dev)
-    hky, hvy = torch.empty_like(hk), torch.empty_like(hv)
 
-    def per_tensor_step():
-        kvq.fp16_to_fp8(hk, hk8, B, o, w)
-        kvq.fp16_to_fp8(hv, hv8, B, o, w)
-        kvq.fp8_to_fp16(hk8, hky, B, o, w)
-        kvq.fp8_to_fp16(hv8, hvy, B, o, w)
+    def per_tensor_step(i):
+        t = step.sets[i % len(step.sets)]
+        kvq.fp16_to_fp8(t["k"], t["k8"], B, o, w)
+        kvq.fp16_to_fp8(t["v"], t["v8"], B, o, w)
+        kvq.fp8_to_fp16(t["k8"], t["ky"], B, o, w)
+        kvq.fp8_to_fp16(t["v8"], t["vy"], B, o, w)
     record("fp8_step_single_tensor_calls", "headline window, fp16_to_fp8(K), (V), fp8_to_fp16(K), (V): 4 launches",
-           4 * BYTES_PER_ELEM["fp8"] * B * w * H * D, per_tensor_step)
-    del hk, hv, hk8, hv8, hky, hvy
+           4 * BYTES_PER_ELEM["fp8"] * B * w * H * D, per_tensor_step, sets=len(step.sets))
 
-    # contiguous Q4 / Q6, channel outliers [16, 8192, 8, 128]
+    # contiguous Q4 / Q6 / Q8, channel outliers [16, 8192, 8, 128] (537 MB of FP16 K+V)
     k, v = workloads.channel_outliers(device=dev)
     B, S, H, D = k.shape
     n = 2 * k.numel()
@@ -350,22 +472,27 @@ def per_op_measurements(kvq, dev, peak, steps, flush, include_model=True):
         vs = torch.empty_like(ks)
         cfg = f"contiguous [16,8192,8,128] K+V wbits={wb}"
         record(f"fp16_to_q_kv/q{wb}", cfg, BYTES_PER_ELEM[wb] * n,
-               lambda: kvq.fp16_to_q_kv(k, kc, ks, v, vc, vs, B, 0, S, 0, None, None, wb))
+               lambda i: kvq.fp16_to_q_kv(k, kc, ks, v, vc, vs, B, 0, S, 0, None, None, wb))
         record(f"q_to_fp16_kv/q{wb}", cfg, BYTES_PER_ELEM[wb] * n,
-               lambda: kvq.q_to_fp16_kv(kc, ky, ks, vc, vy, vs, B, 0, S, 0, None, None, wb))
+               lambda i: kvq.q_to_fp16_kv(kc, ky, ks, vc, vy, vs, B, 0, S, 0, None, None, wb))
         del kc, vc, ks, vs
     # FP8 alone on the big tensor
     k8 = torch.empty(k.shape, dtype=torch.uint8, device=dev)
     record("fp16_to_fp8", "contiguous [16,8192,8,128] K", 3.0 * k.numel(),
-           lambda: kvq.fp16_to_fp8(k, k8, B, 0, S))
+           lambda i: kvq.fp16_to_fp8(k, k8, B, 0, S))
     record("fp8_to_fp16", "contiguous [16,8192,8,128] K", 3.0 * k.numel(),
-           lambda: kvq.fp8_to_fp16(k8, ky, B, 0, S))
+           lambda i: kvq.fp8_to_fp16(k8, ky, B, 0, S))
     del k, v, ky, vy, k8
     torch.cuda.empty_cache()
 
-    # paged Q4 decode / prefill on the 2048-page pool
+    # paged Q4 / FP8 decode and prefill on the 2048-page pool.  Input copy r of the
+    # prefill rows is the same pool read through a block table whose pages are shifted by
+    # 256 r (mod 2048): the windows land on other physical pages.
     pool = workloads.paged_pool(device=dev)
     P, ps, H, D = pool.k.shape
+    sets = STREAM_SETS
+    bts = [torch.where(pool.block_table >= 0, (pool.block_table + (P // sets) * r) % P, pool.block_table)
+           for r in range(sets)]
     cs, ss = kvq.q_shapes(tuple(pool.k.shape), 4)
     kc = torch.zeros(cs, dtype=torch.uint8, device=dev)
     vc = torch.zeros_like(kc)
@@ -374,40 +501,40 @@ def per_op_measurements(kvq, dev, peak, steps, flush, include_model=True):
     lens = pool.cache_seqlens.cpu()
     k8p, v8p = torch.zeros(pool.k.shape, dtype=torch.uint8, device=dev), torch.zeros(pool.k.shape, dtype=torch.uint8,
                                                                                     device=dev)
+    sl = pool.cache_seqlens
     for phase, off, w in (("decode", 0, 1), ("prefill", -512, 512)):
         npos = sum(max(0, int(L) + off + w) - max(0, int(L) + off) for L in lens)
         nb8 = BYTES_PER_ELEM["fp8"] * 2 * npos * H * D
         cfg8 = f"paged 2048x256x8x128 pool, 32 seqs, {phase} width={w}, K+V"
         record(f"fp16_to_fp8_kv/{phase}", cfg8, nb8,
-               lambda: kvq.fp16_to_fp8_kv(pool.k, k8p, pool.v, v8p, 32, off, w, ps, pool.cache_seqlens,
-                                          pool.block_table))
+               lambda i: kvq.fp16_to_fp8_kv(pool.k, k8p, pool.v, v8p, 32, off, w, ps, sl, bts[i % sets]), sets)
         record(f"fp8_to_fp16_kv/{phase}", cfg8, nb8,
-               lambda: kvq.fp8_to_fp16_kv(k8p, pool.k, v8p, pool.v, 32, off, w, ps, pool.cache_seqlens,
-                                          pool.block_table))
+               lambda i: kvq.fp8_to_fp16_kv(k8p, pool.k, v8p, pool.v, 32, off, w, ps, sl, bts[i % sets]), sets)
         nb = BYTES_PER_ELEM[4] * 2 * npos * H * D
         cfg = f"paged 2048x256x8x128 pool, 32 seqs, {phase} width={w}"
         record(f"fp16_to_q_kv/q4/{phase}", cfg, nb,
-               lambda: kvq.fp16_to_q_kv(pool.k, kc, ks, pool.v, vc, vs, 32, off, w, ps,
-                                        pool.cache_seqlens, pool.block_table, 4))
+               lambda i: kvq.fp16_to_q_kv(pool.k, kc, ks, pool.v, vc, vs, 32, off, w, ps, sl, bts[i % sets], 4),
+               sets)
         record(f"q_to_fp16_kv/q4/{phase}", cfg, nb,
-               lambda: kvq.q_to_fp16_kv(kc, pool.k, ks, vc, pool.v, vs, 32, off, w, ps,
-                                        pool.cache_seqlens, pool.block_table, 4))
+               lambda i: kvq.q_to_fp16_kv(kc, pool.k, ks, vc, pool.v, vs, 32, off, w, ps, sl, bts[i % sets], 4),
+               sets)
     del kc, vc, ks, vs, k8p, v8p
     torch.cuda.empty_cache()
 
     # decode attention straight from the quantized pool: 32 sequences, 32 query heads
-    # (4 per kv head), one new token each, every cached position attended
+    # (4 per kv head), one new token each, every cached position attended (>= 280 MB of
+    # codes and scales per launch)
     for wb in (4, 6, 8):
         fn, nb = attention_setup(kvq, dev, pool, wb)
         record(f"decode_attention_q/q{wb}/paged",
-               f"paged 2048x256x8x128 pool, 32 seqs, 32 query heads, wbits={wb}", nb, fn)
+               f"paged 2048x256x8x128 pool, 32 seqs, 32 query heads, wbits={wb}", nb, lambda i: fn())
         del fn
         torch.cuda.empty_cache()
     del pool
     torch.cuda.empty_cache()
 
     if include_model:
-        out.extend(model_layers(kvq, dev, peak, max(3, steps // 10), flush))
+        out.extend(model_layers(kvq, dev, peak, min(20, max(3, steps // 10)), flush))
     return out
 
 
@@ -477,10 +604,9 @@ def model_layers(kvq, dev, peak, steps, flush, layers=32):
     res = []
     cfg = "paged Q6, 32 layers x K/V 8x32768x8x128, page 256, shuffled block_table"
     for name, fn in (("q_to_fp16_kv/q6/model32", deq), ("fp16_to_q_kv/q6/model32", qnt)):
-        per, _ = time_device(lambda ev: fn(), steps, 2, flush, collective=False)
-        ms = statistics.mean(per)
+        ms = time_stream(lambda i: fn(), 1, steps, 3, flush, collective=False)
         res.append({"op": name, "config": cfg, "bytes": int(nb), "us": round(ms * 1e3, 1),
-                    "gbs": round(nb / ms / 1e6, 1), "frac": round(nb / ms / 1e6 / peak, 3)})
+                    "gbs": round(nb / ms / 1e6, 1), "frac": round(nb / ms / 1e6 / peak, 3), "timing": "stream"})
     del L
     torch.cuda.empty_cache()
     return res
@@ -611,7 +737,7 @@ def oracle_step_sample(batch=4, max_seconds=12.0, min_reps=1):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-per-op", action="store_true", help="skip the per-op table")
@@ -658,30 +784,34 @@ def main():
     # each rank converts its own 4 sequences: a global batch of 4 * world (weak scaling)
     batch = HEADLINE["shape"][0]
     step = Fp8Step(kvq, dev, batch, seed_shift=rank)
-    # timed region: the step graph replayed as it is (no event nodes inside it)
-    per_step, _ = time_device(step.run, args.steps, args.warmup, flush, sampler)
-    ms_local = statistics.mean(per_step)
+    # timed region: `steps` consecutive steps over rotating input copies (inputs larger
+    # than L2), one pair of CUDA events around all of them, max over ranks
+    ms_local = time_stream(step.run, len(step.sets), args.steps, args.warmup, flush, sampler)
     ms = max_over_ranks(ms_local, dev)
-    # per-launch durations: the same graph with events between its launches
-    _, segs = time_device(step.run, max(50, args.steps // 10), 3, flush, None, n_marks=1)
+    # per-launch durations inside the step: the step time split in the proportions of an
+    # event-marked pass; the dominant launch is then timed on its own, as a stream of
+    # `steps` launches of it over the same rotating input copies
+    share, seg_ms = stream_shares(step, len(step.sets))
     names = step.names
-    seg_ms = [statistics.mean(s[i] for s in segs) for i in range(2)]
-    # Event nodes between launches cost time of their own, so each launch's duration
-    # inside the timed (unmarked) step is the step time split in the proportions of
-    # the marked segments.
-    share = [t / sum(seg_ms) for t in seg_ms]
     launch_ms = [ms_local * f for f in share]
     dom_i = 0 if launch_ms[0] >= launch_ms[1] else 1
-    dom = (names[dom_i], launch_ms[dom_i])
+    dom_ms = time_stream(lambda i: step.launch(dom_i, i), len(step.sets), args.steps, args.warmup, flush,
+                         collective=False)
+    dom = (names[dom_i], dom_ms)
     achieved = step.launch_bytes / dom[1] / 1e6
-    dom_isolated_ms = seg_ms[dom_i]
+    # one step on its own (L2 flushed before it, CUDA events around it): the latency of a
+    # single isolated call, launch and event overhead included
+    iso, iso_segs = time_device(lambda ev: step.run(0, ev[0] if ev else None), 200, 5, flush, None, n_marks=1,
+                                collective=False)
+    iso_ms = statistics.mean(iso)
+    iso_seg_ms = [statistics.mean(x[i] for x in iso_segs) for i in range(2)]
 
     e2e_ms, h2d, d2h = e2e_fp8(kvq, step, max(10, args.steps // 10), 3, dev)
     e2e_ms = max_over_ranks(e2e_ms, dev)
 
     per_op = []
     if world == 1 and not args.no_per_op:
-        per_op = per_op_measurements(kvq, dev, peak, max(20, args.steps // 5), flush,
+        per_op = per_op_measurements(kvq, dev, peak, min(200, max(20, args.steps // 5)), flush, step,
                                      include_model=not args.no_model)
     if sampler:
         sampler.stop()
@@ -716,20 +846,30 @@ def main():
         "config": {"workload": HEADLINE["workload"], "shape": list(HEADLINE["shape"]),
                    "global_batch": batch * world, "offset": HEADLINE["offset"], "width": HEADLINE["width"],
                    "ops": ["fp16_to_fp8 of K and V (one fused launch)", "fp8_to_fp16 of K and V (one fused launch)"],
-                   "launch": "CUDA graph of the 2 fused K+V conversions, replayed once per step", "l2": "flushed between steps (256 MiB write + 256 MiB read, outside the per-step events)",
+                   "launch": f"{args.steps} consecutive steps (2 fused K+V launches each) replayed from CUDA graphs, "
+                             "one pair of CUDA events around them",
+                   "l2": f"inputs larger than L2: step i converts input copy i % {len(step.sets)} "
+                         f"({len(step.sets)} x {step.set_bytes / 1e6:.0f} MB), L2 flushed once before the timed steps",
                    "parallelism": f"replicas x{world}, each rank its own 4 sequences"},
         "roofline": {"bound": "hbm", "kernel": dom[0], "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 3), "peak_kind": peak_kind,
                      "bytes_per_launch": int(step.launch_bytes), "us_per_launch": round(dom[1] * 1e3, 2),
-                     "duration": "timed step x this launch's share of the event-marked step",
-                     "us_per_launch_marked": round(dom_isolated_ms * 1e3, 2),
+                     "duration": f"CUDA events around {args.steps} back-to-back launches of this kernel alone, "
+                                 "rotating through the same input copies as the step",
+                     "us_per_launch_in_step": round(launch_ms[dom_i] * 1e3, 2),
+                     "in_step": "timed step time x this launch's share of an event-marked pass of the same stream",
                      "traffic": recorded_traffic(dom[0])},
         "per_kernel_us": {n: round(t * 1e3, 2) for n, t in zip(names, launch_ms)},
         "per_kernel_us_marked": {n: round(t * 1e3, 2) for n, t in zip(names, seg_ms)},
+        "isolated": {"us_per_step": round(iso_ms * 1e3, 2),
+                     "per_kernel_us": {n: round(t * 1e3, 2) for n, t in zip(names, iso_seg_ms)},
+                     "gbs": round(step.bytes_per_step / iso_ms / 1e6, 1),
+                     "how": "one step at a time: L2 flushed, CUDA events around the step's graph and "
+                            "between its launches (includes ~6 us of event and launch overhead)"},
         "cpu_baseline": cpu,
         "e2e": {"value": round(world * step.bytes_per_step / e2e_ms / 1e6, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": step.launches_per_step * args.steps,
+        "gpu_launches": step.launches_per_step * args.steps,  # in the timed region
         "clocks": sampler.summary() if sampler else None,
         "per_op": per_op,
     }
@@ -737,9 +877,15 @@ def main():
     return 0
 
 
+REF_SECONDS = 60.0  # the reference arm's timed steps take about this long in all
+
+
 def run_reference(args):
-    """The CPU oracle as the reference arm: each step = the headline step on batch 1 (one of the
-    four sequences), single-threaded, on this host."""
+    """The CPU oracle as the reference arm: each step is a bounded sample of the headline
+    step, FP8 encode + decode of K and V over the first n positions of one sequence's
+    window, single-threaded, on this host; n (a multiple of 16, at most the window) is
+    chosen from a calibration step so that the `steps` timed steps take about
+    REF_SECONDS."""
     import numpy as np
 
     import oracle
@@ -752,9 +898,19 @@ def run_reference(args):
     k8, v8 = np.zeros(kn.shape, np.uint8), np.zeros(vn.shape, np.uint8)
     ky, vy = np.zeros(kn.shape, np.uint16), np.zeros(vn.shape, np.uint16)
 
+    def once_n(n):
+        oracle.fp16_to_fp8_kv(kn, k8, vn, v8, 1, o, n)
+        oracle.fp8_to_fp16_kv(k8, ky, v8, vy, 1, o, n)
+
+    t0 = time.perf_counter()
+    once_n(16)
+    per_pos = (time.perf_counter() - t0) / 16
+    n = int(REF_SECONDS / max(1, args.steps) / per_pos) // 16 * 16
+    n = max(16, min(w, n))
+
     def once():
-        oracle.fp16_to_fp8_kv(kn, k8, vn, v8, 1, o, w)
-        oracle.fp8_to_fp16_kv(k8, ky, v8, vy, 1, o, w)
+        oracle.fp16_to_fp8_kv(kn, k8, vn, v8, 1, o, n)
+        oracle.fp8_to_fp16_kv(k8, ky, v8, vy, 1, o, n)
 
     for _ in range(args.warmup):
         once()
@@ -762,9 +918,9 @@ def run_reference(args):
     for _ in range(args.steps):
         once()
     dt = (time.perf_counter() - t0) / args.steps
-    nbytes = 4 * BYTES_PER_ELEM["fp8"] * w * H * D
+    nbytes = 4 * BYTES_PER_ELEM["fp8"] * n * H * D
     value = nbytes / dt / 1e9
-    sample = f"batch 1 of 4 per step (window {o}..{o + w}, K and V, encode + decode)"
+    sample = f"per step: positions {o}..{o + n} of one of the 4 sequences (of the window {o}..{o + w}), K and V, encode + decode"
     line = {
         "impl": "reference",
         "metric": "KV-cache convert GB/s (read+write), FP8 E5M2 encode+decode of K and V",

@@ -150,18 +150,48 @@ kvq_status launch_pdl(Kernel kernel, dim3 grid, int threads, int smem, void* str
   return launch_status();
 }
 
-template <class Op>
-kvq_status launch_ldg(Params p, int nkv, void* stream) {
+// CTAs of `kernel` that the current device holds at once (SMs x resident
+// CTAs per SM), cached per device in `cache`; 0 if it cannot be queried.
+template <class Kernel>
+long long first_wave_ctas(Kernel kernel, int threads, std::atomic<long long>* cache, int max_devices) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= max_devices) {
+    cudaGetLastError();
+    return 0;
+  }
+  long long n = cache[dev].load();
+  if (n == 0) {
+    int sms = 0, per_sm = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    n = static_cast<long long>(sms) * per_sm;
+    cache[dev].store(n);
+  }
+  return n;
+}
+
+template <class Op, bool kPaged>
+kvq_status launch_ldg_mode(Params p, int nkv, void* stream) {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<long long> wave[kMaxDevices];
+  p.prefetch_ctas = first_wave_ctas(convert_kernel<Op, kPaged>, LdgCfg<Op>::kThreads, wave, kMaxDevices);
   // Paged tiles are four CTA rounds long: each CTA pays one block-table lookup
   // before its first data load, and a longer tile amortizes it.
-  const long long target = static_cast<long long>(ldg_tile_elems<Op>()) * (p.g.page_size > 0 ? 4 : 1);
+  const long long target = static_cast<long long>(ldg_tile_elems<Op>()) * (kPaged ? 4 : 1);
   p.g.tile_pos = pick_tile_pos(p.g.hd, p.g.page_size, target);
-  const int paged = p.g.page_size > 0;
-  const long long tiles = (static_cast<long long>(p.g.width) + p.g.tile_pos - 1) / p.g.tile_pos + paged;
+  const long long tiles = (static_cast<long long>(p.g.width) + p.g.tile_pos - 1) / p.g.tile_pos + (kPaged ? 1 : 0);
   if (tiles > 0x7FFFFFFFLL) return KVQ_ERR_RANGE;
   const dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(p.g.batch < 65535 ? p.g.batch : 65535),
                   static_cast<unsigned>(nkv));
-  return launch_pdl(convert_kernel<Op>, grid, LdgCfg<Op>::kThreads, 0, stream, p);
+  return launch_pdl(convert_kernel<Op, kPaged>, grid, LdgCfg<Op>::kThreads, 0, stream, p);
+}
+
+template <class Op>
+kvq_status launch_ldg(const Params& p, int nkv, void* stream) {
+  return p.g.page_size > 0 ? launch_ldg_mode<Op, true>(p, nkv, stream) : launch_ldg_mode<Op, false>(p, nkv, stream);
 }
 
 // The bulk engine needs every tile of the input stream 16-byte aligned and a

@@ -33,24 +33,71 @@ constexpr int ldg_tile_elems() {
   return LdgCfg<Op>::kThreads * LdgCfg<Op>::kUnroll * LdgCfg<Op>::kUnitElems;
 }
 
-template <class Op>
+__device__ __forceinline__ void prefetch_l2_range(const void* base, long long bytes, int tid, int nthreads) {
+  if (bytes <= 0) return;
+  const char* b = static_cast<const char*>(base);
+  for (long long off = static_cast<long long>(tid) * 128; off < bytes; off += static_cast<long long>(nthreads) * 128)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(b + off));
+  if (tid == 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(b + bytes - 1));
+}
+
+// Ask L2 for the input bytes of this CTA's first round of loads before
+// waiting on the previous grid, so that this grid's DRAM reads start while the
+// previous one drains.  Only CTAs of the first wave (those that can be
+// resident before the previous grid ends) do it; later CTAs start after it
+// has finished anyway.  A prefetch only fills L2, which is also where every
+// write of the previous grid lands, so it can never make a later load see
+// stale data.  Paged tiles need the sequence length and the block-table
+// entry: warp 0 reads them at L2 (bypassing L1, which other SMs' writes do
+// not refresh), and since they may be stale they only steer the hint; the
+// page index is range checked, so every prefetched address lies inside the
+// cache.
+template <class Op, bool kPaged>
+__device__ __forceinline__ void prefetch_first_round(const Params& p, int kv) {
+  using C = LdgCfg<Op>;
+  const long long cta =
+      blockIdx.x + static_cast<long long>(gridDim.x) * (blockIdx.y + static_cast<long long>(gridDim.y) * blockIdx.z);
+  const int seq = blockIdx.y;
+  if (cta >= p.prefetch_ctas || seq >= p.g.batch) return;
+  long long row0 = 0;
+  int nrows = 0;
+  int tid = threadIdx.x, nthreads = C::kThreads;
+  if (!kPaged) {
+    if (!contiguous_tile(p.g, seq, blockIdx.x, row0, nrows)) return;
+  } else {
+    if (threadIdx.x >= 32) return;
+    nthreads = 32;
+    if (!paged_tile(p.g, seq, blockIdx.x, __ldcg(p.g.seqlens + seq), nullptr, false, row0, nrows, true)) return;
+  }
+  const long long elems = min(static_cast<long long>(nrows) * p.g.hd, static_cast<long long>(ldg_tile_elems<Op>()));
+  prefetch_l2_range(static_cast<const uint8_t*>(p.in[kv]) + row0 * p.g.hd * Op::kInNum / Op::kInDen,
+                    elems * Op::kInNum / Op::kInDen, tid, nthreads);
+  if (Op::kReadsScales)
+    prefetch_l2_range(static_cast<const __half*>(p.scales[kv]) + row0 * p.g.hd / kBlockElems,
+                      elems / kBlockElems * 2, tid, nthreads);
+}
+
+// One instantiation per mode: contiguous grids carry no paging code at all.
+template <class Op, bool kPaged>
 __global__ void __launch_bounds__(LdgCfg<Op>::kThreads, LdgCfg<Op>::kMinBlocksPerSM)
     convert_kernel(const __grid_constant__ Params p) {
   using C = LdgCfg<Op>;
+  prefetch_first_round<Op, kPaged>(p, blockIdx.z);
   // Programmatic dependent launch: this grid may be launched while the
   // previous kernel on the stream is still running; wait for it to finish (and
-  // its writes to become visible) before touching global memory, and let the
-  // next kernel start launching as soon as every CTA of this grid has started.
+  // its writes to become visible) before loading anything it may have written,
+  // and let the next kernel start launching as soon as every CTA of this grid
+  // has started.
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  __shared__ int s_bt[C::kThreads];
+  __shared__ int s_bt[kPaged ? C::kThreads : 1];
   __shared__ int s_seqlen;
   const int kv = blockIdx.z;
   for (int seq = blockIdx.y; seq < p.g.batch; seq += gridDim.y) {
     long long row0 = 0;
     int nrows = 0;
     bool ok;
-    if (p.g.page_size == 0) {
+    if (!kPaged) {
       ok = contiguous_tile(p.g, seq, blockIdx.x, row0, nrows);
     } else {
       // Stage the sequence's block-table row (when it fits) together with its

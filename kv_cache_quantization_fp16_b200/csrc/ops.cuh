@@ -31,6 +31,7 @@ struct SharedSrc {
 // FP8 encode: 8 binary16 (16 bytes) in, 8 bytes out per thread step.
 struct Fp8Encode {
   static constexpr int kInNum = 2, kInDen = 1;  // input bytes per element
+  static constexpr bool kReadsScales = false;
   template <class Src, int NT, int U>
   __device__ static void body(const Params& p, int kv, long long row0, int nrows, const void* in, int tid) {
     const long long e0 = row0 * p.g.hd;
@@ -56,6 +57,7 @@ struct Fp8Encode {
 // FP8 decode: 8 bytes in, 8 binary16 out per thread step.
 struct Fp8Decode {
   static constexpr int kInNum = 1, kInDen = 1;
+  static constexpr bool kReadsScales = false;
   template <class Src, int NT, int U>
   __device__ static void body(const Params& p, int kv, long long row0, int nrows, const void* in, int tid) {
     const long long e0 = row0 * p.g.hd;
@@ -85,6 +87,7 @@ struct Fp8Decode {
 template <int B>
 struct QEncode {
   static constexpr int kInNum = 2, kInDen = 1;
+  static constexpr bool kReadsScales = false;
   template <class Src, int NT, int U>
   __device__ static void body(const Params& p, int kv, long long row0, int nrows, const void* in, int tid) {
     const long long e0 = row0 * p.g.hd;
@@ -139,6 +142,7 @@ struct QEncode {
 template <int B>
 struct QDecode {
   static constexpr int kInNum = B, kInDen = 8;
+  static constexpr bool kReadsScales = true;
   template <class Src, int NT, int U>
   __device__ static void body(const Params& p, int kv, long long row0, int nrows, const void* in, int tid) {
     const long long e0 = row0 * p.g.hd;

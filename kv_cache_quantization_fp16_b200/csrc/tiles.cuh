@@ -51,8 +51,10 @@ __device__ __forceinline__ bool contiguous_tile(const Geometry& g, int seq, int 
 // one page).  `bt_row` is the sequence's block-table row staged in shared
 // memory (or null: read it from global memory).  Bad metadata is recorded by
 // the thread with `report` set and the tile is skipped.
+// With `l2_only` the block-table entry is read at L2 (bypassing L1).
 __device__ __forceinline__ bool paged_tile(const Geometry& g, int seq, int tile_x, int seqlen,
-                                           const int* bt_row, bool report, long long& row0, int& nrows) {
+                                           const int* bt_row, bool report, long long& row0, int& nrows,
+                                           bool l2_only = false) {
   const long long start = static_cast<long long>(seqlen) + g.offset;
   const long long lo = start < 0 ? 0 : start;
   const long long hi = start + g.width;
@@ -66,7 +68,8 @@ __device__ __forceinline__ bool paged_tile(const Geometry& g, int seq, int tile_
     if (report) record_error(KVQ_DEV_BAD_PAGE_INDEX);
     return false;
   }
-  const int page = bt_row ? bt_row[lp] : g.block_table[static_cast<long long>(seq) * g.bt_stride + lp];
+  const int32_t* entry = g.block_table + static_cast<long long>(seq) * g.bt_stride + lp;
+  const int page = bt_row ? bt_row[lp] : (l2_only ? __ldcg(entry) : *entry);
   if (page < 0 || page >= g.dim0) {
     if (report) record_error(KVQ_DEV_BAD_PAGE);
     return false;
@@ -81,6 +84,9 @@ struct Params {
   const void* in[2];
   void* out[2];
   void* scales[2];  // Q encode: written; Q decode: read
+  // CTAs (in launch order) that can be resident while the previous grid on the
+  // stream is still draining: only they prefetch before the dependency wait.
+  long long prefetch_ctas;
 };
 
 }  // namespace kvq

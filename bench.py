@@ -315,31 +315,37 @@ def _stream_graph(launch, n):
     return g
 
 
-def time_stream(launch, sets, steps, warmup, flush, sampler=None, collective=True):
+def time_stream(launch, sets, steps, warmup, flush, sampler=None, collective=True, chunk=None):
     """Mean device time (ms) per step of `steps` consecutive steps, timed by one pair of
     CUDA events around all of them.  Step i is launch(i); it converts input copy i % sets,
     so no step finds its inputs in L2 (sets = 1 for workloads larger than L2).  The steps
-    are replayed from a CUDA graph of `sets` steps (plus one of steps % sets), L2 is
-    flushed once before the timed region, and with `collective` a barrier over all ranks
-    brackets it."""
+    are replayed from CUDA graphs of `chunk` steps (a multiple of `sets`; about 256 by
+    default, so that graph boundaries, which break the chaining of launches, are rare),
+    plus one graph for the remainder.  L2 is flushed once before the timed region, and
+    with `collective` a barrier over all ranks brackets it."""
+    if chunk is None:
+        chunk = sets * max(1, 256 // sets)
     cur = torch.cuda.current_stream()
     side = torch.cuda.Stream()
     side.wait_stream(cur)
-    with torch.cuda.stream(side):  # eager first calls (library set-up) before capture
-        for i in range(sets):
+    eager = min(warmup, sets)  # the first warm-up steps run eagerly, so first-call set-up precedes capture
+    with torch.cuda.stream(side):
+        for i in range(eager):
             launch(i)
     cur.wait_stream(side)
     torch.cuda.synchronize()
-    full = _stream_graph(launch, sets)
-    tails = {n: _stream_graph(launch, n) for n in {steps % sets, warmup % sets} if n}
+    graphs = {}
 
     def run(n):
-        for _ in range(n // sets):
-            full.replay()
-        if n % sets:
-            tails[n % sets].replay()
+        for m in [chunk] * (n // chunk) + ([n % chunk] if n % chunk else []):
+            if m not in graphs:
+                graphs[m] = _stream_graph(launch, m)
+            graphs[m].replay()
 
-    run(warmup)
+    run(warmup - eager)
+    for m in {chunk if steps >= chunk else 0, steps % chunk} - {0}:  # capture before timing
+        if m not in graphs:
+            graphs[m] = _stream_graph(launch, m)
     flush()
     torch.cuda.synchronize()
     if collective:
@@ -357,7 +363,7 @@ def time_stream(launch, sets, steps, warmup, flush, sampler=None, collective=Tru
     if collective:
         _barrier()
     ms = s.elapsed_time(e) / steps
-    del full, tails
+    graphs.clear()
     return ms
 
 
@@ -604,7 +610,7 @@ def model_layers(kvq, dev, peak, steps, flush, layers=32):
     res = []
     cfg = "paged Q6, 32 layers x K/V 8x32768x8x128, page 256, shuffled block_table"
     for name, fn in (("q_to_fp16_kv/q6/model32", deq), ("fp16_to_q_kv/q6/model32", qnt)):
-        ms = time_stream(lambda i: fn(), 1, steps, 3, flush, collective=False)
+        ms = time_stream(lambda i: fn(), 1, steps, 3, flush, collective=False, chunk=1)
         res.append({"op": name, "config": cfg, "bytes": int(nb), "us": round(ms * 1e3, 1),
                     "gbs": round(nb / ms / 1e6, 1), "frac": round(nb / ms / 1e6 / peak, 3), "timing": "stream"})
     del L

@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(kBulkThreads, 1)
     if (!mbar_wait(&full_bar[s], static_cast<uint32_t>((it / kBulkStages) & 1), &abort_flag)) break;
     const long long row0 = meta_row0[s];
     if (row0 >= 0) {
-      Op::template body<SharedSrc, kBulkConsumers, BulkCfg<Op>::kUnroll>(p, meta_kv[s], row0, meta_nrows[s],
+      Op::template body<SharedSrc, kBulkConsumers, BulkCfg<Op>::kUnroll, false>(p, meta_kv[s], row0, meta_nrows[s],
                                                                            stage_mem + s * kBulkStageBytes, ctid);
     }
     __syncwarp();

@@ -9,8 +9,10 @@
 //
 // Each body is templated on where its main input stream is read from (`Src`:
 // global memory through the non-coherent path, or a shared-memory copy of
-// the tile), on the number of threads that share the tile (NT) and on how
-// many independent loads each thread issues before it computes (U).
+// the tile), on the number of threads that share the tile (NT), on how many
+// independent loads each thread issues before it computes (U: one round of
+// loads), and on whether each round asks L2 for the next round's input
+// (kPf, for tiles of several rounds read from global memory).
 #pragma once
 
 #include "codec.cuh"
@@ -19,26 +21,52 @@
 namespace kvq {
 
 struct GlobalSrc {
+  static constexpr bool kGlobal = true;
   template <class T>
   __device__ __forceinline__ static T load(const T* p) { return __ldg(p); }
 };
 
 struct SharedSrc {
+  static constexpr bool kGlobal = false;
   template <class T>
   __device__ __forceinline__ static T load(const T* p) { return *p; }
 };
+
+// L2 prefetch of `bytes` bytes from `base`: one 128-byte line per thread and
+// step (plus the last byte, so a range that starts mid-line is covered).
+__device__ __forceinline__ void prefetch_l2_range(const void* base, long long bytes, int tid, int nthreads) {
+  if (bytes <= 0) return;
+  const char* b = static_cast<const char*>(base);
+  for (long long off = static_cast<long long>(tid) * 128; off < bytes; off += static_cast<long long>(nthreads) * 128)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(b + off));
+  if (tid == 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(b + bytes - 1));
+}
+
+// In a tile of several rounds (paged tiles), ask L2 for the next round's
+// input units [next, next + per_round) while this round is converted, so that
+// DRAM keeps streaming between the rounds of a CTA.  Units are `unit_bytes`
+// apart in the input stream.  A prefetch never changes what a load returns.
+template <bool kOn>
+__device__ __forceinline__ void prefetch_next_round(const void* in, int unit_bytes, int next, int total,
+                                                    int per_round, int tid, int nt) {
+  if (!kOn || next >= total) return;
+  const int units = min(per_round, total - next);
+  prefetch_l2_range(static_cast<const uint8_t*>(in) + static_cast<long long>(next) * unit_bytes,
+                    static_cast<long long>(units) * unit_bytes, tid, nt);
+}
 
 // FP8 encode: 8 binary16 (16 bytes) in, 8 bytes out per thread step.
 struct Fp8Encode {
   static constexpr int kInNum = 2, kInDen = 1;  // input bytes per element
   static constexpr bool kReadsScales = false;
-  template <class Src, int NT, int U>
+  template <class Src, int NT, int U, bool kPf>
   __device__ static void body(const Params& p, int kv, long long row0, int nrows, const void* in, int tid) {
     const long long e0 = row0 * p.g.hd;
     const uint4* src = static_cast<const uint4*>(in);
     uint2* dst = reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.out[kv]) + e0);
     const int nvec = static_cast<int>(nrows * p.g.hd / 8);
     for (int base = 0; base < nvec; base += NT * U) {
+      prefetch_next_round<kPf>(in, 16, base + NT * U, nvec, NT * U, tid, NT);
       uint4 x[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -58,13 +86,14 @@ struct Fp8Encode {
 struct Fp8Decode {
   static constexpr int kInNum = 1, kInDen = 1;
   static constexpr bool kReadsScales = false;
-  template <class Src, int NT, int U>
+  template <class Src, int NT, int U, bool kPf>
   __device__ static void body(const Params& p, int kv, long long row0, int nrows, const void* in, int tid) {
     const long long e0 = row0 * p.g.hd;
     const uint2* src = static_cast<const uint2*>(in);
     uint4* dst = reinterpret_cast<uint4*>(static_cast<__half*>(p.out[kv]) + e0);
     const int nvec = static_cast<int>(nrows * p.g.hd / 8);
     for (int base = 0; base < nvec; base += NT * U) {
+      prefetch_next_round<kPf>(in, 8, base + NT * U, nvec, NT * U, tid, NT);
       uint2 x[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -88,7 +117,7 @@ template <int B>
 struct QEncode {
   static constexpr int kInNum = 2, kInDen = 1;
   static constexpr bool kReadsScales = false;
-  template <class Src, int NT, int U>
+  template <class Src, int NT, int U, bool kPf>
   __device__ static void body(const Params& p, int kv, long long row0, int nrows, const void* in, int tid) {
     const long long e0 = row0 * p.g.hd;
     const uint4* src = static_cast<const uint4*>(in);
@@ -96,6 +125,7 @@ struct QEncode {
     __half* scales = static_cast<__half*>(p.scales[kv]) + e0 / kBlockElems;
     const int nblk = static_cast<int>(nrows * p.g.hd / kBlockElems);
     for (int base = 0; base < nblk; base += NT * U) {
+      prefetch_next_round<kPf>(in, 64, base + NT * U, nblk, NT * U, tid, NT);
       uint4 x[U][4];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -143,7 +173,7 @@ template <int B>
 struct QDecode {
   static constexpr int kInNum = B, kInDen = 8;
   static constexpr bool kReadsScales = true;
-  template <class Src, int NT, int U>
+  template <class Src, int NT, int U, bool kPf>
   __device__ static void body(const Params& p, int kv, long long row0, int nrows, const void* in, int tid) {
     const long long e0 = row0 * p.g.hd;
     const uint8_t* codes = static_cast<const uint8_t*>(in);
@@ -151,6 +181,8 @@ struct QDecode {
     uint4* dst = reinterpret_cast<uint4*>(static_cast<__half*>(p.out[kv]) + e0);
     const int nvec = static_cast<int>(nrows * p.g.hd / 8);
     for (int base = 0; base < nvec; base += NT * U) {
+      prefetch_next_round<kPf>(in, B, base + NT * U, nvec, NT * U, tid, NT);  // codes: B bytes per 8 elements
+      prefetch_next_round<kPf>(scales, 2, (base + NT * U) / 4, nvec / 4, NT * U / 4, tid, NT);
       uint32_t lo[U], hi[U];
       __half s[U];
 #pragma unroll

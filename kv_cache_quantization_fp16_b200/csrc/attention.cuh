@@ -5,28 +5,36 @@
 //
 // One new query per sequence and head; GQA: `group` query heads share a kv
 // head.  Keys and values are the dequantized codes, bit for bit what
-// q_to_fp16_kv writes (dequantized in registers with the same arithmetic).
+// q_to_fp16_kv writes: RN16((code - z) * s), with (code - z) formed exactly
+// in binary16 and one rounding in the multiply.
 //
 // Split-K flash decoding.  Kernel 1 (attn_partial_kernel): one CTA per
-// (chunk of positions, kv head, sequence), four warps.  The CTA first copies
-// its whole chunk of K and V codes and scales into shared memory with
-// cp.async (all copies in flight at once, so a CTA keeps tens of KB of
-// loads outstanding), then each warp takes 16 positions at a time and
-//   * dequantizes K for the 16 positions into mma.sync m16n8k16 A fragments
-//     (positions are the M dimension, the query heads of the group the N
-//     dimension, padded to 8), multiplies by the preloaded query fragments
-//     (fp16 inputs, fp32 accumulation: products are exact);
-//   * updates an online softmax (base 2) per query head;
-//   * dequantizes V for the 16 positions into A fragments of O^T = V^T P^T
-//     (head_dim is the M dimension) and accumulates with P split into a
-//     binary16 high part and a binary16 residual (two MMAs), so the weights
-//     keep about 22 significant bits.
-// The head_dim order inside a fragment is permuted so that every lane's
-// slice of a cache row is contiguous (one wide load, one scale); the query
-// and the output use the same permutation.  The four warps' states merge
-// in shared memory and the chunk's (max, sum, accumulator) goes to the
-// workspace.  Kernel 2 (attn_combine_kernel) merges the chunks of each
-// (sequence, head) and writes binary16 outputs.
+// (chunk of positions, kv head, sequence), four warps.  The CTA copies its
+// whole chunk of K and V codes and scales into shared memory with cp.async
+// (every copy in flight at once), then each warp takes 16 positions at a
+// time:
+//   * S = Q K^T on mma.sync m16n8k16 with the query heads as the M dimension
+//     (rows >= group are zero) and 8 positions per N tile: each lane
+//     dequantizes one contiguous span of D/4 elements of one position (a B
+//     fragment needs 4 head_dim elements per k-step, and the head_dim order
+//     inside the MMA is permuted so that a lane's elements over all k-steps
+//     are that span); the query fragments use the same permutation;
+//   * online softmax (base 2) per query head with lazy rescaling: the
+//     reference maximum only moves when a score exceeds it by more than
+//     kAttnRescaleLog2, so the accumulators are rarely touched and every
+//     weight stays below 2^kAttnRescaleLog2;
+//   * O^T += V^T P^T: the S accumulators of two N tiles are exactly the B
+//     fragment of P^T for a 16-position k-step (no data movement); P is split
+//     into a binary16 high part and a binary16 residual (two MMAs), so the
+//     weights keep about 22 significant bits; V^T A fragments pair two
+//     positions at one head_dim index, built by interleaving the bytes of two
+//     rows before the codes are unpacked.
+// Code unpacking avoids per-code shifts: `(w & 0x000F000F) | 0x64006400` is
+// the binary16 pair (1024 + c0, 1024 + c4) of a Q4 word, and the high-nibble
+// pair is 16x that, brought back exactly with an FMA by 1/16.
+// The four warps' states merge in shared memory and the chunk's (max, sum,
+// accumulator) goes to the workspace.  Kernel 2 (attn_combine_kernel) merges
+// the chunks of each (sequence, head) and writes binary16 outputs.
 #pragma once
 
 #include "codec.cuh"
@@ -36,7 +44,8 @@ namespace kvq {
 
 constexpr int kAttnWarps = 4;
 constexpr int kAttnThreads = 32 * kAttnWarps;
-constexpr int kAttnMaxGroup = 8;  // query heads per kv head (one MMA N block)
+constexpr int kAttnMaxGroup = 8;        // query heads per kv head (one MMA N block of P^T)
+constexpr float kAttnRescaleLog2 = 8.0f;  // lazy-rescale threshold (log2 units)
 
 struct AttnParams {
   const __half* q;  // [batch, n_heads, D]
@@ -53,12 +62,13 @@ struct AttnParams {
   float scale_log2;  // softmax_scale * log2(e)
 };
 
-__device__ __forceinline__ void mma_16816(float c[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
+__device__ __forceinline__ void mma_16816(float c[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};\n"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
@@ -66,24 +76,206 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Shared-memory staging of one CTA's chunk: K codes, V codes (rows padded
-// by 16 bytes so that the fragment reads of neighbouring rows fall in
-// different banks), K scales, V scales, then each position's cache row index.
-// Rows of up to 64 code bytes take 256-position chunks, longer rows 128.
+__device__ __forceinline__ __half2 as_h2(uint32_t x) { return *reinterpret_cast<const __half2*>(&x); }
+__device__ __forceinline__ uint32_t as_u32(__half2 x) { return *reinterpret_cast<const uint32_t*>(&x); }
+
+// (code - z) of a binary16 pair holding 1024 + code (exact).
+template <int Z>
+__device__ __forceinline__ uint32_t minus_z(uint32_t h) {
+  const __half2 off = __halves2half2(__ushort_as_half(static_cast<unsigned short>(0x6400 + Z)),
+                                     __ushort_as_half(static_cast<unsigned short>(0x6400 + Z)));
+  return as_u32(__hsub2_rn(as_h2(h), off));
+}
+
+// (code - z) of a binary16 pair holding 1024 + 16 * code: h / 16 - (64 + z),
+// exact (h / 16 is exact, the difference is a small integer).
+template <int Z>
+__device__ __forceinline__ uint32_t minus_z_x16(uint32_t h) {
+  static_assert(Z == 8, "the 16x form is used for 4-bit codes only");
+  // 1/16 = 0x2C00, -(64 + 8) = -72 = 0xD480 in binary16
+  const __half2 sixteenth = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));
+  const __half2 off = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));
+  return as_u32(__hfma2(as_h2(h), sixteenth, off));
+}
+
+// 2^x for the softmax weights: the hardware approximation (relative error
+// about 2^-22 over the range used; results below 2^-126 flush to zero, which
+// only drops weights that cannot matter next to the reference weight 1).
+__device__ __forceinline__ float exp2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t scale_pair(uint32_t d, __half2 s2) { return as_u32(__hmul2_rn(as_h2(d), s2)); }
+
+// ---------------------------------------------------------------------------
+// Unpacking of one row's span (same-row pairs) and of two rows' spans
+// (cross-row pairs), per code width.  Results are (code - z) in binary16,
+// exact; the caller multiplies by the scale.
+//
+// Same-row pair order (`row_pair_elem`): pair r of a span holds elements
+// (e0, e1) = row_pair_elem(r, 0 / 1).  Cross-row order (`xrow_elem`): pair r
+// holds element xrow_elem(r) of row 0 (low half) and of row 1 (high half).
+// ---------------------------------------------------------------------------
+
+template <int B>
+struct AttnCodec;
+
+template <>
+struct AttnCodec<4> {
+  static constexpr int kZ = 8;
+  // pairs per 32-bit word: (0,4), (1,5), (2,6), (3,7)
+  __host__ __device__ static constexpr int row_pair_elem(int r, int e) { return 8 * (r >> 2) + (r & 3) + 4 * e; }
+  __host__ __device__ static constexpr int xrow_elem(int r) { return r; }
+  template <int NW>
+  __device__ static void row_pairs(const uint32_t (&w)[NW], uint32_t (&out)[4 * NW]) {
+#pragma unroll
+    for (int i = 0; i < NW; ++i) {
+      const uint32_t x = w[i], y = w[i] >> 8;
+      out[4 * i + 0] = minus_z<kZ>((x & 0x000F000Fu) | 0x64006400u);
+      out[4 * i + 1] = minus_z_x16<kZ>((x & 0x00F000F0u) | 0x64006400u);
+      out[4 * i + 2] = minus_z<kZ>((y & 0x000F000Fu) | 0x64006400u);
+      out[4 * i + 3] = minus_z_x16<kZ>((y & 0x00F000F0u) | 0x64006400u);
+    }
+  }
+  // rows r0, r1 (NW words each) -> 8 * NW cross-row pairs, element order 0..8NW-1
+  template <int NW>
+  __device__ static void xrow_pairs(const uint32_t (&w0)[NW], const uint32_t (&w1)[NW], uint32_t (&out)[8 * NW]) {
+#pragma unroll
+    for (int i = 0; i < NW; ++i) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        // bytes 2h, 2h+1 of each row: elements 8i + 4h .. 8i + 4h + 3
+        const uint32_t x = __byte_perm(w0[i], w1[i], h ? 0x7632 : 0x5410);
+        const uint32_t y = x >> 8;
+        out[8 * i + 4 * h + 0] = minus_z<kZ>((x & 0x000F000Fu) | 0x64006400u);
+        out[8 * i + 4 * h + 1] = minus_z_x16<kZ>((x & 0x00F000F0u) | 0x64006400u);
+        out[8 * i + 4 * h + 2] = minus_z<kZ>((y & 0x000F000Fu) | 0x64006400u);
+        out[8 * i + 4 * h + 3] = minus_z_x16<kZ>((y & 0x00F000F0u) | 0x64006400u);
+      }
+    }
+  }
+};
+
+template <>
+struct AttnCodec<8> {
+  static constexpr int kZ = 128;
+  // pairs per 32-bit word: (0,1), (2,3)
+  __host__ __device__ static constexpr int row_pair_elem(int r, int e) { return 2 * r + e; }
+  __host__ __device__ static constexpr int xrow_elem(int r) { return r; }
+  template <int NW>
+  __device__ static void row_pairs(const uint32_t (&w)[NW], uint32_t (&out)[2 * NW]) {
+#pragma unroll
+    for (int i = 0; i < NW; ++i) {
+      out[2 * i + 0] = minus_z<kZ>(__byte_perm(w[i], 0x64646464u, 0x5140));
+      out[2 * i + 1] = minus_z<kZ>(__byte_perm(w[i], 0x64646464u, 0x7362));
+    }
+  }
+  template <int NW>
+  __device__ static void xrow_pairs(const uint32_t (&w0)[NW], const uint32_t (&w1)[NW], uint32_t (&out)[4 * NW]) {
+#pragma unroll
+    for (int i = 0; i < NW; ++i) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        // t = [r0.c(2h), r0.c(2h+1), r1.c(2h), r1.c(2h+1)]
+        const uint32_t t = __byte_perm(w0[i], w1[i], h ? 0x7632 : 0x5410);
+        out[4 * i + 2 * h + 0] = minus_z<kZ>(__byte_perm(t, 0x64646464u, 0x4240));
+        out[4 * i + 2 * h + 1] = minus_z<kZ>(__byte_perm(t, 0x64646464u, 0x4341));
+      }
+    }
+  }
+};
+
+// Q6: a 16-code group is 12 bytes (three little-endian words, code k at bits
+// [6k, 6k + 6)).  Eight codes are six bytes B0..B5; pairs (q, q + 4) sit at
+// the same bit offsets of (B0..B2) and (B3..B5), so one byte permute puts
+// them 16 bits apart: (0,4) = B0 | B3, (1,5) = (B0 B1 | B3 B4) >> 6,
+// (2,6) = (B1 B2 | B4 B5) >> 4, (3,7) = (B2 | B5) >> 2.
+template <>
+struct AttnCodec<6> {
+  static constexpr int kZ = 32;
+  __host__ __device__ static constexpr int row_pair_elem(int r, int e) { return 8 * (r >> 2) + (r & 3) + 4 * e; }
+  __host__ __device__ static constexpr int xrow_elem(int r) { return 8 * (r >> 3) + ((r >> 1) & 3) + 4 * (r & 1); }
+  // 8 codes from bytes B0..B5 = bytes o..o+5 of the pair (a, b) (o = 0 or 2):
+  // four (1024 + code) pairs (q, q + 4)
+  __device__ static void raw8_at(uint32_t a, uint32_t b, uint32_t o, uint32_t (&r)[4]) {
+    const uint32_t add = o * 0x1111u;  // every selector nibble moves up by o bytes
+    const uint32_t p0 = __byte_perm(a, b, 0x3300u + add);  // B0, B0, B3, B3
+    const uint32_t p1 = __byte_perm(a, b, 0x4310u + add);  // B0, B1, B3, B4
+    const uint32_t p2 = __byte_perm(a, b, 0x5421u + add);  // B1, B2, B4, B5
+    const uint32_t p3 = __byte_perm(a, b, 0x5522u + add);  // B2, B2, B5, B5
+    r[0] = (p0 & 0x003F003Fu) | 0x64006400u;
+    r[1] = ((p1 >> 6) & 0x003F003Fu) | 0x64006400u;
+    r[2] = ((p2 >> 4) & 0x003F003Fu) | 0x64006400u;
+    r[3] = ((p3 >> 2) & 0x003F003Fu) | 0x64006400u;
+  }
+  // NG groups (3 words each) -> 8 * NG same-row pairs
+  template <int NG>
+  __device__ static void row_pairs_g(const uint32_t (&w)[3 * NG], uint32_t (&out)[8 * NG]) {
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+      uint32_t r0[4], r1[4];
+      raw8_at(w[3 * g], w[3 * g + 1], 0, r0);
+      raw8_at(w[3 * g + 1], w[3 * g + 2], 2, r1);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        out[8 * g + q] = minus_z<kZ>(r0[q]);
+        out[8 * g + 4 + q] = minus_z<kZ>(r1[q]);
+      }
+    }
+  }
+  // two rows, NG groups each -> 16 * NG cross-row pairs in xrow_elem order
+  template <int NG>
+  __device__ static void xrow_pairs_g(const uint32_t (&w0)[3 * NG], const uint32_t (&w1)[3 * NG],
+                                      uint32_t (&out)[16 * NG]) {
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+#pragma unroll
+      for (int hg = 0; hg < 2; ++hg) {
+        uint32_t a[4], b[4];
+        raw8_at(w0[3 * g + hg], w0[3 * g + hg + 1], 2 * hg, a);
+        raw8_at(w1[3 * g + hg], w1[3 * g + hg + 1], 2 * hg, b);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          // element q of both rows, then element q + 4 of both rows
+          out[16 * g + 8 * hg + 2 * q] = minus_z<kZ>(__byte_perm(a[q], b[q], 0x5410));
+          out[16 * g + 8 * hg + 2 * q + 1] = minus_z<kZ>(__byte_perm(a[q], b[q], 0x7632));
+        }
+      }
+    }
+  }
+};
+
+// Per-warp shared-memory staging.  A work item is one (sequence, kv head,
+// 128-position chunk); a warp streams it through two buffers of kSub
+// positions each (K codes, V codes, K scales, V scales), filling one while it
+// computes on the other.  Row strides are padded where that removes bank
+// conflicts of the fragment reads (K: one span per lane of eight consecutive
+// rows; V: four rows per lane, byte-interleaved in pairs).
 template <int B, int D>
 struct AttnTile {
   static constexpr int kRowBytes = D * B / 8;
-  static constexpr int kStride = kRowBytes + 16;
+  static constexpr int kStrideK = kRowBytes + (kRowBytes % 128 == 0 ? 16 : 0);
+  static constexpr int kStrideV = kRowBytes + ((B == 6 && D == 64) ? 0 : 16);
   static constexpr int kScales = D / 32;
-  static constexpr int kChunk = kRowBytes <= 64 ? 256 : 128;
-  static constexpr int kCodeBytes = kChunk * kStride;
-  static constexpr int kScaleBytes = kChunk * kScales * 2;
-  static constexpr int kStageBytes = 2 * (kCodeBytes + kScaleBytes);
-  static constexpr int kAccBytes = kAttnWarps * D * (kAttnMaxGroup + 1) * 4;  // merge area (aliases the stage)
-  static constexpr int kRowIdxOffset = kStageBytes > kAccBytes ? kStageBytes : kAccBytes;
-  static constexpr int kSmemBytes = kRowIdxOffset + kChunk * 8;
+  static constexpr int kChunk = 128;                        // positions per work item / workspace entry
+  static constexpr int kSub = kRowBytes <= 64 ? 32 : 16;   // positions per staged buffer
+  static constexpr int kBufK = kSub * kStrideK;
+  static constexpr int kBufV = kSub * kStrideV;
+  static constexpr int kBufS = kSub * kScales * 2;
+  static constexpr int kBufBytes = (kBufK + kBufV + 2 * kBufS + 15) / 16 * 16;
+  static constexpr int kQBytes = kAttnMaxGroup * D * 2;  // the item's query rows (copied with its first sub-chunk)
+  static constexpr int kWarpBytes = 2 * kBufBytes + kQBytes;
+  static constexpr int kSeqlenSlots = 256;  // sequence lengths staged per CTA (larger batches read global memory)
+  static constexpr int kSmemBytes = kAttnWarps * kWarpBytes + kSeqlenSlots * 4;
+  static constexpr int KN = D / 4;   // K elements per lane per position (one contiguous span)
+  static constexpr int VN = D / 8;   // V elements per lane per row (one contiguous span)
+  static constexpr int KS = D / 16;  // k-steps of Q K^T = m-tiles of V^T P^T
+  static constexpr int kKSpanBytes = KN * B / 8;
+  static constexpr int kVSpanBytes = VN * B / 8;
 };
-constexpr int kAttnMinChunk = 128;  // smallest chunk any (B, D) uses: sizes the workspace
+constexpr int kAttnMinChunk = 128;  // positions per workspace entry (every (B, D))
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
@@ -99,24 +291,11 @@ __device__ __forceinline__ void cp_async_small(void* dst, const void* src) {
                : "memory");
 }
 
-// Dequantize N consecutive elements [d, d + N) of one staged row (d a
-// multiple of N, N a multiple of 8) into N / 2 half2 registers (element
-// pairs (d + 2e, d + 2e + 1)).  Every 32-element block inside the span
-// starts at a multiple of 32, so 8-element unit u uses scale (d >> 5) + (u >> 2).
-template <int B, int N>
-__device__ __forceinline__ void dequant_span(const uint8_t* row, const __half* srow, int d, uint32_t out[N / 2]) {
-  static_assert(N % 8 == 0, "whole 8-element units");
-  constexpr int NB = N * B / 8;  // bytes of the span; the span starts at a multiple of NB
-  const uint8_t* p = row + d * B / 8;
-  uint32_t w[(NB + 3) / 4 + 1];
-  if constexpr (B == 6 && N == 8) {
-    // 6 bytes at a 2-byte offset: the two words of the 12-byte group half
-    const uint32_t* grp = reinterpret_cast<const uint32_t*>(row + (d >> 4) * 12);
-    const int half = (d >> 3) & 1;
-    const uint32_t a = grp[half], b = grp[half + 1];
-    w[0] = __funnelshift_r(a, b, 16 * half);
-    w[1] = (b >> (16 * half)) & 0xFFFFu;
-  } else if constexpr (NB % 16 == 0) {
+// NB bytes (a multiple of 4) from shared memory at p, aligned to the widest
+// access NB and the offset allow, as 32-bit words.
+template <int NB>
+__device__ __forceinline__ void lds_words(const uint8_t* p, uint32_t (&w)[NB / 4]) {
+  if constexpr (NB % 16 == 0) {
 #pragma unroll
     for (int v = 0; v < NB / 16; ++v) {
       const uint4 x = reinterpret_cast<const uint4*>(p)[v];
@@ -132,294 +311,434 @@ __device__ __forceinline__ void dequant_span(const uint8_t* row, const __half* s
 #pragma unroll
     for (int v = 0; v < NB / 4; ++v) w[v] = reinterpret_cast<const uint32_t*>(p)[v];
   }
+}
+
+// The K span of one lane (KN elements starting at element KN * j of a staged
+// row) as (code - z) pairs times the scale: KN / 2 half2 registers in
+// row_pair_elem order.
+template <int B, int D>
+__device__ __forceinline__ void k_span(const uint8_t* row, const __half* srow, int j, uint32_t (&out)[D / 8]) {
+  using T = AttnTile<B, D>;
+  constexpr int KN = T::KN, NB = T::kKSpanBytes;
+  uint32_t w[NB / 4];
+  lds_words<NB>(row + j * NB, w);
+  if constexpr (B == 6) {
+    AttnCodec<6>::row_pairs_g<NB / 12>(w, out);
+  } else {
+    AttnCodec<B>::template row_pairs<NB / 4>(w, out);
+  }
+  // scales: one 32-element block per 16 registers (KN <= 32: one block)
+  constexpr int kRegsPerBlock = 16;
 #pragma unroll
-  for (int u = 0; u < N / 8; ++u) {
-    const __half s = srow[(d >> 5) + (u >> 2)];
+  for (int b = 0; b < (KN + 31) / 32; ++b) {
+    const __half s = srow[(KN * j) / 32 + b];
     const __half2 s2 = __halves2half2(s, s);
-    uint4 r;
-    if constexpr (B == 4) {
-      r = dequant_q4_v8(w[u], s2);
-    } else if constexpr (B == 8) {
-      r = dequant_q8_v8(w[2 * u], w[2 * u + 1], s2);
-    } else if constexpr (N == 8) {
-      r = dequant_q6_v8(w[0], w[1], s2);
-    } else {
-      const int q = u >> 1;  // 16-code group: words 3q .. 3q + 2
-      r = (u & 1) ? dequant_q6_v8(__funnelshift_r(w[3 * q + 1], w[3 * q + 2], 16), w[3 * q + 2] >> 16, s2)
-                  : dequant_q6_v8(w[3 * q], w[3 * q + 1] & 0xFFFFu, s2);
-    }
-    out[4 * u + 0] = r.x;
-    out[4 * u + 1] = r.y;
-    out[4 * u + 2] = r.z;
-    out[4 * u + 3] = r.w;
+#pragma unroll
+    for (int r = b * kRegsPerBlock; r < (b + 1) * kRegsPerBlock && r < KN / 2; ++r) out[r] = scale_pair(out[r], s2);
   }
 }
 
-// Physical row of logical position p of sequence `seq`, or -1 when the paging
-// metadata points outside the cache.
-__device__ __forceinline__ long long attn_row(const AttnParams& a, int seq, long long p, const int* bt_chunk,
-                                              long long lp0) {
-  if (a.page_size == 0) return static_cast<long long>(seq) * a.dim1 + p;
-  const long long lp = p / a.page_size;
-  if (lp >= a.bt_stride) return -1;
-  const int page = bt_chunk[lp - lp0];
-  if (page < 0 || page >= a.dim0) return -1;
-  return static_cast<long long>(page) * a.page_size + p % a.page_size;
+// The V spans of one lane for a pair of rows (VN elements starting at element
+// VN * g): VN cross-row pairs (row r0 low half, r1 high half) times the two
+// rows' scales, in xrow_elem order.
+template <int B, int D>
+__device__ __forceinline__ void v_span_pair(const uint8_t* r0, const uint8_t* r1, __half s0, __half s1, int g,
+                                            uint32_t (&out)[D / 8]) {
+  using T = AttnTile<B, D>;
+  constexpr int VN = T::VN, NB = T::kVSpanBytes;
+  if constexpr (B == 6 && VN == 8) {
+    // 6 bytes at byte 6g: the aligned 8 bytes around them, bytes o..o+5 (o = 0 or 2)
+    const int base = (6 * g) & ~3;
+    const uint32_t o = (6 * g) & 3;
+    const uint32_t a0 = reinterpret_cast<const uint32_t*>(r0 + base)[0], b0 = reinterpret_cast<const uint32_t*>(r0 + base)[1];
+    const uint32_t a1 = reinterpret_cast<const uint32_t*>(r1 + base)[0], b1 = reinterpret_cast<const uint32_t*>(r1 + base)[1];
+    uint32_t x[4], y[4];
+    AttnCodec<6>::raw8_at(a0, b0, o, x);
+    AttnCodec<6>::raw8_at(a1, b1, o, y);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      out[2 * q] = minus_z<32>(__byte_perm(x[q], y[q], 0x5410));
+      out[2 * q + 1] = minus_z<32>(__byte_perm(x[q], y[q], 0x7632));
+    }
+  } else {
+    uint32_t w0[NB / 4], w1[NB / 4];
+    lds_words<NB>(r0 + g * NB, w0);
+    lds_words<NB>(r1 + g * NB, w1);
+    if constexpr (B == 6) {
+      AttnCodec<6>::xrow_pairs_g<NB / 12>(w0, w1, out);
+    } else {
+      AttnCodec<B>::template xrow_pairs<NB / 4>(w0, w1, out);
+    }
+  }
+  const __half2 s2 = __halves2half2(s0, s1);
+#pragma unroll
+  for (int r = 0; r < VN; ++r) out[r] = scale_pair(out[r], s2);
+}
+
+
+// One sub-chunk of one work item, as a warp walks its items.
+struct AttnCursor {
+  long long item;       // work item index, or -1 past the end
+  int seq, chunk, kvh;  // what the item is
+  int sub;              // sub-chunk within the item
+  int n;                // positions of this sub-chunk (<= kSub)
+  bool last;            // last sub-chunk of the item
+};
+
+template <int B, int D>
+struct AttnWalk {
+  using T = AttnTile<B, D>;
+  const AttnParams& a;
+  const int* s_len;  // staged sequence lengths (or null)
+  long long stride;  // warps in the grid
+
+  __device__ long long max_len() const {
+    return a.page_size == 0 ? static_cast<long long>(a.dim1) : static_cast<long long>(a.max_chunks) * T::kChunk;
+  }
+  // sequence length, clamped to what the cache (or the launched chunks) can hold
+  __device__ int length(int seq) const {
+    long long L = s_len ? s_len[seq] : a.seqlens[seq];
+    if (L < 0) L = 0;
+    const long long m = max_len();
+    return static_cast<int>(L > m ? m : L);
+  }
+  // first sub-chunk of the first non-empty item at or after `item`
+  __device__ AttnCursor seek(long long item) const {
+    const long long n_items = static_cast<long long>(a.batch) * a.max_chunks * a.kv_heads;
+    AttnCursor c;
+    for (; item < n_items; item += stride) {
+      const long long t = item / a.kv_heads;
+      c.kvh = static_cast<int>(item - t * a.kv_heads);
+      c.seq = static_cast<int>(t / a.max_chunks);
+      c.chunk = static_cast<int>(t - static_cast<long long>(c.seq) * a.max_chunks);
+      const int L = length(c.seq);
+      const int p0 = c.chunk * T::kChunk;
+      if (p0 < L) {
+        c.item = item;
+        c.sub = 0;
+        const int rest = min(L - p0, T::kChunk);
+        c.n = min(rest, T::kSub);
+        c.last = rest <= T::kSub;
+        return c;
+      }
+    }
+    c.item = -1;
+    return c;
+  }
+  __device__ AttnCursor next(const AttnCursor& c) const {
+    if (c.last) return seek(c.item + stride);
+    AttnCursor d = c;
+    d.sub = c.sub + 1;
+    const int rest = min(length(c.seq) - c.chunk * T::kChunk, T::kChunk) - d.sub * T::kSub;
+    d.n = min(rest, T::kSub);
+    d.last = rest <= T::kSub;
+    return d;
+  }
+};
+
+// Issue the copies of one sub-chunk into a warp buffer (and, for the first
+// sub-chunk of an item, its query rows into the warp's query area); returns
+// the bit mask of its positions that hold data (bit i: position i).
+template <int B, int D>
+__device__ __forceinline__ uint32_t attn_issue(const AttnParams& a, const AttnCursor& c, uint8_t* buf, uint8_t* sq,
+                                               int lane) {
+  using T = AttnTile<B, D>;
+  constexpr int SC = T::kSub, P = T::kRowBytes / 16;
+  uint8_t* const sk = buf;
+  uint8_t* const sv = buf + T::kBufK;
+  __half* const sks = reinterpret_cast<__half*>(buf + T::kBufK + T::kBufV);
+  __half* const svs = sks + SC * T::kScales;
+  // cache row of this lane's position (lanes < SC): -1 bad paging metadata, -2 past the window
+  long long hr = -2;
+  if (lane < c.n) {
+    const int p = c.chunk * T::kChunk + c.sub * SC + lane;
+    long long row;
+    if (a.page_size == 0) {
+      row = static_cast<long long>(c.seq) * a.dim1 + p;
+    } else {
+      const int lp = p / a.page_size;
+      const int page = lp < a.bt_stride ? a.block_table[static_cast<long long>(c.seq) * a.bt_stride + lp] : -1;
+      row = (page < 0 || page >= a.dim0) ? -1 : static_cast<long long>(page) * a.page_size + (p - lp * a.page_size);
+      if (row < 0) record_error(KVQ_DEV_BAD_PAGE);
+    }
+    hr = row < 0 ? -1 : row * a.kv_heads + c.kvh;
+  }
+  const uint32_t mask = __ballot_sync(0xFFFFFFFFu, hr >= 0);
+  // codes: task t = (row t / P, 16-byte part t % P), 32 tasks per pass
+#pragma unroll
+  for (int t0 = 0; t0 < SC * P; t0 += 32) {
+    const int t = t0 + lane, r = t / P, part = t - r * P;
+    const long long h = __shfl_sync(0xFFFFFFFFu, hr, r);
+    if (h >= 0) {
+      const long long src = h * T::kRowBytes + part * 16;
+      cp_async16(sk + r * T::kStrideK + part * 16, a.k_codes + src);
+      cp_async16(sv + r * T::kStrideV + part * 16, a.v_codes + src);
+    }
+  }
+  // scales; rows without data get zero scales, which dequantize whatever codes
+  // the buffer holds to zero
+  if (lane < SC) {
+    if (hr >= 0) {
+      cp_async_small<T::kScales * 2>(sks + lane * T::kScales, a.k_scales + hr * T::kScales);
+      cp_async_small<T::kScales * 2>(svs + lane * T::kScales, a.v_scales + hr * T::kScales);
+    } else {
+#pragma unroll
+      for (int e = 0; e < T::kScales; ++e) sks[lane * T::kScales + e] = svs[lane * T::kScales + e] = __ushort_as_half(0);
+    }
+  }
+  // the item's query rows travel with its first sub-chunk
+  if (c.sub == 0) {
+    const __half* q = a.q + (static_cast<long long>(c.seq) * a.n_heads + static_cast<long long>(c.kvh) * a.group) * D;
+    for (int t = lane; t < a.group * D / 8; t += 32) cp_async16(sq + t * 16, q + t * 8);
+  }
+  return mask;
 }
 
 template <int B, int D>
-__global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(const __grid_constant__ AttnParams a) {
+__global__ void __launch_bounds__(kAttnThreads, D > 128 ? 2 : 4) attn_partial_kernel(const __grid_constant__ AttnParams a) {
   using T = AttnTile<B, D>;
-  constexpr int KS = D / 16;  // k-steps of Q K^T, m-blocks of V^T P^T
-  constexpr int KN = D / 4;   // K elements per lane per position
-  constexpr int VN = D / 8;   // V elements per lane per position
-  constexpr int C = T::kChunk;
+  using Codec = AttnCodec<B>;
+  constexpr int KS = T::KS;  // k-steps of Q K^T, m-tiles of V^T P^T
+  constexpr int KR = D / 8;  // registers of one K span / one V span pair
+  constexpr int SC = T::kSub;
 
   extern __shared__ __align__(16) uint8_t smem[];
-  uint8_t* const sk = smem;
-  uint8_t* const sv = smem + T::kCodeBytes;
-  __half* const sks = reinterpret_cast<__half*>(smem + 2 * T::kCodeBytes);
-  __half* const svs = sks + C * T::kScales;
-  long long* const s_hr = reinterpret_cast<long long*>(smem + T::kRowIdxOffset);
-  float(*const s_acc)[D][kAttnMaxGroup + 1] = reinterpret_cast<float(*)[D][kAttnMaxGroup + 1]>(smem);
-  __shared__ int s_bt[C + 1];
-  __shared__ float s_p[kAttnWarps][16][kAttnMaxGroup + 1];
-  __shared__ float s_m[kAttnWarps][kAttnMaxGroup];
-  __shared__ float s_l[kAttnWarps][kAttnMaxGroup];
-  __shared__ int s_bad;
-
-  const int chunk = blockIdx.x, kvh = blockIdx.y, seq = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, j = lane & 3;
+  uint8_t* const wbuf = smem + warp * T::kWarpBytes;
+  int* const s_len = reinterpret_cast<int*>(smem + kAttnWarps * T::kWarpBytes);
 
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  if (threadIdx.x == 0) s_bad = 0;
+  const bool staged = a.batch <= T::kSeqlenSlots;
+  if (staged)
+    for (int i = threadIdx.x; i < a.batch; i += kAttnThreads) s_len[i] = a.seqlens[i];
+  __syncthreads();  // the only CTA-wide barrier: from here on every warp walks its own items
 
-  long long L = a.seqlens[seq];
-  if (L < 0) L = 0;
-  const long long max_len = a.page_size == 0 ? static_cast<long long>(a.dim1)
-                                             : static_cast<long long>(a.max_chunks) * C;
-  if (L > max_len) {  // longer than the cache (contiguous) or than the launched chunks (paged)
-    if (threadIdx.x == 0 && chunk == 0 && kvh == 0) record_error(KVQ_DEV_BAD_PAGE_INDEX);
-    L = max_len;
-  }
-  const long long p0 = static_cast<long long>(chunk) * C;
-  if (p0 >= L) return;  // the whole CTA leaves together
-  const long long p1 = min(L, p0 + C);
-  const int n = static_cast<int>(p1 - p0);
+  const AttnWalk<B, D> walk{a, staged ? s_len : nullptr, static_cast<long long>(gridDim.x) * kAttnWarps};
+  uint8_t* const sq_area = wbuf + 2 * T::kBufBytes;
+  AttnCursor cur = walk.seek(static_cast<long long>(blockIdx.x) * kAttnWarps + warp);
+  if (cur.item < 0) return;
+  uint32_t mask_cur = attn_issue<B, D>(a, cur, wbuf, sq_area, lane);
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+  int b = 0;
 
-  // block-table entries of the chunk's logical pages, staged once
-  long long lp0 = 0;
-  if (a.page_size > 0) {
-    lp0 = p0 / a.page_size;
-    const long long lp1 = (p1 - 1) / a.page_size;
-    for (long long lp = lp0 + threadIdx.x; lp <= lp1; lp += kAttnThreads)
-      s_bt[lp - lp0] = lp < a.bt_stride ? a.block_table[static_cast<long long>(seq) * a.bt_stride + lp] : -1;
-  }
-  __syncthreads();
-
-  // cache row of every position of the chunk (-1: bad paging metadata, -2: past the window)
-  for (int i = threadIdx.x; i < C; i += kAttnThreads) {
-    long long hr = -2;
-    if (i < n) {
-      const long long row = attn_row(a, seq, p0 + i, s_bt, lp0);
-      if (row < 0) s_bad = 1;
-      hr = row < 0 ? -1 : row * a.kv_heads + kvh;
-    }
-    s_hr[i] = hr;
-  }
-  __syncthreads();
-
-  // issue every copy of the chunk; rows without data get zero scales, which
-  // dequantize whatever codes the buffer holds to zero
-  {
-    constexpr int P = T::kRowBytes / 16;
-    for (int t = threadIdx.x; t < C * P; t += kAttnThreads) {
-      const int i = t / P, part = t - i * P;
-      const long long hr = s_hr[i];
-      if (hr >= 0) {
-        const long long off = hr * T::kRowBytes + part * 16;
-        cp_async16(sk + i * T::kStride + part * 16, a.k_codes + off);
-        cp_async16(sv + i * T::kStride + part * 16, a.v_codes + off);
-      }
-    }
-    for (int i = threadIdx.x; i < C; i += kAttnThreads) {
-      const long long hr = s_hr[i];
-      if (hr >= 0) {
-        cp_async_small<T::kScales * 2>(sks + i * T::kScales, a.k_scales + hr * T::kScales);
-        cp_async_small<T::kScales * 2>(svs + i * T::kScales, a.v_scales + hr * T::kScales);
-      } else {
-#pragma unroll
-        for (int e = 0; e < T::kScales; ++e) sks[i * T::kScales + e] = svs[i * T::kScales + e] = __ushort_as_half(0);
-      }
-    }
-    asm volatile("cp.async.commit_group;\n" ::: "memory");
-  }
-
-  // query fragments (B operand of Q K^T): head g of the group, this lane's
-  // permuted head_dim slice d = KN*j + 4s + {0..3}; loaded while the copies fly
-  uint32_t qf[KS][2];
-  {
-    const bool live = g < a.group;
-    const __half* qrow = a.q + (static_cast<long long>(seq) * a.n_heads + kvh * a.group + (live ? g : 0)) * D;
-#pragma unroll
-    for (int s = 0; s < KS; ++s) {
-      const int d0 = KN * j + 4 * s;
-      qf[s][0] = live ? __ldg(reinterpret_cast<const uint32_t*>(qrow + d0)) : 0u;
-      qf[s][1] = live ? __ldg(reinterpret_cast<const uint32_t*>(qrow + d0 + 2)) : 0u;
-    }
-  }
-  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
-  __syncthreads();
-
-  float m_run[2] = {-INFINITY, -INFINITY};  // heads 2j, 2j+1 (log2 domain)
-  float l_run[2] = {0.0f, 0.0f};
+  uint32_t qa0[KS], qa2[KS];
+  float m_ref = -INFINITY, l_part = 0.0f;
   float acc[KS][4];
-#pragma unroll
-  for (int mb = 0; mb < KS; ++mb) acc[mb][0] = acc[mb][1] = acc[mb][2] = acc[mb][3] = 0.0f;
 
-  for (int t0 = 16 * warp; t0 < n; t0 += 16 * kAttnWarps) {
-    // ---- K: positions t0 + g and t0 + g + 8, elements [KN*j, KN*j + KN)
-    uint32_t kd[2][KN / 2];
-    bool kvalid[2];
+  // Per iteration: wait for the current sub-chunk, take the item's query
+  // fragments if it starts here, issue the next sub-chunk's copies into the
+  // other buffer, then compute on the current one.
+  while (true) {
+    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+    __syncwarp();
+    if (cur.sub == 0) {
+      // a new item: query fragments (A operand of Q K^T, rows = heads of the
+      // group, rows >= 8 zero; lane j's head_dim elements follow the K span
+      // order) and a fresh softmax state
+      const __half(*sq)[D] = reinterpret_cast<const __half(*)[D]>(sq_area);
+      const bool live = g < a.group;
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int i = t0 + g + 8 * r;
-      kvalid[r] = s_hr[i] >= 0;
-      dequant_span<B, KN>(sk + i * T::kStride, sks + i * T::kScales, KN * j, kd[r]);
+      for (int s = 0; s < KS; ++s) {
+        const int d00 = T::KN * j + Codec::row_pair_elem(2 * s, 0), d01 = T::KN * j + Codec::row_pair_elem(2 * s, 1);
+        const int d10 = T::KN * j + Codec::row_pair_elem(2 * s + 1, 0);
+        const int d11 = T::KN * j + Codec::row_pair_elem(2 * s + 1, 1);
+        const __half* qr = sq[live ? g : 0];
+        qa0[s] = live ? as_u32(__halves2half2(qr[d00], qr[d01])) : 0u;
+        qa2[s] = live ? as_u32(__halves2half2(qr[d10], qr[d11])) : 0u;
+      }
+      m_ref = -INFINITY;
+      l_part = 0.0f;
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.0f;
+      if (cur.chunk == 0 && cur.kvh == 0 && lane == 0) {
+        const long long L = a.seqlens[cur.seq];
+        if (L > walk.max_len()) record_error(KVQ_DEV_BAD_PAGE_INDEX);  // window longer than the cache
+      }
+      __syncwarp();  // the query area may be refilled below
     }
-    float sc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-    for (int s = 0; s < KS; ++s) {
-      const uint32_t af[4] = {kd[0][2 * s], kd[1][2 * s], kd[0][2 * s + 1], kd[1][2 * s + 1]};
-      mma_16816(sc, af, qf[s][0], qf[s][1]);
+    const AttnCursor nxt = walk.next(cur);
+    uint32_t mask_nxt = 0;
+    if (nxt.item >= 0) {
+      mask_nxt = attn_issue<B, D>(a, nxt, wbuf + (b ^ 1) * T::kBufBytes, sq_area, lane);
+      asm volatile("cp.async.commit_group;\n" ::: "memory");
     }
-    // scores: sc[0] = (pos g, head 2j), sc[1] = (g, 2j+1), sc[2] = (g+8, 2j), sc[3] = (g+8, 2j+1)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) sc[e] = kvalid[e >> 1] ? sc[e] * a.scale_log2 : -INFINITY;
 
-    // ---- online softmax for heads 2j, 2j+1 over the 16 positions
-    float p_[4];
+    const uint8_t* const buf = wbuf + b * T::kBufBytes;
+    const uint8_t* const sk = buf;
+    const uint8_t* const sv = buf + T::kBufK;
+    const __half* const sks = reinterpret_cast<const __half*>(buf + T::kBufK + T::kBufV);
+    const __half* const svs = sks + SC * T::kScales;
+
+    for (int t0 = 0; t0 < cur.n; t0 += 16) {
+      // ---- S = Q K^T for positions t0 + 8t + (0..7): lane supplies position t0 + 8t + g
+      float sc[2][4];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      float mx = fmaxf(sc[h], sc[2 + h]);
-      mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 4));
-      mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 8));
-      mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 16));
-      const float m_new = fmaxf(m_run[h], mx);
-      const float alpha = (m_new == -INFINITY) ? 1.0f : exp2f(m_run[h] - m_new);
-      p_[h] = (sc[h] == -INFINITY) ? 0.0f : exp2f(sc[h] - m_new);
-      p_[2 + h] = (sc[2 + h] == -INFINITY) ? 0.0f : exp2f(sc[2 + h] - m_new);
-      float sum = p_[h] + p_[2 + h];
-      sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 4);
-      sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 8);
-      sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 16);
-      l_run[h] = l_run[h] * alpha + sum;
-      m_run[h] = m_new;
-      if (alpha != 1.0f) {
+      for (int t = 0; t < 2; ++t) {
+        const int i = t0 + 8 * t + g;
+        uint32_t kb[KR];
+        k_span<B, D>(sk + i * T::kStrideK, sks + i * T::kScales, j, kb);
+        sc[t][0] = sc[t][1] = sc[t][2] = sc[t][3] = 0.0f;
 #pragma unroll
-        for (int mb = 0; mb < KS; ++mb) {
-          acc[mb][h] *= alpha;
-          acc[mb][2 + h] *= alpha;
+        for (int s = 0; s < KS; ++s) mma_16816(sc[t], qa0[s], 0u, qa2[s], 0u, kb[2 * s], kb[2 * s + 1]);
+      }
+      // scores of head g at positions t0 + 8t + 2j + e (c0, c1); positions without data -inf
+      float p[2][2];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int i = t0 + 8 * t + 2 * j + e;
+          const float v = ((mask_cur >> i) & 1u) ? sc[t][e] * a.scale_log2 : -INFINITY;
+          p[t][e] = v;
+          mx = fmaxf(mx, v);
+        }
+      }
+      mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
+      // lazy rescale: move the reference only when a score exceeds it by more than the threshold
+      const bool grow = mx > m_ref + kAttnRescaleLog2;
+      if (__any_sync(0xFFFFFFFFu, grow)) {
+        const float m_new = grow ? mx : m_ref;
+        const float alpha = (m_ref == -INFINITY) ? 0.0f : exp2_approx(m_ref - m_new);
+        l_part *= alpha;
+        // accumulators hold heads 2j, 2j+1: their factors live in quads 2j, 2j+1
+        const float a0 = __shfl_sync(0xFFFFFFFFu, alpha, 8 * j);
+        const float a1 = __shfl_sync(0xFFFFFFFFu, alpha, 8 * j + 4);
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+          acc[mt][0] *= a0;
+          acc[mt][1] *= a1;
+          acc[mt][2] *= a0;
+          acc[mt][3] *= a1;
+        }
+        m_ref = m_new;
+      }
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          p[t][e] = (p[t][e] == -INFINITY) ? 0.0f : exp2_approx(p[t][e] - m_ref);
+          l_part += p[t][e];
+        }
+      }
+      // ---- P^T B fragment: b0 = P[g][2j, 2j+1] (tile 0), b1 = P[g][8 + 2j, 8 + 2j + 1] (tile 1),
+      // as a binary16 high part and a binary16 residual
+      const uint32_t bh0 = pack_half2(p[0][0], p[0][1]), bh1 = pack_half2(p[1][0], p[1][1]);
+      const float2 f0 = __half22float2(as_h2(bh0)), f1 = __half22float2(as_h2(bh1));
+      const uint32_t bl0 = pack_half2(p[0][0] - f0.x, p[0][1] - f0.y);
+      const uint32_t bl1 = pack_half2(p[1][0] - f1.x, p[1][1] - f1.y);
+
+      // ---- O^T += V^T P^T: row pairs (2j, 2j+1) and (2j+8, 2j+9) of the 16 positions
+      uint32_t va[KR], vb[KR];
+      {
+        const int i0 = t0 + 2 * j, i1 = i0 + 8;
+        const int sblk = (T::VN * g) / 32;
+        v_span_pair<B, D>(sv + i0 * T::kStrideV, sv + (i0 + 1) * T::kStrideV, svs[i0 * T::kScales + sblk],
+                          svs[(i0 + 1) * T::kScales + sblk], g, va);
+        v_span_pair<B, D>(sv + i1 * T::kStrideV, sv + (i1 + 1) * T::kStrideV, svs[i1 * T::kScales + sblk],
+                          svs[(i1 + 1) * T::kScales + sblk], g, vb);
+      }
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        mma_16816(acc[mt], va[2 * mt], va[2 * mt + 1], vb[2 * mt], vb[2 * mt + 1], bh0, bh1);
+        mma_16816(acc[mt], va[2 * mt], va[2 * mt + 1], vb[2 * mt], vb[2 * mt + 1], bl0, bl1);
+      }
+    }
+
+    if (cur.last) {
+      // the item's partial result: (max, sum, accumulator) of every head of the group
+      float l_sum = l_part;
+      l_sum += __shfl_xor_sync(0xFFFFFFFFu, l_sum, 1);
+      l_sum += __shfl_xor_sync(0xFFFFFFFFu, l_sum, 2);
+      const long long head0 = static_cast<long long>(cur.seq) * a.n_heads + static_cast<long long>(cur.kvh) * a.group;
+      float* const ws = a.ws + (head0 * a.max_chunks + cur.chunk) * (D + 2);
+      const long long hstride = static_cast<long long>(a.max_chunks) * (D + 2);  // next head, same chunk
+      if (j == 0 && g < a.group) {
+        ws[g * hstride] = m_ref;
+        ws[g * hstride + 1] = l_sum;
+      }
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        const int da = T::VN * g + Codec::xrow_elem(2 * mt), db = T::VN * g + Codec::xrow_elem(2 * mt + 1);
+        if (2 * j < a.group) {
+          ws[(2 * j) * hstride + 2 + da] = acc[mt][0];
+          ws[(2 * j) * hstride + 2 + db] = acc[mt][2];
+        }
+        if (2 * j + 1 < a.group) {
+          ws[(2 * j + 1) * hstride + 2 + da] = acc[mt][1];
+          ws[(2 * j + 1) * hstride + 2 + db] = acc[mt][3];
         }
       }
     }
-
-    // ---- P^T as the B operand: lane needs P[head g][pos 2j, 2j+1, 2j+8, 2j+9]
-    s_p[warp][g][2 * j] = p_[0];
-    s_p[warp][g][2 * j + 1] = p_[1];
-    s_p[warp][g + 8][2 * j] = p_[2];
-    s_p[warp][g + 8][2 * j + 1] = p_[3];
-    __syncwarp();
-    const float b0 = s_p[warp][2 * j][g], b1 = s_p[warp][2 * j + 1][g];
-    const float b2 = s_p[warp][2 * j + 8][g], b3 = s_p[warp][2 * j + 9][g];
-    __syncwarp();
-    const uint32_t bh0 = pack_half2(b0, b1), bh1 = pack_half2(b2, b3);
-    const __half2 h0 = *reinterpret_cast<const __half2*>(&bh0), h1 = *reinterpret_cast<const __half2*>(&bh1);
-    const float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
-    const uint32_t bl0 = pack_half2(b0 - f0.x, b1 - f0.y), bl1 = pack_half2(b2 - f1.x, b3 - f1.y);
-
-    // ---- V: positions t0 + {2j, 2j+1, 2j+8, 2j+9}, elements [VN*g, VN*g + VN)
-    uint32_t vd[4][VN / 2];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int i = t0 + 2 * j + (r & 1) + 8 * (r >> 1);
-      dequant_span<B, VN>(sv + i * T::kStride, svs + i * T::kScales, VN * g, vd[r]);
-    }
-#pragma unroll
-    for (int mb = 0; mb < KS; ++mb) {
-      // rows d = VN*g + 2mb (+1 for rows g+8); columns = positions
-      const uint32_t af[4] = {__byte_perm(vd[0][mb], vd[1][mb], 0x5410), __byte_perm(vd[0][mb], vd[1][mb], 0x7632),
-                              __byte_perm(vd[2][mb], vd[3][mb], 0x5410), __byte_perm(vd[2][mb], vd[3][mb], 0x7632)};
-      mma_16816(acc[mb], af, bh0, bh1);
-      mma_16816(acc[mb], af, bl0, bl1);
-    }
-  }
-
-  // ---- merge the four warps: acc[mb] holds O^T[d][h] for d = VN*g + 2mb (c0, c1: heads 2j, 2j+1)
-  // and d + 1 (c2, c3).  The merge area aliases the staged chunk.
-  __syncthreads();
-  if (g == 0) {
-    s_m[warp][2 * j] = m_run[0];
-    s_m[warp][2 * j + 1] = m_run[1];
-    s_l[warp][2 * j] = l_run[0];
-    s_l[warp][2 * j + 1] = l_run[1];
-  }
-#pragma unroll
-  for (int mb = 0; mb < KS; ++mb) {
-    const int d = VN * g + 2 * mb;
-    s_acc[warp][d][2 * j] = acc[mb][0];
-    s_acc[warp][d][2 * j + 1] = acc[mb][1];
-    s_acc[warp][d + 1][2 * j] = acc[mb][2];
-    s_acc[warp][d + 1][2 * j + 1] = acc[mb][3];
-  }
-  __syncthreads();
-  if (threadIdx.x == 0 && s_bad) record_error(KVQ_DEV_BAD_PAGE);
-  const int slots = a.group * (D + 2);
-  for (int t = threadIdx.x; t < slots; t += kAttnThreads) {
-    const int h = t / (D + 2), col = t % (D + 2);
-    float mstar = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kAttnWarps; ++w) mstar = fmaxf(mstar, s_m[w][h]);
-    float v = 0.0f;
-    if (col == 0) {
-      v = mstar;
-    } else {
-#pragma unroll
-      for (int w = 0; w < kAttnWarps; ++w) {
-        const float f = (s_m[w][h] == -INFINITY) ? 0.0f : exp2f(s_m[w][h] - mstar);
-        v += f * (col == 1 ? s_l[w][h] : s_acc[w][col - 2][h]);
-      }
-    }
-    const long long slot = (static_cast<long long>(seq) * a.n_heads + kvh * a.group + h) * a.max_chunks + chunk;
-    a.ws[slot * (D + 2) + col] = v;
+    __syncwarp();  // every lane is done with this buffer before it is refilled
+    if (nxt.item < 0) break;
+    cur = nxt;
+    mask_cur = mask_nxt;
+    b ^= 1;
   }
 }
 
-// Merge the chunks of every (sequence, head): thread d of CTA (head, sequence).
+// Merge the chunks of every (sequence, head): CTA (head, sequence) of four
+// warps.  The chunk maxima are reduced by all threads at once; then warp w
+// sums chunks w, w + 4, ... (lane l owns head_dim elements l, l + 32, ...), so
+// that many chunks' loads are in flight, and the warps' sums meet in shared
+// memory.
+constexpr int kCombineThreads = 128;
+
 template <int D>
-__global__ void __launch_bounds__(D) attn_combine_kernel(const __grid_constant__ AttnParams a) {
+__global__ void __launch_bounds__(kCombineThreads) attn_combine_kernel(const __grid_constant__ AttnParams a) {
+  constexpr int kWarps = kCombineThreads / 32, DPL = D / 32;
+  __shared__ float s_red[kWarps];
+  __shared__ float s_l[kWarps];
+  __shared__ float s_o[kWarps][D];
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int h = blockIdx.x, seq = blockIdx.y, d = threadIdx.x;
+  const int h = blockIdx.x, seq = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   long long L = a.seqlens[seq];
   if (L < 0) L = 0;
   if (a.page_size == 0 && L > a.dim1) L = a.dim1;
   long long nch = (L + a.chunk - 1) / a.chunk;
   if (nch > a.max_chunks) nch = a.max_chunks;
   const float* ws = a.ws + (static_cast<long long>(seq) * a.n_heads + h) * a.max_chunks * (D + 2);
-  float mstar = -INFINITY;
-  for (long long c = 0; c < nch; ++c) mstar = fmaxf(mstar, ws[c * (D + 2)]);
-  float l = 0.0f, o = 0.0f;
-  for (long long c = 0; c < nch; ++c) {
-    const float mc = ws[c * (D + 2)];
+  float mx = -INFINITY;
+  for (long long c = threadIdx.x; c < nch; c += kCombineThreads) mx = fmaxf(mx, ws[c * (D + 2)]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+  if (lane == 0) s_red[warp] = mx;
+  __syncthreads();
+  float mstar = s_red[0];
+#pragma unroll
+  for (int w = 1; w < kWarps; ++w) mstar = fmaxf(mstar, s_red[w]);
+  float l = 0.0f, acc[DPL];
+#pragma unroll
+  for (int k = 0; k < DPL; ++k) acc[k] = 0.0f;
+#pragma unroll 4
+  for (long long c = warp; c < nch; c += kWarps) {
+    const float* e = ws + c * (D + 2);
+    const float mc = e[0];
     const float f = (mc == -INFINITY) ? 0.0f : exp2f(mc - mstar);
-    l += f * ws[c * (D + 2) + 1];
-    o += f * ws[c * (D + 2) + 2 + d];
+    l += f * e[1];
+#pragma unroll
+    for (int k = 0; k < DPL; ++k) acc[k] += f * e[2 + lane + 32 * k];
   }
-  const float y = (l > 0.0f) ? o / l : 0.0f;
-  a.out[(static_cast<long long>(seq) * a.n_heads + h) * D + d] = __float2half_rn(y);
+#pragma unroll
+  for (int k = 0; k < DPL; ++k) s_o[warp][lane + 32 * k] = acc[k];
+  if (lane == 0) s_l[warp] = l;
+  __syncthreads();
+  float lt = 0.0f;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) lt += s_l[w];
+  for (int d = threadIdx.x; d < D; d += kCombineThreads) {
+    float o = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) o += s_o[w][d];
+    const float y = (lt > 0.0f) ? o / lt : 0.0f;
+    a.out[(static_cast<long long>(seq) * a.n_heads + h) * D + d] = __float2half_rn(y);
+  }
 }
 
 }  // namespace kvq

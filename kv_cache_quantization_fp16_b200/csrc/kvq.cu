@@ -153,7 +153,7 @@ kvq_status launch_pdl(Kernel kernel, dim3 grid, int threads, int smem, void* str
 // CTAs of `kernel` that the current device holds at once (SMs x resident
 // CTAs per SM), cached per device in `cache`; 0 if it cannot be queried.
 template <class Kernel>
-long long first_wave_ctas(Kernel kernel, int threads, std::atomic<long long>* cache, int max_devices) {
+long long first_wave_ctas(Kernel kernel, int threads, int smem, std::atomic<long long>* cache, int max_devices) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= max_devices) {
     cudaGetLastError();
@@ -163,7 +163,7 @@ long long first_wave_ctas(Kernel kernel, int threads, std::atomic<long long>* ca
   if (n == 0) {
     int sms = 0, per_sm = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess) {
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess) {
       cudaGetLastError();
       return 0;
     }
@@ -177,7 +177,7 @@ template <class Op, bool kPaged>
 kvq_status launch_ldg_mode(Params p, int nkv, void* stream) {
   constexpr int kMaxDevices = 64;
   static std::atomic<long long> wave[kMaxDevices];
-  p.prefetch_ctas = first_wave_ctas(convert_kernel<Op, kPaged>, LdgCfg<Op>::kThreads, wave, kMaxDevices);
+  p.prefetch_ctas = first_wave_ctas(convert_kernel<Op, kPaged>, LdgCfg<Op>::kThreads, 0, wave, kMaxDevices);
   // Paged tiles are four CTA rounds long: each CTA pays one block-table lookup
   // before its first data load, and a longer tile amortizes it.
   const long long target = static_cast<long long>(ldg_tile_elems<Op>()) * (kPaged ? 4 : 1);
@@ -456,6 +456,9 @@ bool allow_attention_smem() {
   return true;
 }
 
+// Persistent grid of the partial kernel: every (sequence, 128-position chunk,
+// kv head) work item goes to one warp; as many CTAs as the device holds at
+// once (occupancy cached per device), never more than there are items.
 template <int B, int D>
 kvq_status launch_attention(kvq::AttnParams a, const kvq_cache_desc* desc, void* stream) {
   using T = kvq::AttnTile<B, D>;
@@ -464,10 +467,17 @@ kvq_status launch_attention(kvq::AttnParams a, const kvq_cache_desc* desc, void*
   if (max_chunks < 1 || max_chunks > 0x7FFFFFFFLL) return KVQ_ERR_RANGE;
   a.max_chunks = static_cast<int>(max_chunks);
   if (!allow_attention_smem<B, D>()) return KVQ_ERR_CUDA;
-  kvq_status st = launch_pdl(kvq::attn_partial_kernel<B, D>, dim3(a.max_chunks, a.kv_heads, a.batch),
-                             kvq::kAttnThreads, T::kSmemBytes, stream, a);
+  constexpr int kMaxDevices = 64;
+  static std::atomic<long long> resident[kMaxDevices];
+  const long long ctas_max = first_wave_ctas(kvq::attn_partial_kernel<B, D>, kvq::kAttnThreads, T::kSmemBytes,
+                                             resident, kMaxDevices);
+  if (ctas_max < 1) return KVQ_ERR_CUDA;
+  const long long items = static_cast<long long>(a.batch) * a.max_chunks * a.kv_heads;
+  const long long need = (items + kvq::kAttnWarps - 1) / kvq::kAttnWarps;
+  const unsigned grid = static_cast<unsigned>(need < ctas_max ? need : ctas_max);
+  kvq_status st = launch_pdl(kvq::attn_partial_kernel<B, D>, dim3(grid), kvq::kAttnThreads, T::kSmemBytes, stream, a);
   if (st != KVQ_OK) return st;
-  return launch_pdl(kvq::attn_combine_kernel<D>, dim3(a.n_heads, a.batch), D, 0, stream, a);
+  return launch_pdl(kvq::attn_combine_kernel<D>, dim3(a.n_heads, a.batch), kvq::kCombineThreads, 0, stream, a);
 }
 
 template <int B>

@@ -24,8 +24,10 @@ Extra keys:
   cpu_baseline  the CPU oracle (single-threaded C++) timed on this host on the
                 same step;
   e2e           the same metric through the public Python API with pinned host
-                buffers: host->device copy of the window, the four conversions,
-                device->host copy of the decoded window, all inside the events;
+                buffers: host->device copy of the windows, the two conversions,
+                device->host copy of the decoded windows every step, all inside
+                the events; steps pipelined over three streams (upload,
+                convert, download) and two buffer sets;
   per_op        every other conversion on its own workload (contiguous Q4/Q6,
                 paged Q4 decode / prefill, the model-sized paged Q6 layers), each
                 as GB/s and fraction of the HBM peak (--per-op, on by default).
@@ -400,34 +402,59 @@ def stream_shares(step, sets, reps=20):
 
 
 def e2e_fp8(kvq, step: Fp8Step, steps, warmup, dev):
-    """Same step through the public API from pinned host buffers: H2D of the K/V windows,
-    the four conversions, D2H of the decoded windows, all inside the CUDA events."""
+    """The headline step end to end through the public Python API, from pinned host
+    buffers: every step copies its K/V windows host -> device, runs the two fused
+    conversions and copies the decoded windows device -> host.  Steps are pipelined
+    the way a serving loop would run them: uploads on one stream, conversions on a
+    second, downloads on a third, two device buffer sets used alternately, so step
+    i+1's upload overlaps step i's download (PCIe is full duplex).  The timed region
+    runs from before the first upload to after the last download."""
     B, S, H, D = step.k.shape
     o, w = step.off, step.w
-    hk = step.k.cpu().pin_memory()
-    hv = step.v.cpu().pin_memory()
-    hy_k = torch.empty_like(hk).pin_memory()
-    hy_v = torch.empty_like(hv).pin_memory()
+    sets = step.sets[:2]
+    host_in = [(t["k"].cpu().pin_memory(), t["v"].cpu().pin_memory()) for t in sets]
+    host_out = [(torch.empty_like(hk).pin_memory(), torch.empty_like(hv).pin_memory()) for hk, hv in host_in]
+    s_in, s_cv, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in sets]
+    ev_cv = [torch.cuda.Event() for _ in sets]
+    ev_out = [torch.cuda.Event() for _ in sets]
+    for e in ev_cv + ev_out:
+        e.record()
 
-    def once():
-        for b in range(B):
-            step.k[b, o:o + w].copy_(hk[b, o:o + w], non_blocking=True)
-            step.v[b, o:o + w].copy_(hv[b, o:o + w], non_blocking=True)
-        step.run()
-        for b in range(B):
-            hy_k[b, o:o + w].copy_(step.ky[b, o:o + w], non_blocking=True)
-            hy_v[b, o:o + w].copy_(step.vy[b, o:o + w], non_blocking=True)
+    def once(i):
+        r = i % 2
+        t, (hk, hv), (yk, yv) = sets[r], host_in[r], host_out[r]
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_cv[r])  # the conversions of step i-2 are done with this set's inputs
+            for b in range(B):
+                t["k"][b, o:o + w].copy_(hk[b, o:o + w], non_blocking=True)
+                t["v"][b, o:o + w].copy_(hv[b, o:o + w], non_blocking=True)
+            ev_in[r].record(s_in)
+        with torch.cuda.stream(s_cv):
+            s_cv.wait_event(ev_in[r])
+            s_cv.wait_event(ev_out[r])  # the download of step i-2 is done with this set's outputs
+            kvq.fp16_to_fp8_kv(t["k"], t["k8"], t["v"], t["v8"], B, o, w)
+            kvq.fp8_to_fp16_kv(t["k8"], t["ky"], t["v8"], t["vy"], B, o, w)
+            ev_cv[r].record(s_cv)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_cv[r])
+            for b in range(B):
+                yk[b, o:o + w].copy_(t["ky"][b, o:o + w], non_blocking=True)
+                yv[b, o:o + w].copy_(t["vy"][b, o:o + w], non_blocking=True)
+            ev_out[r].record(s_out)
 
-    for _ in range(warmup):
-        once()
+    for i in range(warmup):
+        once(i)
     torch.cuda.synchronize()
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
-    for _ in range(steps):
-        once()
-    e.record()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(s_in)
+    for i in range(steps):
+        once(i)
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(s_cv)
+    end.record(s_out)
     torch.cuda.synchronize()
-    ms = s.elapsed_time(e) / steps
+    ms = start.elapsed_time(end) / steps
     win_bytes = B * w * H * D * 2
     return ms, 2 * win_bytes, 2 * win_bytes
 
@@ -440,11 +467,15 @@ def per_op_measurements(kvq, dev, peak, steps, flush, step, include_model=True):
     launch on its own instead (L2 flushed before it, CUDA events around it)."""
     out = []
 
-    def record(name, config, nbytes, launch, sets=1, n=steps):
-        if nbytes >= 1 << 20:
+    def record(name, config, nbytes, launch, sets=1, n=steps, stream=None):
+        if stream is None:
+            stream = nbytes >= 1 << 20
+        if stream:
             ms, timing = time_stream(launch, sets, n, 3, flush, collective=False), "stream"
             if sets > 1:
                 timing += f", {sets} rotating input copies"
+            if nbytes < 1 << 20:
+                timing += " (inputs stay in L2, as a just-written decode token's would)"
         else:
             per, _ = time_device(lambda ev: launch(0), n, 3, flush, collective=False)
             ms, timing = statistics.mean(per), "isolated launch, L2 flushed"
@@ -524,6 +555,13 @@ def per_op_measurements(kvq, dev, peak, steps, flush, step, include_model=True):
         record(f"q_to_fp16_kv/q4/{phase}", cfg, nb,
                lambda i: kvq.q_to_fp16_kv(kc, pool.k, ks, vc, pool.v, vs, 32, off, w, ps, sl, bts[i % sets], 4),
                sets)
+        if phase == "decode":  # the same single-token launches back to back
+            record("fp16_to_q_kv/q4/decode/stream", cfg, nb,
+                   lambda i: kvq.fp16_to_q_kv(pool.k, kc, ks, pool.v, vc, vs, 32, off, w, ps, sl, bts[i % sets], 4),
+                   sets, stream=True)
+            record("fp16_to_fp8_kv/decode/stream", cfg8, nb8,
+                   lambda i: kvq.fp16_to_fp8_kv(pool.k, k8p, pool.v, v8p, 32, off, w, ps, sl, bts[i % sets]),
+                   sets, stream=True)
     del kc, vc, ks, vs, k8p, v8p
     torch.cuda.empty_cache()
 

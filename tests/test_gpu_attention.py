@@ -132,9 +132,23 @@ def test_paged_pool_full_size_sampled(kvq, oracle_mod, dev, wbits):
                                                 1.0 / math.sqrt(D), D)
     assert st == oracle_mod.OK
     got = out[pick].float().cpu().numpy().astype(np.float64)
-    vmax = float(ks.float().abs().max().cpu()) * (1 << (wbits - 1))
+    vmax = float(vs.float().abs().max().cpu()) * (1 << (wbits - 1))
     tol = np.spacing(np.maximum(np.abs(ex), 2.0 ** -14).astype(np.float16)).astype(np.float64) + 2.0 ** -14 * vmax
     assert np.all(np.abs(got - ex) <= tol)
+
+
+def test_many_short_sequences(kvq, oracle_mod, dev):
+    """More sequences than the kernel stages lengths for in shared memory (its lengths
+    then come from global memory), lengths 0..150 so that most work items are empty or
+    partial, and two 128-position chunks for the longest ones."""
+    B, S, H, D, NH = 300, 150, 2, 64, 4
+    k, v = workloads.normal_kv((B, S, H, D), 23)
+    kc, ks, vc, vs = quantize_on_gpu(kvq, k, v, 4, dev)
+    g = torch.Generator().manual_seed(5)
+    lens = torch.randint(0, S + 1, (B,), generator=g, dtype=torch.int32)
+    lens[:3] = torch.tensor([0, 1, S], dtype=torch.int32)
+    q = torch.randn(B, NH, D, generator=g).half()
+    check(kvq, oracle_mod, q, kc, ks, vc, vs, lens, 4, 1.0 / math.sqrt(D), dev)
 
 
 def test_bad_paging_reported(kvq, dev):

@@ -309,12 +309,27 @@ def _barrier():
         dist.barrier()
 
 
+def _upload_graph(g):
+    """Upload an instantiated CUDA graph to the device (driver cuGraphUpload) so that its
+    first replay inside a timed region costs what later replays cost; a no-op where the
+    driver call is unavailable."""
+    import ctypes
+
+    try:
+        drv = ctypes.CDLL("libcuda.so.1")
+        drv.cuGraphUpload(ctypes.c_void_p(g.raw_cuda_graph_exec()),
+                          ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    except (OSError, AttributeError, RuntimeError):
+        pass
+
+
 def _stream_graph(launch, n):
-    """CUDA graph of steps 0..n-1 of `launch(i)`, back to back."""
+    """CUDA graph of steps 0..n-1 of `launch(i)`, back to back, uploaded to the device."""
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         for i in range(n):
             launch(i)
+    _upload_graph(g)
     return g
 
 

@@ -467,7 +467,7 @@ bool allow_attention_smem() {
   return true;
 }
 
-// Persistent grid of the partial kernel: every (sequence, 128-position chunk,
+// Persistent grid of the partial kernel: every (sequence, 256-position chunk,
 // kv head) work item goes to one warp; as many CTAs as the device holds at
 // once (occupancy cached per device), never more than there are items.
 template <int B, int D>

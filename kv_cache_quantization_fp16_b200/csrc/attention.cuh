@@ -261,7 +261,7 @@ struct AttnTile {
   static constexpr int kStrideV = kRowBytes + ((B == 6 && D == 64) ? 0 : 16);
   static constexpr int kScales = D / 32;
   static constexpr int kChunk = 256;                        // positions per work item / workspace entry
-  static constexpr int kSub = kRowBytes <= 64 ? 32 : 16;   // positions per staged buffer
+  static constexpr int kSub = kRowBytes <= 96 ? 32 : 16;   // positions per staged buffer (measured)
   static constexpr int kBufK = kSub * kStrideK;
   static constexpr int kBufV = kSub * kStrideV;
   static constexpr int kBufS = kSub * kScales * 2;

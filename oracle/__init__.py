@@ -55,6 +55,9 @@ def lib() -> ctypes.CDLL:
         L.kvqref_decode_attention_q.argtypes = [u16p, u8p, u16p, u8p, u16p, u16p, f64p] + [I] * 7 + \
             [i32p, i32p, I, I, ctypes.c_double]
         L.kvqref_decode_attention_q.restype = ctypes.c_int
+        L.kvqref_decode_attention_fp8.argtypes = [u16p, u8p, u8p, u16p, f64p] + [I] * 7 + \
+            [i32p, i32p, I, ctypes.c_double]
+        L.kvqref_decode_attention_fp8.restype = ctypes.c_int
         i64p = ctypes.POINTER(ctypes.c_int64)
         LL = ctypes.c_longlong
         L.kvqref_count_match.argtypes = [i64p, LL, i64p, LL, LL]
@@ -264,4 +267,27 @@ def decode_attention_q(q, k_codes, k_scales, v_codes, v_scales, batch_size, n_he
         _p(np.ascontiguousarray(_bits(v_scales)), ctypes.c_uint16), _p(out, ctypes.c_uint16),
         _p(ex, ctypes.c_double), d0, d1, H, head_dim, batch_size, n_heads, page_size,
         _p(sl, ctypes.c_int32), _p(bt, ctypes.c_int32), stride, wbits, float(softmax_scale))
+    return st, out, ex
+
+
+def decode_attention_fp8(q, k_fp8, v_fp8, batch_size, n_heads, page_size, cache_seqlens, block_table,
+                         softmax_scale):
+    """fp64 decode attention over an FP8 (E5M2) cache, keys and values decoded exactly.
+    q: [batch, n_heads, D] float16/uint16; k_fp8, v_fp8: [d0, d1, H, D] uint8.  Returns
+    (status, out uint16 [batch, n_heads, D], exact float64 [batch, n_heads, D])."""
+    d0, d1, H, D = k_fp8.shape
+    qb = np.ascontiguousarray(_bits(q))
+    out = np.zeros((batch_size, n_heads, D), np.uint16)
+    ex = np.zeros((batch_size, n_heads, D), np.float64)
+    sl = np.ascontiguousarray(cache_seqlens, np.int32)
+    if page_size:
+        bt = np.ascontiguousarray(block_table, np.int32)
+        stride = bt.shape[1]
+    else:
+        bt, stride = None, 0
+    st = lib().kvqref_decode_attention_fp8(
+        _p(qb, ctypes.c_uint16), _p(np.ascontiguousarray(k_fp8, np.uint8), ctypes.c_uint8),
+        _p(np.ascontiguousarray(v_fp8, np.uint8), ctypes.c_uint8), _p(out, ctypes.c_uint16),
+        _p(ex, ctypes.c_double), d0, d1, H, D, batch_size, n_heads, page_size,
+        _p(sl, ctypes.c_int32), _p(bt, ctypes.c_int32), stride, float(softmax_scale))
     return st, out, ex

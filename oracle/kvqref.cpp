@@ -409,20 +409,22 @@ int kvqref_q_to_fp16_kv(const uint8_t* k_in, uint16_t* k_out, const uint16_t* k_
 // Usage ("convert KV tensors during the attention forward pass"): attention of
 // one new query per sequence over the dequantized cache, in double precision,
 // one position at a time.
-int kvqref_decode_attention_q(const uint16_t* q, const uint8_t* k_codes, const uint16_t* k_scales,
-                              const uint8_t* v_codes, const uint16_t* v_scales, uint16_t* out,
-                              double* out_exact, int dim0, int dim1, int heads, int head_dim,
-                              int batch_size, int n_heads, int page_size, const int32_t* cache_seqlens,
-                              const int32_t* block_table, int bt_stride, int wbits, double softmax_scale) {
-  if (!valid_wbits(wbits) || heads <= 0 || head_dim <= 0 || head_dim % kBlock || head_dim > 65536) return KVQREF_BAD_ARG;
-  if (n_heads <= 0 || n_heads % heads || batch_size < 0 || dim0 < 0 || dim1 < 0 || !cache_seqlens) return KVQREF_BAD_ARG;
-  if (page_size < 0 || (page_size > 0 && (dim1 != page_size || !block_table))) return KVQREF_BAD_ARG;
-  if (page_size == 0 && batch_size > dim0) return KVQREF_BAD_ARG;
+}  // extern "C" (the shared attention loop below is C++)
+
+namespace {
+
+// Decode attention for one query over positions [0, seqlen) of sequence i:
+// `key_row(hr, out)` / `value_row(hr, out)` write the binary16 key / value of
+// cache row hr (row * heads + kv head).  Scores, softmax and the weighted sum
+// in double precision, one position at a time, in the order the definition
+// states them.
+template <class KeyRow, class ValueRow>
+int attention_rows(const uint16_t* q, uint16_t* out, double* out_exact, int dim0, int dim1, int heads, int head_dim,
+                   int batch_size, int n_heads, int page_size, const int32_t* cache_seqlens,
+                   const int32_t* block_table, int bt_stride, double softmax_scale, KeyRow key_row,
+                   ValueRow value_row) {
   const int group = n_heads / heads;
-  const long code_bytes = static_cast<long>(head_dim) * wbits / 8;
-  const long nscales = head_dim / kBlock;
   int status = KVQREF_OK;
-  uint8_t codes[65536];
   uint16_t deq[65536];
   for (int i = 0; i < batch_size; ++i) {
     const long L = cache_seqlens[i] < 0 ? 0 : cache_seqlens[i];
@@ -448,8 +450,7 @@ int kvqref_decode_attention_q(const uint16_t* q, const uint8_t* k_codes, const u
           row = static_cast<long>(page) * page_size + p % page_size;
         }
         const long hr = row * heads + kvh;
-        unpack_row(k_codes + hr * code_bytes, head_dim, wbits, codes);
-        dequantize_row(codes, k_scales + hr * nscales, head_dim, wbits, deq);
+        key_row(hr, deq);
         double dot = 0.0;
         for (int d = 0; d < head_dim; ++d) dot += half_to_double(qh[d]) * half_to_double(deq[d]);
         s[n_valid] = softmax_scale * dot;
@@ -465,8 +466,7 @@ int kvqref_decode_attention_q(const uint16_t* q, const uint8_t* k_codes, const u
       for (int d = 0; d < head_dim; ++d) acc[d] = 0.0;
       for (long j = 0; j < n_valid; ++j) {
         const double w = std::exp(s[j] - m) / denom;
-        unpack_row(v_codes + rows[j] * code_bytes, head_dim, wbits, codes);
-        dequantize_row(codes, v_scales + rows[j] * nscales, head_dim, wbits, deq);
+        value_row(rows[j], deq);
         for (int d = 0; d < head_dim; ++d) acc[d] += w * half_to_double(deq[d]);
       }
       uint16_t* oh = out + (static_cast<long>(i) * n_heads + h) * head_dim;
@@ -480,6 +480,54 @@ int kvqref_decode_attention_q(const uint16_t* q, const uint8_t* k_codes, const u
     }
   }
   return status;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kvqref_decode_attention_q(const uint16_t* q, const uint8_t* k_codes, const uint16_t* k_scales,
+                              const uint8_t* v_codes, const uint16_t* v_scales, uint16_t* out,
+                              double* out_exact, int dim0, int dim1, int heads, int head_dim,
+                              int batch_size, int n_heads, int page_size, const int32_t* cache_seqlens,
+                              const int32_t* block_table, int bt_stride, int wbits, double softmax_scale) {
+  if (!valid_wbits(wbits) || heads <= 0 || head_dim <= 0 || head_dim % kBlock || head_dim > 65536) return KVQREF_BAD_ARG;
+  if (n_heads <= 0 || n_heads % heads || batch_size < 0 || dim0 < 0 || dim1 < 0 || !cache_seqlens) return KVQREF_BAD_ARG;
+  if (page_size < 0 || (page_size > 0 && (dim1 != page_size || !block_table))) return KVQREF_BAD_ARG;
+  if (page_size == 0 && batch_size > dim0) return KVQREF_BAD_ARG;
+  const long code_bytes = static_cast<long>(head_dim) * wbits / 8;
+  const long nscales = head_dim / kBlock;
+  uint8_t codes[65536];
+  // keys and values: the packed codes unpacked and dequantized exactly as kvqref_q_to_fp16_kv does
+  auto k_row = [&](long hr, uint16_t* o) {
+    unpack_row(k_codes + hr * code_bytes, head_dim, wbits, codes);
+    dequantize_row(codes, k_scales + hr * nscales, head_dim, wbits, o);
+  };
+  auto v_row = [&](long hr, uint16_t* o) {
+    unpack_row(v_codes + hr * code_bytes, head_dim, wbits, codes);
+    dequantize_row(codes, v_scales + hr * nscales, head_dim, wbits, o);
+  };
+  return attention_rows(q, out, out_exact, dim0, dim1, heads, head_dim, batch_size, n_heads, page_size, cache_seqlens,
+                        block_table, bt_stride, softmax_scale, k_row, v_row);
+}
+
+int kvqref_decode_attention_fp8(const uint16_t* q, const uint8_t* k_fp8, const uint8_t* v_fp8, uint16_t* out,
+                                double* out_exact, int dim0, int dim1, int heads, int head_dim, int batch_size,
+                                int n_heads, int page_size, const int32_t* cache_seqlens, const int32_t* block_table,
+                                int bt_stride, double softmax_scale) {
+  if (heads <= 0 || head_dim <= 0 || head_dim > 65536) return KVQREF_BAD_ARG;
+  if (n_heads <= 0 || n_heads % heads || batch_size < 0 || dim0 < 0 || dim1 < 0 || !cache_seqlens) return KVQREF_BAD_ARG;
+  if (page_size < 0 || (page_size > 0 && (dim1 != page_size || !block_table))) return KVQREF_BAD_ARG;
+  if (page_size == 0 && batch_size > dim0) return KVQREF_BAD_ARG;
+  // keys and values: each E5M2 byte decoded exactly as kvqref_fp8_to_fp16 does
+  auto k_row = [&](long hr, uint16_t* o) {
+    for (int d = 0; d < head_dim; ++d) o[d] = e5m2_decode(k_fp8[hr * head_dim + d]);
+  };
+  auto v_row = [&](long hr, uint16_t* o) {
+    for (int d = 0; d < head_dim; ++d) o[d] = e5m2_decode(v_fp8[hr * head_dim + d]);
+  };
+  return attention_rows(q, out, out_exact, dim0, dim1, heads, head_dim, batch_size, n_heads, page_size, cache_seqlens,
+                        block_table, bt_stride, softmax_scale, k_row, v_row);
 }
 
 // Description, count_match: compare element by element from the start and

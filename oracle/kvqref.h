@@ -138,6 +138,14 @@ int kvqref_decode_attention_q(const uint16_t* q, const uint8_t* k_codes, const u
                               int batch_size, int n_heads, int page_size, const int32_t* cache_seqlens,
                               const int32_t* block_table, int bt_stride, int wbits, double softmax_scale);
 
+/* Decode attention over an FP8 (E5M2) cache: as kvqref_decode_attention_q,
+ * with keys and values the E5M2 bytes decoded exactly as kvqref_fp8_to_fp16
+ * does.  k_fp8, v_fp8: [dim0, dim1, heads, head_dim] bytes. */
+int kvqref_decode_attention_fp8(const uint16_t* q, const uint8_t* k_fp8, const uint8_t* v_fp8, uint16_t* out,
+                                double* out_exact, int dim0, int dim1, int heads, int head_dim, int batch_size,
+                                int n_heads, int page_size, const int32_t* cache_seqlens, const int32_t* block_table,
+                                int bt_stride, double softmax_scale);
+
 /* count_match (Description; I/O Contract): length of the common prefix of two
  * 64-bit element sequences, looking at no more than max_a elements. */
 long long kvqref_count_match(const int64_t* a, long long a_len, const int64_t* b, long long b_len,

@@ -1,5 +1,6 @@
-"""Pins for the oracle's decode attention over a quantized cache (the consumer the
-page's Usage section names: conversions "during the attention forward pass").
+"""Pins for the oracle's decode attention over a quantized (Q4/Q6/Q8) or FP8 (E5M2) cache
+(the consumer the page's Usage section names: conversions "during the attention forward
+pass").
 
 * one position: the output is that position's dequantized value exactly;
 * zero query: every score is 0, the output is the mean of the values;
@@ -180,4 +181,100 @@ def test_empty_window_and_bad_args(oracle_mod):
     st, _, _ = oracle_mod.decode_attention_q(q3, kc, ks, kc, ks, 1, 3, 0, np.array([2], np.int32), None, 4, 1.0, D)
     assert st == oracle_mod.BAD_ARG  # 3 query heads do not split over 2 kv heads
     st, _, _ = oracle_mod.decode_attention_q(q, kc, ks, kc, ks, 1, 2, 0, np.array([5], np.int32), None, 4, 1.0, D)
+    assert st == oracle_mod.BAD_ARG  # window longer than the cache
+
+
+# ---- decode attention over an FP8 (E5M2) cache -------------------------------------------
+
+def _e5m2_numpy(b: np.ndarray) -> np.ndarray:
+    """E5M2 bytes to float64 without the oracle: the byte is the high byte of a binary16."""
+    return (b.astype(np.uint16) << 8).view(np.float16).astype(np.float64)
+
+
+def _fp8_cache(B, S, H, D, seed):
+    """Random E5M2 bytes drawn directly (independent of the oracle's encoder): random sign and
+    mantissa bits, exponent field in [9, 17], so magnitudes lie in [2^-6, 7] and no byte is
+    Inf or NaN."""
+    g = np.random.default_rng(seed)
+    def draw():
+        b = g.integers(0, 256, (B, S, H, D), dtype=np.uint8)
+        e = g.integers(9, 18, (B, S, H, D), dtype=np.uint8)
+        return ((b & 0x83) | (e << 2)).astype(np.uint8)
+    return draw(), draw()
+
+
+def test_fp8_single_position_returns_value(oracle_mod):
+    B, S, H, D, NH = 2, 3, 2, 64, 4
+    k8, v8 = _fp8_cache(B, S, H, D, 11)
+    q = _np16(torch.randn(B, NH, D).half())
+    st, out, ex = oracle_mod.decode_attention_fp8(q, k8, v8, B, NH, 0, np.array([1, 1], np.int32), None, 0.125)
+    assert st == oracle_mod.OK
+    vv = _e5m2_numpy(v8)
+    for i in range(B):
+        for h in range(NH):
+            assert np.array_equal(ex[i, h], vv[i, 0, h // 2])
+            assert np.array_equal(out[i, h], (v8[i, 0, h // 2].astype(np.uint16) << 8))
+
+
+def test_fp8_zero_query_is_the_mean(oracle_mod):
+    B, S, H, D, NH = 1, 29, 1, 32, 2
+    k8, v8 = _fp8_cache(B, S, H, D, 12)
+    q = np.zeros((B, NH, D), np.uint16)
+    st, out, ex = oracle_mod.decode_attention_fp8(q, k8, v8, B, NH, 0, np.array([S], np.int32), None, 1.0)
+    assert st == oracle_mod.OK
+    assert np.allclose(ex[0, 0], _e5m2_numpy(v8)[0, :, 0].mean(axis=0), rtol=1e-13, atol=1e-15)
+
+
+def test_fp8_two_positions_closed_form(oracle_mod):
+    """k_0 = 0 and k_1[0] = 2 (byte 0x40); q = e_0 and scale ln 3 / 2 give scores 0 and ln 3, so
+    the weights are exactly 1/4 and 3/4; v_0 = 1 (0x3C), v_1 = 2 (0x40) everywhere makes the
+    output exactly 1/4 + 3/2 = 1.75."""
+    D = 16
+    k8 = np.zeros((1, 2, 1, D), np.uint8)
+    k8[0, 1, 0, 0] = 0x40
+    v8 = np.zeros((1, 2, 1, D), np.uint8)
+    v8[0, 0], v8[0, 1] = 0x3C, 0x40
+    q = np.zeros((1, 1, D), np.float16)
+    q[0, 0, 0] = 1.0
+    st, out, ex = oracle_mod.decode_attention_fp8(q.view(np.uint16), k8, v8, 1, 1, 0, np.array([2], np.int32), None,
+                                                  math.log(3.0) / 2.0)
+    assert st == oracle_mod.OK
+    assert np.allclose(ex[0, 0], 1.75, rtol=1e-14, atol=0)
+    assert np.all(out[0, 0] == np.float16(1.75).view(np.uint16))
+
+
+def test_fp8_paged_equals_contiguous_and_matches_numpy(oracle_mod):
+    B, S, H, D, NH, ps = 3, 64, 2, 64, 8, 16
+    k8, v8 = _fp8_cache(B, S, H, D, 13)
+    lens = np.array([64, 1, 40], np.int32)
+    q16 = torch.randn(B, NH, D).half()
+    q = _np16(q16)
+    st, out_c, ex_c = oracle_mod.decode_attention_fp8(q, k8, v8, B, NH, 0, lens, None, 0.125)
+    assert st == oracle_mod.OK
+    pages = (B * S // ps, ps, H, D)
+    ident = workloads.identity_block_table(B, S, ps).numpy()
+    st, out_p, ex_p = oracle_mod.decode_attention_fp8(q, k8.reshape(pages), v8.reshape(pages), B, NH, ps, lens,
+                                                      ident, 0.125)
+    assert st == oracle_mod.OK and np.array_equal(out_c, out_p) and np.array_equal(ex_c, ex_p)
+    perm = np.random.default_rng(1).permutation(pages[0])
+    kp, vp = np.empty_like(k8.reshape(pages)), np.empty_like(v8.reshape(pages))
+    kp[perm], vp[perm] = k8.reshape(pages), v8.reshape(pages)
+    st, out_m, _ = oracle_mod.decode_attention_fp8(q, kp, vp, B, NH, ps, lens, perm[ident].astype(np.int32), 0.125)
+    assert st == oracle_mod.OK and np.array_equal(out_m, out_c)
+    # numpy restatement: decode, softmax, weighted sum
+    kk, vv, qf = _e5m2_numpy(k8), _e5m2_numpy(v8), q16.double().numpy()
+    for i in range(B):
+        for h in range(NH):
+            sc = 0.125 * kk[i, : lens[i], h // 4] @ qf[i, h]
+            w = np.exp(sc - sc.max())
+            assert np.allclose(ex_c[i, h], (w / w.sum()) @ vv[i, : lens[i], h // 4], rtol=1e-12, atol=1e-14)
+
+
+def test_fp8_bad_args(oracle_mod):
+    k8 = np.zeros((1, 4, 2, 16), np.uint8)
+    q3 = np.zeros((1, 3, 16), np.uint16)
+    st, _, _ = oracle_mod.decode_attention_fp8(q3, k8, k8, 1, 3, 0, np.array([2], np.int32), None, 1.0)
+    assert st == oracle_mod.BAD_ARG  # 3 query heads do not split over 2 kv heads
+    q = np.zeros((1, 2, 16), np.uint16)
+    st, _, _ = oracle_mod.decode_attention_fp8(q, k8, k8, 1, 2, 0, np.array([5], np.int32), None, 1.0)
     assert st == oracle_mod.BAD_ARG  # window longer than the cache

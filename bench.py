@@ -595,6 +595,11 @@ def per_op_measurements(kvq, dev, peak, steps, flush, step, include_model=True):
                f"paged 2048x256x8x128 pool, 32 seqs, 32 query heads, wbits={wb}", nb, lambda i: fn())
         del fn
         torch.cuda.empty_cache()
+    fn, nb = attention_setup_fp8(kvq, dev, pool)
+    record("decode_attention_fp8/paged", "paged 2048x256x8x128 pool, 32 seqs, 32 query heads, E5M2", nb,
+           lambda i: fn())
+    del fn
+    torch.cuda.empty_cache()
     del pool
     torch.cuda.empty_cache()
 
@@ -612,6 +617,29 @@ def attention_bytes(lens, kv_heads, head_dim, wbits, n_heads=ATTN_QUERY_HEADS):
     per_row = head_dim * wbits // 8 + 2 * (head_dim // 32)
     npos = sum(int(L) for L in lens)
     return 2 * npos * kv_heads * per_row + 2 * 2 * len(lens) * n_heads * head_dim
+
+
+def attention_setup_fp8(kvq, dev, pool, n_heads=ATTN_QUERY_HEADS):
+    """Encode the whole pool to E5M2 (untimed) and return (launch, algorithmic bytes) of decode
+    attention over it: one byte per cached element, no scales."""
+    P, ps, H, D = pool.k.shape
+    batch = pool.cache_seqlens.numel()
+    k8 = torch.zeros(pool.k.shape, dtype=torch.uint8, device=dev)
+    v8 = torch.zeros_like(k8)
+    full = pool.block_table.shape[1] * ps
+    kvq.fp16_to_fp8_kv(pool.k, k8, pool.v, v8, batch, -full, full, ps, pool.cache_seqlens, pool.block_table)
+    g = torch.Generator(device="cpu").manual_seed(workloads.SEED_BASE + 77)
+    q = torch.randn(batch, n_heads, D, generator=g).half().to(dev)
+    out = torch.empty_like(q)
+    ws = torch.empty(max(16, kvq.attention_workspace_bytes(tuple(pool.k.shape), batch, n_heads, ps,
+                                                           pool.block_table.shape[1])), dtype=torch.uint8, device=dev)
+    scale = 1.0 / math.sqrt(D)
+
+    def fn():
+        kvq.decode_attention_fp8(q, k8, v8, out, batch, pool.cache_seqlens, scale, ps, pool.block_table, ws)
+    fn()
+    npos = sum(int(L) for L in pool.cache_seqlens.cpu().tolist())
+    return fn, 2 * npos * H * D + 2 * 2 * batch * n_heads * D
 
 
 def attention_setup(kvq, dev, pool, wbits, n_heads=ATTN_QUERY_HEADS):
@@ -682,7 +710,7 @@ def model_layers(kvq, dev, peak, steps, flush, layers=32):
 CASES = ("headline_fp8enc_kv", "headline_fp8dec_kv", "headline_fp8enc", "headline_fp8dec", "fp8enc", "fp8dec", "q4enc",
          "q4dec", "q6enc", "q6dec", "q8enc", "q8dec", "paged_prefill_q4enc", "paged_prefill_q4dec",
          "paged_decode_q4enc", "model_layer_q6enc", "model_layer_q6dec", "attn_paged_q4", "attn_paged_q6",
-         "attn_paged_q8")
+         "attn_paged_q8", "attn_paged_fp8")
 
 
 def run_case(kvq, dev, name, batch, steps, warmup, peak, stream=False):
@@ -742,6 +770,9 @@ def run_case(kvq, dev, name, batch, steps, warmup, peak, stream=False):
             fn = (lambda: kvq.fp16_to_q_kv(k, kc, ks, v, vc, vs, B, 0, S, 0, None, None, wb)) \
                 if name.endswith("enc") else (lambda: kvq.q_to_fp16_kv(kc, ky, ks, vc, vy, vs, B, 0, S, 0, None,
                                                                         None, wb))
+    elif name == "attn_paged_fp8":
+        pool = workloads.paged_pool(device=dev)
+        fn, nb = attention_setup_fp8(kvq, dev, pool)
     elif name.startswith("attn_paged"):
         pool = workloads.paged_pool(device=dev)
         fn, nb = attention_setup(kvq, dev, pool, int(name[-1]))

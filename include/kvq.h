@@ -197,8 +197,22 @@ KVQ_API kvq_status kvq_decode_attention_q(const void* q, const void* k_codes, co
                                           float softmax_scale, void* workspace, size_t workspace_bytes,
                                           void* stream);
 
-/* Workspace bytes kvq_decode_attention_q needs for this geometry (0 for bad
- * arguments).  Host-only. */
+/* Decode attention over an FP8 (E5M2) KV cache: kvq_decode_attention_q with
+ * keys and values the E5M2 bytes decoded exactly as kvq_fp8_to_fp16 does (the
+ * page's Usage section converts the FP8 cache during the attention forward
+ * pass as it does the Q cache).  There are no scales.
+ *   k_fp8, v_fp8  [dim0, dim1, kv_heads, head_dim] uint8 (E5M2), 16-byte aligned
+ *   Everything else (q, out, paging, workspace, softmax_scale, stream, errors,
+ *   two kernels enqueued) as for kvq_decode_attention_q; head_dim 64, 128 or 256.
+ *   A stored Inf or NaN byte propagates into the outputs that attend to it. */
+KVQ_API kvq_status kvq_decode_attention_fp8(const void* q, const void* k_fp8, const void* v_fp8, void* out,
+                                            const kvq_cache_desc* desc, int batch_size, int n_heads, int page_size,
+                                            const int32_t* cache_seqlens, const int32_t* block_table,
+                                            float softmax_scale, void* workspace, size_t workspace_bytes,
+                                            void* stream);
+
+/* Workspace bytes kvq_decode_attention_q and kvq_decode_attention_fp8 need for
+ * this geometry (0 for bad arguments).  Host-only. */
 KVQ_API size_t kvq_decode_attention_workspace_size(const kvq_cache_desc* desc, int batch_size, int n_heads,
                                                    int page_size);
 

@@ -28,7 +28,7 @@ import torch
 __all__ = ["fp16_to_fp8", "fp8_to_fp16", "fp16_to_fp8_kv", "fp8_to_fp16_kv", "fp16_to_q_kv", "q_to_fp16_kv", "poll_device_error",
            "selfcheck_code_rounding", "count_match", "decode_attention_q", "decode_attention_q_noalloc",
            "attention_workspace_bytes", "q_shapes", "set_engine", "get_engine", "engine", "KVQError",
-           "LIB_PATH", "library"]
+           "LIB_PATH", "library", "decode_attention_fp8"]
 
 ENGINES = {"auto": 0, "ldg": 1, "bulk": 2}
 
@@ -73,6 +73,9 @@ def _load() -> ctypes.CDLL:
     L.kvq_decode_attention_q.argtypes = [vp, vp, vp, vp, vp, vp, dp, I, I, I, vp, vp, I, ctypes.c_float, vp,
                                          ctypes.c_size_t, vp]
     L.kvq_decode_attention_q.restype = I
+    L.kvq_decode_attention_fp8.argtypes = [vp, vp, vp, vp, dp, I, I, I, vp, vp, ctypes.c_float, vp, ctypes.c_size_t,
+                                           vp]
+    L.kvq_decode_attention_fp8.restype = I
     L.kvq_decode_attention_q_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, dp, I, I, I, vp, vp, I, ctypes.c_float,
                                                  vp]
     L.kvq_decode_attention_q_noalloc.restype = I
@@ -368,6 +371,45 @@ def decode_attention_q(q, k_codes, k_scales, v_codes, v_scales, out, batch_size,
                                          int(n_heads), int(page_size), cache_seqlens.data_ptr(), bt_ptr, int(wbits),
                                          float(softmax_scale), workspace.data_ptr(), workspace.numel(), _stream(dev))
     _check(st, "decode_attention_q")
+
+
+def decode_attention_fp8(q, k_fp8, v_fp8, out, batch_size, cache_seqlens, softmax_scale, page_size=0,
+                         block_table=None, workspace=None) -> None:
+    """Decode attention reading an FP8 (E5M2) cache directly, the bytes decoded exactly as
+    fp8_to_fp16 does (no FP16 cache is written).
+
+    q, out: [batch, n_heads, head_dim] float16 CUDA tensors; k_fp8, v_fp8: [d0, d1, kv_heads,
+    head_dim] uint8 as written by fp16_to_fp8 / fp16_to_fp8_kv; cache_seqlens, paging and
+    ``workspace`` as for decode_attention_q."""
+    _require(isinstance(q, torch.Tensor) and q.dtype == torch.float16 and q.is_cuda and q.dim() == 3
+             and q.is_contiguous(), "q must be a contiguous [batch, n_heads, head_dim] float16 CUDA tensor")
+    _require(out.shape == q.shape and out.dtype == torch.float16 and out.is_contiguous() and out.device == q.device,
+             "out must match q")
+    D = q.shape[2]
+    for t, n in ((k_fp8, "k_fp8"), (v_fp8, "v_fp8")):
+        _cuda4(t, torch.uint8, n)
+        _require(t.shape[3] == D and t.device == q.device, f"{n} must be [d0, d1, kv_heads, {D}] on q's device")
+    _require(k_fp8.shape == v_fp8.shape, "k_fp8 and v_fp8 must have one shape")
+    dev = q.device
+    _require(cache_seqlens is not None and cache_seqlens.dtype == torch.int32 and cache_seqlens.device == dev
+             and cache_seqlens.is_contiguous() and cache_seqlens.numel() >= batch_size,
+             "cache_seqlens must be a contiguous int32 tensor on the caches' device with batch_size entries")
+    stride, _, bt_ptr = _paging(page_size, cache_seqlens, block_table, batch_size, dev)
+    d0, d1, H, _ = k_fp8.shape
+    desc = _Desc(d0, d1, H, D, stride)
+    n_heads = q.shape[1]
+    need = int(_lib.kvq_decode_attention_workspace_size(ctypes.byref(desc), int(batch_size), int(n_heads),
+                                                        int(page_size)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _require(workspace.is_cuda and workspace.device == dev and workspace.numel() >= need,
+             f"workspace must hold at least {need} bytes on the caches' device")
+    with torch.cuda.device(dev):
+        st = _lib.kvq_decode_attention_fp8(q.data_ptr(), k_fp8.data_ptr(), v_fp8.data_ptr(), out.data_ptr(),
+                                           ctypes.byref(desc), int(batch_size), int(n_heads), int(page_size),
+                                           cache_seqlens.data_ptr(), bt_ptr, float(softmax_scale),
+                                           workspace.data_ptr(), workspace.numel(), _stream(dev))
+    _check(st, "decode_attention_fp8")
 
 
 ATTENTION_SCRATCH_BYTES = 16 << 20  # KVQ_ATTENTION_SCRATCH_BYTES

@@ -6,7 +6,8 @@
 // One new query per sequence and head; GQA: `group` query heads share a kv
 // head.  Keys and values are the dequantized codes, bit for bit what
 // q_to_fp16_kv writes: RN16((code - z) * s), with (code - z) formed exactly
-// in binary16 and one rounding in the multiply.
+// in binary16 and one rounding in the multiply; or, for an FP8 cache (format
+// code 0), the E5M2 bytes decoded exactly as fp8_to_fp16 does.
 //
 // Split-K flash decoding.  Kernel 1 (attn_partial_kernel): one CTA per
 // (chunk of positions, kv head, sequence), four warps.  The CTA copies its
@@ -158,6 +159,36 @@ struct AttnCodec<4> {
   }
 };
 
+// FP8 (E5M2; format code 0): the byte is the high byte of the binary16 value,
+// so a byte permute against zero decodes two values exactly; no scale.
+template <>
+struct AttnCodec<0> {
+  // pairs per 32-bit word: (0,1), (2,3)
+  __host__ __device__ static constexpr int row_pair_elem(int r, int e) { return 2 * r + e; }
+  __host__ __device__ static constexpr int xrow_elem(int r) { return r; }
+  template <int NW>
+  __device__ static void row_pairs(const uint32_t (&w)[NW], uint32_t (&out)[2 * NW]) {
+#pragma unroll
+    for (int i = 0; i < NW; ++i) {
+      out[2 * i + 0] = __byte_perm(w[i], 0u, 0x1404);  // [0, b0, 0, b1]
+      out[2 * i + 1] = __byte_perm(w[i], 0u, 0x3424);  // [0, b2, 0, b3]
+    }
+  }
+  // rows r0, r1 (NW words each) -> 4 * NW cross-row pairs, element order 0..4NW-1
+  template <int NW>
+  __device__ static void xrow_pairs(const uint32_t (&w0)[NW], const uint32_t (&w1)[NW], uint32_t (&out)[4 * NW]) {
+#pragma unroll
+    for (int i = 0; i < NW; ++i) {
+      const uint32_t a = w0[i] << 8, b = w1[i] << 8;    // [0, b0, b1, b2] of each row
+      const uint32_t c = w0[i] >> 16, d = w1[i] >> 16;  // [b2, b3, 0, 0] of each row
+      out[4 * i + 0] = __byte_perm(a, b, 0x5410);
+      out[4 * i + 1] = __byte_perm(a, b, 0x6420);
+      out[4 * i + 2] = __byte_perm(a, b, 0x7430);
+      out[4 * i + 3] = __byte_perm(c, d, 0x5612);
+    }
+  }
+};
+
 template <>
 struct AttnCodec<8> {
   static constexpr int kZ = 128;
@@ -256,10 +287,11 @@ struct AttnCodec<6> {
 // rows; V: four rows per lane, byte-interleaved in pairs).
 template <int B, int D>
 struct AttnTile {
-  static constexpr int kRowBytes = D * B / 8;
+  static constexpr int kBits = B == 0 ? 8 : B;  // bits per cached element (format 0: E5M2 bytes)
+  static constexpr int kRowBytes = D * kBits / 8;
   static constexpr int kStrideK = kRowBytes + (kRowBytes % 128 == 0 ? 16 : 0);
   static constexpr int kStrideV = kRowBytes + ((B == 6 && D == 64) ? 0 : 16);
-  static constexpr int kScales = D / 32;
+  static constexpr int kScales = B == 0 ? 0 : D / 32;  // binary16 scales per row
   static constexpr int kChunk = 256;                        // positions per work item / workspace entry
   static constexpr int kSub = kRowBytes <= 96 ? 32 : 16;   // positions per staged buffer (measured)
   static constexpr int kBufK = kSub * kStrideK;
@@ -273,8 +305,8 @@ struct AttnTile {
   static constexpr int KN = D / 4;   // K elements per lane per position (one contiguous span)
   static constexpr int VN = D / 8;   // V elements per lane per row (one contiguous span)
   static constexpr int KS = D / 16;  // k-steps of Q K^T = m-tiles of V^T P^T
-  static constexpr int kKSpanBytes = KN * B / 8;
-  static constexpr int kVSpanBytes = VN * B / 8;
+  static constexpr int kKSpanBytes = KN * kBits / 8;
+  static constexpr int kVSpanBytes = VN * kBits / 8;
 };
 constexpr int kAttnMinChunk = 128;  // sizes the workspace: no (B, D) uses a shorter chunk
 
@@ -328,10 +360,10 @@ __device__ __forceinline__ void k_span(const uint8_t* row, const __half* srow, i
   } else {
     AttnCodec<B>::template row_pairs<NB / 4>(w, out);
   }
-  // scales: one 32-element block per 16 registers (KN <= 32: one block)
+  // scales: one 32-element block per 16 registers (KN <= 32: one block); E5M2 has none
   constexpr int kRegsPerBlock = 16;
 #pragma unroll
-  for (int b = 0; b < (KN + 31) / 32; ++b) {
+  for (int b = 0; b < (T::kScales ? (KN + 31) / 32 : 0); ++b) {
     const __half s = srow[(KN * j) / 32 + b];
     const __half2 s2 = __halves2half2(s, s);
 #pragma unroll
@@ -371,9 +403,11 @@ __device__ __forceinline__ void v_span_pair(const uint8_t* r0, const uint8_t* r1
       AttnCodec<B>::template xrow_pairs<NB / 4>(w0, w1, out);
     }
   }
-  const __half2 s2 = __halves2half2(s0, s1);
+  if constexpr (T::kScales > 0) {
+    const __half2 s2 = __halves2half2(s0, s1);
 #pragma unroll
-  for (int r = 0; r < VN; ++r) out[r] = scale_pair(out[r], s2);
+    for (int r = 0; r < VN; ++r) out[r] = scale_pair(out[r], s2);
+  }
 }
 
 
@@ -483,15 +517,27 @@ __device__ __forceinline__ uint32_t attn_issue(const AttnParams& a, const AttnCu
       cp_async16(sv + r * T::kStrideV + part * 16, a.v_codes + src);
     }
   }
-  // scales; rows without data get zero scales, which dequantize whatever codes
-  // the buffer holds to zero
-  if (lane < SC) {
-    if (hr >= 0) {
-      cp_async_small<T::kScales * 2>(sks + lane * T::kScales, a.k_scales + hr * T::kScales);
-      cp_async_small<T::kScales * 2>(svs + lane * T::kScales, a.v_scales + hr * T::kScales);
-    } else {
+  if constexpr (T::kScales > 0) {
+    // scales; rows without data get zero scales, which dequantize whatever codes
+    // the buffer holds to zero
+    if (lane < SC) {
+      if (hr >= 0) {
+        cp_async_small<T::kScales * 2>(sks + lane * T::kScales, a.k_scales + hr * T::kScales);
+        cp_async_small<T::kScales * 2>(svs + lane * T::kScales, a.v_scales + hr * T::kScales);
+      } else {
 #pragma unroll
-      for (int e = 0; e < T::kScales; ++e) sks[lane * T::kScales + e] = svs[lane * T::kScales + e] = __ushort_as_half(0);
+        for (int e = 0; e < T::kScales; ++e)
+          sks[lane * T::kScales + e] = svs[lane * T::kScales + e] = __ushort_as_half(0);
+      }
+    }
+  } else {
+    // E5M2 has no scale: a value row without data is zeroed (its weight is 0, but a
+    // stale Inf or NaN byte would still poison the weighted sum); key rows are masked
+    // by their -inf score instead
+    if (lane < SC && hr < 0) {
+#pragma unroll
+      for (int part = 0; part < P; ++part)
+        *reinterpret_cast<uint4*>(sv + lane * T::kStrideV + part * 16) = make_uint4(0u, 0u, 0u, 0u);
     }
   }
   // the item's query rows travel with its first sub-chunk
@@ -644,10 +690,13 @@ __global__ void __launch_bounds__(kAttnThreads, D > 128 ? 2 : 4) attn_partial_ke
       {
         const int i0 = t0 + 2 * j, i1 = i0 + 8;
         const int sblk = (T::VN * g) / 32;
-        v_span_pair<B, D>(sv + i0 * T::kStrideV, sv + (i0 + 1) * T::kStrideV, svs[i0 * T::kScales + sblk],
-                          svs[(i0 + 1) * T::kScales + sblk], g, va);
-        v_span_pair<B, D>(sv + i1 * T::kStrideV, sv + (i1 + 1) * T::kStrideV, svs[i1 * T::kScales + sblk],
-                          svs[(i1 + 1) * T::kScales + sblk], g, vb);
+        const __half zero = __ushort_as_half(0);
+        const __half s00 = T::kScales ? svs[i0 * T::kScales + sblk] : zero;
+        const __half s01 = T::kScales ? svs[(i0 + 1) * T::kScales + sblk] : zero;
+        const __half s10 = T::kScales ? svs[i1 * T::kScales + sblk] : zero;
+        const __half s11 = T::kScales ? svs[(i1 + 1) * T::kScales + sblk] : zero;
+        v_span_pair<B, D>(sv + i0 * T::kStrideV, sv + (i0 + 1) * T::kStrideV, s00, s01, g, va);
+        v_span_pair<B, D>(sv + i1 * T::kStrideV, sv + (i1 + 1) * T::kStrideV, s10, s11, g, vb);
       }
 #pragma unroll
       for (int mt = 0; mt < KS; ++mt) {

@@ -510,14 +510,21 @@ size_t kvq_decode_attention_workspace_size(const kvq_cache_desc* desc, int batch
          (desc->head_dim + 2) * sizeof(float);
 }
 
-kvq_status kvq_decode_attention_q(const void* q, const void* k_codes, const void* k_scales, const void* v_codes,
-                                  const void* v_scales, void* out, const kvq_cache_desc* desc, int batch_size,
-                                  int n_heads, int page_size, const int32_t* cache_seqlens,
-                                  const int32_t* block_table, int wbits, float softmax_scale, void* workspace,
-                                  size_t workspace_bytes, void* stream) {
-  if (!q || !k_codes || !k_scales || !v_codes || !v_scales || !out || !desc || !cache_seqlens) return KVQ_ERR_NULL;
-  if (wbits != 4 && wbits != 6 && wbits != 8) return KVQ_ERR_WBITS;
-  kvq_status st = check_desc(desc, 32);
+}  // extern "C"
+
+namespace {
+
+// Shared argument checks and launch of the decode-attention entry points:
+// format 4 / 6 / 8 = Q codes with scales, 0 = E5M2 bytes without scales.
+kvq_status decode_attention(const void* q, const void* k_codes, const void* k_scales, const void* v_codes,
+                            const void* v_scales, void* out, const kvq_cache_desc* desc, int batch_size, int n_heads,
+                            int page_size, const int32_t* cache_seqlens, const int32_t* block_table, int format,
+                            float softmax_scale, void* workspace, size_t workspace_bytes, void* stream) {
+  const bool scaled = format != 0;
+  if (!q || !k_codes || !v_codes || !out || !desc || !cache_seqlens) return KVQ_ERR_NULL;
+  if (scaled && (!k_scales || !v_scales)) return KVQ_ERR_NULL;
+  if (format != 0 && format != 4 && format != 6 && format != 8) return KVQ_ERR_WBITS;
+  kvq_status st = check_desc(desc, scaled ? 32 : 8);
   if (st != KVQ_OK) return st;
   const int D = desc->head_dim;
   if (D != 64 && D != 128 && D != 256) return KVQ_ERR_SHAPE;
@@ -560,9 +567,32 @@ kvq_status kvq_decode_attention_q(const void* q, const void* k_codes, const void
   a.page_size = page_size;
   a.bt_stride = desc->block_table_stride;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
-  if (wbits == 4) return launch_attention_b<4>(a, desc, stream);
-  if (wbits == 6) return launch_attention_b<6>(a, desc, stream);
-  return launch_attention_b<8>(a, desc, stream);
+  if (format == 4) return launch_attention_b<4>(a, desc, stream);
+  if (format == 6) return launch_attention_b<6>(a, desc, stream);
+  if (format == 8) return launch_attention_b<8>(a, desc, stream);
+  return launch_attention_b<0>(a, desc, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_decode_attention_q(const void* q, const void* k_codes, const void* k_scales, const void* v_codes,
+                                  const void* v_scales, void* out, const kvq_cache_desc* desc, int batch_size,
+                                  int n_heads, int page_size, const int32_t* cache_seqlens,
+                                  const int32_t* block_table, int wbits, float softmax_scale, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  if (wbits != 4 && wbits != 6 && wbits != 8) return KVQ_ERR_WBITS;
+  return decode_attention(q, k_codes, k_scales, v_codes, v_scales, out, desc, batch_size, n_heads, page_size,
+                          cache_seqlens, block_table, wbits, softmax_scale, workspace, workspace_bytes, stream);
+}
+
+kvq_status kvq_decode_attention_fp8(const void* q, const void* k_fp8, const void* v_fp8, void* out,
+                                    const kvq_cache_desc* desc, int batch_size, int n_heads, int page_size,
+                                    const int32_t* cache_seqlens, const int32_t* block_table, float softmax_scale,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  return decode_attention(q, k_fp8, nullptr, v_fp8, nullptr, out, desc, batch_size, n_heads, page_size,
+                          cache_seqlens, block_table, 0, softmax_scale, workspace, workspace_bytes, stream);
 }
 
 long long kvq_count_match(const int64_t* a, long long a_len, const int64_t* b, long long b_len, long long max_a) {

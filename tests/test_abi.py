@@ -164,6 +164,33 @@ def test_decode_attention_validation(kvq):
     assert call(bs=0, wsp=None, wsb=0) == 0             # empty batch enqueues nothing
 
 
+def test_decode_attention_fp8_validation(kvq):
+    L = kvq.library()
+    by = ctypes.byref
+    d = _desc(kvq, d0=2, d1=16, H=2, D=64)
+    ws = kvq.attention_workspace_bytes((2, 16, 2, 64), 2, 4)
+    P = [FAKE] * 4  # q, k_fp8, v_fp8, out
+
+    def call(*args, desc=d, bs=2, nh=4, ps=0, lens=FAKE, bt=None, wsp=FAKE, wsb=ws):
+        return L.kvq_decode_attention_fp8(*(args or P), by(desc) if desc else None, bs, nh, ps, lens, bt,
+                                          ctypes.c_float(0.125), wsp, wsb, None)
+
+    assert call(None, *P[1:]) == 1
+    assert call(FAKE, None, *P[2:]) == 1
+    assert call(lens=None) == 1
+    assert call(desc=None) == 1
+    assert call(wsp=None) == 1
+    assert call(desc=_desc(kvq, D=96)) == 2             # head_dim 64, 128 or 256
+    assert call(nh=3) == 2
+    assert call(bs=3) == 4
+    assert call(wsb=ws - 1) == 4
+    assert call(P[0], P[1] + 4, *P[2:]) == 5            # 16-byte alignment
+    dp = _desc(kvq, d0=10, d1=16, H=2, D=64, stride=4)
+    assert call(desc=dp, ps=16) == 1                    # paged needs a block table
+    assert call(desc=dp, ps=8, bt=FAKE) == 4            # page_size must equal dim1
+    assert call(bs=0, wsp=None, wsb=0) == 0             # empty batch enqueues nothing
+
+
 def test_decode_attention_noalloc_validation(kvq):
     L = kvq.library()
     by = ctypes.byref

@@ -162,3 +162,82 @@ def test_bad_paging_reported(kvq, dev):
     kvq.decode_attention_q(torch.randn(1, 2, D).half().to(dev), kc, ks, vc, vs, out, 1, lens, 4, 0.1, ps, bt)
     assert kvq.poll_device_error() != 0
     assert not torch.isnan(out.float()).any()
+
+
+# ---- decode attention over an FP8 (E5M2) cache -------------------------------------------
+
+def fp8_on_gpu(kvq, k, v, dev):
+    d0, d1 = k.shape[:2]
+    k8 = torch.zeros(k.shape, dtype=torch.uint8, device=dev)
+    v8 = torch.zeros_like(k8)
+    kvq.fp16_to_fp8_kv(k.to(dev), k8, v.to(dev), v8, d0, 0, d1)
+    return k8, v8
+
+
+def check_fp8(kvq, oracle_mod, q, k8, v8, lens, scale, dev, page_size=0, bt=None, pick=None):
+    B, NH, D = q.shape
+    out = torch.full((B, NH, D), float("nan"), dtype=torch.float16, device=dev)
+    kvq.decode_attention_fp8(q.to(dev), k8, v8, out, B, lens.to(dev), scale, page_size,
+                             bt.to(dev) if bt is not None else None)
+    assert kvq.poll_device_error() == 0
+    rows = list(range(B)) if pick is None else pick
+    qs = q[rows].contiguous()
+    ls = lens.cpu()[rows].contiguous()
+    bts = bt.cpu()[rows].contiguous() if bt is not None else None
+    st, ref, ex = oracle_mod.decode_attention_fp8(u16(qs), k8.cpu().numpy(), v8.cpu().numpy(), len(rows), NH,
+                                                  page_size, ls.numpy(), bts.numpy() if bts is not None else None,
+                                                  scale)
+    assert st == oracle_mod.OK
+    got = out[rows].float().cpu().numpy().astype(np.float64)
+    assert not np.isnan(got).any()
+    vals = np.abs((v8.cpu().numpy().astype(np.uint16) << 8).view(np.float16).astype(np.float64))
+    vmax = float(vals[np.isfinite(vals)].max())  # finite values only: bytes past a window may hold NaN
+    tol = np.spacing(np.maximum(np.abs(ex), 2.0 ** -14).astype(np.float16)).astype(np.float64) + 2.0 ** -14 * vmax
+    err = np.abs(got - ex)
+    bad = np.nonzero(err > tol)
+    assert bad[0].size == 0, f"{bad[0].size} outputs off, worst {err.max():.3g} (tol there {tol[bad][0]:.3g})"
+    return float((ref == u16(out[rows])).mean())
+
+
+@pytest.mark.parametrize("D,H,NH", [(128, 2, 8), (64, 4, 4), (256, 1, 8), (128, 1, 2)])
+def test_fp8_contiguous(kvq, oracle_mod, dev, D, H, NH):
+    B, S = 3, 600
+    k, v = workloads.fp8_window(shape=(B, S, H, D))  # N(0,1) with outliers and subnormals
+    k8, v8 = fp8_on_gpu(kvq, k, v, dev)
+    q = torch.randn(B, NH, D).half()
+    lens = torch.tensor([600, 37, 257], dtype=torch.int32)
+    same = check_fp8(kvq, oracle_mod, q, k8, v8, lens, 1.0 / math.sqrt(D), dev)
+    assert same > 0.9
+
+
+@pytest.mark.parametrize("ps", [256, 16, 7])
+def test_fp8_paged(kvq, oracle_mod, dev, ps):
+    pool = workloads.paged_pool(num_pages=4000 // ps + 40, page_size=ps, heads=2, head_dim=128, batch=5,
+                                max_len=700)
+    k8, v8 = fp8_on_gpu(kvq, pool.k, pool.v, dev)
+    q = torch.randn(5, 8, 128).half()
+    lens = pool.cache_seqlens.clone()
+    lens[0], lens[1] = 0, 1
+    check_fp8(kvq, oracle_mod, q, k8, v8, lens, 0.088, dev, page_size=ps, bt=pool.block_table)
+
+
+def test_fp8_paged_pool_full_size_sampled(kvq, oracle_mod, dev):
+    """The 2048-page pool (32 sequences up to 16384 positions, 8 kv heads, 32 query heads) in
+    E5M2, checked against the oracle on 6 sequences (all heads)."""
+    pool = workloads.paged_pool(device=dev)
+    k8, v8 = fp8_on_gpu(kvq, pool.k, pool.v, dev)
+    q = torch.randn(32, 32, 128, generator=torch.Generator().manual_seed(8)).half()
+    check_fp8(kvq, oracle_mod, q, k8, v8, pool.cache_seqlens.cpu(), 1.0 / math.sqrt(128), dev, page_size=256,
+              bt=pool.block_table.cpu(), pick=[0, 5, 11, 17, 23, 31])
+
+
+def test_fp8_stale_nan_bytes_do_not_leak(kvq, oracle_mod, dev):
+    """Positions past a sequence's length whose bytes are NaN patterns get weight 0 and must
+    not turn the output into NaN (the kernel zeroes value rows without data)."""
+    B, S, H, D, NH = 2, 96, 1, 64, 2
+    k, v = workloads.normal_kv((B, S, H, D), 31)
+    k8, v8 = fp8_on_gpu(kvq, k, v, dev)
+    k8[:, 40:] = 0x7E  # NaN bytes beyond the attended window
+    v8[:, 40:] = 0xFF
+    q = torch.randn(B, NH, D).half()
+    check_fp8(kvq, oracle_mod, q, k8, v8, torch.tensor([40, 33], dtype=torch.int32), 0.125, dev)

@@ -217,7 +217,7 @@ class Fp8Step:
         self.kvq, self.batch = kvq, batch
         self.sets = []
         for r in range(sets):
-            k, v = workloads.fp8_window(seed=workloads.SEED_BASE + 2 + seed_shift + 100 * r, shape=shape,
+            k, v = workloads.fp8_window(seed=workloads.SEED_BASE + 2 + seed_shift + 100003 * r, shape=shape,
                                         device=dev)
             self.sets.append(dict(k=k, v=v, k8=torch.zeros(shape, dtype=torch.uint8, device=dev),
                                   v8=torch.zeros(shape, dtype=torch.uint8, device=dev),
@@ -897,9 +897,12 @@ def main():
     flush = L2Flush(dev)
     sampler = ClockSampler(local_rank).start() if rank == 0 else None
 
-    # each rank converts its own 4 sequences: a global batch of 4 * world (weak scaling)
-    batch = HEADLINE["shape"][0]
-    step = Fp8Step(kvq, dev, batch, seed_shift=rank)
+    # weak scaling: a global batch of 4 sequences per rank; rank r converts its shard of
+    # it (4 sequences), its inputs seeded by the shard's first global sequence index
+    global_batch = HEADLINE["shape"][0] * world
+    lo, hi = shard_range(global_batch, rank, world)
+    batch = hi - lo
+    step = Fp8Step(kvq, dev, batch, seed_shift=lo)
     # timed region: `steps` consecutive steps over rotating input copies (inputs larger
     # than L2), one pair of CUDA events around all of them, max over ranks
     ms_local = time_stream(step.run, len(step.sets), args.steps, args.warmup, flush, sampler)
@@ -960,7 +963,7 @@ def main():
         "dtype": "f16->u8->f16",
         "data": "synthetic (seeded N(0,1) with 1% outliers and 0.1% subnormals, drawn on device)",
         "config": {"workload": HEADLINE["workload"], "shape": list(HEADLINE["shape"]),
-                   "global_batch": batch * world, "offset": HEADLINE["offset"], "width": HEADLINE["width"],
+                   "global_batch": global_batch, "offset": HEADLINE["offset"], "width": HEADLINE["width"],
                    "ops": ["fp16_to_fp8 of K and V (one fused launch)", "fp8_to_fp16 of K and V (one fused launch)"],
                    "launch": f"{args.steps} consecutive steps (2 fused K+V launches each) replayed from CUDA graphs, "
                              "one pair of CUDA events around them",

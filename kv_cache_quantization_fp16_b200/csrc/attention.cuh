@@ -9,11 +9,13 @@
 // in binary16 and one rounding in the multiply; or, for an FP8 cache (format
 // code 0), the E5M2 bytes decoded exactly as fp8_to_fp16 does.
 //
-// Split-K flash decoding.  Kernel 1 (attn_partial_kernel): one CTA per
-// (chunk of positions, kv head, sequence), four warps.  The CTA copies its
-// whole chunk of K and V codes and scales into shared memory with cp.async
-// (every copy in flight at once), then each warp takes 16 positions at a
-// time:
+// Split-K flash decoding.  Kernel 1 (attn_partial_kernel) is a persistent
+// grid (one wave of CTAs of four warps).  Every (sequence, 256-position chunk,
+// kv head) is a work item; the warps take items round-robin and each walks its
+// own: it streams the item through two shared-memory buffers of 16 or 32
+// positions (cp.async copies of K and V codes, scales and, with the first
+// sub-chunk, the group's query rows), filling one while it computes on the
+// other, 16 positions at a time:
 //   * S = Q K^T on mma.sync m16n8k16 with the query heads as the M dimension
 //     (rows >= group are zero) and 8 positions per N tile: each lane
 //     dequantizes one contiguous span of D/4 elements of one position (a B
@@ -33,9 +35,9 @@
 // Code unpacking avoids per-code shifts: `(w & 0x000F000F) | 0x64006400` is
 // the binary16 pair (1024 + c0, 1024 + c4) of a Q4 word, and the high-nibble
 // pair is 16x that, brought back exactly with an FMA by 1/16.
-// The four warps' states merge in shared memory and the chunk's (max, sum,
-// accumulator) goes to the workspace.  Kernel 2 (attn_combine_kernel) merges
-// the chunks of each (sequence, head) and writes binary16 outputs.
+// At the end of an item the warp writes its (max, sum, accumulator) per query
+// head to the workspace entry of that chunk.  Kernel 2 (attn_combine_kernel)
+// merges the chunks of each (sequence, head) and writes binary16 outputs.
 #pragma once
 
 #include "codec.cuh"

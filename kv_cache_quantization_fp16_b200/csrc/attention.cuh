@@ -11,8 +11,9 @@
 //
 // Split-K flash decoding.  Kernel 1 (attn_partial_kernel) is a persistent
 // grid (one wave of CTAs of four warps).  Every (sequence, 256-position chunk,
-// kv head) is a work item; the warps take items round-robin and each walks its
-// own: it streams the item through two shared-memory buffers of 16 or 32
+// kv head) that holds data is a work item; warp w of W takes items w, w + W,
+// ... of a compact enumeration of them (so the warps' shares differ by at most
+// one item) and walks each: it streams the item through two shared-memory buffers of 16 or 32
 // positions (cp.async copies of K and V codes, scales and, with the first
 // sub-chunk, the group's query rows), filling one while it computes on the
 // other, 16 positions at a time:
@@ -39,6 +40,8 @@
 // head to the workspace entry of that chunk.  Kernel 2 (attn_combine_kernel)
 // merges the chunks of each (sequence, head) and writes binary16 outputs.
 #pragma once
+
+#include <type_traits>
 
 #include "codec.cuh"
 #include "tiles.cuh"
@@ -302,8 +305,10 @@ struct AttnTile {
   static constexpr int kBufBytes = (kBufK + kBufV + 2 * kBufS + 15) / 16 * 16;
   static constexpr int kQBytes = kAttnMaxGroup * D * 2;  // the item's query rows (copied with its first sub-chunk)
   static constexpr int kWarpBytes = 2 * kBufBytes + kQBytes;
-  static constexpr int kSeqlenSlots = 256;  // sequence lengths staged per CTA (larger batches read global memory)
-  static constexpr int kSmemBytes = kAttnWarps * kWarpBytes + kSeqlenSlots * 4;
+  // sequence lengths staged per CTA, with the running count of work items
+  // (larger batches read global memory and walk every item slot)
+  static constexpr int kSeqlenSlots = 256;
+  static constexpr int kSmemBytes = kAttnWarps * kWarpBytes + 2 * kSeqlenSlots * 4 + 16;
   static constexpr int KN = D / 4;   // K elements per lane per position (one contiguous span)
   static constexpr int VN = D / 8;   // V elements per lane per row (one contiguous span)
   static constexpr int KS = D / 16;  // k-steps of Q K^T = m-tiles of V^T P^T
@@ -414,64 +419,109 @@ __device__ __forceinline__ void v_span_pair(const uint8_t* r0, const uint8_t* r1
 
 
 // One sub-chunk of one work item, as a warp walks its items.
+template <class I>
 struct AttnCursor {
-  long long item;       // work item index, or -1 past the end
+  I item;               // work item index, or -1 past the end
   int seq, chunk, kvh;  // what the item is
   int sub;              // sub-chunk within the item
   int n;                // positions of this sub-chunk (<= kSub)
   bool last;            // last sub-chunk of the item
 };
 
-template <int B, int D>
+// Work items in walk order, two ways (the launch picks one).
+// kCompact: only items that hold data are enumerated.  The CTA stages the
+// batch in shared memory: kSeqlenSlots sequence lengths, then kSeqlenSlots
+// running item counts (entry i counts the items of sequences 0..i:
+// ceil(length / chunk) chunks times kv heads each), then the item total.  Item
+// k is found by a binary search over the running counts, and every warp gets
+// the same number of items to within one.  The launch guarantees that the
+// batch fits the slots and that every item count fits an int.
+// Otherwise: every (sequence, chunk, kv head) slot up to the cache's capacity
+// is visited and empty ones are skipped (lengths staged when the batch fits).
+template <int B, int D, bool kCompact>
 struct AttnWalk {
   using T = AttnTile<B, D>;
+  using Item = typename std::conditional<kCompact, int, long long>::type;
+  using Cursor = AttnCursor<Item>;
   const AttnParams& a;
-  const int* s_len;  // staged sequence lengths (or null)
-  long long stride;  // warps in the grid
+  bool staged;  // the batch's lengths are in shared memory
+
+  // the staged block, after the warps' buffers in dynamic shared memory
+  __device__ static int* block() {
+    extern __shared__ __align__(16) uint8_t smem[];
+    return reinterpret_cast<int*>(smem + kAttnWarps * T::kWarpBytes);
+  }
+  // warps in the grid
+  __device__ static Item stride() { return static_cast<Item>(gridDim.x) * kAttnWarps; }
 
   __device__ long long max_len() const {
     return a.page_size == 0 ? static_cast<long long>(a.dim1) : static_cast<long long>(a.max_chunks) * T::kChunk;
   }
   // sequence length, clamped to what the cache (or the launched chunks) can hold
   __device__ int length(int seq) const {
-    long long L = s_len ? s_len[seq] : a.seqlens[seq];
+    long long L = staged ? block()[seq] : a.seqlens[seq];
     if (L < 0) L = 0;
     const long long m = max_len();
     return static_cast<int>(L > m ? m : L);
   }
-  // first sub-chunk of the first non-empty item at or after `item`
-  __device__ AttnCursor seek(long long item) const {
-    const long long n_items = static_cast<long long>(a.batch) * a.max_chunks * a.kv_heads;
-    AttnCursor c;
-    for (; item < n_items; item += stride) {
-      if (n_items < (1LL << 31)) {  // 32-bit index arithmetic suffices
-        const unsigned it = static_cast<unsigned>(item), t = it / static_cast<unsigned>(a.kv_heads);
-        c.kvh = static_cast<int>(it - t * static_cast<unsigned>(a.kv_heads));
-        c.seq = static_cast<int>(t / static_cast<unsigned>(a.max_chunks));
-        c.chunk = static_cast<int>(t - static_cast<unsigned>(c.seq) * static_cast<unsigned>(a.max_chunks));
-      } else {
-        const long long t = item / a.kv_heads;
-        c.kvh = static_cast<int>(item - t * a.kv_heads);
-        c.seq = static_cast<int>(t / a.max_chunks);
-        c.chunk = static_cast<int>(t - static_cast<long long>(c.seq) * a.max_chunks);
-      }
-      const int L = length(c.seq);
-      const int p0 = c.chunk * T::kChunk;
-      if (p0 < L) {
-        c.item = item;
-        c.sub = 0;
-        const int rest = min(L - p0, T::kChunk);
-        c.n = min(rest, T::kSub);
-        c.last = rest <= T::kSub;
+  // first sub-chunk of item `item` (kCompact), or of the first non-empty item slot at or after it
+  __device__ Cursor seek(Item item) const {
+    Cursor c;
+    if constexpr (kCompact) {
+      const int* const s_items = block() + T::kSeqlenSlots;
+      if (item >= s_items[T::kSeqlenSlots]) {
+        c.item = -1;
         return c;
       }
+      int lo = 0, hi = a.batch - 1;  // the first sequence whose running count exceeds the item
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (s_items[mid] > item) hi = mid;
+        else lo = mid + 1;
+      }
+      const unsigned r = static_cast<unsigned>(item - (lo ? s_items[lo - 1] : 0));
+      const unsigned chunk = r / static_cast<unsigned>(a.kv_heads);
+      c.seq = lo;
+      c.chunk = static_cast<int>(chunk);
+      c.kvh = static_cast<int>(r - chunk * static_cast<unsigned>(a.kv_heads));
+      const int rest = min(length(c.seq) - c.chunk * T::kChunk, T::kChunk);
+      c.item = item;
+      c.sub = 0;
+      c.n = min(rest, T::kSub);
+      c.last = rest <= T::kSub;
+      return c;
+    } else {
+      const long long n_items = static_cast<long long>(a.batch) * a.max_chunks * a.kv_heads;
+      for (; item < n_items; item += stride()) {
+        if (n_items < (1LL << 31)) {  // 32-bit index arithmetic suffices
+          const unsigned it = static_cast<unsigned>(item), t = it / static_cast<unsigned>(a.kv_heads);
+          c.kvh = static_cast<int>(it - t * static_cast<unsigned>(a.kv_heads));
+          c.seq = static_cast<int>(t / static_cast<unsigned>(a.max_chunks));
+          c.chunk = static_cast<int>(t - static_cast<unsigned>(c.seq) * static_cast<unsigned>(a.max_chunks));
+        } else {
+          const long long t = item / a.kv_heads;
+          c.kvh = static_cast<int>(item - t * a.kv_heads);
+          c.seq = static_cast<int>(t / a.max_chunks);
+          c.chunk = static_cast<int>(t - static_cast<long long>(c.seq) * a.max_chunks);
+        }
+        const int L = length(c.seq);
+        const int p0 = c.chunk * T::kChunk;
+        if (p0 < L) {
+          c.item = item;
+          c.sub = 0;
+          const int rest = min(L - p0, T::kChunk);
+          c.n = min(rest, T::kSub);
+          c.last = rest <= T::kSub;
+          return c;
+        }
+      }
+      c.item = -1;
+      return c;
     }
-    c.item = -1;
-    return c;
   }
-  __device__ AttnCursor next(const AttnCursor& c) const {
-    if (c.last) return seek(c.item + stride);
-    AttnCursor d = c;
+  __device__ Cursor next(const Cursor& c) const {
+    if (c.last) return seek(c.item + stride());
+    Cursor d = c;
     d.sub = c.sub + 1;
     const int rest = min(length(c.seq) - c.chunk * T::kChunk, T::kChunk) - d.sub * T::kSub;
     d.n = min(rest, T::kSub);
@@ -483,8 +533,8 @@ struct AttnWalk {
 // Issue the copies of one sub-chunk into a warp buffer (and, for the first
 // sub-chunk of an item, its query rows into the warp's query area); returns
 // the bit mask of its positions that hold data (bit i: position i).
-template <int B, int D>
-__device__ __forceinline__ uint32_t attn_issue(const AttnParams& a, const AttnCursor& c, uint8_t* buf, uint8_t* sq,
+template <int B, int D, class Cursor>
+__device__ __forceinline__ uint32_t attn_issue(const AttnParams& a, const Cursor& c, uint8_t* buf, uint8_t* sq,
                                                int lane) {
   using T = AttnTile<B, D>;
   constexpr int SC = T::kSub, P = T::kRowBytes / 16;
@@ -550,7 +600,7 @@ __device__ __forceinline__ uint32_t attn_issue(const AttnParams& a, const AttnCu
   return mask;
 }
 
-template <int B, int D>
+template <int B, int D, bool kCompact>
 __global__ void __launch_bounds__(kAttnThreads, D > 128 ? 2 : 4) attn_partial_kernel(const __grid_constant__ AttnParams a) {
   using T = AttnTile<B, D>;
   using Codec = AttnCodec<B>;
@@ -563,17 +613,39 @@ __global__ void __launch_bounds__(kAttnThreads, D > 128 ? 2 : 4) attn_partial_ke
   const int g = lane >> 2, j = lane & 3;
   uint8_t* const wbuf = smem + warp * T::kWarpBytes;
   int* const s_len = reinterpret_cast<int*>(smem + kAttnWarps * T::kWarpBytes);
+  using Walk = AttnWalk<B, D, kCompact>;
 
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const bool staged = a.batch <= T::kSeqlenSlots;
+  const bool staged = kCompact || a.batch <= T::kSeqlenSlots;
   if (staged)
     for (int i = threadIdx.x; i < a.batch; i += kAttnThreads) s_len[i] = a.seqlens[i];
-  __syncthreads();  // the only CTA-wide barrier: from here on every warp walks its own items
+  __syncthreads();
+  if (kCompact && warp == 0) {
+    // running item counts over the batch (a warp-wide inclusive scan per 32
+    // sequences; the launch guarantees that the total fits an int)
+    int* const s_items = s_len + T::kSeqlenSlots;
+    const Walk w0{a, true};
+    int run = 0;
+    for (int base = 0; base < a.batch; base += 32) {
+      const int i = base + lane;
+      int n = i < a.batch ? (w0.length(i) + T::kChunk - 1) / T::kChunk * a.kv_heads : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xFFFFFFFFu, n, o);
+        if (lane >= o) n += t;
+      }
+      n += run;
+      if (i < a.batch) s_items[i] = n;
+      run = __shfl_sync(0xFFFFFFFFu, n, 31);
+    }
+    if (lane == 0) s_items[T::kSeqlenSlots] = run;
+  }
+  __syncthreads();  // the last CTA-wide barrier: from here on every warp walks its own items
 
-  const AttnWalk<B, D> walk{a, staged ? s_len : nullptr, static_cast<long long>(gridDim.x) * kAttnWarps};
+  const Walk walk{a, staged};
   uint8_t* const sq_area = wbuf + 2 * T::kBufBytes;
-  AttnCursor cur = walk.seek(static_cast<long long>(blockIdx.x) * kAttnWarps + warp);
+  typename Walk::Cursor cur = walk.seek(static_cast<typename Walk::Item>(blockIdx.x) * kAttnWarps + warp);
   if (cur.item < 0) return;
   uint32_t mask_cur = attn_issue<B, D>(a, cur, wbuf, sq_area, lane);
   asm volatile("cp.async.commit_group;\n" ::: "memory");
@@ -614,7 +686,7 @@ __global__ void __launch_bounds__(kAttnThreads, D > 128 ? 2 : 4) attn_partial_ke
       }
       __syncwarp();  // the query area may be refilled below
     }
-    const AttnCursor nxt = walk.next(cur);
+    const typename Walk::Cursor nxt = walk.next(cur);
     uint32_t mask_nxt = 0;
     if (nxt.item >= 0) {
       mask_nxt = attn_issue<B, D>(a, nxt, wbuf + (b ^ 1) * T::kBufBytes, sq_area, lane);

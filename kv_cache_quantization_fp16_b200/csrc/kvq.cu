@@ -449,16 +449,16 @@ long long attn_max_chunks(const kvq_cache_desc* d, int page_size, int chunk) {
   return (max_len + chunk - 1) / chunk;
 }
 
-// Dynamic shared memory opt-in, once per device for each (B, D) kernel
+// Dynamic shared memory opt-in, once per device for each partial kernel
 // (static plus dynamic shared memory above 48 KB needs it).
-template <int B, int D>
+template <int B, int D, bool kCompact>
 bool allow_attention_smem() {
   constexpr int kMaxDevices = 64;
   static std::atomic<bool> done[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
   if (done[dev].load()) return true;
-  if (cudaFuncSetAttribute(kvq::attn_partial_kernel<B, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(kvq::attn_partial_kernel<B, D, kCompact>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kvq::AttnTile<B, D>::kSmemBytes) != cudaSuccess) {
     cudaGetLastError();
     return false;
@@ -469,7 +469,25 @@ bool allow_attention_smem() {
 
 // Persistent grid of the partial kernel: every (sequence, 256-position chunk,
 // kv head) work item goes to one warp; as many CTAs as the device holds at
-// once (occupancy cached per device), never more than there are items.
+// once (occupancy cached per device), never more than there are item slots.
+template <int B, int D, bool kCompact>
+kvq_status launch_partial(const kvq::AttnParams& a, long long items, void* stream) {
+  using T = kvq::AttnTile<B, D>;
+  if (!allow_attention_smem<B, D, kCompact>()) return KVQ_ERR_CUDA;
+  constexpr int kMaxDevices = 64;
+  static std::atomic<long long> resident[kMaxDevices];
+  const long long ctas_max = first_wave_ctas(kvq::attn_partial_kernel<B, D, kCompact>, kvq::kAttnThreads,
+                                             T::kSmemBytes, resident, kMaxDevices);
+  if (ctas_max < 1) return KVQ_ERR_CUDA;
+  const long long need = (items + kvq::kAttnWarps - 1) / kvq::kAttnWarps;
+  const unsigned grid = static_cast<unsigned>(need < ctas_max ? need : ctas_max);
+  return launch_pdl(kvq::attn_partial_kernel<B, D, kCompact>, dim3(grid), kvq::kAttnThreads, T::kSmemBytes, stream,
+                    a);
+}
+
+// The partial kernel walks only the items that hold data when the batch fits
+// its shared-memory slots and every item count fits an int; otherwise it
+// visits every item slot.  Then the combine kernel.
 template <int B, int D>
 kvq_status launch_attention(kvq::AttnParams a, const kvq_cache_desc* desc, void* stream) {
   using T = kvq::AttnTile<B, D>;
@@ -477,16 +495,10 @@ kvq_status launch_attention(kvq::AttnParams a, const kvq_cache_desc* desc, void*
   const long long max_chunks = attn_max_chunks(desc, a.page_size, T::kChunk);
   if (max_chunks < 1 || max_chunks > 0x7FFFFFFFLL) return KVQ_ERR_RANGE;
   a.max_chunks = static_cast<int>(max_chunks);
-  if (!allow_attention_smem<B, D>()) return KVQ_ERR_CUDA;
-  constexpr int kMaxDevices = 64;
-  static std::atomic<long long> resident[kMaxDevices];
-  const long long ctas_max = first_wave_ctas(kvq::attn_partial_kernel<B, D>, kvq::kAttnThreads, T::kSmemBytes,
-                                             resident, kMaxDevices);
-  if (ctas_max < 1) return KVQ_ERR_CUDA;
   const long long items = static_cast<long long>(a.batch) * a.max_chunks * a.kv_heads;
-  const long long need = (items + kvq::kAttnWarps - 1) / kvq::kAttnWarps;
-  const unsigned grid = static_cast<unsigned>(need < ctas_max ? need : ctas_max);
-  kvq_status st = launch_pdl(kvq::attn_partial_kernel<B, D>, dim3(grid), kvq::kAttnThreads, T::kSmemBytes, stream, a);
+  const bool compact = a.batch <= T::kSeqlenSlots && items <= 0x7FFFFFFFLL;
+  const kvq_status st = compact ? launch_partial<B, D, true>(a, items, stream)
+                                : launch_partial<B, D, false>(a, items, stream);
   if (st != KVQ_OK) return st;
   return launch_pdl(kvq::attn_combine_kernel<D>, dim3(a.n_heads, a.batch), kvq::kCombineThreads, 0, stream, a);
 }

@@ -82,7 +82,7 @@ def test_contiguous(kvq, oracle_mod, dev, wbits, D, H, NH):
     B, S = 3, 600
     k, v = workloads.channel_outliers(shape=(B, S, H, D))
     kc, ks, vc, vs = quantize_on_gpu(kvq, k, v, wbits, dev)
-    q = torch.randn(B, NH, D).half()
+    q = torch.randn(B, NH, D, generator=torch.Generator().manual_seed(100)).half()
     lens = torch.tensor([600, 37, 257], dtype=torch.int32)
     err, same = check(kvq, oracle_mod, q, kc, ks, vc, vs, lens, wbits, 1.0 / math.sqrt(D), dev)
     assert same > 0.9  # nearly every output is the correctly rounded fp64 result
@@ -94,7 +94,7 @@ def test_paged(kvq, oracle_mod, dev, wbits, ps):
     pool = workloads.paged_pool(num_pages=4000 // ps + 40, page_size=ps, heads=2, head_dim=128, batch=5,
                                 max_len=700)
     kc, ks, vc, vs = quantize_on_gpu(kvq, pool.k, pool.v, wbits, dev)
-    q = torch.randn(5, 8, 128).half()
+    q = torch.randn(5, 8, 128, generator=torch.Generator().manual_seed(101)).half()
     lens = pool.cache_seqlens.clone()
     lens[0] = 0
     lens[1] = 1
@@ -107,7 +107,7 @@ def test_sharp_and_flat_softmax(kvq, oracle_mod, dev):
     k, v = workloads.normal_kv((B, S, H, D), 11)
     kc, ks, vc, vs = quantize_on_gpu(kvq, k, v, 6, dev)
     lens = torch.tensor([900, 513], dtype=torch.int32)
-    q = torch.randn(B, NH, D).half() * 4
+    q = torch.randn(B, NH, D, generator=torch.Generator().manual_seed(102)).half() * 4
     check(kvq, oracle_mod, q, kc, ks, vc, vs, lens, 6, 2.0, dev)
     check(kvq, oracle_mod, torch.zeros(B, NH, D).half(), kc, ks, vc, vs, lens, 6, 1.0, dev)
 
@@ -159,7 +159,8 @@ def test_bad_paging_reported(kvq, dev):
     lens = torch.tensor([30], dtype=torch.int32, device=dev)
     out = torch.empty(1, 2, D, dtype=torch.float16, device=dev)
     assert kvq.poll_device_error() == 0
-    kvq.decode_attention_q(torch.randn(1, 2, D).half().to(dev), kc, ks, vc, vs, out, 1, lens, 4, 0.1, ps, bt)
+    q = torch.randn(1, 2, D, generator=torch.Generator().manual_seed(103)).half().to(dev)
+    kvq.decode_attention_q(q, kc, ks, vc, vs, out, 1, lens, 4, 0.1, ps, bt)
     assert kvq.poll_device_error() != 0
     assert not torch.isnan(out.float()).any()
 
@@ -204,7 +205,7 @@ def test_fp8_contiguous(kvq, oracle_mod, dev, D, H, NH):
     B, S = 3, 600
     k, v = workloads.fp8_window(shape=(B, S, H, D))  # N(0,1) with outliers and subnormals
     k8, v8 = fp8_on_gpu(kvq, k, v, dev)
-    q = torch.randn(B, NH, D).half()
+    q = torch.randn(B, NH, D, generator=torch.Generator().manual_seed(104)).half()
     lens = torch.tensor([600, 37, 257], dtype=torch.int32)
     same = check_fp8(kvq, oracle_mod, q, k8, v8, lens, 1.0 / math.sqrt(D), dev)
     assert same > 0.9
@@ -215,7 +216,7 @@ def test_fp8_paged(kvq, oracle_mod, dev, ps):
     pool = workloads.paged_pool(num_pages=4000 // ps + 40, page_size=ps, heads=2, head_dim=128, batch=5,
                                 max_len=700)
     k8, v8 = fp8_on_gpu(kvq, pool.k, pool.v, dev)
-    q = torch.randn(5, 8, 128).half()
+    q = torch.randn(5, 8, 128, generator=torch.Generator().manual_seed(105)).half()
     lens = pool.cache_seqlens.clone()
     lens[0], lens[1] = 0, 1
     check_fp8(kvq, oracle_mod, q, k8, v8, lens, 0.088, dev, page_size=ps, bt=pool.block_table)
@@ -239,5 +240,5 @@ def test_fp8_stale_nan_bytes_do_not_leak(kvq, oracle_mod, dev):
     k8, v8 = fp8_on_gpu(kvq, k, v, dev)
     k8[:, 40:] = 0x7E  # NaN bytes beyond the attended window
     v8[:, 40:] = 0xFF
-    q = torch.randn(B, NH, D).half()
+    q = torch.randn(B, NH, D, generator=torch.Generator().manual_seed(106)).half()
     check_fp8(kvq, oracle_mod, q, k8, v8, torch.tensor([40, 33], dtype=torch.int32), 0.125, dev)

@@ -56,7 +56,7 @@ def test_single_position_returns_value(oracle_mod, wbits):
     k, v = _rand_cache(B, S, H, D, 1)
     kc, ks, vc, vs = _quantize(oracle_mod, k, v, wbits)
     _, vy = _dequant(oracle_mod, kc, ks, vc, vs, wbits, D)
-    q = _np16(torch.randn(B, NH, D).half())
+    q = _np16(torch.randn(B, NH, D, generator=torch.Generator().manual_seed(200)).half())
     st, out, ex = oracle_mod.decode_attention_q(q, kc, ks, vc, vs, B, NH, 0, np.array([1, 1], np.int32), None,
                                                 wbits, 0.125, D)
     assert st == oracle_mod.OK
@@ -83,7 +83,7 @@ def test_two_positions_closed_form(oracle_mod):
     D, wbits = 32, 4
     k = np.zeros((1, 2, 1, D), np.float16)
     k[0, 1, 0, 0] = 7.0  # absmax 7 -> s = 1, code 15 -> 7; scale below divides by 7
-    v = _np16(torch.randn(1, 2, 1, D).half())
+    v = _np16(torch.randn(1, 2, 1, D, generator=torch.Generator().manual_seed(201)).half())
     kc, ks, vc, vs = _quantize(oracle_mod, k.view(np.uint16), v, wbits)
     _, vy = _dequant(oracle_mod, kc, ks, vc, vs, wbits, D)
     q = np.zeros((1, 1, D), np.float16)
@@ -113,7 +113,7 @@ def test_paged_equals_contiguous_and_page_order(oracle_mod, wbits):
     k, v = _rand_cache(B, S, H, D, 4)
     kc, ks, vc, vs = _quantize(oracle_mod, k, v, wbits)
     lens = np.array([64, 1, 40], np.int32)
-    q = _np16(torch.randn(B, NH, D).half())
+    q = _np16(torch.randn(B, NH, D, generator=torch.Generator().manual_seed(202)).half())
     st, out_c, ex_c = oracle_mod.decode_attention_q(q, kc, ks, vc, vs, B, NH, 0, lens, None, wbits, 0.125, D)
     assert st == oracle_mod.OK
     pages = (B * S // ps, ps, H)
@@ -139,7 +139,7 @@ def test_gqa_groups(oracle_mod):
     B, S, H, D, NH, wbits = 1, 30, 2, 32, 6, 4
     k, v = _rand_cache(B, S, H, D, 5)
     kc, ks, vc, vs = _quantize(oracle_mod, k, v, wbits)
-    q = _np16(torch.randn(B, NH, D).half())
+    q = _np16(torch.randn(B, NH, D, generator=torch.Generator().manual_seed(203)).half())
     q[0, 1] = q[0, 0]
     q[0, 3] = q[0, 0]  # head 3 is in the second group (kv head 1)
     st, out, ex = oracle_mod.decode_attention_q(q, kc, ks, vc, vs, B, NH, 0, np.array([S], np.int32), None,
@@ -155,7 +155,7 @@ def test_matches_numpy_softmax(oracle_mod, wbits):
     k, v = _rand_cache(B, S, H, D, 6)
     kc, ks, vc, vs = _quantize(oracle_mod, k, v, wbits)
     ky, vy = _dequant(oracle_mod, kc, ks, vc, vs, wbits, D)
-    q16 = torch.randn(B, NH, D).half()
+    q16 = torch.randn(B, NH, D, generator=torch.Generator().manual_seed(204)).half()
     q = _np16(q16)
     qf = q16.double().numpy()
     lens = np.array([50, 17], np.int32)
@@ -206,7 +206,7 @@ def _fp8_cache(B, S, H, D, seed):
 def test_fp8_single_position_returns_value(oracle_mod):
     B, S, H, D, NH = 2, 3, 2, 64, 4
     k8, v8 = _fp8_cache(B, S, H, D, 11)
-    q = _np16(torch.randn(B, NH, D).half())
+    q = _np16(torch.randn(B, NH, D, generator=torch.Generator().manual_seed(205)).half())
     st, out, ex = oracle_mod.decode_attention_fp8(q, k8, v8, B, NH, 0, np.array([1, 1], np.int32), None, 0.125)
     assert st == oracle_mod.OK
     vv = _e5m2_numpy(v8)
@@ -247,7 +247,7 @@ def test_fp8_paged_equals_contiguous_and_matches_numpy(oracle_mod):
     B, S, H, D, NH, ps = 3, 64, 2, 64, 8, 16
     k8, v8 = _fp8_cache(B, S, H, D, 13)
     lens = np.array([64, 1, 40], np.int32)
-    q16 = torch.randn(B, NH, D).half()
+    q16 = torch.randn(B, NH, D, generator=torch.Generator().manual_seed(206)).half()
     q = _np16(q16)
     st, out_c, ex_c = oracle_mod.decode_attention_fp8(q, k8, v8, B, NH, 0, lens, None, 0.125)
     assert st == oracle_mod.OK

@@ -17,6 +17,8 @@
 // bodies in ops.cuh and the arithmetic in codec.cuh.
 //
 // This is a streaming, HBM-bound path: no tensor cores, no collectives.
+// The host side of decode attention over the converted caches lives in
+// attention_api.cuh, included at the end of this file.
 
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -24,7 +26,6 @@
 #include <atomic>
 
 #include "../../include/kvq.h"
-#include "attention.cuh"
 #include "bulk_engine.cuh"
 #include "codec.cuh"
 #include "ldg_engine.cuh"
@@ -439,173 +440,7 @@ kvq_status kvq_poll_device_error(int32_t* code_out, void* stream) {
 
 }  // extern "C"
 
-namespace {
-
-// Chunks of `chunk` positions a sequence can have: the longest window the
-// cache geometry allows.
-long long attn_max_chunks(const kvq_cache_desc* d, int page_size, int chunk) {
-  const long long max_len = page_size > 0 ? static_cast<long long>(d->block_table_stride) * page_size
-                                          : static_cast<long long>(d->dim1);
-  return (max_len + chunk - 1) / chunk;
-}
-
-// Dynamic shared memory opt-in, once per device for each partial kernel
-// (static plus dynamic shared memory above 48 KB needs it).
-template <int B, int D, bool kCompact>
-bool allow_attention_smem() {
-  constexpr int kMaxDevices = 64;
-  static std::atomic<bool> done[kMaxDevices];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
-  if (done[dev].load()) return true;
-  if (cudaFuncSetAttribute(kvq::attn_partial_kernel<B, D, kCompact>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kvq::AttnTile<B, D>::kSmemBytes) != cudaSuccess) {
-    cudaGetLastError();
-    return false;
-  }
-  done[dev].store(true);
-  return true;
-}
-
-// Persistent grid of the partial kernel: every (sequence, 256-position chunk,
-// kv head) work item goes to one warp; as many CTAs as the device holds at
-// once (occupancy cached per device), never more than there are item slots.
-template <int B, int D, bool kCompact>
-kvq_status launch_partial(const kvq::AttnParams& a, long long items, void* stream) {
-  using T = kvq::AttnTile<B, D>;
-  if (!allow_attention_smem<B, D, kCompact>()) return KVQ_ERR_CUDA;
-  constexpr int kMaxDevices = 64;
-  static std::atomic<long long> resident[kMaxDevices];
-  const long long ctas_max = first_wave_ctas(kvq::attn_partial_kernel<B, D, kCompact>, kvq::kAttnThreads,
-                                             T::kSmemBytes, resident, kMaxDevices);
-  if (ctas_max < 1) return KVQ_ERR_CUDA;
-  const long long need = (items + kvq::kAttnWarps - 1) / kvq::kAttnWarps;
-  const unsigned grid = static_cast<unsigned>(need < ctas_max ? need : ctas_max);
-  return launch_pdl(kvq::attn_partial_kernel<B, D, kCompact>, dim3(grid), kvq::kAttnThreads, T::kSmemBytes, stream,
-                    a);
-}
-
-// The partial kernel walks only the items that hold data when the batch fits
-// its shared-memory slots and every item count fits an int; otherwise it
-// visits every item slot.  Then the combine kernel.
-template <int B, int D>
-kvq_status launch_attention(kvq::AttnParams a, const kvq_cache_desc* desc, void* stream) {
-  using T = kvq::AttnTile<B, D>;
-  a.chunk = T::kChunk;
-  const long long max_chunks = attn_max_chunks(desc, a.page_size, T::kChunk);
-  if (max_chunks < 1 || max_chunks > 0x7FFFFFFFLL) return KVQ_ERR_RANGE;
-  a.max_chunks = static_cast<int>(max_chunks);
-  const long long items = static_cast<long long>(a.batch) * a.max_chunks * a.kv_heads;
-  const bool compact = a.batch <= T::kSeqlenSlots && items <= 0x7FFFFFFFLL;
-  const kvq_status st = compact ? launch_partial<B, D, true>(a, items, stream)
-                                : launch_partial<B, D, false>(a, items, stream);
-  if (st != KVQ_OK) return st;
-  return launch_pdl(kvq::attn_combine_kernel<D>, dim3(a.n_heads, a.batch), kvq::kCombineThreads, 0, stream, a);
-}
-
-template <int B>
-kvq_status launch_attention_b(const kvq::AttnParams& a, const kvq_cache_desc* desc, void* stream) {
-  if (desc->head_dim == 64) return launch_attention<B, 64>(a, desc, stream);
-  if (desc->head_dim == 128) return launch_attention<B, 128>(a, desc, stream);
-  return launch_attention<B, 256>(a, desc, stream);
-}
-
-}  // namespace
-
 extern "C" {
-
-size_t kvq_decode_attention_workspace_size(const kvq_cache_desc* desc, int batch_size, int n_heads,
-                                           int page_size) {
-  if (!desc || batch_size < 0 || n_heads < 0 || page_size < 0) return 0;
-  // sized for the smallest chunk any wbits / head_dim uses
-  return static_cast<size_t>(batch_size) * n_heads * attn_max_chunks(desc, page_size, kvq::kAttnMinChunk) *
-         (desc->head_dim + 2) * sizeof(float);
-}
-
-}  // extern "C"
-
-namespace {
-
-// Shared argument checks and launch of the decode-attention entry points:
-// format 4 / 6 / 8 = Q codes with scales, 0 = E5M2 bytes without scales.
-kvq_status decode_attention(const void* q, const void* k_codes, const void* k_scales, const void* v_codes,
-                            const void* v_scales, void* out, const kvq_cache_desc* desc, int batch_size, int n_heads,
-                            int page_size, const int32_t* cache_seqlens, const int32_t* block_table, int format,
-                            float softmax_scale, void* workspace, size_t workspace_bytes, void* stream) {
-  const bool scaled = format != 0;
-  if (!q || !k_codes || !v_codes || !out || !desc || !cache_seqlens) return KVQ_ERR_NULL;
-  if (scaled && (!k_scales || !v_scales)) return KVQ_ERR_NULL;
-  if (format != 0 && format != 4 && format != 6 && format != 8) return KVQ_ERR_WBITS;
-  kvq_status st = check_desc(desc, scaled ? 32 : 8);
-  if (st != KVQ_OK) return st;
-  const int D = desc->head_dim;
-  if (D != 64 && D != 128 && D != 256) return KVQ_ERR_SHAPE;
-  if (n_heads < 1 || n_heads % desc->kv_heads || n_heads / desc->kv_heads > kvq::kAttnMaxGroup) return KVQ_ERR_SHAPE;
-  if (batch_size < 0 || batch_size > 65535 || desc->kv_heads > 65535 || n_heads > 0x7FFFFFFF) return KVQ_ERR_RANGE;
-  if (page_size < 0) return KVQ_ERR_RANGE;
-  if (page_size == 0) {
-    if (batch_size > desc->dim0) return KVQ_ERR_RANGE;
-  } else {
-    if (!block_table) return KVQ_ERR_NULL;
-    if (page_size != desc->dim1 || desc->block_table_stride < 1) return KVQ_ERR_RANGE;
-  }
-  const void* ptrs[7] = {q, k_codes, k_scales, v_codes, v_scales, out, workspace};
-  for (const void* p : ptrs)
-    if (p && !aligned16(p)) return KVQ_ERR_ALIGN;
-  if ((reinterpret_cast<uintptr_t>(cache_seqlens) | reinterpret_cast<uintptr_t>(block_table)) & 3u)
-    return KVQ_ERR_ALIGN;
-  if (batch_size == 0) return KVQ_OK;
-  const long long max_chunks = attn_max_chunks(desc, page_size, kvq::kAttnMinChunk);
-  if (max_chunks < 1 || max_chunks > 0x7FFFFFFFLL) return KVQ_ERR_RANGE;
-  if (!workspace) return KVQ_ERR_NULL;
-  if (workspace_bytes < kvq_decode_attention_workspace_size(desc, batch_size, n_heads, page_size))
-    return KVQ_ERR_RANGE;
-  kvq::AttnParams a{};
-  a.q = static_cast<const __half*>(q);
-  a.k_codes = static_cast<const uint8_t*>(k_codes);
-  a.k_scales = static_cast<const __half*>(k_scales);
-  a.v_codes = static_cast<const uint8_t*>(v_codes);
-  a.v_scales = static_cast<const __half*>(v_scales);
-  a.out = static_cast<__half*>(out);
-  a.ws = static_cast<float*>(workspace);
-  a.seqlens = cache_seqlens;
-  a.block_table = block_table;
-  a.dim0 = desc->dim0;
-  a.dim1 = desc->dim1;
-  a.kv_heads = desc->kv_heads;
-  a.batch = batch_size;
-  a.n_heads = n_heads;
-  a.group = n_heads / desc->kv_heads;
-  a.page_size = page_size;
-  a.bt_stride = desc->block_table_stride;
-  a.scale_log2 = softmax_scale * 1.4426950408889634f;
-  if (format == 4) return launch_attention_b<4>(a, desc, stream);
-  if (format == 6) return launch_attention_b<6>(a, desc, stream);
-  if (format == 8) return launch_attention_b<8>(a, desc, stream);
-  return launch_attention_b<0>(a, desc, stream);
-}
-
-}  // namespace
-
-extern "C" {
-
-kvq_status kvq_decode_attention_q(const void* q, const void* k_codes, const void* k_scales, const void* v_codes,
-                                  const void* v_scales, void* out, const kvq_cache_desc* desc, int batch_size,
-                                  int n_heads, int page_size, const int32_t* cache_seqlens,
-                                  const int32_t* block_table, int wbits, float softmax_scale, void* workspace,
-                                  size_t workspace_bytes, void* stream) {
-  if (wbits != 4 && wbits != 6 && wbits != 8) return KVQ_ERR_WBITS;
-  return decode_attention(q, k_codes, k_scales, v_codes, v_scales, out, desc, batch_size, n_heads, page_size,
-                          cache_seqlens, block_table, wbits, softmax_scale, workspace, workspace_bytes, stream);
-}
-
-kvq_status kvq_decode_attention_fp8(const void* q, const void* k_fp8, const void* v_fp8, void* out,
-                                    const kvq_cache_desc* desc, int batch_size, int n_heads, int page_size,
-                                    const int32_t* cache_seqlens, const int32_t* block_table, float softmax_scale,
-                                    void* workspace, size_t workspace_bytes, void* stream) {
-  return decode_attention(q, k_fp8, nullptr, v_fp8, nullptr, out, desc, batch_size, n_heads, page_size,
-                          cache_seqlens, block_table, 0, softmax_scale, workspace, workspace_bytes, stream);
-}
 
 long long kvq_count_match(const int64_t* a, long long a_len, const int64_t* b, long long b_len, long long max_a) {
   long long n = a_len < b_len ? a_len : b_len;
@@ -641,58 +476,5 @@ kvq_status kvq_selfcheck_code_rounding(int wbits, unsigned long long* mismatches
 
 }  // extern "C"
 
-// ---------------------------------------------------------------------------
-// Decode attention with library-owned scratch.
-//
-// Some callers cannot allocate device memory where they call attention: a
-// serving loop whose HBM is all handed to its own KV-page pool up front has
-// no allocator to draw a workspace from, and cudaMalloc / cudaFree may
-// synchronize the device, which a per-token decode step on a busy stream
-// cannot afford.  This entry point takes its split-K workspace from a fixed
-// array compiled into the library instead, so it allocates nothing.
-
-static __device__ __align__(256) unsigned char g_attention_scratch[KVQ_ATTENTION_SCRATCH_BYTES];
-
-namespace {
-
-constexpr int kScratchMaxDevices = 64;
-std::atomic<void*> g_attention_scratch_ptr[kScratchMaxDevices];
-
-// Device address of this device's copy of the array, looked up on the first
-// call made with the device current.  Null on failure.
-void* attention_scratch() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kScratchMaxDevices) {
-    cudaGetLastError();
-    return nullptr;
-  }
-  void* ptr = g_attention_scratch_ptr[dev].load();
-  if (ptr) return ptr;
-  if (cudaGetSymbolAddress(&ptr, g_attention_scratch) != cudaSuccess || !ptr) {
-    cudaGetLastError();
-    return nullptr;
-  }
-  g_attention_scratch_ptr[dev].store(ptr);
-  return ptr;
-}
-
-}  // namespace
-
-extern "C" {
-
-kvq_status kvq_decode_attention_q_noalloc(const void* q, const void* k_codes, const void* k_scales,
-                                          const void* v_codes, const void* v_scales, void* out,
-                                          const kvq_cache_desc* desc, int batch_size, int n_heads, int page_size,
-                                          const int32_t* cache_seqlens, const int32_t* block_table, int wbits,
-                                          float softmax_scale, void* stream) {
-  if (!desc) return KVQ_ERR_NULL;
-  if (kvq_decode_attention_workspace_size(desc, batch_size, n_heads, page_size) > KVQ_ATTENTION_SCRATCH_BYTES)
-    return KVQ_ERR_RANGE;
-  void* scratch = attention_scratch();
-  if (!scratch) return KVQ_ERR_CUDA;
-  return kvq_decode_attention_q(q, k_codes, k_scales, v_codes, v_scales, out, desc, batch_size, n_heads,
-                                page_size, cache_seqlens, block_table, wbits, softmax_scale, scratch,
-                                KVQ_ATTENTION_SCRATCH_BYTES, stream);
-}
-
-}  // extern "C"
+// Decode attention over the converted caches: host side.
+#include "attention_api.cuh"

@@ -813,17 +813,19 @@ __global__ void __launch_bounds__(kAttnThreads, D > 128 ? 2 : 4) attn_partial_ke
 }
 
 // Merge the chunks of every (sequence, head): CTA (head, sequence) of four
-// warps.  The chunk maxima are reduced by all threads at once; then warp w
-// sums chunks w, w + 4, ... (lane l owns head_dim elements l, l + 32, ...), so
-// that many chunks' loads are in flight, and the warps' sums meet in shared
-// memory.
+// warps.  Warp w takes chunks w, w + 4, ... in batches of kCombineBatch<D>
+// whose loads are all issued before any is used (lane l owns head_dim elements
+// l, l + 32, ...), and folds each batch into a running (max, sum, accumulator)
+// that it rescales when the maximum moves; the four warps' results meet in
+// shared memory.
 constexpr int kCombineThreads = 128;
+template <int D>
+constexpr int kCombineBatch = 1024 / D;  // chunks per warp in flight: 32 loaded values per lane
 
 template <int D>
-__global__ void __launch_bounds__(kCombineThreads) attn_combine_kernel(const __grid_constant__ AttnParams a) {
-  constexpr int kWarps = kCombineThreads / 32, DPL = D / 32;
-  __shared__ float s_red[kWarps];
-  __shared__ float s_l[kWarps];
+__global__ void __launch_bounds__(kCombineThreads, 8) attn_combine_kernel(const __grid_constant__ AttnParams a) {
+  constexpr int kWarps = kCombineThreads / 32, DPL = D / 32, NB = kCombineBatch<D>;
+  __shared__ float s_m[kWarps], s_l[kWarps];
   __shared__ float s_o[kWarps][D];
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -835,38 +837,57 @@ __global__ void __launch_bounds__(kCombineThreads) attn_combine_kernel(const __g
   long long nch = (L + a.chunk - 1) / a.chunk;
   if (nch > a.max_chunks) nch = a.max_chunks;
   const float* ws = a.ws + (static_cast<long long>(seq) * a.n_heads + h) * a.max_chunks * (D + 2);
-  float mx = -INFINITY;
-  for (long long c = threadIdx.x; c < nch; c += kCombineThreads) mx = fmaxf(mx, ws[c * (D + 2)]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-  if (lane == 0) s_red[warp] = mx;
-  __syncthreads();
-  float mstar = s_red[0];
-#pragma unroll
-  for (int w = 1; w < kWarps; ++w) mstar = fmaxf(mstar, s_red[w]);
-  float l = 0.0f, acc[DPL];
+  float m_run = -INFINITY, l_run = 0.0f, acc[DPL];
 #pragma unroll
   for (int k = 0; k < DPL; ++k) acc[k] = 0.0f;
-#pragma unroll 4
-  for (long long c = warp; c < nch; c += kWarps) {
-    const float* e = ws + c * (D + 2);
-    const float mc = e[0];
-    const float f = (mc == -INFINITY) ? 0.0f : exp2f(mc - mstar);
-    l += f * e[1];
+  for (long long c0 = warp; c0 < nch; c0 += static_cast<long long>(kWarps) * NB) {
+    float mc[NB], lc[NB], x[NB][DPL];
 #pragma unroll
-    for (int k = 0; k < DPL; ++k) acc[k] += f * e[2 + lane + 32 * k];
+    for (int i = 0; i < NB; ++i) {
+      const long long c = c0 + static_cast<long long>(i) * kWarps;
+      const bool in = c < nch;
+      const float* e = ws + (in ? c : 0) * (D + 2);
+      mc[i] = in ? e[0] : -INFINITY;
+      lc[i] = in ? e[1] : 0.0f;
+#pragma unroll
+      for (int k = 0; k < DPL; ++k) x[i][k] = in ? e[2 + lane + 32 * k] : 0.0f;
+    }
+    float mb = m_run;
+#pragma unroll
+    for (int i = 0; i < NB; ++i) mb = fmaxf(mb, mc[i]);
+    const float r = (m_run == -INFINITY) ? 0.0f : exp2f(m_run - mb);
+    l_run *= r;
+#pragma unroll
+    for (int k = 0; k < DPL; ++k) acc[k] *= r;
+#pragma unroll
+    for (int i = 0; i < NB; ++i) {
+      const float f = (mc[i] == -INFINITY) ? 0.0f : exp2f(mc[i] - mb);
+      l_run += f * lc[i];
+#pragma unroll
+      for (int k = 0; k < DPL; ++k) acc[k] += f * x[i][k];
+    }
+    m_run = mb;
+  }
+  if (lane == 0) {
+    s_m[warp] = m_run;
+    s_l[warp] = l_run;
   }
 #pragma unroll
   for (int k = 0; k < DPL; ++k) s_o[warp][lane + 32 * k] = acc[k];
-  if (lane == 0) s_l[warp] = l;
   __syncthreads();
-  float lt = 0.0f;
+  float mstar = s_m[0];
 #pragma unroll
-  for (int w = 0; w < kWarps; ++w) lt += s_l[w];
+  for (int w = 1; w < kWarps; ++w) mstar = fmaxf(mstar, s_m[w]);
+  float fw[kWarps], lt = 0.0f;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    fw[w] = (s_m[w] == -INFINITY) ? 0.0f : exp2f(s_m[w] - mstar);
+    lt += fw[w] * s_l[w];
+  }
   for (int d = threadIdx.x; d < D; d += kCombineThreads) {
     float o = 0.0f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) o += s_o[w][d];
+    for (int w = 0; w < kWarps; ++w) o += fw[w] * s_o[w][d];
     const float y = (lt > 0.0f) ? o / lt : 0.0f;
     a.out[(static_cast<long long>(seq) * a.n_heads + h) * D + d] = __float2half_rn(y);
   }

@@ -151,6 +151,18 @@ def test_many_short_sequences(kvq, oracle_mod, dev):
     check(kvq, oracle_mod, q, kc, ks, vc, vs, lens, 4, 1.0 / math.sqrt(D), dev)
 
 
+def test_small_batches_long_sequences(kvq, oracle_mod, dev):
+    """Batches far too small to give every resident warp a work item: one sequence of up to
+    5000 positions, and 8 sequences of up to 8192, over 8 kv heads and 32 query heads."""
+    for (B, S, H, D, NH), seed in [((1, 5000, 8, 128, 32), 51), ((8, 8192, 8, 128, 32), 52)]:
+        k, v = workloads.normal_kv((B, S, H, D), seed)
+        kc, ks, vc, vs = quantize_on_gpu(kvq, k, v, 4, dev)
+        g = torch.Generator().manual_seed(seed)
+        lens = torch.randint(S // 2, S + 1, (B,), generator=g, dtype=torch.int32)
+        q = torch.randn(B, NH, D, generator=g).half()
+        check(kvq, oracle_mod, q, kc, ks, vc, vs, lens, 4, 1.0 / math.sqrt(D), dev)
+
+
 def test_bad_paging_reported(kvq, dev):
     ps, H, D = 16, 1, 64
     k, v = workloads.small(shape=(4, ps, H, D))

@@ -600,6 +600,15 @@ def per_op_measurements(kvq, dev, peak, steps, flush, step, include_model=True):
            lambda i: fn())
     del fn
     torch.cuda.empty_cache()
+
+    # the small-batch end of decode: one sequence of 16384 positions (contiguous Q4
+    # [1, 16384, 8, 128], 32 query heads); 8 independent caches rotate, so that the 18.9 MB a
+    # launch reads is not in L2
+    fns, nb = attention_batch1_setup(kvq, dev)
+    record("decode_attention_q/q4/batch1", "contiguous [1, 16384, 8, 128] Q4, 1 sequence, 32 query heads", nb,
+           lambda i: fns[i % len(fns)](), sets=len(fns))
+    del fns
+    torch.cuda.empty_cache()
     del pool
     torch.cuda.empty_cache()
 
@@ -617,6 +626,32 @@ def attention_bytes(lens, kv_heads, head_dim, wbits, n_heads=ATTN_QUERY_HEADS):
     per_row = head_dim * wbits // 8 + 2 * (head_dim // 32)
     npos = sum(int(L) for L in lens)
     return 2 * npos * kv_heads * per_row + 2 * 2 * len(lens) * n_heads * head_dim
+
+
+def attention_batch1_setup(kvq, dev, seq_len=16384, copies=8, n_heads=ATTN_QUERY_HEADS):
+    """`copies` independent Q4 caches of one sequence ([1, seq_len, 8, 128], quantized untimed)
+    and the decode-attention launch over each; returns (launches, algorithmic bytes per launch)."""
+    H, D = 8, 128
+    shape = (1, seq_len, H, D)
+    cs, ss = kvq.q_shapes(shape, 4)
+    lens = torch.full((1,), seq_len, dtype=torch.int32, device=dev)
+    ws = torch.empty(max(16, kvq.attention_workspace_bytes(shape, 1, n_heads)), dtype=torch.uint8, device=dev)
+    fns = []
+    for i in range(copies):
+        k, v = workloads.normal_kv(shape, workloads.SEED_BASE + 90 + i, device=dev)
+        kc, vc = (torch.empty(cs, dtype=torch.uint8, device=dev) for _ in range(2))
+        ks, vs = (torch.empty(ss, dtype=torch.float16, device=dev) for _ in range(2))
+        kvq.fp16_to_q_kv(k, kc, ks, v, vc, vs, 1, 0, seq_len, 0, None, None, 4)
+        del k, v
+        g = torch.Generator(device="cpu").manual_seed(workloads.SEED_BASE + 78 + i)
+        q = torch.randn(1, n_heads, D, generator=g).half().to(dev)
+        out = torch.empty_like(q)
+
+        def fn(q=q, kc=kc, ks=ks, vc=vc, vs=vs, out=out):
+            kvq.decode_attention_q(q, kc, ks, vc, vs, out, 1, lens, 4, 1.0 / math.sqrt(D), workspace=ws)
+        fn()
+        fns.append(fn)
+    return fns, attention_bytes([seq_len], H, D, 4, n_heads)
 
 
 def attention_setup_fp8(kvq, dev, pool, n_heads=ATTN_QUERY_HEADS):

@@ -13,7 +13,9 @@
 // grid (one wave of CTAs of four warps).  Every (sequence, 256-position chunk,
 // kv head) that holds data is a work item; warp w of W takes items w, w + W,
 // ... of a compact enumeration of them (so the warps' shares differ by at most
-// one item) and walks each: it streams the item through two shared-memory buffers of 16 or 32
+// one item; when there are no more items than CTAs, the four warps of a CTA
+// take a quarter of each item instead and merge the quarters in shared
+// memory) and walks each: it streams the item through two shared-memory buffers of 16 or 32
 // positions (cp.async copies of K and V codes, scales and, with the first
 // sub-chunk, the group's query rows), filling one while it computes on the
 // other, 16 positions at a time:
@@ -438,21 +440,45 @@ struct AttnCursor {
 // batch fits the slots and that every item count fits an int.
 // Otherwise: every (sequence, chunk, kv head) slot up to the cache's capacity
 // is visited and empty ones are skipped (lengths staged when the batch fits).
-template <int B, int D, bool kCompact>
+// kSplit (with kCompact, for batches too small to give every warp an item):
+// a CTA takes items in turn and each of its four warps a quarter of the
+// item's positions, every warp walking the same kSplitSubs sub-chunks per item
+// (empty ones where its quarter runs past the sequence), so that the CTA can
+// merge the four partial results at the end of each item.
+template <int B, int D, bool kCompact, bool kSplit = false>
 struct AttnWalk {
+  static_assert(kCompact || !kSplit, "the split walk enumerates compactly");
   using T = AttnTile<B, D>;
   using Item = typename std::conditional<kCompact, int, long long>::type;
   using Cursor = AttnCursor<Item>;
+  static constexpr int kQuarter = T::kChunk / kAttnWarps;  // positions per warp and item (kSplit)
+  static constexpr int kSplitSubs = kQuarter / T::kSub;     // sub-chunks per warp and item (kSplit)
   const AttnParams& a;
   bool staged;  // the batch's lengths are in shared memory
+
+  // first position of this warp's part of an item
+  __device__ static int offset() { return kSplit ? kQuarter * static_cast<int>(threadIdx.x >> 5) : 0; }
+  // positions and last-sub-chunk flag of sub-chunk `sub` of an item of sequence length L
+  __device__ void set_sub(Cursor& c, int L, int sub) const {
+    c.sub = sub;
+    if constexpr (kSplit) {
+      const int rest = L - c.chunk * T::kChunk - offset() - sub * T::kSub;
+      c.n = max(0, min(rest, T::kSub));
+      c.last = sub == kSplitSubs - 1;
+    } else {
+      const int rest = min(L - c.chunk * T::kChunk, T::kChunk) - sub * T::kSub;
+      c.n = min(rest, T::kSub);
+      c.last = rest <= T::kSub;
+    }
+  }
 
   // the staged block, after the warps' buffers in dynamic shared memory
   __device__ static int* block() {
     extern __shared__ __align__(16) uint8_t smem[];
     return reinterpret_cast<int*>(smem + kAttnWarps * T::kWarpBytes);
   }
-  // warps in the grid
-  __device__ static Item stride() { return static_cast<Item>(gridDim.x) * kAttnWarps; }
+  // walkers in the grid: warps, or CTAs with kSplit
+  __device__ static Item stride() { return static_cast<Item>(gridDim.x) * (kSplit ? 1 : kAttnWarps); }
 
   __device__ long long max_len() const {
     return a.page_size == 0 ? static_cast<long long>(a.dim1) : static_cast<long long>(a.max_chunks) * T::kChunk;
@@ -484,11 +510,8 @@ struct AttnWalk {
       c.seq = lo;
       c.chunk = static_cast<int>(chunk);
       c.kvh = static_cast<int>(r - chunk * static_cast<unsigned>(a.kv_heads));
-      const int rest = min(length(c.seq) - c.chunk * T::kChunk, T::kChunk);
       c.item = item;
-      c.sub = 0;
-      c.n = min(rest, T::kSub);
-      c.last = rest <= T::kSub;
+      set_sub(c, length(c.seq), 0);
       return c;
     } else {
       const long long n_items = static_cast<long long>(a.batch) * a.max_chunks * a.kv_heads;
@@ -508,10 +531,7 @@ struct AttnWalk {
         const int p0 = c.chunk * T::kChunk;
         if (p0 < L) {
           c.item = item;
-          c.sub = 0;
-          const int rest = min(L - p0, T::kChunk);
-          c.n = min(rest, T::kSub);
-          c.last = rest <= T::kSub;
+          set_sub(c, L, 0);
           return c;
         }
       }
@@ -522,10 +542,7 @@ struct AttnWalk {
   __device__ Cursor next(const Cursor& c) const {
     if (c.last) return seek(c.item + stride());
     Cursor d = c;
-    d.sub = c.sub + 1;
-    const int rest = min(length(c.seq) - c.chunk * T::kChunk, T::kChunk) - d.sub * T::kSub;
-    d.n = min(rest, T::kSub);
-    d.last = rest <= T::kSub;
+    set_sub(d, length(c.seq), c.sub + 1);
     return d;
   }
 };
@@ -534,8 +551,8 @@ struct AttnWalk {
 // sub-chunk of an item, its query rows into the warp's query area); returns
 // the bit mask of its positions that hold data (bit i: position i).
 template <int B, int D, class Cursor>
-__device__ __forceinline__ uint32_t attn_issue(const AttnParams& a, const Cursor& c, uint8_t* buf, uint8_t* sq,
-                                               int lane) {
+__device__ __forceinline__ uint32_t attn_issue(const AttnParams& a, const Cursor& c, int offset, uint8_t* buf,
+                                               uint8_t* sq, int lane) {
   using T = AttnTile<B, D>;
   constexpr int SC = T::kSub, P = T::kRowBytes / 16;
   uint8_t* const sk = buf;
@@ -545,7 +562,7 @@ __device__ __forceinline__ uint32_t attn_issue(const AttnParams& a, const Cursor
   // cache row of this lane's position (lanes < SC): -1 bad paging metadata, -2 past the window
   long long hr = -2;
   if (lane < c.n) {
-    const int p = c.chunk * T::kChunk + c.sub * SC + lane;
+    const int p = c.chunk * T::kChunk + offset + c.sub * SC + lane;
     long long row;
     if (a.page_size == 0) {
       row = static_cast<long long>(c.seq) * a.dim1 + p;
@@ -600,7 +617,7 @@ __device__ __forceinline__ uint32_t attn_issue(const AttnParams& a, const Cursor
   return mask;
 }
 
-template <int B, int D, bool kCompact>
+template <int B, int D, bool kCompact, bool kSplit>
 __global__ void __launch_bounds__(kAttnThreads, D > 128 ? 2 : 4) attn_partial_kernel(const __grid_constant__ AttnParams a) {
   using T = AttnTile<B, D>;
   using Codec = AttnCodec<B>;
@@ -613,7 +630,8 @@ __global__ void __launch_bounds__(kAttnThreads, D > 128 ? 2 : 4) attn_partial_ke
   const int g = lane >> 2, j = lane & 3;
   uint8_t* const wbuf = smem + warp * T::kWarpBytes;
   int* const s_len = reinterpret_cast<int*>(smem + kAttnWarps * T::kWarpBytes);
-  using Walk = AttnWalk<B, D, kCompact>;
+  using Walk = AttnWalk<B, D, kCompact, kSplit>;
+  static_assert(!kSplit || kAttnMaxGroup * (D + 2) * 4 <= T::kBufBytes, "a warp's partial result fits its buffer");
 
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -645,9 +663,12 @@ __global__ void __launch_bounds__(kAttnThreads, D > 128 ? 2 : 4) attn_partial_ke
 
   const Walk walk{a, staged};
   uint8_t* const sq_area = wbuf + 2 * T::kBufBytes;
-  typename Walk::Cursor cur = walk.seek(static_cast<typename Walk::Item>(blockIdx.x) * kAttnWarps + warp);
+  const int offset = Walk::offset();
+  typename Walk::Cursor cur =
+      walk.seek(kSplit ? static_cast<typename Walk::Item>(blockIdx.x)
+                       : static_cast<typename Walk::Item>(blockIdx.x) * kAttnWarps + warp);
   if (cur.item < 0) return;
-  uint32_t mask_cur = attn_issue<B, D>(a, cur, wbuf, sq_area, lane);
+  uint32_t mask_cur = attn_issue<B, D>(a, cur, offset, wbuf, sq_area, lane);
   asm volatile("cp.async.commit_group;\n" ::: "memory");
   int b = 0;
 
@@ -689,7 +710,7 @@ __global__ void __launch_bounds__(kAttnThreads, D > 128 ? 2 : 4) attn_partial_ke
     const typename Walk::Cursor nxt = walk.next(cur);
     uint32_t mask_nxt = 0;
     if (nxt.item >= 0) {
-      mask_nxt = attn_issue<B, D>(a, nxt, wbuf + (b ^ 1) * T::kBufBytes, sq_area, lane);
+      mask_nxt = attn_issue<B, D>(a, nxt, offset, wbuf + (b ^ 1) * T::kBufBytes, sq_area, lane);
       asm volatile("cp.async.commit_group;\n" ::: "memory");
     }
 
@@ -785,8 +806,13 @@ __global__ void __launch_bounds__(kAttnThreads, D > 128 ? 2 : 4) attn_partial_ke
       l_sum += __shfl_xor_sync(0xFFFFFFFFu, l_sum, 1);
       l_sum += __shfl_xor_sync(0xFFFFFFFFu, l_sum, 2);
       const long long head0 = static_cast<long long>(cur.seq) * a.n_heads + static_cast<long long>(cur.kvh) * a.group;
-      float* const ws = a.ws + (head0 * a.max_chunks + cur.chunk) * (D + 2);
-      const long long hstride = static_cast<long long>(a.max_chunks) * (D + 2);  // next head, same chunk
+      float* const entry = a.ws + (head0 * a.max_chunks + cur.chunk) * (D + 2);
+      const long long entry_stride = static_cast<long long>(a.max_chunks) * (D + 2);  // next head, same chunk
+      // kSplit: the warp's quarter goes to its own buffer (free now: the next
+      // sub-chunk streams into the other one), one (D + 2)-float row per head
+      float* const ws = kSplit ? reinterpret_cast<float*>(wbuf + b * T::kBufBytes) : entry;
+      const long long hstride = kSplit ? D + 2 : entry_stride;
+      if (kSplit) __syncwarp();  // every lane is done reading the buffer
       if (j == 0 && g < a.group) {
         ws[g * hstride] = m_ref;
         ws[g * hstride + 1] = l_sum;
@@ -802,6 +828,35 @@ __global__ void __launch_bounds__(kAttnThreads, D > 128 ? 2 : 4) attn_partial_ke
           ws[(2 * j + 1) * hstride + 2 + da] = acc[mt][1];
           ws[(2 * j + 1) * hstride + 2 + db] = acc[mt][3];
         }
+      }
+      if constexpr (kSplit) {
+        // Merge the four quarters into the item's workspace entry.  Every warp
+        // of the CTA walks the same items with the same number of sub-chunks,
+        // so all four reach these barriers together and use the same buffer b.
+        __syncthreads();
+        for (int e = threadIdx.x; e < a.group * D; e += kAttnThreads) {
+          const int h = e / D, d = e - h * D;
+          const float* part[kAttnWarps];
+          float mx = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < kAttnWarps; ++w) {
+            part[w] = reinterpret_cast<const float*>(smem + w * T::kWarpBytes + b * T::kBufBytes) + h * (D + 2);
+            mx = fmaxf(mx, part[w][0]);
+          }
+          float o = 0.0f, l = 0.0f;
+#pragma unroll
+          for (int w = 0; w < kAttnWarps; ++w) {
+            const float f = (part[w][0] == -INFINITY) ? 0.0f : exp2f(part[w][0] - mx);
+            o += f * part[w][2 + d];
+            l += f * part[w][1];
+          }
+          entry[h * entry_stride + 2 + d] = o;
+          if (d == 0) {
+            entry[h * entry_stride] = mx;
+            entry[h * entry_stride + 1] = l;
+          }
+        }
+        __syncthreads();  // the buffers are refilled from the next iteration on
       }
     }
     __syncwarp();  // every lane is done with this buffer before it is refilled

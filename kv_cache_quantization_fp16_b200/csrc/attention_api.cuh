@@ -19,15 +19,15 @@ long long attn_max_chunks(const kvq_cache_desc* d, int page_size, int chunk) {
 
 // Dynamic shared memory opt-in, once per device for each partial kernel
 // (static plus dynamic shared memory above 48 KB needs it).
-template <int B, int D, bool kCompact>
+template <int B, int D, bool kCompact, bool kSplit>
 bool allow_attention_smem() {
   constexpr int kMaxDevices = 64;
   static std::atomic<bool> done[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
   if (done[dev].load()) return true;
-  if (cudaFuncSetAttribute(kvq::attn_partial_kernel<B, D, kCompact>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kvq::AttnTile<B, D>::kSmemBytes) != cudaSuccess) {
+  if (cudaFuncSetAttribute(kvq::attn_partial_kernel<B, D, kCompact, kSplit>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, kvq::AttnTile<B, D>::kSmemBytes) != cudaSuccess) {
     cudaGetLastError();
     return false;
   }
@@ -35,27 +35,36 @@ bool allow_attention_smem() {
   return true;
 }
 
-// Persistent grid of the partial kernel: every (sequence, 256-position chunk,
-// kv head) work item goes to one warp; as many CTAs as the device holds at
-// once (occupancy cached per device), never more than there are item slots.
-template <int B, int D, bool kCompact>
-kvq_status launch_partial(const kvq::AttnParams& a, long long items, void* stream) {
-  using T = kvq::AttnTile<B, D>;
-  if (!allow_attention_smem<B, D, kCompact>()) return KVQ_ERR_CUDA;
+// CTAs of a partial kernel the device holds at once (occupancy cached per
+// device), 0 on failure.
+template <int B, int D, bool kCompact, bool kSplit>
+long long partial_ctas() {
+  if (!allow_attention_smem<B, D, kCompact, kSplit>()) return 0;
   constexpr int kMaxDevices = 64;
   static std::atomic<long long> resident[kMaxDevices];
-  const long long ctas_max = first_wave_ctas(kvq::attn_partial_kernel<B, D, kCompact>, kvq::kAttnThreads,
-                                             T::kSmemBytes, resident, kMaxDevices);
+  return first_wave_ctas(kvq::attn_partial_kernel<B, D, kCompact, kSplit>, kvq::kAttnThreads,
+                         kvq::AttnTile<B, D>::kSmemBytes, resident, kMaxDevices);
+}
+
+// Persistent grid of the partial kernel: every (sequence, 256-position chunk,
+// kv head) work item goes to one warp (to one CTA with kSplit); as many CTAs
+// as the device holds at once, never more than there are item slots.
+template <int B, int D, bool kCompact, bool kSplit>
+kvq_status launch_partial(const kvq::AttnParams& a, long long items, long long ctas_max, void* stream) {
+  using T = kvq::AttnTile<B, D>;
   if (ctas_max < 1) return KVQ_ERR_CUDA;
-  const long long need = (items + kvq::kAttnWarps - 1) / kvq::kAttnWarps;
+  const long long need = kSplit ? items : (items + kvq::kAttnWarps - 1) / kvq::kAttnWarps;
   const unsigned grid = static_cast<unsigned>(need < ctas_max ? need : ctas_max);
-  return launch_pdl(kvq::attn_partial_kernel<B, D, kCompact>, dim3(grid), kvq::kAttnThreads, T::kSmemBytes, stream,
-                    a);
+  return launch_pdl(kvq::attn_partial_kernel<B, D, kCompact, kSplit>, dim3(grid), kvq::kAttnThreads, T::kSmemBytes,
+                    stream, a);
 }
 
 // The partial kernel walks only the items that hold data when the batch fits
 // its shared-memory slots and every item count fits an int; otherwise it
-// visits every item slot.  Then the combine kernel.
+// visits every item slot.  When the cache geometry has no more item slots
+// than the device holds CTAs (batches of one or two long sequences; head_dim
+// <= 128), the four warps of a CTA share each item (measured: 10% faster
+// there, slower from two items per CTA on).  Then the combine kernel.
 template <int B, int D>
 kvq_status launch_attention(kvq::AttnParams a, const kvq_cache_desc* desc, void* stream) {
   using T = kvq::AttnTile<B, D>;
@@ -65,8 +74,16 @@ kvq_status launch_attention(kvq::AttnParams a, const kvq_cache_desc* desc, void*
   a.max_chunks = static_cast<int>(max_chunks);
   const long long items = static_cast<long long>(a.batch) * a.max_chunks * a.kv_heads;
   const bool compact = a.batch <= T::kSeqlenSlots && items <= 0x7FFFFFFFLL;
-  const kvq_status st = compact ? launch_partial<B, D, true>(a, items, stream)
-                                : launch_partial<B, D, false>(a, items, stream);
+  kvq_status st;
+  if (!compact) {
+    st = launch_partial<B, D, false, false>(a, items, partial_ctas<B, D, false, false>(), stream);
+  } else {
+    const long long ctas = partial_ctas<B, D, true, false>();
+    if (D <= 128 && items <= ctas)
+      st = launch_partial<B, D, true, D <= 128>(a, items, partial_ctas<B, D, true, D <= 128>(), stream);
+    else
+      st = launch_partial<B, D, true, false>(a, items, ctas, stream);
+  }
   if (st != KVQ_OK) return st;
   return launch_pdl(kvq::attn_combine_kernel<D>, dim3(a.n_heads, a.batch), kvq::kCombineThreads, 0, stream, a);
 }

@@ -232,7 +232,8 @@ KVQ_API size_t kvq_decode_attention_workspace_size(const kvq_cache_desc* desc, i
  *   kvq_decode_attention_workspace_size(...) exceeds
  *   KVQ_ATTENTION_SCRATCH_BYTES returns KVQ_ERR_RANGE and enqueues nothing
  *   (for example, batch 8 x 32 query heads x head_dim 128 with up to 8192
- *   positions needs 8.5 MB and fits).
+ *   positions needs 4.3 MB and fits; batch 16 with up to 16384 positions
+ *   needs 17 MB and does not).
  *   The first call on each device, made with that device current, looks up
  *   the array's device address; make that first call before any stream
  *   capture.  KVQ_ERR_CUDA if the lookup fails.

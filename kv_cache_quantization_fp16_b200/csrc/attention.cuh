@@ -299,7 +299,7 @@ struct AttnTile {
   static constexpr int kStrideK = kRowBytes + (kRowBytes % 128 == 0 ? 16 : 0);
   static constexpr int kStrideV = kRowBytes + ((B == 6 && D == 64) ? 0 : 16);
   static constexpr int kScales = B == 0 ? 0 : D / 32;  // binary16 scales per row
-  static constexpr int kChunk = 256;                        // positions per work item / workspace entry
+  static constexpr int kChunk = 256;  // positions per work item / workspace entry (kAttnMinChunk)
   static constexpr int kSub = kRowBytes <= 96 ? 32 : 16;   // positions per staged buffer (measured)
   static constexpr int kBufK = kSub * kStrideK;
   static constexpr int kBufV = kSub * kStrideV;
@@ -317,7 +317,7 @@ struct AttnTile {
   static constexpr int kKSpanBytes = KN * kBits / 8;
   static constexpr int kVSpanBytes = VN * kBits / 8;
 };
-constexpr int kAttnMinChunk = 128;  // sizes the workspace: no (B, D) uses a shorter chunk
+constexpr int kAttnMinChunk = 256;  // sizes the workspace: every (B, D) uses 256-position chunks
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),

@@ -102,7 +102,7 @@ extern "C" {
 size_t kvq_decode_attention_workspace_size(const kvq_cache_desc* desc, int batch_size, int n_heads,
                                            int page_size) {
   if (!desc || batch_size < 0 || n_heads < 0 || page_size < 0) return 0;
-  // sized for the smallest chunk any wbits / head_dim uses
+  // one entry per (sequence, query head, 256-position chunk slot)
   return static_cast<size_t>(batch_size) * n_heads * attn_max_chunks(desc, page_size, kvq::kAttnMinChunk) *
          (desc->head_dim + 2) * sizeof(float);
 }

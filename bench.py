@@ -745,7 +745,7 @@ def model_layers(kvq, dev, peak, steps, flush, layers=32):
 CASES = ("headline_fp8enc_kv", "headline_fp8dec_kv", "headline_fp8enc", "headline_fp8dec", "fp8enc", "fp8dec", "q4enc",
          "q4dec", "q6enc", "q6dec", "q8enc", "q8dec", "paged_prefill_q4enc", "paged_prefill_q4dec",
          "paged_decode_q4enc", "model_layer_q6enc", "model_layer_q6dec", "attn_paged_q4", "attn_paged_q6",
-         "attn_paged_q8", "attn_paged_fp8")
+         "attn_paged_q8", "attn_paged_fp8", "attn_batch1_q4")
 
 
 def run_case(kvq, dev, name, batch, steps, warmup, peak, stream=False):
@@ -805,6 +805,9 @@ def run_case(kvq, dev, name, batch, steps, warmup, peak, stream=False):
             fn = (lambda: kvq.fp16_to_q_kv(k, kc, ks, v, vc, vs, B, 0, S, 0, None, None, wb)) \
                 if name.endswith("enc") else (lambda: kvq.q_to_fp16_kv(kc, ky, ks, vc, vy, vs, B, 0, S, 0, None,
                                                                         None, wb))
+    elif name == "attn_batch1_q4":
+        fns, nb = attention_batch1_setup(kvq, dev, copies=1)
+        fn = fns[0]
     elif name == "attn_paged_fp8":
         pool = workloads.paged_pool(device=dev)
         fn, nb = attention_setup_fp8(kvq, dev, pool)

@@ -212,7 +212,8 @@ KVQ_API kvq_status kvq_decode_attention_fp8(const void* q, const void* k_fp8, co
                                             void* stream);
 
 /* Workspace bytes kvq_decode_attention_q and kvq_decode_attention_fp8 need for
- * this geometry (0 for bad arguments).  Host-only. */
+ * this geometry (0 for bad arguments, SIZE_MAX when the size overflows size_t,
+ * which the attention calls reject with KVQ_ERR_RANGE).  Host-only. */
 KVQ_API size_t kvq_decode_attention_workspace_size(const kvq_cache_desc* desc, int batch_size, int n_heads,
                                                    int page_size);
 

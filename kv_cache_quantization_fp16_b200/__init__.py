@@ -315,6 +315,9 @@ def count_match(a: torch.Tensor, b: torch.Tensor, max_a: int) -> int:
     return int(n)
 
 
+_SIZE_MAX = (1 << (8 * ctypes.sizeof(ctypes.c_size_t))) - 1  # the workspace size query's overflow value
+
+
 def attention_workspace_bytes(cache_shape, batch_size: int, n_heads: int, page_size: int = 0,
                               block_table_stride: int = 0) -> int:
     """Workspace bytes decode_attention_q needs: cache_shape is the FP16 cache shape
@@ -361,6 +364,7 @@ def decode_attention_q(q, k_codes, k_scales, v_codes, v_scales, out, batch_size,
     n_heads = q.shape[1]
     need = int(_lib.kvq_decode_attention_workspace_size(ctypes.byref(desc), int(batch_size), int(n_heads),
                                                         int(page_size)))
+    _require(need < _SIZE_MAX, "the workspace this geometry needs does not fit in size_t")
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     _require(workspace.is_cuda and workspace.device == dev and workspace.numel() >= need,
@@ -400,6 +404,7 @@ def decode_attention_fp8(q, k_fp8, v_fp8, out, batch_size, cache_seqlens, softma
     n_heads = q.shape[1]
     need = int(_lib.kvq_decode_attention_workspace_size(ctypes.byref(desc), int(batch_size), int(n_heads),
                                                         int(page_size)))
+    _require(need < _SIZE_MAX, "the workspace this geometry needs does not fit in size_t")
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     _require(workspace.is_cuda and workspace.device == dev and workspace.numel() >= need,

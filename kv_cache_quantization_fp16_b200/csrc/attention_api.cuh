@@ -101,10 +101,18 @@ extern "C" {
 
 size_t kvq_decode_attention_workspace_size(const kvq_cache_desc* desc, int batch_size, int n_heads,
                                            int page_size) {
-  if (!desc || batch_size < 0 || n_heads < 0 || page_size < 0) return 0;
-  // one entry per (sequence, query head, 256-position chunk slot)
-  return static_cast<size_t>(batch_size) * n_heads * attn_max_chunks(desc, page_size, kvq::kAttnMinChunk) *
-         (desc->head_dim + 2) * sizeof(float);
+  if (!desc || batch_size < 0 || n_heads < 0 || page_size < 0 || desc->head_dim < 0 || desc->dim1 < 0 ||
+      desc->block_table_stride < 0)
+    return 0;
+  // one entry per (sequence, query head, 256-position chunk slot); SIZE_MAX when that overflows
+  const long long chunks = attn_max_chunks(desc, page_size, kvq::kAttnMinChunk);
+  size_t n = static_cast<size_t>(batch_size);
+  if (__builtin_mul_overflow(n, static_cast<size_t>(n_heads), &n) ||
+      __builtin_mul_overflow(n, static_cast<size_t>(chunks), &n) ||
+      __builtin_mul_overflow(n, static_cast<size_t>(desc->head_dim) + 2, &n) ||
+      __builtin_mul_overflow(n, sizeof(float), &n))
+    return SIZE_MAX;
+  return n;
 }
 
 }  // extern "C"
@@ -143,8 +151,8 @@ kvq_status decode_attention(const void* q, const void* k_codes, const void* k_sc
   const long long max_chunks = attn_max_chunks(desc, page_size, kvq::kAttnMinChunk);
   if (max_chunks < 1 || max_chunks > 0x7FFFFFFFLL) return KVQ_ERR_RANGE;
   if (!workspace) return KVQ_ERR_NULL;
-  if (workspace_bytes < kvq_decode_attention_workspace_size(desc, batch_size, n_heads, page_size))
-    return KVQ_ERR_RANGE;
+  const size_t need = kvq_decode_attention_workspace_size(desc, batch_size, n_heads, page_size);
+  if (need == SIZE_MAX || workspace_bytes < need) return KVQ_ERR_RANGE;
   kvq::AttnParams a{};
   a.q = static_cast<const __half*>(q);
   a.k_codes = static_cast<const uint8_t*>(k_codes);

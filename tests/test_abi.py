@@ -170,6 +170,24 @@ def test_decode_attention_validation(kvq):
     assert call(bs=0, wsp=None, wsb=0) == 0             # empty batch enqueues nothing
 
 
+def test_decode_attention_workspace_size_overflow(kvq):
+    """A geometry whose workspace size overflows size_t: the size query returns SIZE_MAX and
+    the attention call is rejected before anything is enqueued, whatever workspace it is
+    handed (a wrapped size would otherwise admit a small one)."""
+    L = kvq.library()
+    by = ctypes.byref
+    # paged: 65535 sequences x 524280 query heads x (2^31 - 1) chunk slots x 258 floats
+    d = _desc(kvq, d0=1, d1=256, H=65535, D=256, stride=(1 << 31) - 1)
+    size_max = (1 << (8 * ctypes.sizeof(ctypes.c_size_t))) - 1
+    assert L.kvq_decode_attention_workspace_size(by(d), 65535, 8 * 65535, 256) == size_max
+    P = [FAKE] * 6
+    st = L.kvq_decode_attention_q(*P, by(d), 65535, 8 * 65535, 256, FAKE, FAKE, 4, ctypes.c_float(1.0), FAKE,
+                                  1 << 20, None)
+    assert st == 4  # KVQ_ERR_RANGE
+    assert L.kvq_decode_attention_q_noalloc(*P, by(d), 65535, 8 * 65535, 256, FAKE, FAKE, 4, ctypes.c_float(1.0),
+                                            None) == 4
+
+
 def test_decode_attention_fp8_validation(kvq):
     L = kvq.library()
     by = ctypes.byref

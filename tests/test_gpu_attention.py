@@ -151,6 +151,21 @@ def test_many_short_sequences(kvq, oracle_mod, dev):
     check(kvq, oracle_mod, q, kc, ks, vc, vs, lens, 4, 1.0 / math.sqrt(D), dev)
 
 
+@pytest.mark.parametrize("wbits", [4, 8])
+def test_per_warp_items_with_empty_and_short_sequences(kvq, oracle_mod, dev, wbits):
+    """A batch with more work-item slots than the GPU holds CTAs, so that every warp walks
+    its own items (not the CTA-shared split used for one or two sequences), with empty,
+    one-position and chunk-boundary sequence lengths among random ones."""
+    B, S, H, D, NH = 48, 600, 8, 64, 16
+    k, v = workloads.normal_kv((B, S, H, D), 61)
+    kc, ks, vc, vs = quantize_on_gpu(kvq, k, v, wbits, dev)
+    g = torch.Generator().manual_seed(62)
+    lens = torch.randint(0, S + 1, (B,), generator=g, dtype=torch.int32)
+    lens[:6] = torch.tensor([0, 1, 255, 256, 257, S], dtype=torch.int32)
+    q = torch.randn(B, NH, D, generator=g).half()
+    check(kvq, oracle_mod, q, kc, ks, vc, vs, lens, wbits, 1.0 / math.sqrt(D), dev)
+
+
 def test_small_batches_long_sequences(kvq, oracle_mod, dev):
     """Batches far too small to give every resident warp a work item: one sequence of up to
     5000 positions, and 8 sequences of up to 8192, over 8 kv heads and 32 query heads."""

@@ -12,13 +12,13 @@
 // Split-K flash decoding.  Kernel 1 (attn_partial_kernel) is a persistent
 // grid (one wave of CTAs of four warps).  Every (sequence, 256-position chunk,
 // kv head) that holds data is a work item; warp w of W takes items w, w + W,
-// ... of a compact enumeration of them (so the warps' shares differ by at most
-// one item; when there are no more items than CTAs, the four warps of a CTA
+// ... of a compact enumeration of them, so the warps' shares differ by at most
+// one item.  (When there are no more items than CTAs, the four warps of a CTA
 // take a quarter of each item instead and merge the quarters in shared
-// memory) and walks each: it streams the item through two shared-memory buffers of 16 or 32
-// positions (cp.async copies of K and V codes, scales and, with the first
-// sub-chunk, the group's query rows), filling one while it computes on the
-// other, 16 positions at a time:
+// memory.)  A warp streams its part of an item through two shared-memory
+// buffers of 16 or 32 positions (cp.async copies of K and V codes, scales
+// and, with the first sub-chunk, the group's query rows), filling one while it
+// computes on the other, 16 positions at a time:
 //   * S = Q K^T on mma.sync m16n8k16 with the query heads as the M dimension
 //     (rows >= group are zero) and 8 positions per N tile: each lane
 //     dequantizes one contiguous span of D/4 elements of one position (a B
@@ -66,7 +66,7 @@ struct AttnParams {
   const int32_t* seqlens;
   const int32_t* block_table;
   int dim0, dim1, kv_heads, batch, n_heads, group, page_size, bt_stride, max_chunks;
-  int chunk;  // positions per CTA (AttnTile<B, D>::kChunk)
+  int chunk;  // positions per work item (AttnTile<B, D>::kChunk)
   float scale_log2;  // softmax_scale * log2(e)
 };
 
@@ -320,7 +320,8 @@ struct AttnTile {
 constexpr int kAttnMinChunk = 256;  // sizes the workspace: every (B, D) uses 256-position chunks
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n"
+               ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
                "l"(src)
                : "memory");
 }
@@ -328,7 +329,8 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
 template <int N>
 __device__ __forceinline__ void cp_async_small(void* dst, const void* src) {
   static_assert(N == 4 || N == 8 || N == 16, "cp.async sizes");
-  asm volatile("cp.async.ca.shared.global [%0], [%1], %2;\n" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+  asm volatile("cp.async.ca.shared.global [%0], [%1], %2;\n"
+               ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
                "l"(src), "n"(N)
                : "memory");
 }
@@ -392,8 +394,10 @@ __device__ __forceinline__ void v_span_pair(const uint8_t* r0, const uint8_t* r1
     // 6 bytes at byte 6g: the aligned 8 bytes around them, bytes o..o+5 (o = 0 or 2)
     const int base = (6 * g) & ~3;
     const uint32_t o = (6 * g) & 3;
-    const uint32_t a0 = reinterpret_cast<const uint32_t*>(r0 + base)[0], b0 = reinterpret_cast<const uint32_t*>(r0 + base)[1];
-    const uint32_t a1 = reinterpret_cast<const uint32_t*>(r1 + base)[0], b1 = reinterpret_cast<const uint32_t*>(r1 + base)[1];
+    const uint32_t* const w0 = reinterpret_cast<const uint32_t*>(r0 + base);
+    const uint32_t* const w1 = reinterpret_cast<const uint32_t*>(r1 + base);
+    const uint32_t a0 = w0[0], b0 = w0[1];
+    const uint32_t a1 = w1[0], b1 = w1[1];
     uint32_t x[4], y[4];
     AttnCodec<6>::raw8_at(a0, b0, o, x);
     AttnCodec<6>::raw8_at(a1, b1, o, y);
@@ -618,7 +622,8 @@ __device__ __forceinline__ uint32_t attn_issue(const AttnParams& a, const Cursor
 }
 
 template <int B, int D, bool kCompact, bool kSplit>
-__global__ void __launch_bounds__(kAttnThreads, D > 128 ? 2 : 4) attn_partial_kernel(const __grid_constant__ AttnParams a) {
+__global__ void __launch_bounds__(kAttnThreads, D > 128 ? 2 : 4)
+    attn_partial_kernel(const __grid_constant__ AttnParams a) {
   using T = AttnTile<B, D>;
   using Codec = AttnCodec<B>;
   constexpr int KS = T::KS;  // k-steps of Q K^T, m-tiles of V^T P^T

@@ -27,7 +27,8 @@ bool allow_attention_smem() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
   if (done[dev].load()) return true;
   if (cudaFuncSetAttribute(kvq::attn_partial_kernel<B, D, kCompact, kSplit>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, kvq::AttnTile<B, D>::kSmemBytes) != cudaSuccess) {
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kvq::AttnTile<B, D>::kSmemBytes) != cudaSuccess) {
     cudaGetLastError();
     return false;
   }

@@ -282,6 +282,15 @@ KVQ_API int kvq_get_engine(void);
  * pairs whose codes differ (0 expected).  Asynchronous on `stream`. */
 KVQ_API kvq_status kvq_selfcheck_code_rounding(int wbits, unsigned long long* mismatches, void* stream);
 
+/* Self-check of the bulk engine's bounded waits (no counterpart on the page):
+ * one CTA waits, with the same bounded wait the bulk engine's pipeline uses,
+ * on a shared-memory mbarrier that nothing ever arrives on.  After the wait's
+ * limit (1 s) it gives up, writes 1 to *waited_out (a caller-owned device
+ * int32, written 0 first) and records KVQ_DEV_TIMEOUT in the device error
+ * word, and the kernel ends; no fault, no hang, and the context stays usable.
+ * Asynchronous on `stream`. */
+KVQ_API kvq_status kvq_selfcheck_wait_timeout(int32_t* waited_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

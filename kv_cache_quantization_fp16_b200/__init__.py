@@ -69,6 +69,7 @@ def _load() -> ctypes.CDLL:
     L.kvq_status_string.restype = ctypes.c_char_p
     L.kvq_poll_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), vp]
     L.kvq_selfcheck_code_rounding.argtypes = [I, vp, vp]
+    L.kvq_selfcheck_wait_timeout.argtypes = [vp, vp]
     LL = ctypes.c_longlong
     L.kvq_decode_attention_q.argtypes = [vp, vp, vp, vp, vp, vp, dp, I, I, I, vp, vp, I, ctypes.c_float, vp,
                                          ctypes.c_size_t, vp]
@@ -88,7 +89,8 @@ def _load() -> ctypes.CDLL:
     L.kvq_get_engine.restype = I
     for f in ("kvq_fp16_to_fp8", "kvq_fp8_to_fp16", "kvq_fp16_to_fp8_kv", "kvq_fp8_to_fp16_kv",
               "kvq_fp16_to_q_kv", "kvq_q_to_fp16_kv",
-              "kvq_poll_device_error", "kvq_selfcheck_code_rounding", "kvq_set_engine"):
+              "kvq_poll_device_error", "kvq_selfcheck_code_rounding", "kvq_selfcheck_wait_timeout",
+              "kvq_set_engine"):
         getattr(L, f).restype = I
     return L
 
@@ -269,6 +271,18 @@ def selfcheck_code_rounding(wbits: int, device=None) -> int:
     with torch.cuda.device(dev):
         st = _lib.kvq_selfcheck_code_rounding(int(wbits), out.data_ptr(), _stream(dev))
     _check(st, "selfcheck_code_rounding")
+    return int(out.item())
+
+
+def selfcheck_wait_timeout(device=None) -> int:
+    """Run the bulk engine's bounded wait against an mbarrier nothing arrives on (about
+    1 s).  Returns 1 when the wait gave up as designed; the device error word then holds
+    KVQ_DEV_TIMEOUT (read it with poll_device_error)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    out = torch.full((1,), -1, dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        st = _lib.kvq_selfcheck_wait_timeout(out.data_ptr(), _stream(dev))
+    _check(st, "selfcheck_wait_timeout")
     return int(out.item())
 
 

@@ -21,3 +21,24 @@ def oracle_mod():
 
     oracle.lib()  # builds oracle/libkvqref.so if it is missing or stale
     return oracle
+
+
+def build_library():
+    """Build libkvq.so when it is missing or stale, without importing the package first
+    (the package's __init__ loads the library); returns the imported package."""
+    import importlib.util
+
+    spec = importlib.util.spec_from_file_location(
+        "kvq_build", os.path.join(ROOT, "kv_cache_quantization_fp16_b200", "_build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+    import kv_cache_quantization_fp16_b200
+
+    return kv_cache_quantization_fp16_b200
+
+
+@pytest.fixture(scope="session")
+def kvq_built():
+    return build_library()
+

@@ -15,13 +15,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 @pytest.fixture(scope="module")
-def kvq():
-    from kv_cache_quantization_fp16_b200 import _build
-
-    _build.build()
-    import kv_cache_quantization_fp16_b200 as m
-
-    return m
+def kvq(kvq_built):
+    return kvq_built
 
 
 def _declared_functions():

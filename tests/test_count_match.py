@@ -46,11 +46,8 @@ def test_oracle_count_match_bruteforce(oracle_mod):
         assert oracle_mod.count_match(a, b, m) == brute(a.tolist(), b.tolist(), m)
 
 
-def test_library_count_match_matches_oracle(oracle_mod):
-    from kv_cache_quantization_fp16_b200 import _build
-
-    _build.build()
-    import kv_cache_quantization_fp16_b200 as kvq
+def test_library_count_match_matches_oracle(oracle_mod, kvq_built):
+    kvq = kvq_built
 
     for a, b, m in cases():
         ref = oracle_mod.count_match(a, b, m)

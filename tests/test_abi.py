@@ -101,6 +101,7 @@ def test_selfcheck_validation(kvq):
     L = kvq.library()
     assert L.kvq_selfcheck_code_rounding(4, None, None) == 1
     assert L.kvq_selfcheck_code_rounding(5, FAKE, None) == 3
+    assert L.kvq_selfcheck_wait_timeout(None, None) == 1
     assert L.kvq_poll_device_error(None, None) == 1
 
 

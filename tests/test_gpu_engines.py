@@ -176,3 +176,20 @@ def test_fp8_kv_bad_block_table(kvq, dev, eng):
     assert kvq.poll_device_error() == 0
     kvq.fp16_to_fp8_kv(kd, k8, vd, v8, 2, 0, 8, ps, lens, bt)
     assert kvq.poll_device_error() in (1, 2)
+
+
+def test_bounded_wait_gives_up_and_context_stays_usable(kvq, oracle_mod, dev):
+    """The bulk engine's bounded pipeline wait, run against an mbarrier that nothing
+    arrives on, gives up after its 1 s limit and records KVQ_DEV_TIMEOUT (no fault, no
+    hang); the bulk engine then still converts bit-exactly."""
+    import time
+
+    assert kvq.poll_device_error() == 0
+    t0 = time.perf_counter()
+    assert kvq.selfcheck_wait_timeout() == 1
+    assert time.perf_counter() - t0 >= 0.9
+    assert kvq.poll_device_error() == 3  # KVQ_DEV_TIMEOUT
+    assert kvq.poll_device_error() == 0  # read and cleared
+    with kvq.engine("bulk"):
+        k, v = workloads.channel_outliers(shape=(2, 512, 8, 128))
+        run_q(kvq, oracle_mod, k, v, 4, 2, 3, 500, dev)

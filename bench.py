@@ -1085,8 +1085,9 @@ def run_reference(args):
         "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16->u8->f16",
         "data": "synthetic (seeded, same recipe as the GPU arm)",
+        # the GPU arm's workload (its global batch at this N); each step times the sample above
         "config": {"workload": HEADLINE["workload"], "shape": list(HEADLINE["shape"]),
-                   "global_batch": 1, "offset": o, "width": w},
+                   "global_batch": HEADLINE["shape"][0] * max(1, args.gpus), "offset": o, "width": w},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

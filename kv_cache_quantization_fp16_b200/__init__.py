@@ -25,10 +25,11 @@ import os
 
 import torch
 
-__all__ = ["fp16_to_fp8", "fp8_to_fp16", "fp16_to_fp8_kv", "fp8_to_fp16_kv", "fp16_to_q_kv", "q_to_fp16_kv", "poll_device_error",
-           "selfcheck_code_rounding", "count_match", "decode_attention_q", "decode_attention_q_noalloc",
+__all__ = ["fp16_to_fp8", "fp8_to_fp16", "fp16_to_fp8_kv", "fp8_to_fp16_kv", "fp16_to_q_kv", "q_to_fp16_kv",
+           "poll_device_error", "decode_attention_q", "decode_attention_q_noalloc", "decode_attention_fp8",
+           "ATTENTION_SCRATCH_BYTES", "count_match", "selfcheck_code_rounding", "selfcheck_wait_timeout",
            "attention_workspace_bytes", "q_shapes", "set_engine", "get_engine", "engine", "KVQError",
-           "LIB_PATH", "library", "decode_attention_fp8"]
+           "LIB_PATH", "library"]
 
 ENGINES = {"auto": 0, "ldg": 1, "bulk": 2}
 
@@ -42,6 +43,28 @@ if not os.path.exists(LIB_PATH):
 class _Desc(ctypes.Structure):
     _fields_ = [("dim0", ctypes.c_int32), ("dim1", ctypes.c_int32), ("kv_heads", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("block_table_stride", ctypes.c_int32)]
+
+
+def _i32(x, name: str) -> int:
+    """An int argument of the C ABI, refused when it does not fit (ctypes would wrap it)."""
+    x = int(x)
+    if not -0x80000000 <= x <= 0x7FFFFFFF:
+        raise ValueError(f"{name} = {x} does not fit the library's int32 argument")
+    return x
+
+
+def _i32s(**args) -> tuple:
+    """_i32 of each keyword argument, in order."""
+    return tuple(_i32(v, k) for k, v in args.items())
+
+
+def _desc(d0, d1, H, D, stride) -> _Desc:
+    """The cache descriptor, after checking that every field fits its int32 (ctypes would
+    wrap a larger value silently into a different geometry)."""
+    for name, x in (("dim0", d0), ("dim1", d1), ("kv_heads", H), ("head_dim", D), ("block_table_stride", stride)):
+        if not 0 <= int(x) <= 0x7FFFFFFF:
+            raise ValueError(f"{name} = {int(x)} does not fit the library's int32 cache descriptor")
+    return _Desc(int(d0), int(d1), int(H), int(D), int(stride))
 
 
 _STATUS = {0: "ok", 1: "null pointer", 2: "bad shape", 3: "wbits must be 4, 6 or 8",
@@ -131,12 +154,13 @@ def q_shapes(shape, wbits: int):
 
 
 def _fp8(fn, in_tensor, out_tensor, batch_size, offset, width, in_dtype, out_dtype, where):
+    batch_size, offset, width = _i32s(batch_size=batch_size, offset=offset, width=width)
     _cuda4(in_tensor, in_dtype, "in_tensor")
     _cuda4(out_tensor, out_dtype, "out_tensor")
     _require(in_tensor.shape == out_tensor.shape, "in_tensor and out_tensor must have the same shape")
     _require(in_tensor.device == out_tensor.device, "tensors must be on one device")
     d0, d1, H, D = in_tensor.shape
-    desc = _Desc(d0, d1, H, D, 0)
+    desc = _desc(d0, d1, H, D, 0)
     with torch.cuda.device(in_tensor.device):
         st = fn(in_tensor.data_ptr(), out_tensor.data_ptr(), ctypes.byref(desc), int(batch_size),
                 int(offset), int(width), _stream(in_tensor.device))
@@ -175,6 +199,7 @@ def _paging(page_size, cache_seqlens, block_table, batch_size, dev):
 
 def _fp8_kv(fn, k_in, k_out, v_in, v_out, batch_size, offset, width, page_size, cache_seqlens, block_table,
             in_dtype, out_dtype, where):
+    batch_size, offset, width, page_size = _i32s(batch_size=batch_size, offset=offset, width=width, page_size=page_size)
     for t, n in ((k_in, "k_in"), (v_in, "v_in")):
         _cuda4(t, in_dtype, n)
     for t, n in ((k_out, "k_out"), (v_out, "v_out")):
@@ -185,7 +210,7 @@ def _fp8_kv(fn, k_in, k_out, v_in, v_out, batch_size, offset, width, page_size, 
         _require(t.device == dev, "tensors must be on one device")
     stride, sl_ptr, bt_ptr = _paging(page_size, cache_seqlens, block_table, batch_size, dev)
     d0, d1, H, D = k_in.shape
-    desc = _Desc(d0, d1, H, D, stride)
+    desc = _desc(d0, d1, H, D, stride)
     with torch.cuda.device(dev):
         st = fn(k_in.data_ptr(), k_out.data_ptr(), v_in.data_ptr(), v_out.data_ptr(), ctypes.byref(desc),
                 int(batch_size), int(offset), int(width), int(page_size), sl_ptr, bt_ptr, _stream(dev))
@@ -209,6 +234,8 @@ def fp8_to_fp16_kv(k_in, k_out, v_in, v_out, batch_size, offset, width, page_siz
 
 def _q(fn, fp16_is_input, k_in, k_out, k_scales, v_in, v_out, v_scales, batch_size, offset, width,
        page_size, cache_seqlens, block_table, wbits, where):
+    batch_size, offset, width, page_size, wbits = _i32s(
+        batch_size=batch_size, offset=offset, width=width, page_size=page_size, wbits=wbits)
     k16, kq = (k_in, k_out) if fp16_is_input else (k_out, k_in)
     v16, vq = (v_in, v_out) if fp16_is_input else (v_out, v_in)
     for t, n in ((k16, "FP16 K"), (v16, "FP16 V")):
@@ -230,7 +257,7 @@ def _q(fn, fp16_is_input, k_in, k_out, k_scales, v_in, v_out, v_scales, batch_si
         _require(t.device == dev, "tensors must be on one device")
     stride, sl_ptr, bt_ptr = _paging(page_size, cache_seqlens, block_table, batch_size, dev)
     d0, d1, H, D = k16.shape
-    desc = _Desc(d0, d1, H, D, stride)
+    desc = _desc(d0, d1, H, D, stride)
     with torch.cuda.device(dev):
         st = fn(k_in.data_ptr(), k_out.data_ptr(), k_scales.data_ptr(), v_in.data_ptr(), v_out.data_ptr(),
                 v_scales.data_ptr(), ctypes.byref(desc), int(batch_size), int(offset), int(width),
@@ -336,8 +363,9 @@ def attention_workspace_bytes(cache_shape, batch_size: int, n_heads: int, page_s
                               block_table_stride: int = 0) -> int:
     """Workspace bytes decode_attention_q needs: cache_shape is the FP16 cache shape
     [d0, d1, kv_heads, head_dim] the codes were made from."""
+    batch_size, n_heads, page_size = _i32s(batch_size=batch_size, n_heads=n_heads, page_size=page_size)
     d0, d1, H, D = cache_shape
-    desc = _Desc(d0, d1, H, D, block_table_stride if page_size else 0)
+    desc = _desc(d0, d1, H, D, block_table_stride if page_size else 0)
     return int(_lib.kvq_decode_attention_workspace_size(ctypes.byref(desc), int(batch_size), int(n_heads),
                                                         int(page_size)))
 
@@ -351,6 +379,7 @@ def decode_attention_q(q, k_codes, k_scales, v_codes, v_scales, out, batch_size,
     head_dim / 32] float16); cache_seqlens [batch] int32 (positions [0, len) are attended);
     paged mode with page_size > 0 and block_table.  ``workspace`` is a CUDA uint8 tensor of at
     least attention_workspace_bytes(...) bytes; when omitted one is allocated with torch."""
+    batch_size, page_size, wbits = _i32s(batch_size=batch_size, page_size=page_size, wbits=wbits)
     _require(isinstance(q, torch.Tensor) and q.dtype == torch.float16 and q.is_cuda and q.dim() == 3
              and q.is_contiguous(), "q must be a contiguous [batch, n_heads, head_dim] float16 CUDA tensor")
     _require(out.shape == q.shape and out.dtype == torch.float16 and out.is_contiguous() and out.device == q.device,
@@ -374,7 +403,7 @@ def decode_attention_q(q, k_codes, k_scales, v_codes, v_scales, out, batch_size,
              "cache_seqlens must be a contiguous int32 tensor on the caches' device with batch_size entries")
     stride, _, bt_ptr = _paging(page_size, cache_seqlens, block_table, batch_size, dev)
     d0, d1, H, _ = k_codes.shape
-    desc = _Desc(d0, d1, H, D, stride)
+    desc = _desc(d0, d1, H, D, stride)
     n_heads = q.shape[1]
     need = int(_lib.kvq_decode_attention_workspace_size(ctypes.byref(desc), int(batch_size), int(n_heads),
                                                         int(page_size)))
@@ -399,6 +428,7 @@ def decode_attention_fp8(q, k_fp8, v_fp8, out, batch_size, cache_seqlens, softma
     q, out: [batch, n_heads, head_dim] float16 CUDA tensors; k_fp8, v_fp8: [d0, d1, kv_heads,
     head_dim] uint8 as written by fp16_to_fp8 / fp16_to_fp8_kv; cache_seqlens, paging and
     ``workspace`` as for decode_attention_q."""
+    batch_size, page_size = _i32s(batch_size=batch_size, page_size=page_size)
     _require(isinstance(q, torch.Tensor) and q.dtype == torch.float16 and q.is_cuda and q.dim() == 3
              and q.is_contiguous(), "q must be a contiguous [batch, n_heads, head_dim] float16 CUDA tensor")
     _require(out.shape == q.shape and out.dtype == torch.float16 and out.is_contiguous() and out.device == q.device,
@@ -414,7 +444,7 @@ def decode_attention_fp8(q, k_fp8, v_fp8, out, batch_size, cache_seqlens, softma
              "cache_seqlens must be a contiguous int32 tensor on the caches' device with batch_size entries")
     stride, _, bt_ptr = _paging(page_size, cache_seqlens, block_table, batch_size, dev)
     d0, d1, H, _ = k_fp8.shape
-    desc = _Desc(d0, d1, H, D, stride)
+    desc = _desc(d0, d1, H, D, stride)
     n_heads = q.shape[1]
     need = int(_lib.kvq_decode_attention_workspace_size(ctypes.byref(desc), int(batch_size), int(n_heads),
                                                         int(page_size)))
@@ -441,6 +471,7 @@ def decode_attention_q_noalloc(q, k_codes, k_scales, v_codes, v_scales, out, bat
     allocated, by torch or by CUDA.  Geometries needing more workspace than
     ATTENTION_SCRATCH_BYTES are rejected.  Calls that overlap on the GPU share the array
     and race; make the first call on a device before any stream capture."""
+    batch_size, page_size, wbits = _i32s(batch_size=batch_size, page_size=page_size, wbits=wbits)
     _require(isinstance(q, torch.Tensor) and q.dtype == torch.float16 and q.is_cuda and q.dim() == 3
              and q.is_contiguous(), "q must be a contiguous [batch, n_heads, head_dim] float16 CUDA tensor")
     _require(out.shape == q.shape and out.dtype == torch.float16 and out.is_contiguous() and out.device == q.device,
@@ -464,7 +495,7 @@ def decode_attention_q_noalloc(q, k_codes, k_scales, v_codes, v_scales, out, bat
              "cache_seqlens must be a contiguous int32 tensor on the caches' device with batch_size entries")
     stride, _, bt_ptr = _paging(page_size, cache_seqlens, block_table, batch_size, dev)
     d0, d1, H, _ = k_codes.shape
-    desc = _Desc(d0, d1, H, D, stride)
+    desc = _desc(d0, d1, H, D, stride)
     n_heads = q.shape[1]
     need = int(_lib.kvq_decode_attention_workspace_size(ctypes.byref(desc), int(batch_size), int(n_heads),
                                                         int(page_size)))

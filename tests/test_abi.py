@@ -220,3 +220,20 @@ def test_decode_attention_noalloc_validation(kvq):
     assert L.kvq_decode_attention_q_noalloc(*P, None, 2, 4, 0, FAKE, None, 4, ctypes.c_float(1.0), None) == 1
     # beyond the scratch array: rejected on the host, nothing enqueued
     assert L.kvq_decode_attention_q_noalloc(*P, by(big), 64, 64, 0, FAKE, None, 4, ctypes.c_float(1.0), None) == 4
+
+
+def test_binding_rejects_dimensions_beyond_int32(kvq):
+    """A cache dimension the int32 descriptor cannot hold is refused by the binding
+    instead of wrapping into another geometry."""
+    with pytest.raises(ValueError, match="int32"):
+        kvq._desc(1, (1 << 32) + 5, 8, 128, 0)
+    with pytest.raises(ValueError, match="int32"):
+        kvq._desc(1, 16, 8, 128, -1)
+    d = kvq._desc(2, 16, 2, 64, 0)
+    assert (d.dim0, d.dim1, d.kv_heads, d.head_dim, d.block_table_stride) == (2, 16, 2, 64, 0)
+
+
+def test_binding_rejects_int_arguments_beyond_int32(kvq):
+    assert kvq._i32(-5, "offset") == -5
+    with pytest.raises(ValueError, match="width"):
+        kvq._i32(1 << 32, "width")

@@ -532,7 +532,8 @@ struct AttnWalk {
           c.chunk = static_cast<int>(t - static_cast<long long>(c.seq) * a.max_chunks);
         }
         const int L = length(c.seq);
-        const int p0 = c.chunk * T::kChunk;
+        // 64-bit: a slot's chunk can reach max_chunks (up to 2^31 - 1), far past any length
+        const long long p0 = static_cast<long long>(c.chunk) * T::kChunk;
         if (p0 < L) {
           c.item = item;
           set_sub(c, L, 0);

@@ -150,8 +150,9 @@ def test_gqa_groups(oracle_mod):
 
 
 @pytest.mark.parametrize("wbits", [4, 6, 8])
-def test_matches_numpy_softmax(oracle_mod, wbits):
-    B, S, H, D, NH = 2, 50, 2, 128, 4
+@pytest.mark.parametrize("D,NH", [(64, 2), (128, 4), (256, 16)])
+def test_matches_numpy_softmax(oracle_mod, wbits, D, NH):
+    B, S, H = 2, 50, 2
     k, v = _rand_cache(B, S, H, D, 6)
     kc, ks, vc, vs = _quantize(oracle_mod, k, v, wbits)
     ky, vy = _dequant(oracle_mod, kc, ks, vc, vs, wbits, D)
@@ -161,13 +162,16 @@ def test_matches_numpy_softmax(oracle_mod, wbits):
     lens = np.array([50, 17], np.int32)
     st, out, ex = oracle_mod.decode_attention_q(q, kc, ks, vc, vs, B, NH, 0, lens, None, wbits, 0.0883883, D)
     assert st == oracle_mod.OK
+    group = NH // H
     for i in range(B):
         for h in range(NH):
-            kk, vv = ky[i, : lens[i], h // 2], vy[i, : lens[i], h // 2]
+            kk, vv = ky[i, : lens[i], h // group], vy[i, : lens[i], h // group]
             sc = 0.0883883 * kk @ qf[i, h]
             w = np.exp(sc - sc.max())
             ref = (w / w.sum()) @ vv
             assert np.allclose(ex[i, h], ref, rtol=1e-12, atol=1e-14)
+    # the binary16 outputs are the exact results rounded to nearest even
+    assert np.array_equal(out, ex.astype(np.float16).view(np.uint16))
 
 
 def test_empty_window_and_bad_args(oracle_mod):

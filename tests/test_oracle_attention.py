@@ -247,8 +247,9 @@ def test_fp8_two_positions_closed_form(oracle_mod):
     assert np.all(out[0, 0] == np.float16(1.75).view(np.uint16))
 
 
-def test_fp8_paged_equals_contiguous_and_matches_numpy(oracle_mod):
-    B, S, H, D, NH, ps = 3, 64, 2, 64, 8, 16
+@pytest.mark.parametrize("D,NH", [(64, 8), (128, 2), (256, 16)])
+def test_fp8_paged_equals_contiguous_and_matches_numpy(oracle_mod, D, NH):
+    B, S, H, ps = 3, 64, 2, 16
     k8, v8 = _fp8_cache(B, S, H, D, 13)
     lens = np.array([64, 1, 40], np.int32)
     q16 = torch.randn(B, NH, D, generator=torch.Generator().manual_seed(206)).half()
@@ -267,11 +268,13 @@ def test_fp8_paged_equals_contiguous_and_matches_numpy(oracle_mod):
     assert st == oracle_mod.OK and np.array_equal(out_m, out_c)
     # numpy restatement: decode, softmax, weighted sum
     kk, vv, qf = _e5m2_numpy(k8), _e5m2_numpy(v8), q16.double().numpy()
+    group = NH // H
     for i in range(B):
         for h in range(NH):
-            sc = 0.125 * kk[i, : lens[i], h // 4] @ qf[i, h]
+            sc = 0.125 * kk[i, : lens[i], h // group] @ qf[i, h]
             w = np.exp(sc - sc.max())
-            assert np.allclose(ex_c[i, h], (w / w.sum()) @ vv[i, : lens[i], h // 4], rtol=1e-12, atol=1e-14)
+            assert np.allclose(ex_c[i, h], (w / w.sum()) @ vv[i, : lens[i], h // group], rtol=1e-12, atol=1e-14)
+    assert np.array_equal(out_c, ex_c.astype(np.float16).view(np.uint16))
 
 
 def test_fp8_bad_args(oracle_mod):

@@ -185,3 +185,29 @@ __global__ void __launch_bounds__(kBulkThreads, 1)
 }
 
 }  // namespace kvq
+
+// ---------------------------------------------------------------------------
+// Self-check of the bounded pipeline wait: one thread waits on an mbarrier
+// that expects one arrival that never comes; mbar_wait gives up after its
+// limit and records KVQ_DEV_TIMEOUT.
+// ---------------------------------------------------------------------------
+
+namespace kvq {
+
+__global__ void selfcheck_wait_timeout_kernel(int32_t* waited_out) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  *waited_out = mbar_wait(&bar, 0, nullptr) ? 0 : 1;
+}
+
+}  // namespace kvq
+
+extern "C" kvq_status kvq_selfcheck_wait_timeout(int32_t* waited_out, void* stream) {
+  if (!waited_out) return KVQ_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(waited_out, 0, sizeof(int32_t), s) != cudaSuccess) return KVQ_ERR_CUDA;
+  kvq::selfcheck_wait_timeout_kernel<<<1, 32, 0, s>>>(waited_out);
+  return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}

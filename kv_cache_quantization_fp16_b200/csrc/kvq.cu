@@ -70,20 +70,6 @@ __global__ void selfcheck_rounding_kernel(unsigned long long* mismatches) {
   if (bad) atomicAdd(mismatches, bad);
 }
 
-// ---------------------------------------------------------------------------
-// Self-check of the bounded pipeline wait: one thread waits on an mbarrier
-// that expects one arrival that never comes; mbar_wait gives up after its
-// limit and records KVQ_DEV_TIMEOUT.
-// ---------------------------------------------------------------------------
-
-__global__ void selfcheck_wait_timeout_kernel(int32_t* waited_out) {
-  __shared__ uint64_t bar;
-  if (threadIdx.x != 0) return;
-  mbar_init(&bar, 1);
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  *waited_out = mbar_wait(&bar, 0, nullptr) ? 0 : 1;
-}
-
 }  // namespace kvq
 
 // ===========================================================================
@@ -473,14 +459,6 @@ kvq_status kvq_set_engine(int engine) {
 }
 
 int kvq_get_engine(void) { return g_engine.load(); }
-
-kvq_status kvq_selfcheck_wait_timeout(int32_t* waited_out, void* stream) {
-  if (!waited_out) return KVQ_ERR_NULL;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(waited_out, 0, sizeof(int32_t), s) != cudaSuccess) return KVQ_ERR_CUDA;
-  kvq::selfcheck_wait_timeout_kernel<<<1, 32, 0, s>>>(waited_out);
-  return launch_status();
-}
 
 kvq_status kvq_selfcheck_code_rounding(int wbits, unsigned long long* mismatches, void* stream) {
   if (!mismatches) return KVQ_ERR_NULL;

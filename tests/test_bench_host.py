@@ -63,3 +63,33 @@ def test_max_over_ranks_gloo_two_ranks():
 
 def test_max_over_ranks_without_group():
     assert bench.max_over_ranks(2.25) == 2.25
+
+
+def test_algorithmic_bytes_per_element():
+    """The roofline numerators: FP16 in (2 B) plus the format's bytes out (or the reverse),
+    scales at 2 B per 32 elements."""
+    assert bench.BYTES_PER_ELEM["fp8"] == 3.0
+    assert bench.BYTES_PER_ELEM[4] == 2.5625 and bench.BYTES_PER_ELEM[6] == 2.8125
+    assert bench.BYTES_PER_ELEM[8] == 3.0625
+    B, S, H, D = bench.HEADLINE["shape"]
+    assert (B, S, H, D) == (4, 4096, 8, 128) and bench.HEADLINE["width"] == 2048
+    # one fused K+V encode launch of the headline window: 3 B x 2 x 4 x 2048 x 8 x 128
+    assert 3 * 2 * B * bench.HEADLINE["width"] * H * D == 50331648
+
+
+def test_attention_bytes():
+    # Q4, D = 128: per position and kv head 64 B of codes + 8 B of scales, for K and V;
+    # plus the queries read and the outputs written (2 B each)
+    assert bench.attention_bytes([10, 0], 8, 128, 4, 32) == 2 * 10 * 8 * 72 + 2 * 2 * 2 * 32 * 128
+    assert bench.attention_bytes([16384], 8, 128, 4, 32) == 18890752
+
+
+def test_recorded_traffic_follows_the_source_digest(tmp_path, monkeypatch):
+    f = tmp_path / "traffic.txt"
+    f.write_text(f"# comment\nfp16_to_fp8_kv 1234 {bench.kernel_source_digest()}\nother 5 0000000000000000\n")
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(f))
+    assert bench.recorded_traffic("fp16_to_fp8_kv") == 1234
+    assert bench.recorded_traffic("other") is None           # stale digest
+    assert bench.recorded_traffic("missing") is None
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "absent.txt"))
+    assert bench.recorded_traffic("fp16_to_fp8_kv") is None

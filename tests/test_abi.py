@@ -237,3 +237,36 @@ def test_binding_rejects_int_arguments_beyond_int32(kvq):
     assert kvq._i32(-5, "offset") == -5
     with pytest.raises(ValueError, match="width"):
         kvq._i32(1 << 32, "width")
+
+
+def test_header_is_plain_c_and_links(kvq, tmp_path):
+    """include/kvq.h compiles as C99 with warnings as errors, and a C program links against
+    libkvq.so and calls the host-only entry points (no device work)."""
+    import shutil
+    import subprocess
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_kvq.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "kvq.h"
+int main(void) {
+  const long long a[4] = {1, 2, 3, 4}, b[4] = {1, 2, 9, 4};
+  kvq_cache_desc d = {2, 16, 2, 64, 0};
+  if (kvq_count_match((const int64_t*)a, 4, (const int64_t*)b, 4, 4) != 2) return 1;
+  if (kvq_decode_attention_workspace_size(&d, 2, 4, 0) == 0) return 2;
+  if (strcmp(kvq_status_string(KVQ_OK), kvq_status_string(KVQ_ERR_NULL)) == 0) return 3;
+  if (kvq_fp16_to_fp8(NULL, NULL, &d, 1, 0, 1, NULL) != KVQ_ERR_NULL) return 4;
+  puts("ok");
+  return 0;
+}
+''')
+    exe = tmp_path / "use_kvq"
+    lib = os.path.dirname(kvq.LIB_PATH)
+    subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                    "-L", lib, "-lkvq", f"-Wl,-rpath,{lib}"], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", (out.returncode, out.stdout, out.stderr)

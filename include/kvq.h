@@ -235,8 +235,10 @@ KVQ_API size_t kvq_decode_attention_workspace_size(const kvq_cache_desc* desc, i
  *   (for example, batch 8 x 32 query heads x head_dim 128 with up to 8192
  *   positions needs 4.3 MB and fits; batch 16 with up to 16384 positions
  *   needs 17 MB and does not).
- *   The first call on each device, made with that device current, looks up
- *   the array's device address; make that first call before any stream
+ *   Every call looks up the device address of the current device's copy of
+ *   the array (a host-side query that enqueues nothing), so a reset and
+ *   re-created device context is picked up; the first call on a device may
+ *   also load the library's device code there, so make it before any stream
  *   capture.  KVQ_ERR_CUDA if the lookup fails.
  *   Every call on a device shares the one array and leaves its partial
  *   results there; nothing in it has to start at zero, because each call

@@ -217,24 +217,16 @@ static __device__ __align__(256) unsigned char g_attention_scratch[KVQ_ATTENTION
 
 namespace {
 
-constexpr int kScratchMaxDevices = 64;
-std::atomic<void*> g_attention_scratch_ptr[kScratchMaxDevices];
-
-// Device address of this device's copy of the array, looked up on the first
-// call made with the device current.  Null on failure.
+// Device address of the current device's copy of the array, or null on
+// failure.  Looked up on every call (a host-side query that enqueues nothing):
+// an address kept from an earlier call would dangle once the device's primary
+// context has been reset and re-created.
 void* attention_scratch() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kScratchMaxDevices) {
-    cudaGetLastError();
-    return nullptr;
-  }
-  void* ptr = g_attention_scratch_ptr[dev].load();
-  if (ptr) return ptr;
+  void* ptr = nullptr;
   if (cudaGetSymbolAddress(&ptr, g_attention_scratch) != cudaSuccess || !ptr) {
     cudaGetLastError();
     return nullptr;
   }
-  g_attention_scratch_ptr[dev].store(ptr);
   return ptr;
 }
 

@@ -222,6 +222,26 @@ def test_decode_attention_noalloc_validation(kvq):
     assert L.kvq_decode_attention_q_noalloc(*P, by(big), 64, 64, 0, FAKE, None, 4, ctypes.c_float(1.0), None) == 4
 
 
+def test_scratch_size_matches_the_header(kvq):
+    """The binding's pre-check uses the scratch size include/kvq.h defines: the two must
+    not drift apart (the binding would then reject valid calls, or pass calls the
+    library refuses)."""
+    text = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    m = re.search(r"#define\s+KVQ_ATTENTION_SCRATCH_BYTES\s+\(\(size_t\)(\d+)\s*<<\s*(\d+)\)", text)
+    assert m, "KVQ_ATTENTION_SCRATCH_BYTES not found in include/kvq.h"
+    assert kvq.ATTENTION_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
+    # and the library agrees at the boundary: the largest geometry that fits is accepted by
+    # the size check, one entry more is refused (host-side validation only)
+    L = kvq.library()
+    by = ctypes.byref
+    d = _desc(kvq, d0=1, d1=256, H=1, D=126)  # one 256-position chunk, 128 floats per entry
+    per_head = L.kvq_decode_attention_workspace_size(by(d), 1, 1, 0)
+    assert per_head == 128 * 4
+    heads_fit = kvq.ATTENTION_SCRATCH_BYTES // per_head
+    assert L.kvq_decode_attention_workspace_size(by(d), 1, heads_fit, 0) <= kvq.ATTENTION_SCRATCH_BYTES
+    assert L.kvq_decode_attention_workspace_size(by(d), 1, heads_fit + 1, 0) > kvq.ATTENTION_SCRATCH_BYTES
+
+
 def test_binding_rejects_dimensions_beyond_int32(kvq):
     """A cache dimension the int32 descriptor cannot hold is refused by the binding
     instead of wrapping into another geometry."""

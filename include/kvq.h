@@ -284,6 +284,21 @@ KVQ_API int kvq_get_engine(void);
  * pairs whose codes differ (0 expected).  Asynchronous on `stream`. */
 KVQ_API kvq_status kvq_selfcheck_code_rounding(int wbits, unsigned long long* mismatches, void* stream);
 
+/* Self-check (no counterpart on the page): measures, on the device, the
+ * arithmetic constants the decode-attention error bound is built from.
+ * `results` is a caller-owned device pointer to three doubles (8-byte
+ * aligned), zeroed and then filled with:
+ *   [0] the largest relative error of the hardware 2^x approximation the
+ *       softmax uses (ex2.approx.ftz.f32), over every binary32 x in [-126, 8];
+ *   [1] the largest relative error of exp2f over every binary32 x in
+ *       [-126, 0] (the chunk merge factors);
+ *   [2] the largest error of one mma.sync m16n8k16 step (binary16 products,
+ *       binary32 accumulator) over 310 M adversarial random accumulations,
+ *       in units of 2^-23 times the largest magnitude among the step's 16
+ *       products and its accumulator (the bound assumes at most 18).
+ * Asynchronous on `stream`; a few hundred milliseconds of device time. */
+KVQ_API kvq_status kvq_selfcheck_attention_numerics(double* results, void* stream);
+
 /* Self-check of the bulk engine's bounded waits (no counterpart on the page):
  * one CTA waits, with the same bounded wait the bulk engine's pipeline uses,
  * on a shared-memory mbarrier that nothing ever arrives on.  After the wait's

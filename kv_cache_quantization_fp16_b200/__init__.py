@@ -28,6 +28,7 @@ import torch
 __all__ = ["fp16_to_fp8", "fp8_to_fp16", "fp16_to_fp8_kv", "fp8_to_fp16_kv", "fp16_to_q_kv", "q_to_fp16_kv",
            "poll_device_error", "decode_attention_q", "decode_attention_q_noalloc", "decode_attention_fp8",
            "ATTENTION_SCRATCH_BYTES", "count_match", "selfcheck_code_rounding", "selfcheck_wait_timeout",
+           "selfcheck_attention_numerics",
            "attention_workspace_bytes", "q_shapes", "set_engine", "get_engine", "engine", "KVQError",
            "LIB_PATH", "library"]
 
@@ -93,6 +94,7 @@ def _load() -> ctypes.CDLL:
     L.kvq_poll_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), vp]
     L.kvq_selfcheck_code_rounding.argtypes = [I, vp, vp]
     L.kvq_selfcheck_wait_timeout.argtypes = [vp, vp]
+    L.kvq_selfcheck_attention_numerics.argtypes = [vp, vp]
     LL = ctypes.c_longlong
     L.kvq_decode_attention_q.argtypes = [vp, vp, vp, vp, vp, vp, dp, I, I, I, vp, vp, I, ctypes.c_float, vp,
                                          ctypes.c_size_t, vp]
@@ -113,7 +115,7 @@ def _load() -> ctypes.CDLL:
     for f in ("kvq_fp16_to_fp8", "kvq_fp8_to_fp16", "kvq_fp16_to_fp8_kv", "kvq_fp8_to_fp16_kv",
               "kvq_fp16_to_q_kv", "kvq_q_to_fp16_kv",
               "kvq_poll_device_error", "kvq_selfcheck_code_rounding", "kvq_selfcheck_wait_timeout",
-              "kvq_set_engine"):
+              "kvq_selfcheck_attention_numerics", "kvq_set_engine"):
         getattr(L, f).restype = I
     return L
 
@@ -299,6 +301,21 @@ def selfcheck_code_rounding(wbits: int, device=None) -> int:
         st = _lib.kvq_selfcheck_code_rounding(int(wbits), out.data_ptr(), _stream(dev))
     _check(st, "selfcheck_code_rounding")
     return int(out.item())
+
+
+def selfcheck_attention_numerics(device=None) -> dict:
+    """The arithmetic constants the decode-attention error bound rests on, measured on the
+    device: the largest relative error of the softmax's hardware 2^x approximation over
+    [-126, 8] (``ex2_rel``), of exp2f over [-126, 0] (``exp2f_rel``), and the largest
+    error of one mma.sync accumulation step in units of 2^-23 times its largest term
+    (``mma_step_ulps``)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    out = torch.zeros(3, dtype=torch.float64, device=dev)
+    with torch.cuda.device(dev):
+        st = _lib.kvq_selfcheck_attention_numerics(out.data_ptr(), _stream(dev))
+    _check(st, "selfcheck_attention_numerics")
+    r = out.cpu().tolist()
+    return {"ex2_rel": r[0], "exp2f_rel": r[1], "mma_step_ulps": r[2]}
 
 
 def selfcheck_wait_timeout(device=None) -> int:

@@ -476,5 +476,7 @@ kvq_status kvq_selfcheck_code_rounding(int wbits, unsigned long long* mismatches
 
 }  // extern "C"
 
-// Decode attention over the converted caches: host side.
+// Decode attention over the converted caches: host side, and the self-check of
+// the arithmetic its error bound rests on.
 #include "attention_api.cuh"
+#include "attention_selfcheck.cuh"

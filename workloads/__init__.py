@@ -80,6 +80,19 @@ def with_outliers_and_subnormals(x32: torch.Tensor, g, device, p_out=0.01, p_sub
     return torch.where(is_sub, sub, h)
 
 
+def channel_outlier_keys(shape, seed: int, lo: float, hi: float, device="cpu"):
+    """K ~ N(0, 1) FP16 with channel 0 of every (position, head) replaced by +-U(lo, hi)
+    (fair sign), so that query-key scores are dominated by one channel; V drawn by the
+    fp8_window recipe with the next seed."""
+    g = _gen(seed, device)
+    k = _randn(shape, g, device)
+    mag = lo + (hi - lo) * _rand(shape[:-1], g, device)
+    sign = torch.where(_rand(shape[:-1], g, device) < 0.5, -1.0, 1.0)
+    k[..., 0] = sign * mag
+    _, v = fp8_window(seed=seed + 1, shape=shape, device=device)
+    return k.half(), v
+
+
 def fp8_window(seed: int = SEED_BASE + 2, shape=(4, 4096, 8, 128), device="cpu"):
     g = _gen(seed, device)
     k = with_outliers_and_subnormals(_randn(shape, g, device), g, device)

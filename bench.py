@@ -1,40 +1,41 @@
 """Benchmark of the KV-cache format conversions on B200.
 
-Headline workload (one JSON line on rank 0): the contiguous FP8 partial-window
-workload -- K and V FP16 caches [4, 4096, 8, 128] (N(0,1) with 1% +-U(20,60000)
-outliers and 0.1% subnormals), window offset 1024, width 2048.  One step is
-fp16_to_fp8 of K and V, then fp8_to_fp16 of K and V, through the C ABI's fused
-K+V calls (one launch per direction) on resident device buffers; the same step
-through the single-tensor calls (4 launches) is reported in per_op.  The metric
-is algorithmic GB/s (bytes read + bytes written: 3 bytes per element per
-conversion).
+Headline workload (one JSON line on rank 0): the paged Q6 KV cache of a 32-layer
+model -- per layer, K and V pools of 1024 pages x 256 positions x 8 kv heads x 128
+(8 sequences x 32768 positions, shuffled block table; K N(0,1) times a per-channel
+lognormal scale, V N(0,1)), about 48 GB resident.  One step is the full-window
+q_to_fp16_kv of every layer, then fp16_to_q_kv of every layer, one fused K+V launch
+per layer and direction (64 launches).  The metric is algorithmic GB/s (bytes read
++ bytes written: 2 + 0.75 + 2/32 bytes per element per conversion).
 
-Timing.  `--steps` consecutive steps run back to back (replayed from CUDA
-graphs) between one pair of CUDA events.  The inputs are larger than L2: the
-step keeps 8 independent copies of the workload (about 1.3 GB) and step i
-converts copy i % 8, so every copy has been evicted by the other copies'
-traffic before it comes round again; L2 is flushed once before the timed
-steps.  The latency of one step on its own (L2 flushed before it, events
-around it) is reported beside it under `isolated`.
+Timing.  `--repeats` regions of exactly `--steps` consecutive steps, each between
+one pair of CUDA events with a barrier over the ranks and a device synchronize on
+both sides, the step replayed from a CUDA graph; the value is the median region
+(min and max beside it), the max over ranks of each.  The inputs (48 GB) are far
+larger than L2, so no flush is needed between steps.
 
 Extra keys:
-  roofline      the dominant kernel's achieved GB/s (algorithmic bytes per
-                launch / mean CUDA-event duration) against the measured HBM
-                copy peak in MEASURED_PEAKS.json;
-  cpu_baseline  the CPU oracle (single-threaded C++) timed on this host on the
-                same step;
-  e2e           the same metric through the public Python API with pinned host
-                buffers: host->device copy of the windows, the two conversions,
-                device->host copy of the decoded windows every step, all inside
-                the events; steps pipelined over three streams (upload,
-                convert, download) and two buffer sets;
-  per_op        every other conversion on its own workload (contiguous Q4/Q6,
-                paged Q4 decode / prefill, the model-sized paged Q6 layers), each
-                as GB/s and fraction of the HBM peak (--per-op, on by default).
+  roofline      the dominant direction's layer launch: algorithmic bytes per launch
+                / its CUDA-event duration (that direction's 32 launches alone,
+                `--steps` times between one pair of events), against the measured
+                HBM copy peak in MEASURED_PEAKS.json; `traffic` from the committed
+                ncu record (profiles/traffic.txt) while the kernels are unchanged;
+  cpu_baseline  the CPU oracle timed on this host on bounded samples of layer 0 of
+                the same step, on every core (single-threaded functions over
+                disjoint position ranges) and on one core, with the all-layer step
+                time those rates imply;
+  e2e           the same step through the public Python API from pinned host
+                memory: per layer, Q6 codes and scales host->device, both
+                conversions, codes and scales device->host, all inside the events;
+                three streams, layers pipelined;
+  per_op        every other conversion on its own workload (the FP8 partial-window
+                step, contiguous Q4/Q6/Q8 and FP8, paged Q4 and FP8 decode /
+                prefill, decode attention), each as GB/s and fraction of the HBM
+                peak (on by default; --no-per-op skips it).
 
-Multi-GPU (torchrun, one rank per GPU): every rank converts its own shard of
-sequences (weak scaling, no collective on the data path); the step time is the
-max over ranks.  ``--impl reference`` times the CPU oracle instead (rank 0 only).
+Multi-GPU (torchrun, one rank per GPU): every rank converts its own model's cache
+(weak scaling, no collective on the data path); each region's time is the max over
+ranks.  ``--impl reference`` times the CPU oracle instead (rank 0 only).
 """
 from __future__ import annotations
 
@@ -56,7 +57,10 @@ import torch  # noqa: E402
 
 import workloads  # noqa: E402
 
-HEADLINE = dict(workload="fp8_window_contiguous", shape=(4, 4096, 8, 128), offset=1024, width=2048)
+FP8_WINDOW = dict(workload="fp8_window_contiguous", shape=(4, 4096, 8, 128), offset=1024, width=2048)
+# the headline workload: one model's paged Q6 KV cache, every layer dequantized then quantized
+MODEL32 = dict(workload="paged_q6_model32", layers=32, seqs=8, seq_len=32768, kv_heads=8, head_dim=128,
+               page_size=256, wbits=6)
 FLUSH_BYTES = 256 << 20
 L2_BYTES = 126 << 20  # B200 L2 size
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -212,7 +216,7 @@ class Fp8Step:
     comes round again)."""
 
     def __init__(self, kvq, dev, batch, seed_shift=0, sets=STREAM_SETS):
-        B, S, H, D = HEADLINE["shape"]
+        B, S, H, D = FP8_WINDOW["shape"]
         shape = (batch, S, H, D)
         self.kvq, self.batch = kvq, batch
         self.sets = []
@@ -225,7 +229,7 @@ class Fp8Step:
         first = self.sets[0]
         self.set_bytes = sum(t.numel() * t.element_size() for t in first.values())
         self.k, self.v, self.k8, self.v8, self.ky, self.vy = (first[n] for n in ("k", "v", "k8", "v8", "ky", "vy"))
-        self.off, self.w = HEADLINE["offset"], HEADLINE["width"]
+        self.off, self.w = FP8_WINDOW["offset"], FP8_WINDOW["width"]
         self.elems_per_tensor = batch * self.w * H * D
         self.launch_bytes = BYTES_PER_ELEM["fp8"] * 2 * self.elems_per_tensor  # K and V
         self.bytes_per_step = 2 * self.launch_bytes
@@ -250,6 +254,179 @@ class Fp8Step:
         if ev is not None:
             ev.record()
         kvq.fp8_to_fp16_kv(t["k8"], t["ky"], t["v8"], t["vy"], b, o, w)
+
+
+class ModelStep:
+    """Headline step on one rank: the paged Q6 KV cache of a 32-layer model (per layer K and V
+    pools of 1024 pages x 256 positions x 8 kv heads x 128, 8 sequences x 32768 positions,
+    a shuffled block table), full-window q_to_fp16_kv of every layer, then fp16_to_q_kv of
+    every layer: one fused K+V launch per layer and direction, 64 launches per step.  About
+    48 GB stay resident on the device, far above the L2 size, so no step finds its inputs in
+    L2.  Rank r of a multi-GPU run holds layers seeded 32 r .. 32 r + 31 (its own model
+    replica's cache)."""
+
+    def __init__(self, kvq, dev, layer0=0):
+        m = MODEL32
+        self.kvq, self.wb, self.n = kvq, m["wbits"], m["seq_len"]
+        self.layers = []
+        for i in range(m["layers"]):
+            pool = workloads.model_layer(layer0 + i, seqs=m["seqs"], seq_len=m["seq_len"], page_size=m["page_size"],
+                                         heads=m["kv_heads"], head_dim=m["head_dim"], device=dev)
+            cs, ss = kvq.q_shapes(tuple(pool.k.shape), self.wb)
+            t = dict(pool=pool, kc=torch.empty(cs, dtype=torch.uint8, device=dev),
+                     vc=torch.empty(cs, dtype=torch.uint8, device=dev),
+                     ks=torch.empty(ss, dtype=torch.float16, device=dev),
+                     vs=torch.empty(ss, dtype=torch.float16, device=dev))
+            self.quantize(t)  # set-up, untimed: the Q6 cache the step starts from
+            self.layers.append(t)
+        torch.cuda.synchronize()
+        pool = self.layers[0]["pool"]
+        self.elems_per_launch = 2 * pool.k.numel()  # K and V
+        self.launch_bytes = BYTES_PER_ELEM[self.wb] * self.elems_per_launch
+        self.launches_per_step = 2 * len(self.layers)
+        self.bytes_per_step = self.launches_per_step * self.launch_bytes
+        self.names = ["q_to_fp16_kv/q6/model_layer", "fp16_to_q_kv/q6/model_layer"]
+
+    def _args(self, t):
+        p = t["pool"]
+        return (MODEL32["seqs"], -self.n, self.n, MODEL32["page_size"], p.cache_seqlens, p.block_table, self.wb)
+
+    def dequantize(self, t):
+        p = t["pool"]
+        self.kvq.q_to_fp16_kv(t["kc"], p.k, t["ks"], t["vc"], p.v, t["vs"], *self._args(t))
+
+    def quantize(self, t):
+        p = t["pool"]
+        self.kvq.fp16_to_q_kv(p.k, t["kc"], t["ks"], p.v, t["vc"], t["vs"], *self._args(t))
+
+    def half(self, j):
+        """Launches of direction j (0: dequantize every layer, 1: quantize every layer)."""
+        for t in self.layers:
+            (self.dequantize if j == 0 else self.quantize)(t)
+
+    def run(self, ev=None):
+        self.half(0)
+        if ev is not None:
+            ev.record()
+        self.half(1)
+
+
+def time_repeats(fn, steps, warmup, repeats, sampler=None, collective=True):
+    """`repeats` timed regions, each of exactly `steps` consecutive steps between one pair of
+    CUDA events (a barrier over the ranks and a device synchronize on both sides, the max
+    over ranks taken); fn is captured once as a CUDA graph of one step and replayed.
+    Returns the mean ms per step of every region."""
+    cur = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+    side.wait_stream(cur)
+    with torch.cuda.stream(side):
+        fn()  # first-call set-up precedes capture
+    cur.wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    _upload_graph(g)
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    out = []
+    if sampler:
+        sampler.mark()
+    for _ in range(repeats):
+        if collective:
+            _barrier()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(steps):
+            g.replay()
+        e.record()
+        torch.cuda.synchronize()
+        ms = s.elapsed_time(e) / steps
+        out.append(max_over_ranks(ms, torch.device("cuda", torch.cuda.current_device())) if collective else ms)
+    if collective:
+        _barrier()
+    if sampler:
+        sampler.mark()
+    del g
+    return out
+
+
+def model_shares(step, reps=3):
+    """ms of each direction inside a step: one event recorded between the two halves of a
+    captured step, read over `reps` replays (one event between two 7 ms halves costs
+    nothing measurable)."""
+    marks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        marks[0].record()
+        step.run(marks[1])
+        marks[2].record()
+    seg = [0.0, 0.0]
+    for _ in range(reps):
+        g.replay()
+        torch.cuda.synchronize()
+        seg[0] += marks[0].elapsed_time(marks[1])
+        seg[1] += marks[1].elapsed_time(marks[2])
+    del g
+    return [x / reps for x in seg]
+
+
+def e2e_model(kvq, step: ModelStep, steps, warmup):
+    """The headline step end to end through the public Python API from pinned host memory:
+    per layer, the host -> device copy of its Q6 codes and scales (K and V), the
+    dequantize and quantize launches, and the device -> host copy of the re-quantized
+    codes and scales.  Layers are pipelined as a serving loop would: uploads on one
+    stream, conversions on a second, downloads on a third, so layer i+1's upload and
+    layer i-1's download overlap layer i's conversions (PCIe is full duplex).  Two pinned
+    host buffer sets alternate (layer i reads set i % 2).  Returns (ms per step, host ->
+    device bytes per step, device -> host bytes per step)."""
+    names = ("kc", "ks", "vc", "vs")
+    host_in = [{n: step.layers[r][n].cpu().pin_memory() for n in names} for r in range(2)]
+    host_out = [{n: torch.empty_like(h[n]).pin_memory() for n in names} for h in host_in]
+    s_in, s_cv, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    L = len(step.layers)
+    ev_in = [torch.cuda.Event() for _ in range(L)]
+    ev_cv = [torch.cuda.Event() for _ in range(L)]
+    ev_out = [torch.cuda.Event() for _ in range(L)]
+    for e in ev_out:
+        e.record()
+
+    def once():
+        for i, t in enumerate(step.layers):
+            hi, ho = host_in[i % 2], host_out[i % 2]
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(ev_out[i])  # the previous download of this layer's codes is done
+                for n in names:
+                    t[n].copy_(hi[n], non_blocking=True)
+                ev_in[i].record(s_in)
+            with torch.cuda.stream(s_cv):
+                s_cv.wait_event(ev_in[i])
+                step.dequantize(t)
+                step.quantize(t)
+                ev_cv[i].record(s_cv)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_cv[i])
+                for n in names:
+                    ho[n].copy_(t[n], non_blocking=True)
+                ev_out[i].record(s_out)
+
+    for _ in range(warmup):
+        once()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(s_in)
+    for _ in range(steps):
+        once()
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(s_cv)
+    end.record(s_out)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / steps
+    per_layer = sum(host_in[0][n].numel() * host_in[0][n].element_size() for n in names)
+    return ms, L * per_layer, L * per_layer
 
 
 def capture(fn, n_marks=0):
@@ -390,97 +567,7 @@ def time_stream(launch, sets, steps, warmup, flush, sampler=None, collective=Tru
     return ms
 
 
-def stream_shares(step, sets, reps=20):
-    """Fraction of a stream step taken by each of its two launches: the same stream with an
-    event between every two launches (captured in the graph), averaged over `reps` replays.
-    Event nodes serialize the launches, so only the proportions are used."""
-    n = sets
-    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * n + 1)]
-    cur = torch.cuda.current_stream()
-    side = torch.cuda.Stream()
-    side.wait_stream(cur)
-    with torch.cuda.stream(side):
-        for i in range(n):
-            step.run(i)
-    cur.wait_stream(side)
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        for i in range(n):
-            evs[2 * i].record()
-            step.run(i, evs[2 * i + 1])
-        evs[2 * n].record()
-    seg = [0.0, 0.0]
-    for _ in range(reps):
-        g.replay()
-        torch.cuda.synchronize()
-        for i in range(n):
-            seg[0] += evs[2 * i].elapsed_time(evs[2 * i + 1])
-            seg[1] += evs[2 * i + 1].elapsed_time(evs[2 * i + 2])
-    del g
-    tot = seg[0] + seg[1]
-    return [x / tot for x in seg], [x / (reps * n) for x in seg]
-
-
-def e2e_fp8(kvq, step: Fp8Step, steps, warmup, dev):
-    """The headline step end to end through the public Python API, from pinned host
-    buffers: every step copies its K/V windows host -> device, runs the two fused
-    conversions and copies the decoded windows device -> host.  Steps are pipelined
-    the way a serving loop would run them: uploads on one stream, conversions on a
-    second, downloads on a third, two device buffer sets used alternately, so step
-    i+1's upload overlaps step i's download (PCIe is full duplex).  The timed region
-    runs from before the first upload to after the last download."""
-    B, S, H, D = step.k.shape
-    o, w = step.off, step.w
-    sets = step.sets[:2]
-    host_in = [(t["k"].cpu().pin_memory(), t["v"].cpu().pin_memory()) for t in sets]
-    host_out = [(torch.empty_like(hk).pin_memory(), torch.empty_like(hv).pin_memory()) for hk, hv in host_in]
-    s_in, s_cv, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    ev_in = [torch.cuda.Event() for _ in sets]
-    ev_cv = [torch.cuda.Event() for _ in sets]
-    ev_out = [torch.cuda.Event() for _ in sets]
-    for e in ev_cv + ev_out:
-        e.record()
-
-    def once(i):
-        r = i % 2
-        t, (hk, hv), (yk, yv) = sets[r], host_in[r], host_out[r]
-        with torch.cuda.stream(s_in):
-            s_in.wait_event(ev_cv[r])  # the conversions of step i-2 are done with this set's inputs
-            for b in range(B):
-                t["k"][b, o:o + w].copy_(hk[b, o:o + w], non_blocking=True)
-                t["v"][b, o:o + w].copy_(hv[b, o:o + w], non_blocking=True)
-            ev_in[r].record(s_in)
-        with torch.cuda.stream(s_cv):
-            s_cv.wait_event(ev_in[r])
-            s_cv.wait_event(ev_out[r])  # the download of step i-2 is done with this set's outputs
-            kvq.fp16_to_fp8_kv(t["k"], t["k8"], t["v"], t["v8"], B, o, w)
-            kvq.fp8_to_fp16_kv(t["k8"], t["ky"], t["v8"], t["vy"], B, o, w)
-            ev_cv[r].record(s_cv)
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(ev_cv[r])
-            for b in range(B):
-                yk[b, o:o + w].copy_(t["ky"][b, o:o + w], non_blocking=True)
-                yv[b, o:o + w].copy_(t["vy"][b, o:o + w], non_blocking=True)
-            ev_out[r].record(s_out)
-
-    for i in range(warmup):
-        once(i)
-    torch.cuda.synchronize()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(s_in)
-    for i in range(steps):
-        once(i)
-    s_out.wait_stream(s_in)
-    s_out.wait_stream(s_cv)
-    end.record(s_out)
-    torch.cuda.synchronize()
-    ms = start.elapsed_time(end) / steps
-    win_bytes = B * w * H * D * 2
-    return ms, 2 * win_bytes, 2 * win_bytes
-
-
-def per_op_measurements(kvq, dev, peak, steps, flush, step, include_model=True):
+def per_op_measurements(kvq, dev, peak, steps, flush):
     """Each remaining conversion on its own workload.  Throughput rows time `steps`
     consecutive launches (time_stream) on inputs larger than L2: workloads above the L2
     size as they are, smaller ones rotating through independent input copies.  Rows
@@ -504,9 +591,16 @@ def per_op_measurements(kvq, dev, peak, steps, flush, step, include_model=True):
                     "gbs": round(nbytes / ms / 1e6, 1), "frac": round(nbytes / ms / 1e6 / peak, 3),
                     "timing": timing})
 
-    # the headline step through the page's single-tensor calls (4 launches instead of 2)
-    B, S, H, D = HEADLINE["shape"]
-    o, w = HEADLINE["offset"], HEADLINE["width"]
+    # the FP8 partial-window step (K and V [4, 4096, 8, 128], window 1024..3072): encode then
+    # decode through the fused K+V calls, 2 launches, rotating through 8 input copies
+    step = Fp8Step(kvq, dev, FP8_WINDOW["shape"][0])
+    record("fp8_window_step", "contiguous K+V [4,4096,8,128], window 1024..3072, fp16_to_fp8_kv then "
+           "fp8_to_fp16_kv (2 fused launches)", step.bytes_per_step, step.run, sets=len(step.sets))
+    record("fp8_window_step/fp16_to_fp8_kv", "the same window, the encode launch alone", step.launch_bytes,
+           lambda i: step.launch(0, i), sets=len(step.sets))
+    # the same step through the page's single-tensor calls (4 launches instead of 2)
+    B, S, H, D = FP8_WINDOW["shape"]
+    o, w = FP8_WINDOW["offset"], FP8_WINDOW["width"]
 
     def per_tensor_step(i):
         t = step.sets[i % len(step.sets)]
@@ -514,7 +608,7 @@ def per_op_measurements(kvq, dev, peak, steps, flush, step, include_model=True):
         kvq.fp16_to_fp8(t["v"], t["v8"], B, o, w)
         kvq.fp8_to_fp16(t["k8"], t["ky"], B, o, w)
         kvq.fp8_to_fp16(t["v8"], t["vy"], B, o, w)
-    record("fp8_step_single_tensor_calls", "headline window, fp16_to_fp8(K), (V), fp8_to_fp16(K), (V): 4 launches",
+    record("fp8_step_single_tensor_calls", "FP8 window, fp16_to_fp8(K), (V), fp8_to_fp16(K), (V): 4 launches",
            4 * BYTES_PER_ELEM["fp8"] * B * w * H * D, per_tensor_step, sets=len(step.sets))
 
     # contiguous Q4 / Q6 / Q8, channel outliers [16, 8192, 8, 128] (537 MB of FP16 K+V)
@@ -609,11 +703,8 @@ def per_op_measurements(kvq, dev, peak, steps, flush, step, include_model=True):
            lambda i: fns[i % len(fns)](), sets=len(fns))
     del fns
     torch.cuda.empty_cache()
-    del pool
+    del pool, step
     torch.cuda.empty_cache()
-
-    if include_model:
-        out.extend(model_layers(kvq, dev, peak, min(20, max(3, steps // 10)), flush))
     return out
 
 
@@ -701,48 +792,9 @@ def attention_setup(kvq, dev, pool, wbits, n_heads=ATTN_QUERY_HEADS):
     return fn, attention_bytes(pool.cache_seqlens.cpu().tolist(), H, D, wbits, n_heads)
 
 
-def model_layers(kvq, dev, peak, steps, flush, layers=32):
-    """32 layers x K/V of 8 x 32768 x 8 x 128 FP16 in 256-position pages (~48 GB resident):
-    full-window q_to_fp16_kv over all layers, then fp16_to_q_kv over all layers."""
-    L = []
-    for i in range(layers):
-        pool = workloads.model_layer(i, device=dev)
-        cs, ss = kvq.q_shapes(tuple(pool.k.shape), 6)
-        kc = torch.empty(cs, dtype=torch.uint8, device=dev)
-        vc = torch.empty_like(kc)
-        ks = torch.empty(ss, dtype=torch.float16, device=dev)
-        vs = torch.empty_like(ks)
-        kvq.fp16_to_q_kv(pool.k, kc, ks, pool.v, vc, vs, 8, -32768, 32768, 256, pool.cache_seqlens,
-                         pool.block_table, 6)  # setup, untimed
-        L.append((pool, kc, vc, ks, vs))
-    torch.cuda.synchronize()
-    n = 2 * L[0][0].k.numel() * layers
-    nb = BYTES_PER_ELEM[6] * n
-
-    def deq():
-        for pool, kc, vc, ks, vs in L:
-            kvq.q_to_fp16_kv(kc, pool.k, ks, vc, pool.v, vs, 8, -32768, 32768, 256, pool.cache_seqlens,
-                             pool.block_table, 6)
-
-    def qnt():
-        for pool, kc, vc, ks, vs in L:
-            kvq.fp16_to_q_kv(pool.k, kc, ks, pool.v, vc, vs, 8, -32768, 32768, 256, pool.cache_seqlens,
-                             pool.block_table, 6)
-
-    res = []
-    cfg = "paged Q6, 32 layers x K/V 8x32768x8x128, page 256, shuffled block_table"
-    for name, fn in (("q_to_fp16_kv/q6/model32", deq), ("fp16_to_q_kv/q6/model32", qnt)):
-        ms = time_stream(lambda i: fn(), 1, steps, 3, flush, collective=False, chunk=1)
-        res.append({"op": name, "config": cfg, "bytes": int(nb), "us": round(ms * 1e3, 1),
-                    "gbs": round(nb / ms / 1e6, 1), "frac": round(nb / ms / 1e6 / peak, 3), "timing": "stream"})
-    del L
-    torch.cuda.empty_cache()
-    return res
-
-
 # ------------------------------------------------------ single-op cases ----
 
-CASES = ("headline_fp8enc_kv", "headline_fp8dec_kv", "headline_fp8enc", "headline_fp8dec", "fp8enc", "fp8dec", "q4enc",
+CASES = ("fp8_window_enc_kv", "fp8_window_dec_kv", "fp8_window_enc", "fp8_window_dec", "fp8enc", "fp8dec", "q4enc",
          "q4dec", "q6enc", "q6dec", "q8enc", "q8dec", "paged_prefill_q4enc", "paged_prefill_q4dec",
          "paged_decode_q4enc", "model_layer_q6enc", "model_layer_q6dec", "attn_paged_q4", "attn_paged_q6",
          "attn_paged_q8", "attn_paged_fp8", "attn_batch1_q4")
@@ -754,9 +806,9 @@ def run_case(kvq, dev, name, batch, steps, warmup, peak, stream=False):
     268 MB of FP16 K+V, above the L2 size); paged cases the 2048-page pool; model cases
     one 1024-page layer."""
     flush = L2Flush(dev)
-    if stream and name.startswith("headline") and name.endswith("_kv"):
-        # the fused headline launch alone, rotating through the step's 8 input copies
-        step = Fp8Step(kvq, dev, HEADLINE["shape"][0])
+    if stream and name.startswith("fp8_window") and name.endswith("_kv"):
+        # the fused FP8 window launch alone, rotating through the step's 8 input copies
+        step = Fp8Step(kvq, dev, FP8_WINDOW["shape"][0])
         j = 0 if "enc" in name else 1
         for i in range(len(step.sets)):
             step.run(i)  # valid E5M2 inputs for the decoder
@@ -764,9 +816,9 @@ def run_case(kvq, dev, name, batch, steps, warmup, peak, stream=False):
         nb = step.launch_bytes
         return {"case": name, "batch": batch, "bytes": int(nb), "us": round(ms * 1e3, 2), "gbs": round(nb / ms / 1e6, 1),
                 "frac": round(nb / ms / 1e6 / peak, 3), "timing": "stream, 8 rotating input copies"}
-    if name.startswith("headline") and name.endswith("_kv"):
-        B, S, H, D = HEADLINE["shape"]
-        o, w = HEADLINE["offset"], HEADLINE["width"]
+    if name.startswith("fp8_window") and name.endswith("_kv"):
+        B, S, H, D = FP8_WINDOW["shape"]
+        o, w = FP8_WINDOW["offset"], FP8_WINDOW["width"]
         k, v = workloads.fp8_window(shape=(B, S, H, D), device=dev)
         k8, v8 = torch.zeros(k.shape, dtype=torch.uint8, device=dev), torch.zeros(v.shape, dtype=torch.uint8, device=dev)
         ky, vy = torch.empty_like(k), torch.empty_like(v)
@@ -774,9 +826,9 @@ def run_case(kvq, dev, name, batch, steps, warmup, peak, stream=False):
         nb = 3.0 * 2 * B * w * H * D
         fn = (lambda: kvq.fp16_to_fp8_kv(k, k8, v, v8, B, o, w)) if "enc" in name else \
              (lambda: kvq.fp8_to_fp16_kv(k8, ky, v8, vy, B, o, w))
-    elif name.startswith("headline"):
-        B, S, H, D = HEADLINE["shape"]
-        o, w = HEADLINE["offset"], HEADLINE["width"]
+    elif name.startswith("fp8_window"):
+        B, S, H, D = FP8_WINDOW["shape"]
+        o, w = FP8_WINDOW["offset"], FP8_WINDOW["width"]
         k, _ = workloads.fp8_window(shape=(B, S, H, D), device=dev)
         k8 = torch.zeros(k.shape, dtype=torch.uint8, device=dev)
         y = torch.empty_like(k)
@@ -853,33 +905,103 @@ def run_case(kvq, dev, name, batch, steps, warmup, peak, stream=False):
 
 # -------------------------------------------------------------- CPU oracle ----
 
-def oracle_step_sample(batch=4, max_seconds=12.0, min_reps=1):
-    """Time the CPU oracle on the headline step (all four conversions of the full window),
-    repeating until about max_seconds.  Returns (GB/s, seconds per step, reps, description)."""
+def host_layer(layer_pool, kc, ks, vc, vs):
+    """Host copies of one model layer's Q6 cache (codes, scales, paging tables) and FP16
+    output pools for the oracle."""
     import numpy as np
+
+    def u16(t):
+        return t.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    h = dict(kc=kc.cpu().numpy(), vc=vc.cpu().numpy(), ks=u16(ks), vs=u16(vs),
+             lens=layer_pool.cache_seqlens.cpu().numpy().astype(np.int32),
+             bt=layer_pool.block_table.cpu().numpy().astype(np.int32), ps=layer_pool.page_size)
+    shape = tuple(layer_pool.k.shape)
+    h["ky"], h["vy"] = np.zeros(shape, np.uint16), np.zeros(shape, np.uint16)
+    return h
+
+
+def oracle_model_tasks(h, tasks, threads, wbits=6):
+    """The oracle's q_to_fp16_kv then fp16_to_q_kv (as written: single-threaded functions)
+    over the position ranges `tasks` = [(sequence, first, end)] of a host layer, `threads`
+    ranges at a time on disjoint positions (a harness split; ctypes releases the GIL).
+    Returns (seconds, positions)."""
+    from concurrent.futures import ThreadPoolExecutor
 
     import oracle
 
-    B, S, H, D = HEADLINE["shape"]
-    k, v = workloads.fp8_window(shape=(batch, S, H, D))
-    kn = k.view(torch.int16).numpy().view(np.uint16)
-    vn = v.view(torch.int16).numpy().view(np.uint16)
-    k8 = np.zeros(kn.shape, np.uint8)
-    v8 = np.zeros(vn.shape, np.uint8)
-    ky = np.zeros(kn.shape, np.uint16)
-    vy = np.zeros(vn.shape, np.uint16)
-    o, w = HEADLINE["offset"], HEADLINE["width"]
-    reps, t0 = 0, time.perf_counter()
-    while True:
-        oracle.fp16_to_fp8_kv(kn, k8, vn, v8, batch, o, w)
-        oracle.fp8_to_fp16_kv(k8, ky, v8, vy, batch, o, w)
-        reps += 1
-        if reps >= min_reps and time.perf_counter() - t0 >= max_seconds:
-            break
-    dt = (time.perf_counter() - t0) / reps
-    nbytes = 4 * BYTES_PER_ELEM["fp8"] * batch * w * H * D
-    desc = f"{reps} full step(s): FP8 encode+decode of K and V, batch {batch}, window {o}..{o + w}"
-    return nbytes / dt / 1e9, dt, reps, desc
+    def one(task):
+        i, a, b = task
+        L = int(h["lens"][i])
+        sl, bt = h["lens"][i:i + 1], h["bt"][i:i + 1]
+        assert oracle.q_to_fp16_kv(h["kc"], h["ky"], h["ks"], h["vc"], h["vy"], h["vs"], 1, a - L, b - a, h["ps"],
+                                   sl, bt, wbits) == oracle.OK
+        assert oracle.fp16_to_q_kv(h["ky"], h["kc"], h["ks"], h["vy"], h["vc"], h["vs"], 1, a - L, b - a, h["ps"],
+                                   sl, bt, wbits) == oracle.OK
+
+    t0 = time.perf_counter()
+    if threads == 1:
+        for task in tasks:
+            one(task)
+    else:
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(one, tasks))
+    return time.perf_counter() - t0, sum(b - a for _, a, b in tasks)
+
+
+def position_tasks(lens, npos, chunk):
+    """Ranges of at most `chunk` positions covering the first `npos` positions of the
+    layer, sequence by sequence."""
+    tasks, left = [], npos
+    for i, L in enumerate(lens):
+        for a in range(0, int(L), chunk):
+            if left <= 0:
+                return tasks
+            b = min(int(L), a + chunk, a + left)
+            tasks.append((i, a, b))
+            left -= b - a
+    return tasks
+
+
+def range_positions(npos, cores):
+    """Positions per task of the all-core oracle runs: about four tasks per core, from 64 to
+    512 positions, a multiple of 64."""
+    return max(64, min(512, npos // (4 * cores) // 64 * 64))
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_model_baseline(h, seconds=10.0):
+    """The CPU oracle on bounded samples of layer 0 of the headline step (dequantize then
+    quantize, K and V), on 1 core and on every core; GB/s in the headline's algorithmic
+    bytes, and the all-layer step time these rates imply (extrapolated)."""
+    bpp = 2 * 2 * MODEL32["kv_heads"] * MODEL32["head_dim"] * BYTES_PER_ELEM[MODEL32["wbits"]]  # bytes/position
+    total = int(sum(int(L) for L in h["lens"]))
+    dt, n = oracle_model_tasks(h, position_tasks(h["lens"], 64, 64), 1)  # calibration
+    per_pos = dt / n
+    n1 = max(64, min(total, int(seconds / per_pos) // 64 * 64))
+    t1, p1 = oracle_model_tasks(h, position_tasks(h["lens"], n1, 256), 1)
+    cores = host_cores()
+    nall = max(64, min(total, int(seconds * cores / per_pos) // 64 * 64))
+    tall, pall = oracle_model_tasks(h, position_tasks(h["lens"], nall, range_positions(nall, cores)), cores)
+    step_bytes = 2 * MODEL32["layers"] * 2 * MODEL32["seqs"] * MODEL32["seq_len"] * MODEL32["kv_heads"] * \
+        MODEL32["head_dim"] * BYTES_PER_ELEM[MODEL32["wbits"]]
+    g1, gall = bpp * p1 / t1 / 1e9, bpp * pall / tall / 1e9
+    return {"value": round(gall, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"layer 0 of the headline workload, its first {pall} (of {total}) sequence positions "
+                      f"in ranges of {range_positions(nall, cores)} over {cores} threads: q_to_fp16_kv then "
+                      f"fp16_to_q_kv of K and V (Q6), the oracle's single-threaded functions as written",
+            "seconds": round(tall, 2),
+            "single_core": {"value": round(g1, 4), "unit": "GB/s", "cores": 1, "seconds": round(t1, 2),
+                            "sample": f"layer 0, its first {p1} positions, one thread"},
+            "step_seconds_extrapolated": {"all_cores": round(step_bytes / (gall * 1e9), 1),
+                                          "single_core": round(step_bytes / (g1 * 1e9), 1),
+                                          "how": "the whole 32-layer step at the sampled rates (extrapolated)"}}
 
 
 # ------------------------------------------------------------------- main ----
@@ -887,23 +1009,26 @@ def oracle_step_sample(batch=4, max_seconds=12.0, min_reps=1):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--repeats", type=int, default=25,
+                    help="timed regions of --steps steps each; the value is their median")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-per-op", action="store_true", help="skip the per-op table")
-    ap.add_argument("--no-model", action="store_true", help="skip the 32-layer model-sized rows")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", choices=CASES, action="append",
                     help="time only these single conversions (for sweeps and ncu); no headline line")
     ap.add_argument("--case-batch", type=int, default=4)
     ap.add_argument("--stream", action="store_true",
                     help="with --case: time the launches back to back (one event pair) instead of one at a "
-                         "time with L2 flushed; the headline cases rotate through 8 input copies")
+                         "time with L2 flushed; the FP8 window cases rotate through 8 input copies")
     ap.add_argument("--engine", choices=["auto", "ldg", "bulk"], default="auto",
                     help="load engine of the conversion kernels (plain loads or TMA bulk copies)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.steps < 1 or args.repeats < 1:
+        ap.error("--steps and --repeats must be >= 1")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -921,8 +1046,7 @@ def main():
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     import kv_cache_quantization_fp16_b200 as kvq
 
     peak, peak_kind = hbm_peak()
@@ -932,44 +1056,37 @@ def main():
             print(json.dumps(run_case(kvq, dev, c, args.case_batch, args.steps, args.warmup, peak, args.stream)),
                   flush=True)
         return 0
-    flush = L2Flush(dev)
     sampler = ClockSampler(local_rank).start() if rank == 0 else None
 
-    # weak scaling: a global batch of 4 sequences per rank; rank r converts its shard of
-    # it (4 sequences), its inputs seeded by the shard's first global sequence index
-    global_batch = HEADLINE["shape"][0] * world
-    lo, hi = shard_range(global_batch, rank, world)
-    batch = hi - lo
-    step = Fp8Step(kvq, dev, batch, seed_shift=lo)
-    # timed region: `steps` consecutive steps over rotating input copies (inputs larger
-    # than L2), one pair of CUDA events around all of them, max over ranks
-    ms_local = time_stream(step.run, len(step.sets), args.steps, args.warmup, flush, sampler)
-    ms = max_over_ranks(ms_local, dev)
-    # per-launch durations inside the step: the step time split in the proportions of an
-    # event-marked pass; the dominant launch is then timed on its own, as a stream of
-    # `steps` launches of it over the same rotating input copies
-    share, seg_ms = stream_shares(step, len(step.sets))
-    names = step.names
-    launch_ms = [ms_local * f for f in share]
-    dom_i = 0 if launch_ms[0] >= launch_ms[1] else 1
-    dom_ms = time_stream(lambda i: step.launch(dom_i, i), len(step.sets), args.steps, args.warmup, flush,
-                         collective=False)
-    dom = (names[dom_i], dom_ms)
-    achieved = step.launch_bytes / dom[1] / 1e6
-    # one step on its own (L2 flushed before it, CUDA events around it): the latency of a
-    # single isolated call, launch and event overhead included
-    iso, iso_segs = time_device(lambda ev: step.run(0, ev[0] if ev else None), 200, 5, flush, None, n_marks=1,
-                                collective=False)
-    iso_ms = statistics.mean(iso)
-    iso_seg_ms = [statistics.mean(x[i] for x in iso_segs) for i in range(2)]
-
-    e2e_ms, h2d, d2h = e2e_fp8(kvq, step, max(10, args.steps // 10), 3, dev)
+    # weak scaling: every rank converts its own model replica's 32-layer cache (~48 GB)
+    step = ModelStep(kvq, dev, layer0=MODEL32["layers"] * rank)
+    # timed regions: `repeats` x (exactly `steps` consecutive steps between one pair of CUDA
+    # events, barrier + synchronize on both sides, max over ranks); the value is the median
+    reps = time_repeats(step.run, args.steps, args.warmup, args.repeats, sampler)
+    ms = statistics.median(reps)
+    # the two directions inside a step (one event between the halves), then the dominant one
+    # timed alone: `steps` x its 32 layer launches between one pair of events, 3 regions
+    seg_ms = model_shares(step)
+    dom_i = 0 if seg_ms[0] >= seg_ms[1] else 1
+    dom_reps = time_repeats(lambda: step.half(dom_i), args.steps, 3, 3, collective=False)
+    dom_launch_ms = statistics.median(dom_reps) / len(step.layers)
+    achieved = step.launch_bytes / dom_launch_ms / 1e6
+    # end to end: Q6 codes and scales up from pinned host memory, both conversions, codes and
+    # scales back down, every layer of every step
+    e2e_steps = max(2, min(args.steps, 5))
+    e2e_ms, h2d, d2h = e2e_model(kvq, step, e2e_steps, 1)
     e2e_ms = max_over_ranks(e2e_ms, dev)
+
+    host = None
+    if rank == 0 and not args.no_cpu_baseline:
+        t = step.layers[0]
+        host = host_layer(t["pool"], t["kc"], t["ks"], t["vc"], t["vs"])
+    del step
+    torch.cuda.empty_cache()
 
     per_op = []
     if world == 1 and not args.no_per_op:
-        per_op = per_op_measurements(kvq, dev, peak, min(200, max(20, args.steps // 5)), flush, step,
-                                     include_model=not args.no_model)
+        per_op = per_op_measurements(kvq, dev, peak, min(200, max(20, 10 * args.steps)), L2Flush(dev))
     if sampler:
         sampler.stop()
 
@@ -979,54 +1096,55 @@ def main():
     if rank != 0:
         return 0
 
-    cpu = None
-    if not args.no_cpu_baseline:
-        gbs, dt, reps, desc = oracle_step_sample()
-        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": desc, "seconds_per_step": round(dt, 3)}
-
-    total_bytes = world * step.bytes_per_step
-    value = total_bytes / ms / 1e6
+    cpu = oracle_model_baseline(host) if host is not None else None
+    bytes_per_step = 2 * MODEL32["layers"] * BYTES_PER_ELEM[MODEL32["wbits"]] * 2 * MODEL32["seqs"] * \
+        MODEL32["seq_len"] * MODEL32["kv_heads"] * MODEL32["head_dim"]
+    value = world * bytes_per_step / ms / 1e6
+    launches = 2 * MODEL32["layers"]
+    names = ["q_to_fp16_kv/q6/model_layer", "fp16_to_q_kv/q6/model_layer"]
     line = {
-        "metric": "KV-cache convert GB/s (read+write), FP8 E5M2 encode+decode of K and V",
+        "metric": "KV-cache convert GB/s (read+write), paged Q6 dequantize + quantize of every layer",
         "value": round(value, 1),
         "unit": "GB/s",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(ms, 5),
+        "ms_per_step": round(ms, 4),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f16->u8->f16",
-        "data": "synthetic (seeded N(0,1) with 1% outliers and 0.1% subnormals, drawn on device)",
-        "config": {"workload": HEADLINE["workload"], "shape": list(HEADLINE["shape"]),
-                   "global_batch": global_batch, "offset": HEADLINE["offset"], "width": HEADLINE["width"],
-                   "ops": ["fp16_to_fp8 of K and V (one fused launch)", "fp8_to_fp16 of K and V (one fused launch)"],
-                   "launch": f"{args.steps} consecutive steps (2 fused K+V launches each) replayed from CUDA graphs, "
-                             "one pair of CUDA events around them",
-                   "l2": f"inputs larger than L2: step i converts input copy i % {len(step.sets)} "
-                         f"({len(step.sets)} x {step.set_bytes / 1e6:.0f} MB), L2 flushed once before the timed steps",
-                   "parallelism": f"replicas x{world}, each rank its own 4 sequences"},
-        "roofline": {"bound": "hbm", "kernel": dom[0], "achieved": round(achieved, 1), "peak": peak,
+        "dtype": "f16<->u6 codes + f16 scales",
+        "data": "synthetic (seeded: K N(0,1) x per-channel lognormal scale, V N(0,1), shuffled block tables; "
+                "drawn on the device)",
+        "config": {"workload": MODEL32["workload"], "layers": MODEL32["layers"], "seqs": MODEL32["seqs"],
+                   "seq_len": MODEL32["seq_len"], "kv_heads": MODEL32["kv_heads"], "head_dim": MODEL32["head_dim"],
+                   "page_size": MODEL32["page_size"], "wbits": MODEL32["wbits"],
+                   "ops": ["q_to_fp16_kv of every layer (one fused K+V launch each)",
+                           "fp16_to_q_kv of every layer (one fused K+V launch each)"],
+                   "bytes_per_step": int(bytes_per_step),
+                   "launch": f"{args.steps} consecutive steps ({launches} launches each) replayed from a CUDA graph "
+                             f"of one step between one pair of CUDA events; {args.repeats} such regions, value = "
+                             "the median region",
+                   "repeats_ms_per_step": {"median": round(ms, 4), "min": round(min(reps), 4),
+                                           "max": round(max(reps), 4), "n": len(reps)},
+                   "l2": "inputs larger than L2: ~48 GB resident per rank, no flush needed",
+                   "parallelism": f"replicas x{world}, each rank its own model's 32-layer cache"},
+        "roofline": {"bound": "hbm", "kernel": names[dom_i], "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 3), "peak_kind": peak_kind,
-                     "bytes_per_launch": int(step.launch_bytes), "us_per_launch": round(dom[1] * 1e3, 2),
-                     "duration": f"CUDA events around {args.steps} back-to-back launches of this kernel alone, "
-                                 "rotating through the same input copies as the step",
-                     "us_per_launch_in_step": round(launch_ms[dom_i] * 1e3, 2),
-                     "in_step": "timed step time x this launch's share of an event-marked pass of the same stream",
-                     "traffic": recorded_traffic(dom[0])},
-        "per_kernel_us": {n: round(t * 1e3, 2) for n, t in zip(names, launch_ms)},
-        "per_kernel_us_marked": {n: round(t * 1e3, 2) for n, t in zip(names, seg_ms)},
-        "isolated": {"us_per_step": round(iso_ms * 1e3, 2),
-                     "per_kernel_us": {n: round(t * 1e3, 2) for n, t in zip(names, iso_seg_ms)},
-                     "gbs": round(step.bytes_per_step / iso_ms / 1e6, 1),
-                     "how": "one step at a time: L2 flushed, CUDA events around the step's graph and "
-                            "between its launches (includes ~6 us of event and launch overhead)"},
+                     "bytes_per_launch": int(step_launch_bytes()), "us_per_launch": round(dom_launch_ms * 1e3, 2),
+                     "duration": f"CUDA events around {args.steps} x its {MODEL32['layers']} layer launches, "
+                                 "the direction alone, median of 3 regions",
+                     "us_per_launch_in_step": round(seg_ms[dom_i] / MODEL32["layers"] * 1e3, 2),
+                     "in_step": "its half of a step, one event between the halves, / layers",
+                     "traffic": recorded_traffic(names[dom_i])},
+        "per_direction_ms_in_step": {n: round(t, 4) for n, t in zip(names, seg_ms)},
         "cpu_baseline": cpu,
-        "e2e": {"value": round(world * step.bytes_per_step / e2e_ms / 1e6, 2), "unit": "GB/s",
-                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": step.launches_per_step * args.steps,  # in the timed region
+        "e2e": {"value": round(world * bytes_per_step / e2e_ms / 1e6, 2), "unit": "GB/s",
+                "ms_per_step": round(e2e_ms, 3), "steps": e2e_steps, "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h),
+                "how": "per layer: Q6 codes + scales host->device, dequantize + quantize, codes + scales "
+                       "device->host; three streams, layers pipelined"},
+        "gpu_launches": launches * args.steps * args.repeats,  # in the timed regions
         "clocks": sampler.summary() if sampler else None,
         "per_op": per_op,
     }
@@ -1034,61 +1152,76 @@ def main():
     return 0
 
 
+def step_launch_bytes():
+    """Algorithmic bytes of one layer launch of the headline step (K and V, Q6)."""
+    return BYTES_PER_ELEM[MODEL32["wbits"]] * 2 * MODEL32["seqs"] * MODEL32["seq_len"] * MODEL32["kv_heads"] * \
+        MODEL32["head_dim"]
+
+
 REF_SECONDS = 60.0  # the reference arm's timed steps take about this long in all
 
 
 def run_reference(args):
-    """The CPU oracle as the reference arm: each step is a bounded sample of the headline
-    step, FP8 encode + decode of K and V over the first n positions of one sequence's
-    window, single-threaded, on this host; n (a multiple of 16, at most the window) is
-    chosen from a calibration step so that the `steps` timed steps take about
-    REF_SECONDS."""
+    """The CPU oracle as the reference arm, on the headline workload's metric: each step
+    dequantizes then re-quantizes (Q6, K and V) a bounded sample of one layer -- the first
+    n positions of a layer drawn by the headline recipe (one sequence, shuffled 256-position
+    pages) -- with the oracle's single-threaded functions run over disjoint position
+    ranges on every host core.  n (at most 16384) is chosen from a calibration step so that the
+    `warmup` + `steps` steps take about REF_SECONDS."""
     import numpy as np
 
     import oracle
 
-    B, S, H, D = HEADLINE["shape"]
-    o, w = HEADLINE["offset"], HEADLINE["width"]
-    k, v = workloads.fp8_window(shape=(1, S, H, D))
-    kn = k.view(torch.int16).numpy().view(np.uint16)
-    vn = v.view(torch.int16).numpy().view(np.uint16)
-    k8, v8 = np.zeros(kn.shape, np.uint8), np.zeros(vn.shape, np.uint8)
-    ky, vy = np.zeros(kn.shape, np.uint16), np.zeros(vn.shape, np.uint16)
+    n_max = 16384
+    pool = workloads.model_layer(0, seqs=1, seq_len=n_max, page_size=MODEL32["page_size"],
+                                 heads=MODEL32["kv_heads"], head_dim=MODEL32["head_dim"])
+    kb = pool.k.view(torch.int16).numpy().view(np.uint16)
+    vb = pool.v.view(torch.int16).numpy().view(np.uint16)
+    P, ps, H, D = kb.shape
+    wb = MODEL32["wbits"]
+    kc = np.zeros((P, ps, H, D * wb // 8), np.uint8)
+    vc = np.zeros_like(kc)
+    ks = np.zeros((P, ps, H, D // 32), np.uint16)
+    vs = np.zeros_like(ks)
+    lens = pool.cache_seqlens.numpy().astype(np.int32)
+    bt = pool.block_table.numpy().astype(np.int32)
+    cores = host_cores()
+    h = dict(kc=kc, vc=vc, ks=ks, vs=vs, lens=lens, bt=bt, ps=ps, ky=kb.copy(), vy=vb.copy())
+    # the Q6 cache the steps start from (set-up, untimed): quantize with the oracle
+    from concurrent.futures import ThreadPoolExecutor
 
-    def once_n(n):
-        oracle.fp16_to_fp8_kv(kn, k8, vn, v8, 1, o, n)
-        oracle.fp8_to_fp16_kv(k8, ky, v8, vy, 1, o, n)
-
-    t0 = time.perf_counter()
-    once_n(16)
-    per_pos = (time.perf_counter() - t0) / 16
-    n = int(REF_SECONDS / max(1, args.steps) / per_pos) // 16 * 16
-    n = max(16, min(w, n))
-
-    def once():
-        oracle.fp16_to_fp8_kv(kn, k8, vn, v8, 1, o, n)
-        oracle.fp8_to_fp16_kv(k8, ky, v8, vy, 1, o, n)
-
+    def setup(task):
+        i, a, b = task
+        assert oracle.fp16_to_q_kv(kb, kc, ks, vb, vc, vs, 1, a - n_max, b - a, ps, lens, bt, wb) == oracle.OK
+    with ThreadPoolExecutor(cores) as ex:
+        list(ex.map(setup, position_tasks(lens, n_max, 512)))
+    dt, n = oracle_model_tasks(h, position_tasks(lens, 512, 512), 1)  # calibration, one core
+    per_pos_all = dt / n / cores
+    total_steps = args.steps + args.warmup
+    npos = int(REF_SECONDS / total_steps / per_pos_all) // 512 * 512
+    npos = max(512, min(n_max, npos))
+    tasks = position_tasks(lens, npos, range_positions(npos, cores))
     for _ in range(args.warmup):
-        once()
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        once()
-    dt = (time.perf_counter() - t0) / args.steps
-    nbytes = 4 * BYTES_PER_ELEM["fp8"] * n * H * D
+        oracle_model_tasks(h, tasks, cores)
+    t = sum(oracle_model_tasks(h, tasks, cores)[0] for _ in range(args.steps))
+    dt = t / args.steps
+    nbytes = 2 * 2 * npos * H * D * BYTES_PER_ELEM[wb]
     value = nbytes / dt / 1e9
-    sample = f"per step: positions {o}..{o + n} of one of the 4 sequences (of the window {o}..{o + w}), K and V, encode + decode"
+    sample = (f"per step: positions 0..{npos} of one sequence of a layer drawn by the headline recipe, Q6 "
+              f"q_to_fp16_kv then fp16_to_q_kv of K and V, {range_positions(npos, cores)}-position ranges over "
+              f"{cores} threads")
     line = {
         "impl": "reference",
-        "metric": "KV-cache convert GB/s (read+write), FP8 E5M2 encode+decode of K and V",
+        "metric": "KV-cache convert GB/s (read+write), paged Q6 dequantize + quantize of every layer",
         "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f16->u8->f16",
-        "data": "synthetic (seeded, same recipe as the GPU arm)",
-        # the GPU arm's workload (its global batch at this N); each step times the sample above
-        "config": {"workload": HEADLINE["workload"], "shape": list(HEADLINE["shape"]),
-                   "global_batch": HEADLINE["shape"][0] * max(1, args.gpus), "offset": o, "width": w},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16<->u6 codes + f16 scales",
+        "data": "synthetic (seeded, the GPU arm's recipe)",
+        # the GPU arm's workload (its replicas at this N); each step times the sample above
+        "config": {"workload": MODEL32["workload"], "layers": MODEL32["layers"], "seqs": MODEL32["seqs"],
+                   "seq_len": MODEL32["seq_len"], "kv_heads": H, "head_dim": D, "page_size": ps, "wbits": wb,
+                   "replicas": max(1, args.gpus)},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }

@@ -71,10 +71,59 @@ def test_algorithmic_bytes_per_element():
     assert bench.BYTES_PER_ELEM["fp8"] == 3.0
     assert bench.BYTES_PER_ELEM[4] == 2.5625 and bench.BYTES_PER_ELEM[6] == 2.8125
     assert bench.BYTES_PER_ELEM[8] == 3.0625
-    B, S, H, D = bench.HEADLINE["shape"]
-    assert (B, S, H, D) == (4, 4096, 8, 128) and bench.HEADLINE["width"] == 2048
-    # one fused K+V encode launch of the headline window: 3 B x 2 x 4 x 2048 x 8 x 128
-    assert 3 * 2 * B * bench.HEADLINE["width"] * H * D == 50331648
+    m = bench.MODEL32
+    assert (m["layers"], m["seqs"], m["seq_len"], m["kv_heads"], m["head_dim"], m["wbits"]) == \
+        (32, 8, 32768, 8, 128, 6)
+    # one fused K+V launch of a model layer: 2.8125 B x 2 x 8 x 32768 x 8 x 128
+    assert bench.step_launch_bytes() == 1509949440
+    # the FP8 window per-op row: one fused K+V encode launch is 3 B x 2 x 4 x 2048 x 8 x 128
+    B, S, H, D = bench.FP8_WINDOW["shape"]
+    assert (B, S, H, D) == (4, 4096, 8, 128) and bench.FP8_WINDOW["width"] == 2048
+    assert 3 * 2 * B * bench.FP8_WINDOW["width"] * H * D == 50331648
+
+
+def test_position_tasks_cover_exactly_the_first_positions():
+    lens = [1000, 700, 5]
+    for n in (0, 1, 999, 1000, 1001, 1700, 1705, 5000):
+        tasks = bench.position_tasks(lens, n, 256)
+        covered = [(i, p) for i, a, b in tasks for p in range(a, b)]
+        want = [(i, p) for i, L in enumerate(lens) for p in range(L)][:n]
+        assert covered == want
+        assert all(0 < b - a <= 256 for _, a, b in tasks)
+
+
+def test_oracle_harness_split_gives_the_single_call_result(oracle_mod):
+    """The CPU baseline's split of a layer into position ranges over several threads computes
+    exactly what one oracle call over the whole window computes."""
+    import numpy as np
+    import torch
+
+    import workloads
+
+    pool = workloads.model_layer(0, seqs=2, seq_len=1024, page_size=256, heads=2, head_dim=64)
+    kb = pool.k.view(torch.int16).numpy().view(np.uint16)
+    vb = pool.v.view(torch.int16).numpy().view(np.uint16)
+    P, ps, H, D = kb.shape
+    lens = pool.cache_seqlens.numpy().astype(np.int32)
+    bt = pool.block_table.numpy().astype(np.int32)
+
+    def fresh():
+        kc = np.zeros((P, ps, H, D * 6 // 8), np.uint8)
+        ks = np.zeros((P, ps, H, D // 32), np.uint16)
+        assert oracle_mod.fp16_to_q_kv(kb, kc, ks, vb, kc.copy(), ks.copy(), 2, -1024, 1024, ps, lens, bt, 6) == 0
+        vc, vs = kc.copy(), ks.copy()
+        assert oracle_mod.fp16_to_q_kv(kb, kc, ks, vb, vc, vs, 2, -1024, 1024, ps, lens, bt, 6) == 0
+        return dict(kc=kc, vc=vc, ks=ks, vs=vs, lens=lens, bt=bt, ps=ps, ky=np.zeros_like(kb), vy=np.zeros_like(vb))
+
+    one, split = fresh(), fresh()
+    assert oracle_mod.q_to_fp16_kv(one["kc"], one["ky"], one["ks"], one["vc"], one["vy"], one["vs"], 2, -1024, 1024,
+                                   ps, lens, bt, 6) == 0
+    assert oracle_mod.fp16_to_q_kv(one["ky"], one["kc"], one["ks"], one["vy"], one["vc"], one["vs"], 2, -1024, 1024,
+                                   ps, lens, bt, 6) == 0
+    sec, n = bench.oracle_model_tasks(split, bench.position_tasks(lens, 2048, 100), 3)
+    assert n == 2048 and sec > 0
+    for name in ("kc", "vc", "ks", "vs", "ky", "vy"):
+        assert np.array_equal(one[name], split[name]), name
 
 
 def test_attention_bytes():

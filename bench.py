@@ -880,6 +880,24 @@ def run_case(kvq, dev, name, batch, steps, warmup, peak, stream=False):
         kvq.fp16_to_q_kv(pool.k, kc, ks, pool.v, vc, vs, *args)
         fn = (lambda: kvq.fp16_to_q_kv(pool.k, kc, ks, pool.v, vc, vs, *args)) if name.endswith("enc") else \
              (lambda: kvq.q_to_fp16_kv(kc, pool.k, ks, vc, pool.v, vs, *args))
+        if stream:
+            # the per-op table's stream: input copy r is the pool read through a block table whose
+            # pages are shifted by 256 r, so the windows of consecutive launches differ
+            sets = STREAM_SETS
+            bts = [torch.where(pool.block_table >= 0, (pool.block_table + (P // sets) * r) % P, pool.block_table)
+                   for r in range(sets)]
+            enc = name.endswith("enc")
+
+            def launch(i):
+                a = (32, off, w, ps, pool.cache_seqlens, bts[i % sets], 4)
+                if enc:
+                    kvq.fp16_to_q_kv(pool.k, kc, ks, pool.v, vc, vs, *a)
+                else:
+                    kvq.q_to_fp16_kv(kc, pool.k, ks, vc, pool.v, vs, *a)
+            ms = time_stream(launch, sets, steps, warmup, flush, collective=False)
+            return {"case": name, "batch": 32, "bytes": int(nb), "us": round(ms * 1e3, 2),
+                    "gbs": round(nb / ms / 1e6, 1), "frac": round(nb / ms / 1e6 / peak, 3),
+                    "timing": f"stream, {sets} rotating block tables", "engine": kvq.get_engine()}
     else:
         pool = workloads.model_layer(0, device=dev)
         cs, ss = kvq.q_shapes(tuple(pool.k.shape), 6)
@@ -1022,8 +1040,9 @@ def main():
     ap.add_argument("--stream", action="store_true",
                     help="with --case: time the launches back to back (one event pair) instead of one at a "
                          "time with L2 flushed; the FP8 window cases rotate through 8 input copies")
-    ap.add_argument("--engine", choices=["auto", "ldg", "bulk"], default="auto",
-                    help="load engine of the conversion kernels (plain loads or TMA bulk copies)")
+    ap.add_argument("--engine", choices=["auto", "ldg", "bulk", "ldg_tiled"], default="auto",
+                    help="load engine of the conversion kernels (plain loads, TMA bulk copies, or plain loads "
+                         "with per-sequence paged tiles)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -1053,8 +1072,9 @@ def main():
     kvq.set_engine(args.engine)
     if args.case:
         for c in args.case:
-            print(json.dumps(run_case(kvq, dev, c, args.case_batch, args.steps, args.warmup, peak, args.stream)),
-                  flush=True)
+            r = run_case(kvq, dev, c, args.case_batch, args.steps, args.warmup, peak, args.stream)
+            r.setdefault("engine", kvq.get_engine())
+            print(json.dumps(r), flush=True)
         return 0
     sampler = ClockSampler(local_rank).start() if rank == 0 else None
 

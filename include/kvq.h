@@ -98,14 +98,21 @@ enum {
   KVQ_DEV_TIMEOUT = 3         /* a bulk-engine pipeline wait ran past its limit (1 s) */
 };
 
-/* Load engines (kvq_set_engine).  Both give bit-identical results. */
+/* Load engines and work decompositions (kvq_set_engine).  All give
+ * bit-identical results. */
 enum {
   KVQ_ENGINE_AUTO = 0, /* per operation, the engine measured faster on B200 (default) */
-  KVQ_ENGINE_LDG = 1,  /* one tile per CTA, 16-byte global loads issued up front */
-  KVQ_ENGINE_BULK = 2  /* persistent CTAs, TMA bulk copies (cp.async.bulk, no multicast)
+  KVQ_ENGINE_LDG = 1,  /* 16-byte global loads issued up front; contiguous mode: one tile
+                          per CTA; paged mode: one wave of CTAs splitting the flattened
+                          windows of all sequences into equal position ranges (batches of
+                          up to 1024 sequences whose windows total under 2^31 positions;
+                          otherwise per-sequence tiles as in KVQ_ENGINE_LDG_TILED) */
+  KVQ_ENGINE_BULK = 2, /* persistent CTAs, TMA bulk copies (cp.async.bulk, no multicast)
                           into a 4-stage shared-memory ring, one producer warp and eight
                           consumer warps; used when one position of the input stream is a
                           multiple of 16 bytes, otherwise the LDG engine runs */
+  KVQ_ENGINE_LDG_TILED = 3 /* the LDG engine with per-sequence tiles in paged mode too
+                              (one tile of a sequence's window per CTA) */
 };
 
 /* The shape the torch tensor carried in the original extension. */
@@ -274,6 +281,23 @@ KVQ_API kvq_status kvq_set_engine(int engine);
 
 /* The engine currently selected (a KVQ_ENGINE_* value). */
 KVQ_API int kvq_get_engine(void);
+
+/* Decode-attention kernels (kvq_set_attention_path).  Both compute the same
+ * attention within the error bound stated at kvq_decode_attention_q. */
+enum {
+  KVQ_ATTENTION_AUTO = 0,    /* the kernel measured faster on B200: mma.sync (default) */
+  KVQ_ATTENTION_MMA = 1,     /* warp-level mma.sync tiles for every geometry */
+  KVQ_ATTENTION_TCGEN05 = 2  /* tcgen05.mma with tensor-memory accumulators for head_dim 128
+                                and batches of up to 256 sequences; other geometries run
+                                the mma.sync kernel */
+};
+
+/* Select the decode-attention kernel for all later calls in this process (any
+ * thread).  Returns KVQ_ERR_RANGE for an unknown value.  Host-only. */
+KVQ_API kvq_status kvq_set_attention_path(int path);
+
+/* The decode-attention kernel currently selected (a KVQ_ATTENTION_* value). */
+KVQ_API int kvq_get_attention_path(void);
 
 /* Self-check (no counterpart on the page): compares, on the device, the
  * kernels' fast code rounding (reciprocal, one FMA correction step, rounding

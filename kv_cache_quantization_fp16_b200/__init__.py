@@ -29,10 +29,12 @@ __all__ = ["fp16_to_fp8", "fp8_to_fp16", "fp16_to_fp8_kv", "fp8_to_fp16_kv", "fp
            "poll_device_error", "decode_attention_q", "decode_attention_q_noalloc", "decode_attention_fp8",
            "ATTENTION_SCRATCH_BYTES", "count_match", "selfcheck_code_rounding", "selfcheck_wait_timeout",
            "selfcheck_attention_numerics",
-           "attention_workspace_bytes", "q_shapes", "set_engine", "get_engine", "engine", "KVQError",
+           "attention_workspace_bytes", "q_shapes", "set_engine", "get_engine", "engine", "set_attention_path",
+           "get_attention_path", "attention_path", "ATTENTION_PATHS", "KVQError",
            "LIB_PATH", "library"]
 
-ENGINES = {"auto": 0, "ldg": 1, "bulk": 2}
+ENGINES = {"auto": 0, "ldg": 1, "bulk": 2, "ldg_tiled": 3}
+ATTENTION_PATHS = {"auto": 0, "mma": 1, "tcgen05": 2}
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkvq.so")
 
@@ -112,6 +114,10 @@ def _load() -> ctypes.CDLL:
     L.kvq_set_engine.argtypes = [I]
     L.kvq_get_engine.argtypes = []
     L.kvq_get_engine.restype = I
+    L.kvq_set_attention_path.argtypes = [I]
+    L.kvq_set_attention_path.restype = I
+    L.kvq_get_attention_path.argtypes = []
+    L.kvq_get_attention_path.restype = I
     for f in ("kvq_fp16_to_fp8", "kvq_fp8_to_fp16", "kvq_fp16_to_fp8_kv", "kvq_fp8_to_fp16_kv",
               "kvq_fp16_to_q_kv", "kvq_q_to_fp16_kv",
               "kvq_poll_device_error", "kvq_selfcheck_code_rounding", "kvq_selfcheck_wait_timeout",
@@ -332,8 +338,10 @@ def selfcheck_wait_timeout(device=None) -> int:
 
 def set_engine(name: str) -> None:
     """Select the load engine for all later conversions: "auto" (default: the engine
-    measured faster for each operation), "ldg" (plain 16-byte loads, one tile per CTA)
-    or "bulk" (TMA bulk copies into a shared-memory pipeline)."""
+    measured faster for each operation), "ldg" (plain 16-byte loads; contiguous: one tile
+    per CTA, paged: one wave of CTAs over equal shares of all windows), "bulk" (TMA bulk
+    copies into a shared-memory pipeline) or "ldg_tiled" (plain loads, per-sequence tiles
+    in paged mode too)."""
     _check(_lib.kvq_set_engine(ENGINES[name]), "set_engine")
 
 
@@ -355,6 +363,35 @@ class engine:
 
     def __exit__(self, *exc):
         set_engine(self.prev)
+        return False
+
+
+def set_attention_path(name: str) -> None:
+    """Select the decode-attention kernel for all later calls: "auto" (default), "mma"
+    (warp-level mma.sync tiles) or "tcgen05" (fifth-generation tensor cores with
+    tensor-memory accumulators, for head_dim 128 and batches of up to 256 sequences;
+    other geometries run the mma.sync kernel)."""
+    _check(_lib.kvq_set_attention_path(ATTENTION_PATHS[name]), "set_attention_path")
+
+
+def get_attention_path() -> str:
+    return {v: k for k, v in ATTENTION_PATHS.items()}[_lib.kvq_get_attention_path()]
+
+
+class attention_path:
+    """Context manager: ``with attention_path("mma"): ...`` selects a decode-attention
+    kernel temporarily."""
+
+    def __init__(self, name: str):
+        self.name = name
+
+    def __enter__(self):
+        self.prev = get_attention_path()
+        set_attention_path(self.name)
+        return self
+
+    def __exit__(self, *exc):
+        set_attention_path(self.prev)
         return False
 
 

@@ -6,8 +6,35 @@
 #pragma once
 
 #include "attention.cuh"
+#include "attention_tc.cuh"
 
 namespace {
+
+// Which decode-attention kernel runs (kvq_set_attention_path).
+std::atomic<int> g_attention_path{KVQ_ATTENTION_AUTO};
+
+// CTAs of the tcgen05 kernel the device holds at once (cached per device, after the
+// shared-memory opt-in), 0 on failure.
+template <int B>
+long long tc_ctas() {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<bool> opted[kMaxDevices];
+  static std::atomic<long long> resident[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return 0;
+  }
+  if (!opted[dev].load()) {
+    if (cudaFuncSetAttribute(kvq::attn_tc_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kvq::kTcSmemBytes) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    opted[dev].store(true);
+  }
+  return first_wave_ctas(kvq::attn_tc_kernel<B>, kvq::kTcThreads, kvq::kTcSmemBytes, resident, kMaxDevices);
+}
 
 // Chunks of `chunk` positions a sequence can have: the longest window the
 // cache geometry allows.
@@ -76,6 +103,18 @@ kvq_status launch_attention(kvq::AttnParams a, const kvq_cache_desc* desc, void*
   const long long items = static_cast<long long>(a.batch) * a.max_chunks * a.kv_heads;
   const bool compact = a.batch <= T::kSeqlenSlots && items <= 0x7FFFFFFFLL;
   kvq_status st;
+  const int path = g_attention_path.load(std::memory_order_relaxed);
+  if constexpr (D == kvq::kTcD) {
+    // the tcgen05 kernel: head_dim 128, batches its shared memory stages (<= 256 sequences)
+    if (path == KVQ_ATTENTION_TCGEN05 && compact) {
+      const long long ctas = tc_ctas<B>();
+      if (ctas < 1) return KVQ_ERR_CUDA;
+      st = launch_pdl(kvq::attn_tc_kernel<B>, dim3(static_cast<unsigned>(items < ctas ? items : ctas)),
+                      kvq::kTcThreads, kvq::kTcSmemBytes, stream, a);
+      if (st != KVQ_OK) return st;
+      return launch_pdl(kvq::attn_combine_kernel<D>, dim3(a.n_heads, a.batch), kvq::kCombineThreads, 0, stream, a);
+    }
+  }
   if (!compact) {
     st = launch_partial<B, D, false, false>(a, items, partial_ctas<B, D, false, false>(), stream);
   } else {

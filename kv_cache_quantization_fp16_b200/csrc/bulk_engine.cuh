@@ -102,9 +102,40 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
       : "memory");
 }
 
+// Before the grid dependency wait: an L2-only bulk prefetch of the input of
+// this CTA's first tile, so that its DRAM reads start while the previous grid
+// on the stream drains (every CTA of this persistent grid is in the first
+// wave).  The window and page metadata are read at L2 and only steer the hint
+// (the previous grid may still be writing them); the page is range checked,
+// so the prefetched range lies inside the cache.  Nothing is copied into
+// shared memory before the wait, and a prefetch never changes what a later
+// load returns.
+template <class Op>
+__device__ __forceinline__ void bulk_prefetch_first_tile(const Params& p, int tiles_x, long long total) {
+  const long long t = blockIdx.x;
+  if (t >= total) return;
+  const int x = static_cast<int>(t % tiles_x);
+  const long long rest = t / tiles_x;
+  const int seq = static_cast<int>(rest % p.g.batch);
+  const int kv = static_cast<int>(rest / p.g.batch);
+  long long row0 = 0;
+  int nrows = 0;
+  const bool ok = p.g.page_size == 0
+                      ? contiguous_tile(p.g, seq, x, row0, nrows)
+                      : paged_tile(p.g, seq, x, __ldcg(p.g.seqlens + seq), nullptr, false, row0, nrows, true);
+  if (!ok) return;
+  const long long in_off = row0 * p.g.hd * Op::kInNum / Op::kInDen;
+  const uint32_t bytes = static_cast<uint32_t>(nrows * p.g.hd * Op::kInNum / Op::kInDen);
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(static_cast<const uint8_t*>(p.in[kv]) + in_off),
+               "r"(bytes)
+               : "memory");
+}
+
 template <class Op>
 __global__ void __launch_bounds__(kBulkThreads, 1)
     bulk_kernel(const __grid_constant__ Params p, int tiles_x, int nkv) {
+  if (threadIdx.x == 0)
+    bulk_prefetch_first_tile<Op>(p, tiles_x, static_cast<long long>(tiles_x) * p.g.batch * nkv);
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ __align__(128) uint8_t stage_mem[];

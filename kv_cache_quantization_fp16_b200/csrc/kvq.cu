@@ -201,9 +201,33 @@ kvq_status launch_ldg_mode(Params p, int nkv, void* stream) {
   return launch_pdl(convert_kernel<Op, kPaged>, grid, LdgCfg<Op>::kThreads, 0, stream, p);
 }
 
+// Paged mode on the balanced grid: one wave of CTAs (never more than there are
+// positions to convert), each an equal share of the flattened windows.  Needs
+// the batch to fit the kernel's shared-memory staging and the windows' total
+// to fit an int (the caller checks).
 template <class Op>
-kvq_status launch_ldg(const Params& p, int nkv, void* stream) {
-  return p.g.page_size > 0 ? launch_ldg_mode<Op, true>(p, nkv, stream) : launch_ldg_mode<Op, false>(p, nkv, stream);
+kvq_status launch_balanced(Params p, int nkv, void* stream) {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<long long> wave[kMaxDevices];
+  const long long ctas = first_wave_ctas(convert_balanced_kernel<Op>, LdgCfg<Op>::kThreads, 0, wave, kMaxDevices);
+  if (ctas < 1) return KVQ_ERR_CUDA;
+  const long long most = static_cast<long long>(p.g.batch) * p.g.width * nkv;  // windows are at most `width` long
+  const unsigned grid = static_cast<unsigned>(most < ctas ? most : ctas);
+  return launch_pdl(convert_balanced_kernel<Op>, dim3(grid), LdgCfg<Op>::kThreads, 0, stream, p, nkv);
+}
+
+bool balanced_eligible(const Params& p) {
+  return p.g.page_size > 0 && p.g.batch <= kBalancedMaxBatch &&
+         static_cast<long long>(p.g.batch) * p.g.width < 0x7FFFFFFFLL;
+}
+
+template <class Op>
+kvq_status launch_ldg(const Params& p, int nkv, void* stream, bool tiled) {
+  if (p.g.page_size > 0) {
+    if (!tiled && balanced_eligible(p)) return launch_balanced<Op>(p, nkv, stream);
+    return launch_ldg_mode<Op, true>(p, nkv, stream);
+  }
+  return launch_ldg_mode<Op, false>(p, nkv, stream);
 }
 
 // The bulk engine needs every tile of the input stream 16-byte aligned and a
@@ -254,7 +278,7 @@ kvq_status launch(const Params& p, int nkv, void* stream) {
   int engine = g_engine.load(std::memory_order_relaxed);
   if (engine == KVQ_ENGINE_AUTO) engine = AutoEngine<Op>::pick(p);
   if (engine == KVQ_ENGINE_BULK && bulk_eligible<Op>(p)) return launch_bulk<Op>(p, nkv, stream);
-  return launch_ldg<Op>(p, nkv, stream);
+  return launch_ldg<Op>(p, nkv, stream, engine == KVQ_ENGINE_LDG_TILED);
 }
 
 Geometry make_geometry(const kvq_cache_desc* d, int batch, int offset, int width, int page_size,
@@ -440,6 +464,9 @@ kvq_status kvq_poll_device_error(int32_t* code_out, void* stream) {
 
 }  // extern "C"
 
+// Decode attention over the converted caches: host side.
+#include "attention_api.cuh"
+
 extern "C" {
 
 long long kvq_count_match(const int64_t* a, long long a_len, const int64_t* b, long long b_len, long long max_a) {
@@ -453,12 +480,22 @@ long long kvq_count_match(const int64_t* a, long long a_len, const int64_t* b, l
 }
 
 kvq_status kvq_set_engine(int engine) {
-  if (engine != KVQ_ENGINE_AUTO && engine != KVQ_ENGINE_LDG && engine != KVQ_ENGINE_BULK) return KVQ_ERR_RANGE;
+  if (engine != KVQ_ENGINE_AUTO && engine != KVQ_ENGINE_LDG && engine != KVQ_ENGINE_BULK &&
+      engine != KVQ_ENGINE_LDG_TILED)
+    return KVQ_ERR_RANGE;
   g_engine.store(engine);
   return KVQ_OK;
 }
 
 int kvq_get_engine(void) { return g_engine.load(); }
+
+kvq_status kvq_set_attention_path(int path) {
+  if (path != KVQ_ATTENTION_AUTO && path != KVQ_ATTENTION_MMA && path != KVQ_ATTENTION_TCGEN05) return KVQ_ERR_RANGE;
+  g_attention_path.store(path);
+  return KVQ_OK;
+}
+
+int kvq_get_attention_path(void) { return g_attention_path.load(); }
 
 kvq_status kvq_selfcheck_code_rounding(int wbits, unsigned long long* mismatches, void* stream) {
   if (!mismatches) return KVQ_ERR_NULL;
@@ -476,7 +513,5 @@ kvq_status kvq_selfcheck_code_rounding(int wbits, unsigned long long* mismatches
 
 }  // extern "C"
 
-// Decode attention over the converted caches: host side, and the self-check of
-// the arithmetic its error bound rests on.
-#include "attention_api.cuh"
+// The self-check of the arithmetic the decode-attention error bound rests on.
 #include "attention_selfcheck.cuh"

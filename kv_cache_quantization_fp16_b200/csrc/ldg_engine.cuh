@@ -1,6 +1,9 @@
-// ldg_engine.cuh -- the plain-load engine: one tile per CTA, every thread
-// issues its 16-byte (or 8/4-byte) global loads for the whole tile before it
-// computes.  Grid: x = tiles of a sequence's window, y = sequences, z = K / V.
+// ldg_engine.cuh -- the plain-load engine: every thread issues its 16-byte (or
+// 8/4-byte) global loads for a whole round before it computes.  Two grids:
+// convert_kernel, one tile per CTA (x = tiles of a sequence's window, y =
+// sequences, z = K / V); and, in paged mode, convert_balanced_kernel, one
+// wave of CTAs that split the flattened windows of all sequences (K, then V)
+// into equal ranges of positions.
 #pragma once
 
 #include "ops.cuh"
@@ -114,6 +117,179 @@ __global__ void __launch_bounds__(LdgCfg<Op>::kThreads, LdgCfg<Op>::kMinBlocksPe
       Op::template body<GlobalSrc, C::kThreads, C::kUnroll, kPaged && C::kPrefetchRounds>(p, kv, row0, nrows, in,
                                                                                           threadIdx.x);
     }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Balanced paged grid.  The windows of all sequences (clipped at 0, as
+// paged_tile does) are laid end to end, K's and then V's, and CTA c of G
+// takes positions [c T / G, (c + 1) T / G) of that sequence of T positions, so
+// every CTA moves the same bytes to within one position and one wave of CTAs
+// has no tail.  Each CTA finds the windows itself: the batch's lengths and
+// their running sums are staged in shared memory (no device->host sync); its
+// range is then walked in segments that stay inside one page of one sequence,
+// each converted by the operation's tile body.
+// ---------------------------------------------------------------------------
+
+constexpr int kBalancedMaxBatch = 1024;
+
+struct BalancedShared {
+  int pref[kBalancedMaxBatch + 1];  // pref[i] = positions in the windows of sequences < i
+  long long lo[kBalancedMaxBatch];  // first position of sequence i's window
+  int warp_sum[32];
+  int changed;
+};
+
+// Window of a paged sequence with length `seqlen`: first position and length.
+__device__ __forceinline__ void paged_window(const Geometry& g, int seqlen, long long& lo, int& len) {
+  const long long start = static_cast<long long>(seqlen) + g.offset;
+  lo = start < 0 ? 0 : start;
+  const long long h = start + g.width;
+  len = static_cast<int>(h > lo ? h - lo : 0);
+}
+
+// Stage the windows of the batch: every thread takes `per` consecutive
+// sequences, then a block-wide exclusive scan of the per-thread totals.  With
+// `l2_only`, lengths are read at L2 (a hint before the grid dependency wait).
+// The host guarantees batch <= kBalancedMaxBatch and batch * width < 2^31.
+template <int NT>
+__device__ __forceinline__ void stage_windows(const Geometry& g, BalancedShared& sh, bool l2_only) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int kWarps = NT / 32;
+  const int per = (g.batch + NT - 1) / NT;
+  int total = 0;
+  for (int k = 0; k < per; ++k) {
+    const int i = tid * per + k;
+    if (i < g.batch) {
+      const int L = l2_only ? __ldcg(g.seqlens + i) : g.seqlens[i];
+      long long lo;
+      int len;
+      paged_window(g, L, lo, len);
+      sh.lo[i] = lo;
+      sh.pref[i] = len;  // lengths for now, running sums below
+      total += len;
+    }
+  }
+  int incl = total;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) sh.warp_sum[warp] = incl;
+  __syncthreads();
+  int base = 0;
+  for (int w = 0; w < warp; ++w) base += sh.warp_sum[w];
+  int run = base + incl - total;  // exclusive prefix of this thread's first sequence
+  for (int k = 0; k < per; ++k) {
+    const int i = tid * per + k;
+    if (i < g.batch) {
+      const int len = sh.pref[i];
+      sh.pref[i] = run;
+      run += len;
+    }
+  }
+  if (tid == NT - 1) {
+    int all = 0;
+    for (int w = 0; w < kWarps; ++w) all += sh.warp_sum[w];
+    sh.pref[g.batch] = all;
+  }
+  __syncthreads();
+}
+
+// The segment of the flattened windows starting at position r (< end): which
+// K/V stream, physical first row and positions (within one page of one
+// sequence).  Returns false, after recording the error from thread `report`,
+// when the block table cannot place it (the segment is skipped).
+__device__ __forceinline__ bool balanced_segment(const Geometry& g, const BalancedShared& sh, long long r,
+                                                 long long end, int& kv, long long& row0, int& n, bool report,
+                                                 bool l2_only = false) {
+  const int total = sh.pref[g.batch];
+  kv = static_cast<int>(r / total);
+  const int rr = static_cast<int>(r - static_cast<long long>(kv) * total);
+  int lo = 0, hi = g.batch - 1;  // the last sequence whose running sum is <= rr
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (sh.pref[mid] <= rr) lo = mid;
+    else hi = mid - 1;
+  }
+  const int seq = lo;
+  const long long pos = sh.lo[seq] + (rr - sh.pref[seq]);
+  const long long lp = pos / g.page_size;
+  const long long in_page = pos - lp * g.page_size;
+  long long m = end - r;
+  m = min(m, static_cast<long long>(sh.pref[seq + 1] - rr));
+  m = min(m, static_cast<long long>(g.page_size) - in_page);
+  n = static_cast<int>(m);
+  if (lp >= g.bt_stride) {
+    if (report) record_error(KVQ_DEV_BAD_PAGE_INDEX);
+    return false;
+  }
+  const int32_t* entry = g.block_table + static_cast<long long>(seq) * g.bt_stride + lp;
+  const int page = l2_only ? __ldcg(entry) : *entry;
+  if (page < 0 || page >= g.dim0) {
+    if (report) record_error(KVQ_DEV_BAD_PAGE);
+    return false;
+  }
+  row0 = static_cast<long long>(page) * g.page_size + in_page;
+  return true;
+}
+
+template <class Op>
+__global__ void __launch_bounds__(LdgCfg<Op>::kThreads, LdgCfg<Op>::kMinBlocksPerSM)
+    convert_balanced_kernel(const __grid_constant__ Params p, int nkv) {
+  using C = LdgCfg<Op>;
+  __shared__ BalancedShared sh;
+  const int tid = threadIdx.x;
+  const long long G = gridDim.x, c = blockIdx.x;
+  // Before the grid dependency wait: the windows from lengths read at L2 (a hint:
+  // the previous grid may still be writing), and an L2 prefetch of the first
+  // round of this CTA's first segment, so that its DRAM reads start under the
+  // previous grid's tail.  A prefetch never changes what a later load returns.
+  stage_windows<C::kThreads>(p.g, sh, true);
+  {
+    const long long T = static_cast<long long>(sh.pref[p.g.batch]) * nkv;
+    const long long r0 = T * c / G, r1 = T * (c + 1) / G;
+    int kv, n;
+    long long row0;
+    if (r0 < r1 && balanced_segment(p.g, sh, r0, r1, kv, row0, n, false, true)) {
+      const long long elems = min(static_cast<long long>(n) * p.g.hd, static_cast<long long>(ldg_tile_elems<Op>()));
+      prefetch_l2_range(static_cast<const uint8_t*>(p.in[kv]) + row0 * p.g.hd * Op::kInNum / Op::kInDen,
+                        elems * Op::kInNum / Op::kInDen, tid, C::kThreads);
+      if (Op::kReadsScales)
+        prefetch_l2_range(static_cast<const __half*>(p.scales[kv]) + row0 * p.g.hd / kBlockElems,
+                          elems / kBlockElems * 2, tid, C::kThreads);
+    }
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // The lengths again, now that the previous grid's writes are visible; stage
+  // them anew only if one changed.
+  {
+    const int per = (p.g.batch + C::kThreads - 1) / C::kThreads;
+    int diff = 0;
+    for (int k = 0; k < per; ++k) {
+      const int i = tid * per + k;
+      if (i < p.g.batch) {
+        long long lo;
+        int len;
+        paged_window(p.g, p.g.seqlens[i], lo, len);
+        diff |= (lo != sh.lo[i]) || (len != sh.pref[i + 1] - sh.pref[i]);
+      }
+    }
+    if (__syncthreads_or(diff)) stage_windows<C::kThreads>(p.g, sh, false);
+  }
+  const long long T = static_cast<long long>(sh.pref[p.g.batch]) * nkv;
+  const long long r1 = T * (c + 1) / G;
+  for (long long r = T * c / G; r < r1;) {
+    int kv, n;
+    long long row0;
+    const bool ok = balanced_segment(p.g, sh, r, r1, kv, row0, n, tid == 0);
+    if (ok) {
+      const uint8_t* in = static_cast<const uint8_t*>(p.in[kv]) + row0 * p.g.hd * Op::kInNum / Op::kInDen;
+      Op::template body<GlobalSrc, C::kThreads, C::kUnroll, C::kPrefetchRounds>(p, kv, row0, n, in, tid);
+    }
+    r += n;
   }
 }
 

@@ -38,6 +38,14 @@ def dev(kvq):
     return torch.device("cuda:0")
 
 
+@pytest.fixture(autouse=True, params=["mma", "tcgen05"])
+def apath(request, kvq):
+    """Every attention test runs on both kernels: warp-level mma.sync tiles, and tcgen05
+    with tensor-memory accumulators (head_dim 128; other head sizes fall back to mma.sync)."""
+    with kvq.attention_path(request.param):
+        yield request.param
+
+
 def u16(t):
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
 
@@ -351,10 +359,12 @@ def test_fp8_stale_nan_bytes_do_not_leak(kvq, oracle_mod, dev):
 
 # ---- the arithmetic the bound rests on, and adversarial inputs for it -----------------------
 
-def test_attention_numerics_selfcheck(kvq):
+def test_attention_numerics_selfcheck(kvq, apath):
     """The constants of the derived bound hold on this device: the softmax's 2^x
     approximation and exp2f (exhaustively over the arguments the kernels use) and one
     tensor-core accumulation step (310 M adversarial random cases)."""
+    if apath != "mma":
+        pytest.skip("path-independent")
     r = kvq.selfcheck_attention_numerics()
     print("attention numerics:", r)
     assert 0 < r["ex2_rel"] <= attn_bound.EPS_EXP2

@@ -1,4 +1,5 @@
-"""Both load engines (plain loads and TMA bulk copies) against the CPU oracle, and
+"""The load engines (plain loads on the balanced paged grid, plain loads on per-sequence
+tiles, and TMA bulk copies) against the CPU oracle, and
 against each other, bit for bit: contiguous and paged windows, FP8 and Q4/Q6,
 ragged tails, shapes where the bulk engine is not applicable (it then runs the
 plain-load engine), and the empty-window no-op."""
@@ -28,7 +29,7 @@ def dev(kvq):
     return torch.device("cuda:0")
 
 
-@pytest.fixture(params=["ldg", "bulk"])
+@pytest.fixture(params=["ldg", "ldg_tiled", "bulk"])
 def eng(request, kvq):
     with kvq.engine(request.param):
         yield request.param
@@ -97,6 +98,62 @@ def test_engines_agree_at_scale(kvq, dev):
                              vy.view(torch.int16), f8, fy.view(torch.int16)))
         for a, b in zip(*outs):
             assert torch.equal(a, b)
+    assert kvq.poll_device_error() == 0
+
+
+def test_balanced_grid_edge_windows(kvq, oracle_mod, dev):
+    """The balanced paged grid on windows that are empty, one position long, end exactly
+    at page boundaries, or cross several pages, with more sequences than CTAs would take
+    one each, and a batch above its shared-memory staging (1100 sequences: the tiled grid
+    runs instead); bytes outside the windows stay untouched."""
+    for batch, max_len in ((40, 700), (1100, 60)):
+        g = torch.Generator().manual_seed(workloads.SEED_BASE + 300 + batch)
+        lens = torch.randint(0, max_len + 1, (batch,), generator=g, dtype=torch.int32)
+        lens[:6] = torch.tensor([0, 1, 15, 16, 17, max_len], dtype=torch.int32)
+        num_pages = batch * ((max_len + 1 + 15) // 16)
+        lens, bt = workloads.paged_tables(workloads.SEED_BASE + 301 + batch, batch, max_len, num_pages, 16, lens=lens)
+        k, v = workloads.normal_kv((num_pages, 16, 2, 64), workloads.SEED_BASE + 302 + batch)
+        for offset, width in ((-64, 64), (-33, 32), (0, 1), (-max_len, max_len)):
+            for wbits in (4, 6):
+                run_q(kvq, oracle_mod, k, v, wbits, batch, offset, width, dev, page_size=16, seqlens=lens, bt=bt)
+            run_fp8_kv(kvq, oracle_mod, k, v, batch, offset, width, dev, page_size=16, seqlens=lens, bt=bt)
+
+
+def test_balanced_and_tiled_agree_model_layer(kvq, dev):
+    """One model-sized paged layer (1024 pages x 256 x 8 x 128, shuffled block table), Q6
+    and Q4 both directions and FP8 both directions, on the balanced and the per-sequence
+    tiled grids: identical bytes."""
+    pool = workloads.model_layer(3, device=dev)
+    P, ps, H, D = pool.k.shape
+    args = (8, -32768, 32768, ps, pool.cache_seqlens, pool.block_table)
+    for wbits in (6, 4):
+        outs = []
+        for name in ("ldg", "ldg_tiled"):
+            with kvq.engine(name):
+                cs, ss = kvq.q_shapes(tuple(pool.k.shape), wbits)
+                kc, vc = torch.zeros(cs, dtype=torch.uint8, device=dev), torch.zeros(cs, dtype=torch.uint8, device=dev)
+                ks = torch.zeros(ss, dtype=torch.float16, device=dev)
+                vs = torch.zeros_like(ks)
+                kvq.fp16_to_q_kv(pool.k, kc, ks, pool.v, vc, vs, *args, wbits)
+                ky, vy = torch.zeros_like(pool.k), torch.zeros_like(pool.v)
+                kvq.q_to_fp16_kv(kc, ky, ks, vc, vy, vs, *args, wbits)
+                torch.cuda.synchronize()
+                outs.append((kc, vc, ks.view(torch.int16), vs.view(torch.int16), ky.view(torch.int16),
+                             vy.view(torch.int16)))
+        for a, b in zip(*outs):
+            assert torch.equal(a, b)
+        del outs
+    outs = []
+    for name in ("ldg", "ldg_tiled"):
+        with kvq.engine(name):
+            k8, v8 = (torch.zeros(pool.k.shape, dtype=torch.uint8, device=dev) for _ in range(2))
+            kvq.fp16_to_fp8_kv(pool.k, k8, pool.v, v8, *args)
+            ky, vy = torch.zeros_like(pool.k), torch.zeros_like(pool.v)
+            kvq.fp8_to_fp16_kv(k8, ky, v8, vy, *args)
+            torch.cuda.synchronize()
+            outs.append((k8, v8, ky.view(torch.int16), vy.view(torch.int16)))
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
     assert kvq.poll_device_error() == 0
 
 

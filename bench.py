@@ -1040,6 +1040,9 @@ def main():
     ap.add_argument("--stream", action="store_true",
                     help="with --case: time the launches back to back (one event pair) instead of one at a "
                          "time with L2 flushed; the FP8 window cases rotate through 8 input copies")
+    ap.add_argument("--attention-path", choices=["auto", "mma", "tcgen05"], default="auto",
+                    help="decode-attention kernel (warp-level mma.sync tiles or tcgen05 with tensor-memory "
+                         "accumulators)")
     ap.add_argument("--engine", choices=["auto", "ldg", "bulk", "ldg_tiled"], default="auto",
                     help="load engine of the conversion kernels (plain loads, TMA bulk copies, or plain loads "
                          "with per-sequence paged tiles)")
@@ -1070,10 +1073,13 @@ def main():
 
     peak, peak_kind = hbm_peak()
     kvq.set_engine(args.engine)
+    kvq.set_attention_path(args.attention_path)
     if args.case:
         for c in args.case:
             r = run_case(kvq, dev, c, args.case_batch, args.steps, args.warmup, peak, args.stream)
             r.setdefault("engine", kvq.get_engine())
+            if c.startswith("attn"):
+                r["attention_path"] = kvq.get_attention_path()
             print(json.dumps(r), flush=True)
         return 0
     sampler = ClockSampler(local_rank).start() if rank == 0 else None

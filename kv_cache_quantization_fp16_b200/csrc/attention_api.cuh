@@ -27,13 +27,13 @@ long long tc_ctas() {
   }
   if (!opted[dev].load()) {
     if (cudaFuncSetAttribute(kvq::attn_tc_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kvq::kTcSmemBytes) != cudaSuccess) {
+                             kvq::tc_smem_bytes<B>()) != cudaSuccess) {
       cudaGetLastError();
       return 0;
     }
     opted[dev].store(true);
   }
-  return first_wave_ctas(kvq::attn_tc_kernel<B>, kvq::kTcThreads, kvq::kTcSmemBytes, resident, kMaxDevices);
+  return first_wave_ctas(kvq::attn_tc_kernel<B>, kvq::kTcThreads, kvq::tc_smem_bytes<B>(), resident, kMaxDevices);
 }
 
 // Chunks of `chunk` positions a sequence can have: the longest window the
@@ -110,7 +110,7 @@ kvq_status launch_attention(kvq::AttnParams a, const kvq_cache_desc* desc, void*
       const long long ctas = tc_ctas<B>();
       if (ctas < 1) return KVQ_ERR_CUDA;
       st = launch_pdl(kvq::attn_tc_kernel<B>, dim3(static_cast<unsigned>(items < ctas ? items : ctas)),
-                      kvq::kTcThreads, kvq::kTcSmemBytes, stream, a);
+                      kvq::kTcThreads, kvq::tc_smem_bytes<B>(), stream, a);
       if (st != KVQ_OK) return st;
       return launch_pdl(kvq::attn_combine_kernel<D>, dim3(a.n_heads, a.batch), kvq::kCombineThreads, 0, stream, a);
     }

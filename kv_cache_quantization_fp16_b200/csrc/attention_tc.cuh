@@ -10,10 +10,12 @@
 // CTA: four math warps (one cache position per thread within a 128-position
 // tile, and one output row per thread) and one MMA warp whose elected lane
 // issues every tcgen05.mma.  Per tile:
-//   * each math thread loads its position's K and V codes and scales (issued
-//     one tile ahead, into registers), dequantizes the K row and stores it into
-//     tensor memory (tcgen05.st: lane = position, the A operand of S^T), and
-//     the V row into shared memory (the MN-major A operand of O^T);
+//   * each math thread copies its position's K and V codes and scales into a
+//     shared-memory stage with cp.async (the next tile's K as soon as this
+//     tile's K row is read, its V as soon as this tile's V row is read, so each
+//     copy has about a tile's time to land), dequantizes the K row and stores
+//     it into tensor memory (tcgen05.st: lane = position, the A operand of
+//     S^T), and the V row into shared memory (the MN-major A operand of O^T);
 //   * S^T [128 positions x 16] = K Q^T: eight kind::f16 MMAs (K = 16 each), A
 //     from tensor memory, B = the group's query rows in shared memory (rows
 //     >= group zero), accumulated in binary32 in tensor memory;
@@ -54,9 +56,12 @@ constexpr uint32_t kTcTmemCols = 128;         // K tile 64 columns, S^T 16, O^T 
 constexpr uint32_t kTcColK = 0, kTcColS = 64, kTcColO = 80;
 constexpr int kTcN = 16;                      // MMA N: query heads of the group, zero-padded
 
-// Shared memory of one CTA (dynamic).  The launch requests kTcSmemBytes, more
-// than the struct needs, so that at most four CTAs share an SM and their
-// tensor memory (4 x 128 columns) always fits the SM's 512 columns.
+// Shared memory of one CTA (dynamic): this struct, then the code stage of
+// TcFmt<B>::kStageChunks chunks of 128 x 16 bytes (chunk i of position p at
+// i * 2048 + p * 16: a thread's accesses are 16 bytes apart from its
+// neighbours', free of bank conflicts).  Every format needs more than 64 KB in
+// all, so at most three CTAs share an SM and their tensor memory (3 x 128
+// columns) fits the SM's 512.
 struct TcShared {
   uint8_t v[kTcD * kTcTile * 2];  // V^T operand: (d/8) * 2048 + p * 16 + (d%8) * 2
   uint8_t p_hi[kTcN * kTcTile * 2];  // P^T operand: (n/8) * 2048 + p * 16 + (n%8) * 2
@@ -71,8 +76,6 @@ struct TcShared {
   int items[257];                 // running item counts (compact enumeration), then the total
 };
 
-constexpr int kTcSmemBytes = 57 * 1024;
-static_assert(sizeof(TcShared) <= kTcSmemBytes, "shared memory layout");
 
 // Instruction descriptor of tcgen05.mma kind::f16: binary16 A and B, binary32
 // accumulator, M x N, A / B K-major (0) or MN-major (1).
@@ -154,6 +157,7 @@ struct TcFmt;
 template <>
 struct TcFmt<4> {
   static constexpr bool kPerm = true;
+  static constexpr bool kScaled = true;
   static constexpr int kRowBytes = kTcD / 2;
   __device__ static uint4 chunk(const uint32_t* w, int j, __half2 s2) {
     const uint32_t x = w[j], y = x >> 8;
@@ -169,6 +173,7 @@ struct TcFmt<4> {
 template <>
 struct TcFmt<6> {
   static constexpr bool kPerm = true;
+  static constexpr bool kScaled = true;
   static constexpr int kRowBytes = kTcD * 6 / 8;
   __device__ static uint4 chunk(const uint32_t* w, int j, __half2 s2) {
     const int g = j >> 1, h = j & 1;
@@ -182,6 +187,7 @@ struct TcFmt<6> {
 template <>
 struct TcFmt<8> {
   static constexpr bool kPerm = false;
+  static constexpr bool kScaled = true;
   static constexpr int kRowBytes = kTcD;
   __device__ static uint4 chunk(const uint32_t* w, int j, __half2 s2) {
     const uint32_t a = w[2 * j], b = w[2 * j + 1];
@@ -195,6 +201,7 @@ struct TcFmt<8> {
 template <>
 struct TcFmt<0> {  // E5M2 bytes: the high byte of the binary16 value
   static constexpr bool kPerm = false;
+  static constexpr bool kScaled = false;
   static constexpr int kRowBytes = kTcD;
   __device__ static uint4 chunk(const uint32_t* w, int j, __half2) {
     const uint32_t a = w[2 * j], b = w[2 * j + 1];
@@ -209,29 +216,48 @@ __host__ __device__ constexpr int tc_perm8(int i) {
   return kPerm ? (i >> 1) + 4 * (i & 1) : i;
 }
 
-// The codes of one position of one kv head: K and V rows and their scales.
+// The code stage: K row chunks, V row chunks, then one chunk with the K
+// scales (bytes 0..7) and the V scales (bytes 8..15).
 template <int B>
-struct TcRow {
-  static constexpr int kWords = TcFmt<B>::kRowBytes / 4;
-  uint32_t k[kWords], v[kWords];
-  uint2 ks, vs;  // four binary16 scales each (head_dim 128)
+struct TcStage {
+  static constexpr int kRowChunks = TcFmt<B>::kRowBytes / 16;
+  static constexpr int kK = 0, kV = kRowChunks, kS = 2 * kRowChunks;
+  static constexpr int kChunks = 2 * kRowChunks + (TcFmt<B>::kScaled ? 1 : 0);
+  static constexpr int kBytes = kChunks * kTcTile * 16;
 };
 
 template <int B>
-__device__ __forceinline__ void tc_load_row(const AttnParams& a, long long hr, TcRow<B>& r) {
-  constexpr int NV = TcRow<B>::kWords / 4;
-  const uint4* kp = reinterpret_cast<const uint4*>(a.k_codes + hr * TcFmt<B>::kRowBytes);
-  const uint4* vp = reinterpret_cast<const uint4*>(a.v_codes + hr * TcFmt<B>::kRowBytes);
+constexpr int tc_smem_bytes() {
+  return static_cast<int>((sizeof(TcShared) + 127) / 128 * 128) + TcStage<B>::kBytes;
+}
+
+// Copy position p's K row and K scales (or V row and V scales) of cache row hr
+// into the stage.
+template <int B, bool kValues>
+__device__ __forceinline__ void tc_stage_row(const AttnParams& a, long long hr, uint8_t* stage, int p) {
+  using S = TcStage<B>;
+  const uint8_t* src = (kValues ? a.v_codes : a.k_codes) + hr * TcFmt<B>::kRowBytes;
+  uint8_t* dst = stage + (kValues ? S::kV : S::kK) * (kTcTile * 16) + p * 16;
 #pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const uint4 x = __ldg(kp + i), y = __ldg(vp + i);
-    r.k[4 * i] = x.x, r.k[4 * i + 1] = x.y, r.k[4 * i + 2] = x.z, r.k[4 * i + 3] = x.w;
-    r.v[4 * i] = y.x, r.v[4 * i + 1] = y.y, r.v[4 * i + 2] = y.z, r.v[4 * i + 3] = y.w;
+  for (int i = 0; i < S::kRowChunks; ++i) cp_async16(dst + i * (kTcTile * 16), src + i * 16);
+  if constexpr (TcFmt<B>::kScaled)
+    cp_async_small<8>(stage + S::kS * (kTcTile * 16) + p * 16 + (kValues ? 8 : 0),
+                      (kValues ? a.v_scales : a.k_scales) + hr * (kTcD / 32));
+}
+
+// Position p's K (or V) row words and its four scales from the stage.
+template <int B, bool kValues>
+__device__ __forceinline__ void tc_read_row(const uint8_t* stage, int p, uint32_t (&w)[TcFmt<B>::kRowBytes / 4],
+                                            uint2& sc) {
+  using S = TcStage<B>;
+  const uint8_t* src = stage + (kValues ? S::kV : S::kK) * (kTcTile * 16) + p * 16;
+#pragma unroll
+  for (int i = 0; i < S::kRowChunks; ++i) {
+    const uint4 x = *reinterpret_cast<const uint4*>(src + i * (kTcTile * 16));
+    w[4 * i] = x.x, w[4 * i + 1] = x.y, w[4 * i + 2] = x.z, w[4 * i + 3] = x.w;
   }
-  if constexpr (B != 0) {
-    r.ks = __ldg(reinterpret_cast<const uint2*>(a.k_scales) + hr);
-    r.vs = __ldg(reinterpret_cast<const uint2*>(a.v_scales) + hr);
-  }
+  if constexpr (TcFmt<B>::kScaled)
+    sc = *reinterpret_cast<const uint2*>(stage + S::kS * (kTcTile * 16) + p * 16 + (kValues ? 8 : 0));
 }
 
 __device__ __forceinline__ __half2 tc_scale2(uint2 s, int blk) {
@@ -412,28 +438,62 @@ __global__ void __launch_bounds__(kTcThreads, 2) attn_tc_kernel(const __grid_con
     float m_ref[kAttnMaxGroup], l_part[kAttnMaxGroup], acc[kAttnMaxGroup], alpha_prev[kAttnMaxGroup];
 #pragma unroll
     for (int g = 0; g < kAttnMaxGroup; ++g) m_ref[g] = -INFINITY, l_part[g] = 0.0f, acc[g] = 0.0f, alpha_prev[g] = 1.0f;
+    // fold the previous tile's O^T row into the accumulators (after its MMAs completed)
+    auto fold_o = [&](bool ok) {
+      float o[16];
+      tc_ld16(tmem + lane_base + kTcColO, o);
+#pragma unroll
+      for (int g = 0; g < kAttnMaxGroup; ++g) acc[g] = acc[g] * alpha_prev[g] + (ok ? o[g] : 0.0f);
+    };
+    // the item's (max, sum, accumulator) per head into its workspace entry, then a fresh state
+    auto finish_item = [&](const TcTile& it) {
+#pragma unroll
+      for (int g = 0; g < kAttnMaxGroup; ++g) {
+        float x = l_part[g];
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o2);
+        if (lane == 0) sh.wsum[warp][g] = x;
+      }
+      asm volatile("bar.sync 3, %0;" ::"n"(kTcMathThreads) : "memory");
+      const long long head0 = static_cast<long long>(it.seq) * a.n_heads + static_cast<long long>(it.kvh) * G;
+      const long long stride = static_cast<long long>(a.max_chunks) * (kTcD + 2);
+      float* const entry = a.ws + (head0 * a.max_chunks + it.chunk) * (kTcD + 2);
+#pragma unroll
+      for (int g = 0; g < kAttnMaxGroup; ++g) {
+        if (g >= G) break;
+        entry[g * stride + 2 + d_out] = acc[g];
+        if (p == 0) {
+          entry[g * stride] = m_ref[g];
+          entry[g * stride + 1] = sh.wsum[0][g] + sh.wsum[1][g] + sh.wsum[2][g] + sh.wsum[3][g];
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < kAttnMaxGroup; ++g) m_ref[g] = -INFINITY, l_part[g] = 0.0f, acc[g] = 0.0f;
+    };
 
+    uint8_t* const stage = tc_smem_raw + (sizeof(TcShared) + 127) / 128 * 128;
     TcTile cur = walk.first(blockIdx.x);
-    TcRow<B> row_cur, row_nxt;
-    long long hr_cur = -1;
-    if (cur.item >= 0 && p < cur.n) {
-      hr_cur = tc_cache_row(a, cur.seq, cur.kvh, cur.p0 + p);
-      if (hr_cur >= 0) tc_load_row<B>(a, hr_cur, row_cur);
-    }
     TcTile prev;
     prev.item = -1;
+    long long hr_cur = -1;
+    if (cur.item >= 0 && p < cur.n) hr_cur = tc_cache_row(a, cur.seq, cur.kvh, cur.p0 + p);
+    if (hr_cur >= 0) tc_stage_row<B, false>(a, hr_cur, stage, p);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    if (hr_cur >= 0) tc_stage_row<B, true>(a, hr_cur, stage, p);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    // Copy groups of this thread, oldest first: ..., K(t), V(t), K(t+1), V(t+1).  At
+    // the start of tile t the two youngest are K(t), V(t) (or K(t), V(t) of the first
+    // tile): waiting for all but one lands K(t).
     for (; cur.item >= 0; ++tiles_done) {
       const uint32_t ph = tiles_done & 1u;
       const TcTile nxt = walk.next(cur);
       long long hr_nxt = -1;
-      if (nxt.item >= 0 && p < nxt.n) {
-        hr_nxt = tc_cache_row(a, nxt.seq, nxt.kvh, nxt.p0 + p);
-        if (hr_nxt >= 0) tc_load_row<B>(a, hr_nxt, row_nxt);
-      }
+      if (nxt.item >= 0 && p < nxt.n) hr_nxt = tc_cache_row(a, nxt.seq, nxt.kvh, nxt.p0 + p);
       const bool valid = hr_cur >= 0;
       // a new item: its query rows (perm8 order within each 8 elements), rows < group
       if (cur.t == 0) {
-        if (cur.chunk == 0 && cur.kvh == 0 && p == 0 && static_cast<long long>(sh.seqlen[cur.seq]) > walk.length(cur.seq))
+        if (cur.chunk == 0 && cur.kvh == 0 && p == 0 &&
+            static_cast<long long>(sh.seqlen[cur.seq]) > walk.length(cur.seq))
           record_error(KVQ_DEV_BAD_PAGE_INDEX);  // window longer than the cache
         const int g = p >> 4, j = p & 15;
         if (g < G) {
@@ -448,16 +508,25 @@ __global__ void __launch_bounds__(kTcThreads, 2) attn_tc_kernel(const __grid_con
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       }
       // K row -> tensor memory (the S MMAs of the previous tile are complete)
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+      {
+        uint32_t w[F::kRowBytes / 4];
+        uint2 sc = make_uint2(0, 0);
+        tc_read_row<B, false>(stage, p, w, sc);
 #pragma unroll
-      for (int blk = 0; blk < kTcD / 32; ++blk) {
-        const __half2 s2 = B != 0 ? tc_scale2(row_cur.ks, blk) : __half2();
-        uint32_t r[16];
+        for (int blk = 0; blk < kTcD / 32; ++blk) {
+          const __half2 s2 = F::kScaled ? tc_scale2(sc, blk) : __half2();
+          uint32_t r[16];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint4 u = F::chunk(row_cur.k, 4 * blk + c, s2);
-          r[4 * c] = u.x, r[4 * c + 1] = u.y, r[4 * c + 2] = u.z, r[4 * c + 3] = u.w;
+          for (int c = 0; c < 4; ++c) {
+            const uint4 u = F::chunk(w, 4 * blk + c, s2);
+            r[4 * c] = u.x, r[4 * c + 1] = u.y, r[4 * c + 2] = u.z, r[4 * c + 3] = u.w;
+          }
+          tc_st16(tmem + lane_base + kTcColK + 16 * blk, r);
         }
-        tc_st16(tmem + lane_base + kTcColK + 16 * blk, r);
+        // every word of the staged K row has been used: its slots take the next tile's K codes
+        if (hr_nxt >= 0) tc_stage_row<B, false>(a, hr_nxt, stage, p);
+        asm volatile("cp.async.commit_group;" ::: "memory");
       }
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
@@ -466,42 +535,23 @@ __global__ void __launch_bounds__(kTcThreads, 2) attn_tc_kernel(const __grid_con
       if (prev.item >= 0) {
         const bool ok = mbar_wait(&sh.bar_o, ph ^ 1u, &sh.abort);
         tc_fence_after();
-        float o[16];
-        tc_ld16(tmem + lane_base + kTcColO, o);
-#pragma unroll
-        for (int g = 0; g < kAttnMaxGroup; ++g) acc[g] = acc[g] * alpha_prev[g] + (ok ? o[g] : 0.0f);
-        if (prev.last) {
-          // the item's (max, sum, accumulator) per head
-#pragma unroll
-          for (int g = 0; g < kAttnMaxGroup; ++g) {
-            float x = l_part[g];
-#pragma unroll
-            for (int o2 = 16; o2 > 0; o2 >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o2);
-            if (lane == 0) sh.wsum[warp][g] = x;
-          }
-          asm volatile("bar.sync 3, %0;" ::"n"(kTcMathThreads) : "memory");
-          const long long head0 = static_cast<long long>(prev.seq) * a.n_heads + static_cast<long long>(prev.kvh) * G;
-          const long long stride = static_cast<long long>(a.max_chunks) * (kTcD + 2);
-          float* const entry = a.ws + (head0 * a.max_chunks + prev.chunk) * (kTcD + 2);
-#pragma unroll
-          for (int g = 0; g < kAttnMaxGroup; ++g) {
-            if (g >= G) break;
-            entry[g * stride + 2 + d_out] = acc[g];
-            if (p == 0) {
-              entry[g * stride] = m_ref[g];
-              entry[g * stride + 1] = sh.wsum[0][g] + sh.wsum[1][g] + sh.wsum[2][g] + sh.wsum[3][g];
-            }
-          }
-#pragma unroll
-          for (int g = 0; g < kAttnMaxGroup; ++g) m_ref[g] = -INFINITY, l_part[g] = 0.0f, acc[g] = 0.0f;
-        }
+        fold_o(ok);
+        if (prev.last) finish_item(prev);
       }
       // V row -> shared memory (the O^T MMAs of the previous tile are complete)
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+      {
+        uint32_t w[F::kRowBytes / 4];
+        uint2 sc = make_uint2(0, 0);
+        tc_read_row<B, true>(stage, p, w, sc);
 #pragma unroll
-      for (int j = 0; j < kTcD / 8; ++j) {
-        const __half2 s2 = B != 0 ? tc_scale2(row_cur.vs, j >> 2) : __half2();
-        const uint4 u = valid ? F::chunk(row_cur.v, j, s2) : make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(sh.v + j * 2048 + p * 16) = u;
+        for (int j = 0; j < kTcD / 8; ++j) {
+          const __half2 s2 = F::kScaled ? tc_scale2(sc, j >> 2) : __half2();
+          const uint4 u = valid ? F::chunk(w, j, s2) : make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(sh.v + j * 2048 + p * 16) = u;
+        }
+        if (hr_nxt >= 0) tc_stage_row<B, true>(a, hr_nxt, stage, p);
+        asm volatile("cp.async.commit_group;" ::: "memory");
       }
       // scores of this tile
       const bool ok_s = mbar_wait(&sh.bar_s, ph, &sh.abort);
@@ -545,36 +595,14 @@ __global__ void __launch_bounds__(kTcThreads, 2) attn_tc_kernel(const __grid_con
       prev = cur;
       cur = nxt;
       hr_cur = hr_nxt;
-      row_cur = row_nxt;
     }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
     // the last tile's O^T
     if (prev.item >= 0) {
       const bool ok = mbar_wait(&sh.bar_o, (tiles_done & 1u) ^ 1u, &sh.abort);
       tc_fence_after();
-      float o[16];
-      tc_ld16(tmem + lane_base + kTcColO, o);
-#pragma unroll
-      for (int g = 0; g < kAttnMaxGroup; ++g) acc[g] = acc[g] * alpha_prev[g] + (ok ? o[g] : 0.0f);
-#pragma unroll
-      for (int g = 0; g < kAttnMaxGroup; ++g) {
-        float x = l_part[g];
-#pragma unroll
-        for (int o2 = 16; o2 > 0; o2 >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o2);
-        if (lane == 0) sh.wsum[warp][g] = x;
-      }
-      asm volatile("bar.sync 3, %0;" ::"n"(kTcMathThreads) : "memory");
-      const long long head0 = static_cast<long long>(prev.seq) * a.n_heads + static_cast<long long>(prev.kvh) * G;
-      const long long stride = static_cast<long long>(a.max_chunks) * (kTcD + 2);
-      float* const entry = a.ws + (head0 * a.max_chunks + prev.chunk) * (kTcD + 2);
-#pragma unroll
-      for (int g = 0; g < kAttnMaxGroup; ++g) {
-        if (g >= G) break;
-        entry[g * stride + 2 + d_out] = acc[g];
-        if (p == 0) {
-          entry[g * stride] = m_ref[g];
-          entry[g * stride + 1] = sh.wsum[0][g] + sh.wsum[1][g] + sh.wsum[2][g] + sh.wsum[3][g];
-        }
-      }
+      fold_o(ok);
+      finish_item(prev);
     }
   }
   tc_fence_before();

@@ -443,12 +443,14 @@ __global__ void __launch_bounds__(kTcThreads, 2) attn_tc_kernel(const __grid_con
       float o[16];
       tc_ld16(tmem + lane_base + kTcColO, o);
 #pragma unroll
-      for (int g = 0; g < kAttnMaxGroup; ++g) acc[g] = acc[g] * alpha_prev[g] + (ok ? o[g] : 0.0f);
+      for (int g = 0; g < kAttnMaxGroup; ++g)
+        if (g < G) acc[g] = acc[g] * alpha_prev[g] + (ok ? o[g] : 0.0f);
     };
     // the item's (max, sum, accumulator) per head into its workspace entry, then a fresh state
     auto finish_item = [&](const TcTile& it) {
 #pragma unroll
       for (int g = 0; g < kAttnMaxGroup; ++g) {
+        if (g >= G) break;
         float x = l_part[g];
 #pragma unroll
         for (int o2 = 16; o2 > 0; o2 >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o2);
@@ -561,9 +563,11 @@ __global__ void __launch_bounds__(kTcThreads, 2) attn_tc_kernel(const __grid_con
       float x[kAttnMaxGroup];
 #pragma unroll
       for (int g = 0; g < kAttnMaxGroup; ++g) {
-        x[g] = (valid && ok_s && g < G) ? s[g] * a.scale_log2 : -INFINITY;
-        const float wm = warp_max_f32(x[g]);
-        if (lane == 0) sh.wmax[warp][g] = wm;
+        x[g] = (valid && ok_s) ? s[g] * a.scale_log2 : -INFINITY;
+        if (g < G) {
+          const float wm = warp_max_f32(x[g]);
+          if (lane == 0) sh.wmax[warp][g] = wm;
+        }
       }
       asm volatile("bar.sync 3, %0;" ::"n"(kTcMathThreads) : "memory");
       uint32_t hi[kAttnMaxGroup / 2], lo[kAttnMaxGroup / 2];
@@ -573,6 +577,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) attn_tc_kernel(const __grid_con
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int h = g + e;
+          pw[e] = 0.0f;
+          if (h >= G) continue;  // heads past the group: zero weights
           const float mt = fmaxf(fmaxf(sh.wmax[0][h], sh.wmax[1][h]), fmaxf(sh.wmax[2][h], sh.wmax[3][h]));
           float al = 1.0f;
           if (mt > m_ref[h] + kAttnRescaleLog2) {

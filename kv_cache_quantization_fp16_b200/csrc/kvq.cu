@@ -122,12 +122,12 @@ kvq_status launch_status() {
 std::atomic<int> g_engine{KVQ_ENGINE_AUTO};
 
 // What KVQ_ENGINE_AUTO runs: the engine measured faster on B200 for each
-// operation.  With four-round paged tiles the plain-load engine wins every
-// conversion measured (contiguous and paged, quantize and dequantize), so
-// AUTO is the plain-load engine throughout; the bulk engine stays available.
+// operation.  The plain-load engine with per-sequence tiles wins every
+// conversion measured (contiguous and paged, quantize and dequantize): the
+// bulk engine and the balanced paged grid stay available.
 template <class Op>
 struct AutoEngine {
-  static int pick(const Params&) { return KVQ_ENGINE_LDG; }
+  static int pick(const Params&) { return KVQ_ENGINE_LDG_TILED; }
 };
 
 // Launch with programmatic stream serialization (the kernels wait on the
@@ -213,7 +213,10 @@ kvq_status launch_balanced(Params p, int nkv, void* stream) {
   if (ctas < 1) return KVQ_ERR_CUDA;
   const long long most = static_cast<long long>(p.g.batch) * p.g.width * nkv;  // windows are at most `width` long
   const unsigned grid = static_cast<unsigned>(most < ctas ? most : ctas);
-  return launch_pdl(convert_balanced_kernel<Op>, dim3(grid), LdgCfg<Op>::kThreads, 0, stream, p, nkv);
+  // a unit is one round of loads of the operation: its tile elements in whole positions
+  const long long per_round = ldg_tile_elems<Op>() / p.g.hd;
+  const int unit = static_cast<int>(per_round < 1 ? 1 : (per_round > (1 << 20) ? (1 << 20) : per_round));
+  return launch_pdl(convert_balanced_kernel<Op>, dim3(grid), LdgCfg<Op>::kThreads, 0, stream, p, nkv, unit);
 }
 
 bool balanced_eligible(const Params& p) {

@@ -122,13 +122,18 @@ __global__ void __launch_bounds__(LdgCfg<Op>::kThreads, LdgCfg<Op>::kMinBlocksPe
 
 // ---------------------------------------------------------------------------
 // Balanced paged grid.  The windows of all sequences (clipped at 0, as
-// paged_tile does) are laid end to end, K's and then V's, and CTA c of G
-// takes positions [c T / G, (c + 1) T / G) of that sequence of T positions, so
-// every CTA moves the same bytes to within one position and one wave of CTAs
-// has no tail.  Each CTA finds the windows itself: the batch's lengths and
-// their running sums are staged in shared memory (no device->host sync); its
-// range is then walked in segments that stay inside one page of one sequence,
-// each converted by the operation's tile body.
+// paged_tile does) are laid end to end, K's and then V's: T positions.  One
+// wave of G CTAs walks them in rounds of G units of `unit` positions (one
+// round of loads per thread): in round r CTA c converts positions
+// [(r G + c) unit, (r G + c + 1) unit), so the CTAs of a round cover one
+// contiguous stretch of the caches (as consecutive tiles do), and the last,
+// partial round is split into G equal pieces.  Every CTA moves the same bytes
+// to within one position, and one wave has no tail.  (Giving each CTA one
+// contiguous range instead spread the concurrent accesses over the whole cache
+// and measured 15-25% slower.)  Each CTA finds the windows itself: the batch's
+// lengths and their running sums are staged in shared memory (no device->host
+// sync); a unit is converted in segments that stay inside one page of one
+// sequence.
 // ---------------------------------------------------------------------------
 
 constexpr int kBalancedMaxBatch = 1024;
@@ -235,25 +240,47 @@ __device__ __forceinline__ bool balanced_segment(const Geometry& g, const Balanc
   return true;
 }
 
+// Piece k of this CTA: unit k of the full rounds (k < R), or its share of the
+// last round (k == R); false past the last piece.  Positions count in 32 bits:
+// the host guarantees batch * width < 2^31, so T < 2^32.  Everything is
+// recomputed from shared memory, the launch parameters and the block index, so
+// that nothing of it stays live across a unit's loads.
+__device__ __forceinline__ bool balanced_piece(const BalancedShared& sh, const Geometry& g, int nkv, int unit,
+                                               uint32_t k, uint32_t& b, uint32_t& e) {
+  const uint32_t T = static_cast<uint32_t>(sh.pref[g.batch]) * static_cast<uint32_t>(nkv);
+  const uint32_t G = gridDim.x, c = blockIdx.x;
+  const uint32_t GU = G * static_cast<uint32_t>(unit);
+  const uint32_t R = T / GU;
+  if (k < R) {
+    b = k * GU + c * static_cast<uint32_t>(unit);
+    e = b + static_cast<uint32_t>(unit);
+    return true;
+  }
+  if (k > R) return false;
+  const unsigned long long rem = T - R * GU;
+  b = R * GU + static_cast<uint32_t>(c * rem / G);
+  e = R * GU + static_cast<uint32_t>((c + 1) * rem / G);
+  return true;
+}
+
 template <class Op>
 __global__ void __launch_bounds__(LdgCfg<Op>::kThreads, LdgCfg<Op>::kMinBlocksPerSM)
-    convert_balanced_kernel(const __grid_constant__ Params p, int nkv) {
+    convert_balanced_kernel(const __grid_constant__ Params p, int nkv, int unit) {
   using C = LdgCfg<Op>;
   __shared__ BalancedShared sh;
   const int tid = threadIdx.x;
-  const long long G = gridDim.x, c = blockIdx.x;
   // Before the grid dependency wait: the windows from lengths read at L2 (a hint:
-  // the previous grid may still be writing), and an L2 prefetch of the first
-  // round of this CTA's first segment, so that its DRAM reads start under the
-  // previous grid's tail.  A prefetch never changes what a later load returns.
+  // the previous grid may still be writing), and an L2 prefetch of this CTA's
+  // first unit, so that its DRAM reads start under the previous grid's tail.  A
+  // prefetch never changes what a later load returns.
   stage_windows<C::kThreads>(p.g, sh, true);
   {
-    const long long T = static_cast<long long>(sh.pref[p.g.batch]) * nkv;
-    const long long r0 = T * c / G, r1 = T * (c + 1) / G;
+    uint32_t b, e;
     int kv, n;
     long long row0;
-    if (r0 < r1 && balanced_segment(p.g, sh, r0, r1, kv, row0, n, false, true)) {
-      const long long elems = min(static_cast<long long>(n) * p.g.hd, static_cast<long long>(ldg_tile_elems<Op>()));
+    if (balanced_piece(sh, p.g, nkv, unit, 0, b, e) && b < e &&
+        balanced_segment(p.g, sh, b, e, kv, row0, n, false, true)) {
+      const long long elems = static_cast<long long>(n) * p.g.hd;
       prefetch_l2_range(static_cast<const uint8_t*>(p.in[kv]) + row0 * p.g.hd * Op::kInNum / Op::kInDen,
                         elems * Op::kInNum / Op::kInDen, tid, C::kThreads);
       if (Op::kReadsScales)
@@ -279,17 +306,18 @@ __global__ void __launch_bounds__(LdgCfg<Op>::kThreads, LdgCfg<Op>::kMinBlocksPe
     }
     if (__syncthreads_or(diff)) stage_windows<C::kThreads>(p.g, sh, false);
   }
-  const long long T = static_cast<long long>(sh.pref[p.g.batch]) * nkv;
-  const long long r1 = T * (c + 1) / G;
-  for (long long r = T * c / G; r < r1;) {
-    int kv, n;
-    long long row0;
-    const bool ok = balanced_segment(p.g, sh, r, r1, kv, row0, n, tid == 0);
-    if (ok) {
-      const uint8_t* in = static_cast<const uint8_t*>(p.in[kv]) + row0 * p.g.hd * Op::kInNum / Op::kInDen;
-      Op::template body<GlobalSrc, C::kThreads, C::kUnroll, C::kPrefetchRounds>(p, kv, row0, n, in, tid);
+  uint32_t b, e;
+  for (uint32_t k = 0; balanced_piece(sh, p.g, nkv, unit, k, b, e); ++k) {
+    // the piece in segments that stay inside one page of one sequence
+    for (uint32_t r = b; r < e;) {
+      int kv, n;
+      long long row0;
+      if (balanced_segment(p.g, sh, r, e, kv, row0, n, tid == 0)) {
+        const uint8_t* in = static_cast<const uint8_t*>(p.in[kv]) + row0 * p.g.hd * Op::kInNum / Op::kInDen;
+        Op::template body<GlobalSrc, C::kThreads, C::kUnroll, false>(p, kv, row0, n, in, tid);
+      }
+      r += static_cast<uint32_t>(n);
     }
-    r += n;
   }
 }
 

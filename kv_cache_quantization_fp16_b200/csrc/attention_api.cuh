@@ -26,8 +26,11 @@ long long tc_ctas() {
     return 0;
   }
   if (!opted[dev].load()) {
+    // all of the SM's unified memory as shared memory: two or three CTAs of 64-80 KB
     if (cudaFuncSetAttribute(kvq::attn_tc_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kvq::tc_smem_bytes<B>()) != cudaSuccess) {
+                             kvq::tc_smem_bytes<B>()) != cudaSuccess ||
+        cudaFuncSetAttribute(kvq::attn_tc_kernel<B>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess) {
       cudaGetLastError();
       return 0;
     }

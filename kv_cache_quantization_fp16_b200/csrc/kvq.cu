@@ -213,15 +213,16 @@ kvq_status launch_balanced(Params p, int nkv, void* stream) {
   if (ctas < 1) return KVQ_ERR_CUDA;
   const long long most = static_cast<long long>(p.g.batch) * p.g.width * nkv;  // windows are at most `width` long
   const unsigned grid = static_cast<unsigned>(most < ctas ? most : ctas);
-  // a unit is one round of loads of the operation: its tile elements in whole positions
-  const long long per_round = ldg_tile_elems<Op>() / p.g.hd;
+  // a unit is two rounds of loads of the operation, in whole positions
+  const long long per_round = 2 * ldg_tile_elems<Op>() / p.g.hd;
   const int unit = static_cast<int>(per_round < 1 ? 1 : (per_round > (1 << 20) ? (1 << 20) : per_round));
   return launch_pdl(convert_balanced_kernel<Op>, dim3(grid), LdgCfg<Op>::kThreads, 0, stream, p, nkv, unit);
 }
 
 bool balanced_eligible(const Params& p) {
   return p.g.page_size > 0 && p.g.batch <= kBalancedMaxBatch &&
-         static_cast<long long>(p.g.batch) * p.g.width < 0x7FFFFFFFLL;
+         static_cast<long long>(p.g.batch) * p.g.width < 0x7FFFFFFFLL &&
+         static_cast<long long>(p.g.bt_stride) * p.g.page_size < 0xFFFFFFFFLL;
 }
 
 template <class Op>

@@ -206,30 +206,35 @@ __device__ __forceinline__ void stage_windows(const Geometry& g, BalancedShared&
 // K/V stream, physical first row and positions (within one page of one
 // sequence).  Returns false, after recording the error from thread `report`,
 // when the block table cannot place it (the segment is skipped).
-__device__ __forceinline__ bool balanced_segment(const Geometry& g, const BalancedShared& sh, long long r,
-                                                 long long end, int& kv, long long& row0, int& n, bool report,
+__device__ __forceinline__ bool balanced_segment(const Geometry& g, const BalancedShared& sh, uint32_t r,
+                                                 uint32_t end, int& kv, long long& row0, int& n, bool report,
                                                  bool l2_only = false) {
-  const int total = sh.pref[g.batch];
-  kv = static_cast<int>(r / total);
-  const int rr = static_cast<int>(r - static_cast<long long>(kv) * total);
+  // positions count in 32 bits: the host guarantees batch * width < 2^31, and
+  // K's and V's windows together stay below 2^32
+  const uint32_t total = static_cast<uint32_t>(sh.pref[g.batch]);
+  kv = r >= total ? 1 : 0;
+  const uint32_t rr = r - (kv ? total : 0u);
   int lo = 0, hi = g.batch - 1;  // the last sequence whose running sum is <= rr
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (sh.pref[mid] <= rr) lo = mid;
+    if (static_cast<uint32_t>(sh.pref[mid]) <= rr) lo = mid;
     else hi = mid - 1;
   }
   const int seq = lo;
-  const long long pos = sh.lo[seq] + (rr - sh.pref[seq]);
-  const long long lp = pos / g.page_size;
-  const long long in_page = pos - lp * g.page_size;
-  long long m = end - r;
-  m = min(m, static_cast<long long>(sh.pref[seq + 1] - rr));
-  m = min(m, static_cast<long long>(g.page_size) - in_page);
-  n = static_cast<int>(m);
-  if (lp >= g.bt_stride) {
+  const long long pos = sh.lo[seq] + static_cast<long long>(rr - static_cast<uint32_t>(sh.pref[seq]));
+  if (pos >= static_cast<long long>(g.bt_stride) * g.page_size) {
+    n = static_cast<int>(min(end - r, static_cast<uint32_t>(sh.pref[seq + 1]) - rr));
     if (report) record_error(KVQ_DEV_BAD_PAGE_INDEX);
     return false;
   }
+  const uint32_t p32 = static_cast<uint32_t>(pos);  // < bt_stride * page_size < 2^32
+  const uint32_t ps = static_cast<uint32_t>(g.page_size);
+  const uint32_t lp = p32 / ps;
+  const uint32_t in_page = p32 - lp * ps;
+  uint32_t m = end - r;
+  m = min(m, static_cast<uint32_t>(sh.pref[seq + 1]) - rr);
+  m = min(m, ps - in_page);
+  n = static_cast<int>(m);
   const int32_t* entry = g.block_table + static_cast<long long>(seq) * g.bt_stride + lp;
   const int page = l2_only ? __ldcg(entry) : *entry;
   if (page < 0 || page >= g.dim0) {
@@ -241,10 +246,9 @@ __device__ __forceinline__ bool balanced_segment(const Geometry& g, const Balanc
 }
 
 // Piece k of this CTA: unit k of the full rounds (k < R), or its share of the
-// last round (k == R); false past the last piece.  Positions count in 32 bits:
-// the host guarantees batch * width < 2^31, so T < 2^32.  Everything is
-// recomputed from shared memory, the launch parameters and the block index, so
-// that nothing of it stays live across a unit's loads.
+// last round (k == R); false past the last piece.  Everything is recomputed
+// from shared memory, the launch parameters and the block index, so that
+// nothing of it stays live across a unit's loads.
 __device__ __forceinline__ bool balanced_piece(const BalancedShared& sh, const Geometry& g, int nkv, int unit,
                                                uint32_t k, uint32_t& b, uint32_t& e) {
   const uint32_t T = static_cast<uint32_t>(sh.pref[g.batch]) * static_cast<uint32_t>(nkv);

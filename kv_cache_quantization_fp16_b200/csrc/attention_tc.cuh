@@ -7,9 +7,10 @@
 // work item leaves (max, sum, accumulator) per query head for the combine
 // kernel.
 //
-// CTA: four math warps (one cache position per thread within a 128-position
-// tile, and one output row per thread) and one MMA warp whose elected lane
-// issues every tcgen05.mma.  Per tile:
+// CTA: four warps, one cache position per thread within a 128-position tile
+// and one output row per thread; thread 0 also issues every tcgen05.mma (a
+// fifth, MMA-only warp made the occupancy calculator round the CTA up to eight
+// warps of registers, one CTA per SM).  Per tile:
 //   * each math thread copies its position's K and V codes and scales into a
 //     shared-memory stage with cp.async (the next tile's K as soon as this
 //     tile's K row is read, its V as soon as this tile's V row is read, so each
@@ -51,13 +52,13 @@ constexpr int kTcD = 128;
 constexpr int kTcTile = 128;                  // positions per tile (the MMA's M for S^T)
 constexpr int kTcItem = 256;                  // positions per work item (= workspace chunk)
 constexpr int kTcMathThreads = 128;
-constexpr int kTcThreads = kTcMathThreads + 32;
+constexpr int kTcThreads = kTcMathThreads;
 constexpr uint32_t kTcTmemCols = 128;         // K tile 64 columns, S^T 16, O^T 16
 constexpr uint32_t kTcColK = 0, kTcColS = 64, kTcColO = 80;
 constexpr int kTcN = 16;                      // MMA N: query heads of the group, zero-padded
 
 // Shared memory of one CTA (dynamic): this struct, then the code stage of
-// TcFmt<B>::kStageChunks chunks of 128 x 16 bytes (chunk i of position p at
+// TcStage<B>::kChunks chunks of 128 x 16 bytes (chunk i of position p at
 // i * 2048 + p * 16: a thread's accesses are 16 bytes apart from its
 // neighbours', free of bank conflicts).  Every format needs more than 64 KB in
 // all, so at most three CTAs share an SM and their tensor memory (3 x 128
@@ -137,6 +138,32 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&f)[16]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 16; ++i) f[i] = __uint_as_float(r[i]);
+}
+
+// Wait for the phase with the given parity, the thread suspended in hardware
+// between checks (up to 2 us at a time) instead of spinning; gives up like
+// mbar_wait (abort flag, or 1 s, then KVQ_DEV_TIMEOUT).
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  uint32_t done;
+  const unsigned long long t0 = globaltimer_ns();
+  for (;;) {
+    asm volatile(
+        "{\n"
+        "  .reg .pred p;\n"
+        "  mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        "  selp.u32 %0, 1, 0, p;\n"
+        "}\n"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(2000u)
+        : "memory");
+    if (done) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      record_error(KVQ_DEV_TIMEOUT);
+      return false;
+    }
+  }
 }
 
 // Warp-wide maximum of a binary32 value (order-preserving integer key).
@@ -343,7 +370,7 @@ __device__ __forceinline__ long long tc_cache_row(const AttnParams& a, int seq, 
 }
 
 template <int B>
-__global__ void __launch_bounds__(kTcThreads, 2) attn_tc_kernel(const __grid_constant__ AttnParams a) {
+__global__ void __launch_bounds__(kTcThreads, 3) attn_tc_kernel(const __grid_constant__ AttnParams a) {
   using F = TcFmt<B>;
   constexpr bool kPerm = F::kPerm;
   extern __shared__ __align__(16) uint8_t tc_smem_raw[];
@@ -351,13 +378,13 @@ __global__ void __launch_bounds__(kTcThreads, 2) attn_tc_kernel(const __grid_con
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = a.group;
 
-  if (warp == 4) {
+  if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&sh.tmem)),
                  "r"(kTcTmemCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  if (tid == kTcMathThreads) {
+  if (tid == 0) {
     mbar_init(&sh.bar_kv, kTcMathThreads);
     mbar_init(&sh.bar_p, kTcMathThreads);
     mbar_init(&sh.bar_s, 1);
@@ -402,36 +429,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) attn_tc_kernel(const __grid_con
   const uint32_t tmem = sh.tmem;
   uint32_t tiles_done = 0;  // tiles this CTA has processed: the phase of all four barriers
 
-  if (warp == 4) {
-    // ---------------- MMA issue (one elected lane) ----------------
-    if (lane == 0) {
-      const uint32_t idesc_s = tc_idesc(128, kTcN, 0, 0);
-      const uint32_t idesc_o = tc_idesc(128, kTcN, 1, 1);
-      const uint64_t q_desc = tc_sdesc(smem_addr(sh.q), 128, 2048);
-      const uint64_t v_desc = tc_sdesc(smem_addr(sh.v), 128, 2048);
-      const uint64_t hi_desc = tc_sdesc(smem_addr(sh.p_hi), 128, 2048);
-      const uint64_t lo_desc = tc_sdesc(smem_addr(sh.p_lo), 128, 2048);
-      for (TcTile c = walk.first(blockIdx.x); c.item >= 0; c = walk.next(c), ++tiles_done) {
-        const uint32_t ph = tiles_done & 1u;
-        if (mbar_wait(&sh.bar_kv, ph, &sh.abort)) {
-          tc_fence_after();
-#pragma unroll
-          for (int s = 0; s < kTcD / 16; ++s)
-            tc_mma_ts(tmem + kTcColS, tmem + kTcColK + 8 * s, q_desc + 16 * s, idesc_s, s > 0);
-        }
-        tc_commit(&sh.bar_s);  // arrives once the MMAs above (if any) are done
-        if (mbar_wait(&sh.bar_p, ph, &sh.abort)) {
-          tc_fence_after();
-#pragma unroll
-          for (int s = 0; s < kTcTile / 16; ++s) tc_mma_ss(tmem + kTcColO, v_desc + 16 * s, hi_desc + 16 * s, idesc_o, s > 0);
-#pragma unroll
-          for (int s = 0; s < kTcTile / 16; ++s) tc_mma_ss(tmem + kTcColO, v_desc + 16 * s, lo_desc + 16 * s, idesc_o, 1);
-        }
-        tc_commit(&sh.bar_o);
-      }
-    }
-  } else {
-    // ---------------- math warps ----------------
+  {
+    // ---------------- every thread: one position, one output row ----------------
     const int p = tid;  // position within the tile; output row (tensor-memory lane) of O^T
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const int d_out = (p & ~7) + tc_perm8<kPerm>(p & 7);  // head_dim element of this thread's O^T row
@@ -474,6 +473,34 @@ __global__ void __launch_bounds__(kTcThreads, 2) attn_tc_kernel(const __grid_con
     };
 
     uint8_t* const stage = tc_smem_raw + (sizeof(TcShared) + 127) / 128 * 128;
+    // the MMAs (thread 0): S^T = K Q^T once every thread's K row is in tensor memory,
+    // O^T = V^T P^T once every thread's V row and weights are in shared memory
+    const uint32_t idesc_s = tc_idesc(128, kTcN, 0, 0);
+    const uint32_t idesc_o = tc_idesc(128, kTcN, 1, 1);
+    const uint64_t q_desc = tc_sdesc(smem_addr(sh.q), 128, 2048);
+    const uint64_t v_desc = tc_sdesc(smem_addr(sh.v), 128, 2048);
+    const uint64_t hi_desc = tc_sdesc(smem_addr(sh.p_hi), 128, 2048);
+    const uint64_t lo_desc = tc_sdesc(smem_addr(sh.p_lo), 128, 2048);
+    auto issue_s = [&](uint32_t ph) {
+      if (tc_wait(&sh.bar_kv, ph, &sh.abort)) {
+        tc_fence_after();
+#pragma unroll
+        for (int s = 0; s < kTcD / 16; ++s)
+          tc_mma_ts(tmem + kTcColS, tmem + kTcColK + 8 * s, q_desc + 16 * s, idesc_s, s > 0);
+      }
+      tc_commit(&sh.bar_s);  // arrives once the MMAs above (if any) are done
+    };
+    auto issue_o = [&](uint32_t ph) {
+      if (tc_wait(&sh.bar_p, ph, &sh.abort)) {
+        tc_fence_after();
+#pragma unroll
+        for (int s = 0; s < kTcTile / 16; ++s)
+          tc_mma_ss(tmem + kTcColO, v_desc + 16 * s, hi_desc + 16 * s, idesc_o, s > 0);
+#pragma unroll
+        for (int s = 0; s < kTcTile / 16; ++s) tc_mma_ss(tmem + kTcColO, v_desc + 16 * s, lo_desc + 16 * s, idesc_o, 1);
+      }
+      tc_commit(&sh.bar_o);
+    };
     TcTile cur = walk.first(blockIdx.x);
     TcTile prev;
     prev.item = -1;
@@ -533,9 +560,10 @@ __global__ void __launch_bounds__(kTcThreads, 2) attn_tc_kernel(const __grid_con
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
       mbar_arrive(&sh.bar_kv);
+      if (tid == 0) issue_s(ph);
       // the previous tile's O^T: fold it in, finish its item when it was the last
       if (prev.item >= 0) {
-        const bool ok = mbar_wait(&sh.bar_o, ph ^ 1u, &sh.abort);
+        const bool ok = tc_wait(&sh.bar_o, ph ^ 1u, &sh.abort);
         tc_fence_after();
         fold_o(ok);
         if (prev.last) finish_item(prev);
@@ -556,7 +584,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) attn_tc_kernel(const __grid_con
         asm volatile("cp.async.commit_group;" ::: "memory");
       }
       // scores of this tile
-      const bool ok_s = mbar_wait(&sh.bar_s, ph, &sh.abort);
+      const bool ok_s = tc_wait(&sh.bar_s, ph, &sh.abort);
       tc_fence_after();
       float s[16];
       tc_ld16(tmem + lane_base + kTcColS, s);
@@ -598,6 +626,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) attn_tc_kernel(const __grid_con
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
       mbar_arrive(&sh.bar_p);
+      if (tid == 0) issue_o(ph);
       prev = cur;
       cur = nxt;
       hr_cur = hr_nxt;
@@ -605,7 +634,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) attn_tc_kernel(const __grid_con
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     // the last tile's O^T
     if (prev.item >= 0) {
-      const bool ok = mbar_wait(&sh.bar_o, (tiles_done & 1u) ^ 1u, &sh.abort);
+      const bool ok = tc_wait(&sh.bar_o, (tiles_done & 1u) ^ 1u, &sh.abort);
       tc_fence_after();
       fold_o(ok);
       finish_item(prev);
@@ -613,7 +642,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) attn_tc_kernel(const __grid_con
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 0) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcTmemCols) : "memory");
   }

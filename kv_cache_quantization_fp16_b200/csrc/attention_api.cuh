@@ -15,7 +15,7 @@ std::atomic<int> g_attention_path{KVQ_ATTENTION_AUTO};
 
 // CTAs of the tcgen05 kernel the device holds at once (cached per device, after the
 // shared-memory opt-in), 0 on failure.
-template <int B>
+template <int B, int G>
 long long tc_ctas() {
   constexpr int kMaxDevices = 64;
   static std::atomic<bool> opted[kMaxDevices];
@@ -27,16 +27,42 @@ long long tc_ctas() {
   }
   if (!opted[dev].load()) {
     // all of the SM's unified memory as shared memory: two or three CTAs of 64-80 KB
-    if (cudaFuncSetAttribute(kvq::attn_tc_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(kvq::attn_tc_kernel<B, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kvq::tc_smem_bytes<B>()) != cudaSuccess ||
-        cudaFuncSetAttribute(kvq::attn_tc_kernel<B>, cudaFuncAttributePreferredSharedMemoryCarveout,
+        cudaFuncSetAttribute(kvq::attn_tc_kernel<B, G>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess) {
       cudaGetLastError();
       return 0;
     }
     opted[dev].store(true);
   }
-  return first_wave_ctas(kvq::attn_tc_kernel<B>, kvq::kTcThreads, kvq::tc_smem_bytes<B>(), resident, kMaxDevices);
+  long long n = resident[dev].load();
+  if (n == 0) {
+    // CTAs per SM from the shared memory each needs and the launch bounds (three);
+    // the occupancy query reports one for this kernel
+    int sms = 0, smem_sm = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    long long per_sm = smem_sm / (kvq::tc_smem_bytes<B>() + 1024);
+    if (per_sm > 3) per_sm = 3;
+    if (per_sm < 1) per_sm = 1;
+    n = static_cast<long long>(sms) * per_sm;
+    resident[dev].store(n);
+  }
+  return n;
+}
+
+// The tcgen05 partial kernel for `group` query heads per kv head: as many CTAs
+// as the device holds at once, never more than there are item slots.
+template <int B, int G>
+kvq_status launch_tc(const kvq::AttnParams& a, long long items, void* stream) {
+  const long long ctas = tc_ctas<B, G>();
+  if (ctas < 1) return KVQ_ERR_CUDA;
+  return launch_pdl(kvq::attn_tc_kernel<B, G>, dim3(static_cast<unsigned>(items < ctas ? items : ctas)),
+                    kvq::kTcThreads, kvq::tc_smem_bytes<B>(), stream, a);
 }
 
 // Chunks of `chunk` positions a sequence can have: the longest window the
@@ -110,10 +136,16 @@ kvq_status launch_attention(kvq::AttnParams a, const kvq_cache_desc* desc, void*
   if constexpr (D == kvq::kTcD) {
     // the tcgen05 kernel: head_dim 128, batches its shared memory stages (<= 256 sequences)
     if (path == KVQ_ATTENTION_TCGEN05 && compact) {
-      const long long ctas = tc_ctas<B>();
-      if (ctas < 1) return KVQ_ERR_CUDA;
-      st = launch_pdl(kvq::attn_tc_kernel<B>, dim3(static_cast<unsigned>(items < ctas ? items : ctas)),
-                      kvq::kTcThreads, kvq::tc_smem_bytes<B>(), stream, a);
+      switch (a.group) {
+        case 1: st = launch_tc<B, 1>(a, items, stream); break;
+        case 2: st = launch_tc<B, 2>(a, items, stream); break;
+        case 3: st = launch_tc<B, 3>(a, items, stream); break;
+        case 4: st = launch_tc<B, 4>(a, items, stream); break;
+        case 5: st = launch_tc<B, 5>(a, items, stream); break;
+        case 6: st = launch_tc<B, 6>(a, items, stream); break;
+        case 7: st = launch_tc<B, 7>(a, items, stream); break;
+        default: st = launch_tc<B, 8>(a, items, stream); break;
+      }
       if (st != KVQ_OK) return st;
       return launch_pdl(kvq::attn_combine_kernel<D>, dim3(a.n_heads, a.batch), kvq::kCombineThreads, 0, stream, a);
     }

@@ -53,8 +53,12 @@ constexpr int kTcTile = 128;                  // positions per tile (the MMA's M
 constexpr int kTcItem = 256;                  // positions per work item (= workspace chunk)
 constexpr int kTcMathThreads = 128;
 constexpr int kTcThreads = kTcMathThreads;
-constexpr uint32_t kTcTmemCols = 128;         // K tile 64 columns, S^T 16, O^T 16
-constexpr uint32_t kTcColK = 0, kTcColS = 64, kTcColO = 80;
+constexpr uint32_t kTcTmemCols = 128;         // K tile 64 columns, S^T 2 x 16, O^T 2 x 16
+// S^T is accumulated in two independent halves of the reduction (head_dim 0-63
+// and 64-127), O^T in one accumulator for the weights' high parts and one for
+// their residuals: four chains of four to eight MMAs instead of two of eight
+// and sixteen, summed by the threads that read them.
+constexpr uint32_t kTcColK = 0, kTcColS0 = 64, kTcColS1 = 80, kTcColOh = 96, kTcColOl = 112;
 constexpr int kTcN = 16;                      // MMA N: query heads of the group, zero-padded
 
 // Shared memory of one CTA (dynamic): this struct, then the code stage of
@@ -369,14 +373,14 @@ __device__ __forceinline__ long long tc_cache_row(const AttnParams& a, int seq, 
   return row * a.kv_heads + kvh;
 }
 
-template <int B>
+template <int B, int G>
 __global__ void __launch_bounds__(kTcThreads, 3) attn_tc_kernel(const __grid_constant__ AttnParams a) {
   using F = TcFmt<B>;
   constexpr bool kPerm = F::kPerm;
   extern __shared__ __align__(16) uint8_t tc_smem_raw[];
   TcShared& sh = *reinterpret_cast<TcShared*>(tc_smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int G = a.group;
+  static_assert(G >= 1 && G <= kAttnMaxGroup, "query heads per kv head");
 
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&sh.tmem)),
@@ -439,8 +443,11 @@ __global__ void __launch_bounds__(kTcThreads, 3) attn_tc_kernel(const __grid_con
     for (int g = 0; g < kAttnMaxGroup; ++g) m_ref[g] = -INFINITY, l_part[g] = 0.0f, acc[g] = 0.0f, alpha_prev[g] = 1.0f;
     // fold the previous tile's O^T row into the accumulators (after its MMAs completed)
     auto fold_o = [&](bool ok) {
-      float o[16];
-      tc_ld16(tmem + lane_base + kTcColO, o);
+      float o[16], ol[16];
+      tc_ld16(tmem + lane_base + kTcColOh, o);
+      tc_ld16(tmem + lane_base + kTcColOl, ol);
+#pragma unroll
+      for (int g = 0; g < kAttnMaxGroup; ++g) o[g] += ol[g];
 #pragma unroll
       for (int g = 0; g < kAttnMaxGroup; ++g)
         if (g < G) acc[g] = acc[g] * alpha_prev[g] + (ok ? o[g] : 0.0f);
@@ -485,8 +492,10 @@ __global__ void __launch_bounds__(kTcThreads, 3) attn_tc_kernel(const __grid_con
       if (tc_wait(&sh.bar_kv, ph, &sh.abort)) {
         tc_fence_after();
 #pragma unroll
-        for (int s = 0; s < kTcD / 16; ++s)
-          tc_mma_ts(tmem + kTcColS, tmem + kTcColK + 8 * s, q_desc + 16 * s, idesc_s, s > 0);
+        for (int s = 0; s < kTcD / 32; ++s) {
+          tc_mma_ts(tmem + kTcColS0, tmem + kTcColK + 8 * s, q_desc + 16 * s, idesc_s, s > 0);
+          tc_mma_ts(tmem + kTcColS1, tmem + kTcColK + 32 + 8 * s, q_desc + 64 + 16 * s, idesc_s, s > 0);
+        }
       }
       tc_commit(&sh.bar_s);  // arrives once the MMAs above (if any) are done
     };
@@ -494,10 +503,10 @@ __global__ void __launch_bounds__(kTcThreads, 3) attn_tc_kernel(const __grid_con
       if (tc_wait(&sh.bar_p, ph, &sh.abort)) {
         tc_fence_after();
 #pragma unroll
-        for (int s = 0; s < kTcTile / 16; ++s)
-          tc_mma_ss(tmem + kTcColO, v_desc + 16 * s, hi_desc + 16 * s, idesc_o, s > 0);
-#pragma unroll
-        for (int s = 0; s < kTcTile / 16; ++s) tc_mma_ss(tmem + kTcColO, v_desc + 16 * s, lo_desc + 16 * s, idesc_o, 1);
+        for (int s = 0; s < kTcTile / 16; ++s) {
+          tc_mma_ss(tmem + kTcColOh, v_desc + 16 * s, hi_desc + 16 * s, idesc_o, s > 0);
+          tc_mma_ss(tmem + kTcColOl, v_desc + 16 * s, lo_desc + 16 * s, idesc_o, s > 0);
+        }
       }
       tc_commit(&sh.bar_o);
     };
@@ -586,8 +595,11 @@ __global__ void __launch_bounds__(kTcThreads, 3) attn_tc_kernel(const __grid_con
       // scores of this tile
       const bool ok_s = tc_wait(&sh.bar_s, ph, &sh.abort);
       tc_fence_after();
-      float s[16];
-      tc_ld16(tmem + lane_base + kTcColS, s);
+      float s[16], s1[16];
+      tc_ld16(tmem + lane_base + kTcColS0, s);
+      tc_ld16(tmem + lane_base + kTcColS1, s1);
+#pragma unroll
+      for (int g = 0; g < kAttnMaxGroup; ++g) s[g] += s1[g];
       float x[kAttnMaxGroup];
 #pragma unroll
       for (int g = 0; g < kAttnMaxGroup; ++g) {

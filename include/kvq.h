@@ -103,16 +103,17 @@ enum {
 enum {
   KVQ_ENGINE_AUTO = 0, /* per operation, the engine measured faster on B200 (default) */
   KVQ_ENGINE_LDG = 1,  /* 16-byte global loads issued up front; contiguous mode: one tile
-                          per CTA; paged mode: one wave of CTAs splitting the flattened
-                          windows of all sequences into equal position ranges (batches of
-                          up to 1024 sequences whose windows total under 2^31 positions;
-                          otherwise per-sequence tiles as in KVQ_ENGINE_LDG_TILED) */
+                          per CTA; paged mode: one wave of CTAs taking equal shares of the
+                          flattened windows of all sequences, walked in interleaved rounds
+                          (batches of up to 1024 sequences whose windows total under 2^31
+                          positions; otherwise per-sequence tiles as in
+                          KVQ_ENGINE_LDG_TILED).  Measured slower than the tiles on B200 */
   KVQ_ENGINE_BULK = 2, /* persistent CTAs, TMA bulk copies (cp.async.bulk, no multicast)
                           into a 4-stage shared-memory ring, one producer warp and eight
                           consumer warps; used when one position of the input stream is a
                           multiple of 16 bytes, otherwise the LDG engine runs */
   KVQ_ENGINE_LDG_TILED = 3 /* the LDG engine with per-sequence tiles in paged mode too
-                              (one tile of a sequence's window per CTA) */
+                              (one tile of a sequence's window per CTA): what AUTO runs */
 };
 
 /* The shape the torch tensor carried in the original extension. */
@@ -289,7 +290,7 @@ enum {
   KVQ_ATTENTION_MMA = 1,     /* warp-level mma.sync tiles for every geometry */
   KVQ_ATTENTION_TCGEN05 = 2  /* tcgen05.mma with tensor-memory accumulators for head_dim 128
                                 and batches of up to 256 sequences; other geometries run
-                                the mma.sync kernel */
+                                the mma.sync kernel.  Measured slower than mma.sync on B200 */
 };
 
 /* Select the decode-attention kernel for all later calls in this process (any

@@ -184,8 +184,8 @@ KVQ_API kvq_status kvq_q_to_fp16_kv(const void* k_in, void* k_out, const void* k
  * exactly what kvq_q_to_fp16_kv would produce:
  *   out[i, h, :] = sum_p softmax_p(softmax_scale * q . k_p) * v_p   (binary16),
  * 0 for an empty window.  Arithmetic: fp16 products with fp32 accumulation
- * (tensor cores), base-2 online softmax in fp32; tests bound the difference
- * to the fp64 result by one binary16 ulp plus 2^-14 of the largest |v|.
+ * (tensor cores), base-2 online softmax in fp32; the tests hold every output
+ * to an error bound derived from that arithmetic against the exact result.
  *   q, out     [batch_size, n_heads, head_dim] binary16, 16-byte aligned
  *   k/v codes  [dim0, dim1, kv_heads, head_dim * wbits / 8] uint8
  *   k/v scales [dim0, dim1, kv_heads, head_dim / 32] binary16
@@ -193,8 +193,10 @@ KVQ_API kvq_status kvq_q_to_fp16_kv(const void* k_in, void* k_out, const void* k
  *   dim1); page_size > 0: paged as in kvq_fp16_to_q_kv.  head_dim is 64, 128
  *   or 256; n_heads / kv_heads <= 8; wbits 4, 6 or 8.
  *   workspace: caller-owned device memory of at least
- *   kvq_decode_attention_workspace_size(...) bytes (per-chunk partial
- *   results), 16-byte aligned; its contents on entry do not matter.
+ *   kvq_decode_attention_workspace_size(...) bytes (partial results: 2 +
+ *   head_dim floats per sequence, query head and 128-position chunk the
+ *   cache geometry allows), 16-byte aligned; its contents on entry do not
+ *   matter.
  * Two kernels are enqueued on `stream`.  A window longer than the cache, or
  * paging metadata pointing outside it, skips those positions and sets the
  * device error word. */
@@ -225,9 +227,9 @@ KVQ_API kvq_status kvq_decode_attention_fp8(const void* q, const void* k_fp8, co
 KVQ_API size_t kvq_decode_attention_workspace_size(const kvq_cache_desc* desc, int batch_size, int n_heads,
                                                    int page_size);
 
-/* Size of the scratch array kvq_decode_attention_q_noalloc uses (16 MiB per
+/* Size of the scratch array kvq_decode_attention_q_noalloc uses (32 MiB per
  * device). */
-#define KVQ_ATTENTION_SCRATCH_BYTES ((size_t)16 << 20)
+#define KVQ_ATTENTION_SCRATCH_BYTES ((size_t)32 << 20)
 
 /* kvq_decode_attention_q without a caller workspace.  The pages have no
  * counterpart: this is a convenience of this library for callers that cannot
@@ -240,9 +242,9 @@ KVQ_API size_t kvq_decode_attention_workspace_size(const kvq_cache_desc* desc, i
  *   kvq_decode_attention_q.  A geometry whose
  *   kvq_decode_attention_workspace_size(...) exceeds
  *   KVQ_ATTENTION_SCRATCH_BYTES returns KVQ_ERR_RANGE and enqueues nothing
- *   (for example, batch 8 x 32 query heads x head_dim 128 with up to 8192
- *   positions needs 4.3 MB and fits; batch 16 with up to 16384 positions
- *   needs 17 MB and does not).
+ *   (for example, batch 8 x 32 query heads x head_dim 128 with up to 16384
+ *   positions needs 17 MB and fits; batch 16 with up to 16384 positions
+ *   needs 34 MB and does not).
  *   Every call looks up the device address of the current device's copy of
  *   the array (a host-side query that enqueues nothing), so a reset and
  *   re-created device context is picked up; the first call on a device may

@@ -515,7 +515,7 @@ def decode_attention_fp8(q, k_fp8, v_fp8, out, batch_size, cache_seqlens, softma
     _check(st, "decode_attention_fp8")
 
 
-ATTENTION_SCRATCH_BYTES = 16 << 20  # KVQ_ATTENTION_SCRATCH_BYTES
+ATTENTION_SCRATCH_BYTES = 32 << 20  # KVQ_ATTENTION_SCRATCH_BYTES
 
 
 def decode_attention_q_noalloc(q, k_codes, k_scales, v_codes, v_scales, out, batch_size, cache_seqlens, wbits,

@@ -66,6 +66,7 @@ struct AttnParams {
   const int32_t* seqlens;
   const int32_t* block_table;
   int dim0, dim1, kv_heads, batch, n_heads, group, page_size, bt_stride, max_chunks;
+  int page_shift;  // log2(page_size) when it is a power of two, else -1
   int chunk;  // positions per work item (AttnTile<B, D>::kChunk)
   float scale_log2;  // softmax_scale * log2(e)
 };
@@ -299,7 +300,9 @@ struct AttnTile {
   static constexpr int kStrideK = kRowBytes + (kRowBytes % 128 == 0 ? 16 : 0);
   static constexpr int kStrideV = kRowBytes + ((B == 6 && D == 64) ? 0 : 16);
   static constexpr int kScales = B == 0 ? 0 : D / 32;  // binary16 scales per row
-  static constexpr int kChunk = 256;  // positions per work item / workspace entry (kAttnMinChunk)
+  // positions per work item / workspace entry: 128 for the 4- and 6-bit codes
+  // (their blocked walk), 256 for 8-bit codes and E5M2 (their round-robin walk)
+  static constexpr int kChunk = (B == 4 || B == 6) ? 128 : 256;
   static constexpr int kSub = kRowBytes <= 96 ? 32 : 16;   // positions per staged buffer (measured)
   static constexpr int kBufK = kSub * kStrideK;
   static constexpr int kBufV = kSub * kStrideV;
@@ -317,7 +320,7 @@ struct AttnTile {
   static constexpr int kKSpanBytes = KN * kBits / 8;
   static constexpr int kVSpanBytes = VN * kBits / 8;
 };
-constexpr int kAttnMinChunk = 256;  // sizes the workspace: every (B, D) uses 256-position chunks
+constexpr int kAttnMinChunk = 128;  // sizes the workspace: the smallest kChunk of any (B, D)
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n"
@@ -429,36 +432,59 @@ template <class I>
 struct AttnCursor {
   I item;               // work item index, or -1 past the end
   int seq, chunk, kvh;  // what the item is
+  int nch;              // chunks of the sequence (blocked walk)
   int sub;              // sub-chunk within the item
   int n;                // positions of this sub-chunk (<= kSub)
   bool last;            // last sub-chunk of the item
+  bool fresh;           // the item starts a new softmax state (otherwise it continues the previous one)
 };
 
-// Work items in walk order, two ways (the launch picks one).
+// Work items in walk order.  An item is one (sequence, kChunk-position
+// chunk, kv head); its workspace entry is (sequence, query head, chunk).
 // kCompact: only items that hold data are enumerated.  The CTA stages the
 // batch in shared memory: kSeqlenSlots sequence lengths, then kSeqlenSlots
-// running item counts (entry i counts the items of sequences 0..i:
-// ceil(length / chunk) chunks times kv heads each), then the item total.  Item
-// k is found by a binary search over the running counts, and every warp gets
-// the same number of items to within one.  The launch guarantees that the
-// batch fits the slots and that every item count fits an int.
+// running item counts (entry i counts the items of sequences 0..i), then the
+// total.  The launch guarantees that the batch fits the slots and that every
+// count fits an int.  Without kSplit, one of two walks (chosen per format, by
+// measurement: streams of launches over the paged pool):
+//   Blocked (4- and 6-bit codes, 128-position chunks): items are numbered (kv
+//   head, sequence, chunk), chunk fastest, so the running counts count the
+//   chunks of one kv head.  Warp w of W takes the contiguous range
+//   [w U / W, (w + 1) U / W) of the U items, so the warps' shares differ by at
+//   most one small item.  When W is a multiple of the kv heads, the warps of
+//   every kv head get the same ranges of (sequence, chunk), so the kv heads of
+//   a position are read at about the same time.  Within its range a warp
+//   carries one softmax state over the two chunks of each aligned pair (chunks
+//   2i, 2i + 1 of one sequence and kv head) and writes it to the entry of the
+//   first chunk it took; the entry of the second gets a -inf maximum, which the
+//   combine skips.  A state never spans more than 256 positions.  These codes
+//   cost the most instructions per byte: the balance pays.
+//   Round-robin (8-bit codes and E5M2, 256-position chunks): items are
+//   numbered (sequence, chunk, kv head), kv head fastest, and warp w takes
+//   items w, w + W, ...: the warps of a round read neighbouring items, so the
+//   kv heads of a position, which share DRAM pages, are read together.  These
+//   formats come closest to the DRAM limit, where that locality pays.
+//   kSplit (for batches too small to give every warp an item): items as in
+//   the round-robin walk; a CTA takes items in turn and each of its four warps
+//   a quarter of the item's positions, every warp walking the same kSplitSubs
+//   sub-chunks per item (empty ones where its quarter runs past the sequence),
+//   so that the CTA can merge the four partial results at the end of each item.
 // Otherwise: every (sequence, chunk, kv head) slot up to the cache's capacity
-// is visited and empty ones are skipped (lengths staged when the batch fits).
-// kSplit (with kCompact, for batches too small to give every warp an item):
-// a CTA takes items in turn and each of its four warps a quarter of the
-// item's positions, every warp walking the same kSplitSubs sub-chunks per item
-// (empty ones where its quarter runs past the sequence), so that the CTA can
-// merge the four partial results at the end of each item.
+// is visited in turn (kv head fastest) and empty ones are skipped (lengths
+// staged when the batch fits); every item has its own state and entry.
 template <int B, int D, bool kCompact, bool kSplit = false>
 struct AttnWalk {
   static_assert(kCompact || !kSplit, "the split walk enumerates compactly");
   using T = AttnTile<B, D>;
   using Item = typename std::conditional<kCompact, int, long long>::type;
   using Cursor = AttnCursor<Item>;
+  static constexpr bool kBlocked = kCompact && !kSplit && (B == 4 || B == 6);
   static constexpr int kQuarter = T::kChunk / kAttnWarps;  // positions per warp and item (kSplit)
   static constexpr int kSplitSubs = kQuarter / T::kSub;     // sub-chunks per warp and item (kSplit)
+  static_assert(kSplitSubs >= 1 && kQuarter % T::kSub == 0, "a quarter item is whole sub-chunks");
   const AttnParams& a;
-  bool staged;  // the batch's lengths are in shared memory
+  bool staged;   // the batch's lengths are in shared memory
+  Item end = 0;  // kBlocked: one past this warp's last item
 
   // first position of this warp's part of an item
   __device__ static int offset() { return kSplit ? kQuarter * static_cast<int>(threadIdx.x >> 5) : 0; }
@@ -497,25 +523,40 @@ struct AttnWalk {
   // first sub-chunk of item `item` (kCompact), or of the first non-empty item slot at or after it
   __device__ Cursor seek(Item item) const {
     Cursor c;
+    c.fresh = true;
     if constexpr (kCompact) {
       const int* const s_items = block() + T::kSeqlenSlots;
-      if (item >= s_items[T::kSeqlenSlots]) {
+      if (item >= (kBlocked ? end : s_items[T::kSeqlenSlots])) {
         c.item = -1;
         return c;
+      }
+      int kvh = 0;
+      Item local = item;  // the item among those of its kv head (kBlocked) or of the batch
+      if constexpr (kBlocked) {
+        const unsigned per_head = static_cast<unsigned>(s_items[T::kSeqlenSlots]);
+        kvh = static_cast<int>(static_cast<unsigned>(item) / per_head);
+        local = static_cast<Item>(static_cast<unsigned>(item) - static_cast<unsigned>(kvh) * per_head);
       }
       int lo = 0, hi = a.batch - 1;  // the first sequence whose running count exceeds the item
       while (lo < hi) {
         const int mid = (lo + hi) >> 1;
-        if (s_items[mid] > item) hi = mid;
+        if (s_items[mid] > local) hi = mid;
         else lo = mid + 1;
       }
-      const unsigned r = static_cast<unsigned>(item - (lo ? s_items[lo - 1] : 0));
-      const unsigned chunk = r / static_cast<unsigned>(a.kv_heads);
+      const int prev = lo ? s_items[lo - 1] : 0;
+      const unsigned r = static_cast<unsigned>(local - prev);
       c.seq = lo;
-      c.chunk = static_cast<int>(chunk);
-      c.kvh = static_cast<int>(r - chunk * static_cast<unsigned>(a.kv_heads));
       c.item = item;
-      set_sub(c, length(c.seq), 0);
+      if constexpr (kBlocked) {
+        c.kvh = kvh;
+        c.chunk = static_cast<int>(r);
+        c.nch = s_items[lo] - prev;
+      } else {
+        const unsigned chunk = r / static_cast<unsigned>(a.kv_heads);
+        c.chunk = static_cast<int>(chunk);
+        c.kvh = static_cast<int>(r - chunk * static_cast<unsigned>(a.kv_heads));
+      }
+      set_sub(c, length(lo), 0);
       return c;
     } else {
       const long long n_items = static_cast<long long>(a.batch) * a.max_chunks * a.kv_heads;
@@ -545,16 +586,78 @@ struct AttnWalk {
     }
   }
   __device__ Cursor next(const Cursor& c) const {
-    if (c.last) return seek(c.item + stride());
-    Cursor d = c;
-    set_sub(d, length(c.seq), c.sub + 1);
-    return d;
+    if (!c.last) {
+      Cursor d = c;
+      set_sub(d, length(c.seq), c.sub + 1);
+      return d;
+    }
+    if constexpr (kBlocked) {
+      // the next item of this warp's range: the sequence's next chunk, or a seek
+      if (c.item + 1 >= end) {
+        Cursor d;
+        d.item = -1;
+        return d;
+      }
+      if (c.chunk + 1 < c.nch) {
+        Cursor d = c;
+        d.item = c.item + 1;
+        d.chunk = c.chunk + 1;
+        d.fresh = (d.chunk & 1) == 0;
+        set_sub(d, length(c.seq), 0);
+        return d;
+      }
+      return seek(c.item + 1);
+    } else {
+      return seek(c.item + stride());
+    }
   }
 };
+
+// Scales of one sub-chunk (lane i: position i; rows without data get zero
+// scales, which dequantize whatever codes the buffer holds to zero), the E5M2
+// value rows without data zeroed (a weight of 0 times a stale Inf or NaN byte
+// would still poison the sum; key rows are masked by their -inf score), and,
+// for the first sub-chunk of an item that starts a softmax state, its query rows.
+template <int B, int D, class Cursor>
+__device__ __forceinline__ void attn_issue_rest(const AttnParams& a, const Cursor& c, long long hr, uint8_t* buf,
+                                                uint8_t* sq, int lane) {
+  using T = AttnTile<B, D>;
+  constexpr int SC = T::kSub, P = T::kRowBytes / 16;
+  uint8_t* const sv = buf + T::kBufK;
+  __half* const sks = reinterpret_cast<__half*>(buf + T::kBufK + T::kBufV);
+  __half* const svs = sks + SC * T::kScales;
+  if constexpr (T::kScales > 0) {
+    if (lane < SC) {
+      if (hr >= 0) {
+        cp_async_small<T::kScales * 2>(sks + lane * T::kScales, a.k_scales + hr * T::kScales);
+        cp_async_small<T::kScales * 2>(svs + lane * T::kScales, a.v_scales + hr * T::kScales);
+      } else {
+#pragma unroll
+        for (int e = 0; e < T::kScales; ++e)
+          sks[lane * T::kScales + e] = svs[lane * T::kScales + e] = __ushort_as_half(0);
+      }
+    }
+  } else {
+    if (lane < SC && hr < 0) {
+#pragma unroll
+      for (int part = 0; part < P; ++part)
+        *reinterpret_cast<uint4*>(sv + lane * T::kStrideV + part * 16) = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  if (c.sub == 0 && c.fresh) {
+    const __half* q = a.q + (static_cast<long long>(c.seq) * a.n_heads + static_cast<long long>(c.kvh) * a.group) * D;
+    for (int t = lane; t < a.group * D / 8; t += 32) cp_async16(sq + t * 16, q + t * 8);
+  }
+}
 
 // Issue the copies of one sub-chunk into a warp buffer (and, for the first
 // sub-chunk of an item, its query rows into the warp's query area); returns
 // the bit mask of its positions that hold data (bit i: position i).
+// A sub-chunk starts at a multiple of kSub positions.  When the cache is
+// contiguous or its page size is a multiple of kSub, the sub-chunk's rows are
+// consecutive cache rows: one block-table lookup for the warp, and every lane
+// copies fixed 16-byte parts of rows R apart.  Otherwise every lane resolves
+// its own position's row.
 template <int B, int D, class Cursor>
 __device__ __forceinline__ uint32_t attn_issue(const AttnParams& a, const Cursor& c, int offset, uint8_t* buf,
                                                uint8_t* sq, int lane) {
@@ -562,21 +665,53 @@ __device__ __forceinline__ uint32_t attn_issue(const AttnParams& a, const Cursor
   constexpr int SC = T::kSub, P = T::kRowBytes / 16;
   uint8_t* const sk = buf;
   uint8_t* const sv = buf + T::kBufK;
-  __half* const sks = reinterpret_cast<__half*>(buf + T::kBufK + T::kBufV);
-  __half* const svs = sks + SC * T::kScales;
-  // cache row of this lane's position (lanes < SC): -1 bad paging metadata, -2 past the window
+  const int p0 = c.chunk * T::kChunk + offset + c.sub * SC;  // first position of the sub-chunk
+  if (a.page_size == 0 || a.page_size % SC == 0) {
+    long long row0;
+    int n = c.n;
+    if (a.page_size == 0) {
+      row0 = static_cast<long long>(c.seq) * a.dim1 + p0;
+    } else {
+      const int lp = a.page_shift >= 0 ? p0 >> a.page_shift : p0 / a.page_size;
+      const int page = lp < a.bt_stride ? a.block_table[static_cast<long long>(c.seq) * a.bt_stride + lp] : -1;
+      if (page < 0 || page >= a.dim0) {
+        if (n > 0 && lane == 0) record_error(KVQ_DEV_BAD_PAGE);
+        n = 0;
+      }
+      row0 = static_cast<long long>(page) * a.page_size + (p0 - lp * a.page_size);
+    }
+    const long long hr0 = row0 * a.kv_heads + c.kvh;
+    // lane = (row rl of each group of R rows, 16-byte part pt); R * P <= 32 lanes busy
+    constexpr int R = 32 / P, NPASS = (SC + R - 1) / R;
+    const int rl = lane / P, pt = lane - rl * P;
+    if (lane < R * P && rl < n) {
+      const long long rstride = static_cast<long long>(a.kv_heads) * T::kRowBytes;
+      const long long off = (hr0 + static_cast<long long>(rl) * a.kv_heads) * T::kRowBytes + pt * 16;
+      const uint8_t* ks = a.k_codes + off;
+      const uint8_t* vs = a.v_codes + off;
+#pragma unroll
+      for (int k = 0; k < NPASS; ++k) {
+        const int r = rl + R * k;
+        if (r < n) {
+          cp_async16(sk + r * T::kStrideK + pt * 16, ks);
+          cp_async16(sv + r * T::kStrideV + pt * 16, vs);
+        }
+        ks += R * rstride;
+        vs += R * rstride;
+      }
+    }
+    attn_issue_rest<B, D>(a, c, lane < n ? hr0 + static_cast<long long>(lane) * a.kv_heads : -1, buf, sq, lane);
+    return n >= 32 ? 0xFFFFFFFFu : ((1u << n) - 1u);
+  }
+  // cache row of this lane's position (lanes < n): -1 bad paging metadata, -2 past the window
   long long hr = -2;
   if (lane < c.n) {
-    const int p = c.chunk * T::kChunk + offset + c.sub * SC + lane;
-    long long row;
-    if (a.page_size == 0) {
-      row = static_cast<long long>(c.seq) * a.dim1 + p;
-    } else {
-      const int lp = p / a.page_size;
-      const int page = lp < a.bt_stride ? a.block_table[static_cast<long long>(c.seq) * a.bt_stride + lp] : -1;
-      row = (page < 0 || page >= a.dim0) ? -1 : static_cast<long long>(page) * a.page_size + (p - lp * a.page_size);
-      if (row < 0) record_error(KVQ_DEV_BAD_PAGE);
-    }
+    const int p = p0 + lane;
+    const int lp = p / a.page_size;
+    const int page = lp < a.bt_stride ? a.block_table[static_cast<long long>(c.seq) * a.bt_stride + lp] : -1;
+    const long long row =
+        (page < 0 || page >= a.dim0) ? -1 : static_cast<long long>(page) * a.page_size + (p - lp * a.page_size);
+    if (row < 0) record_error(KVQ_DEV_BAD_PAGE);
     hr = row < 0 ? -1 : row * a.kv_heads + c.kvh;
   }
   const uint32_t mask = __ballot_sync(0xFFFFFFFFu, hr >= 0);
@@ -591,43 +726,28 @@ __device__ __forceinline__ uint32_t attn_issue(const AttnParams& a, const Cursor
       cp_async16(sv + r * T::kStrideV + part * 16, a.v_codes + src);
     }
   }
-  if constexpr (T::kScales > 0) {
-    // scales; rows without data get zero scales, which dequantize whatever codes
-    // the buffer holds to zero
-    if (lane < SC) {
-      if (hr >= 0) {
-        cp_async_small<T::kScales * 2>(sks + lane * T::kScales, a.k_scales + hr * T::kScales);
-        cp_async_small<T::kScales * 2>(svs + lane * T::kScales, a.v_scales + hr * T::kScales);
-      } else {
-#pragma unroll
-        for (int e = 0; e < T::kScales; ++e)
-          sks[lane * T::kScales + e] = svs[lane * T::kScales + e] = __ushort_as_half(0);
-      }
-    }
-  } else {
-    // E5M2 has no scale: a value row without data is zeroed (its weight is 0, but a
-    // stale Inf or NaN byte would still poison the weighted sum); key rows are masked
-    // by their -inf score instead
-    if (lane < SC && hr < 0) {
-#pragma unroll
-      for (int part = 0; part < P; ++part)
-        *reinterpret_cast<uint4*>(sv + lane * T::kStrideV + part * 16) = make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
-  // the item's query rows travel with its first sub-chunk
-  if (c.sub == 0) {
-    const __half* q = a.q + (static_cast<long long>(c.seq) * a.n_heads + static_cast<long long>(c.kvh) * a.group) * D;
-    for (int t = lane; t < a.group * D / 8; t += 32) cp_async16(sq + t * 16, q + t * 8);
-  }
+  attn_issue_rest<B, D>(a, c, hr, buf, sq, lane);
   return mask;
 }
 
-template <int B, int D, bool kCompact, bool kSplit>
+// Transpose of an 8 x 8 binary16 block held across the warp: lane 4r + c holds
+// elements (r, 2c) and (r, 2c + 1) of the block before and of its transpose after.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// kG4 (group <= 4): the query operand repeats the group's heads in columns 4..7,
+// so the lanes holding columns 4..7 compute the same weights as those holding
+// 0..3 and contribute the residual parts: one V^T P^T product per step carries
+// both parts (columns 0..3 high, 4..7 residual), summed when the item ends.
+template <int B, int D, bool kCompact, bool kSplit, bool kG4>
 __global__ void __launch_bounds__(kAttnThreads, D > 128 ? 2 : 4)
     attn_partial_kernel(const __grid_constant__ AttnParams a) {
   using T = AttnTile<B, D>;
   using Codec = AttnCodec<B>;
-  constexpr int KS = T::KS;  // k-steps of Q K^T, m-tiles of V^T P^T
+  constexpr int KS = T::KS;  // k-steps of K Q^T, m-tiles of V^T P^T
   constexpr int KR = D / 8;  // registers of one K span / one V span pair
   constexpr int SC = T::kSub;
 
@@ -653,7 +773,7 @@ __global__ void __launch_bounds__(kAttnThreads, D > 128 ? 2 : 4)
     int run = 0;
     for (int base = 0; base < a.batch; base += 32) {
       const int i = base + lane;
-      int n = i < a.batch ? (w0.length(i) + T::kChunk - 1) / T::kChunk * a.kv_heads : 0;
+      int n = i < a.batch ? (w0.length(i) + T::kChunk - 1) / T::kChunk * (Walk::kBlocked ? 1 : a.kv_heads) : 0;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int t = __shfl_up_sync(0xFFFFFFFFu, n, o);
@@ -667,20 +787,31 @@ __global__ void __launch_bounds__(kAttnThreads, D > 128 ? 2 : 4)
   }
   __syncthreads();  // the last CTA-wide barrier: from here on every warp walks its own items
 
-  const Walk walk{a, staged};
   uint8_t* const sq_area = wbuf + 2 * T::kBufBytes;
   const int offset = Walk::offset();
-  typename Walk::Cursor cur =
-      walk.seek(kSplit ? static_cast<typename Walk::Item>(blockIdx.x)
-                       : static_cast<typename Walk::Item>(blockIdx.x) * kAttnWarps + warp);
+  typename Walk::Item first = kSplit ? static_cast<typename Walk::Item>(blockIdx.x)
+                                     : static_cast<typename Walk::Item>(blockIdx.x) * kAttnWarps + warp;
+  Walk walk{a, staged};
+  if constexpr (Walk::kBlocked) {
+    // this warp's contiguous range of the U = (items of one kv head) x kv heads items
+    const long long U = static_cast<long long>(s_len[2 * T::kSeqlenSlots]) * a.kv_heads;
+    const long long W = static_cast<long long>(gridDim.x) * kAttnWarps;
+    const long long w = static_cast<long long>(blockIdx.x) * kAttnWarps + warp;
+    first = static_cast<typename Walk::Item>(w * U / W);
+    walk.end = static_cast<typename Walk::Item>((w + 1) * U / W);
+  }
+  typename Walk::Cursor cur = walk.seek(first);
   if (cur.item < 0) return;
   uint32_t mask_cur = attn_issue<B, D>(a, cur, offset, wbuf, sq_area, lane);
   asm volatile("cp.async.commit_group;\n" ::: "memory");
   int b = 0;
 
-  uint32_t qa0[KS], qa2[KS];
-  float m_ref = -INFINITY, l_part = 0.0f;
+  // This lane's score columns are 2j and 2j + 1: query heads 2j + e, or with kG4
+  // heads (2j + e) & 3.
+  uint32_t qb0[KS], qb1[KS];
+  float m_ref[2], l_part[2];
   float acc[KS][4];
+  int run_chunk = 0;  // the chunk whose entry receives the current softmax state
 
   // Per iteration: wait for the current sub-chunk, take the item's query
   // fragments if it starts here, issue the next sub-chunk's copies into the
@@ -688,23 +819,36 @@ __global__ void __launch_bounds__(kAttnThreads, D > 128 ? 2 : 4)
   while (true) {
     asm volatile("cp.async.wait_group 0;\n" ::: "memory");
     __syncwarp();
-    if (cur.sub == 0) {
-      // a new item: query fragments (A operand of Q K^T, rows = heads of the
-      // group, rows >= 8 zero; lane j's head_dim elements follow the K span
-      // order) and a fresh softmax state
+    if (cur.sub == 0 && !cur.fresh) {
+      // an item that continues the state: its own entry is marked empty (-inf maximum)
+      if ((!kG4 || j < 2) && g == 0) {
+        const long long head0 = static_cast<long long>(cur.seq) * a.n_heads + static_cast<long long>(cur.kvh) * a.group;
+        float* const entry = a.ws + (head0 * a.max_chunks + cur.chunk) * (D + 2);
+        const long long entry_stride = static_cast<long long>(a.max_chunks) * (D + 2);
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+          if (2 * j + e < a.group) entry[(2 * j + e) * entry_stride] = -INFINITY;
+      }
+    }
+    if (cur.sub == 0 && cur.fresh) {
+      // a new item: query fragments (B operand of K Q^T, column g = head g, or g & 3
+      // with kG4; heads past the group zero; head_dim elements in the K span order)
+      // and a fresh softmax state
       const __half(*sq)[D] = reinterpret_cast<const __half(*)[D]>(sq_area);
-      const bool live = g < a.group;
+      const int hq = kG4 ? (g & 3) : g;
+      const bool live = hq < a.group;
 #pragma unroll
       for (int s = 0; s < KS; ++s) {
         const int d00 = T::KN * j + Codec::row_pair_elem(2 * s, 0), d01 = T::KN * j + Codec::row_pair_elem(2 * s, 1);
         const int d10 = T::KN * j + Codec::row_pair_elem(2 * s + 1, 0);
         const int d11 = T::KN * j + Codec::row_pair_elem(2 * s + 1, 1);
-        const __half* qr = sq[live ? g : 0];
-        qa0[s] = live ? as_u32(__halves2half2(qr[d00], qr[d01])) : 0u;
-        qa2[s] = live ? as_u32(__halves2half2(qr[d10], qr[d11])) : 0u;
+        const __half* qr = sq[live ? hq : 0];
+        qb0[s] = live ? as_u32(__halves2half2(qr[d00], qr[d01])) : 0u;
+        qb1[s] = live ? as_u32(__halves2half2(qr[d10], qr[d11])) : 0u;
       }
-      m_ref = -INFINITY;
-      l_part = 0.0f;
+      m_ref[0] = m_ref[1] = -INFINITY;
+      l_part[0] = l_part[1] = 0.0f;
+      run_chunk = cur.chunk;
 #pragma unroll
       for (int mt = 0; mt < KS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.0f;
       if (cur.chunk == 0 && cur.kvh == 0 && lane == 0) {
@@ -727,64 +871,74 @@ __global__ void __launch_bounds__(kAttnThreads, D > 128 ? 2 : 4)
     const __half* const svs = sks + SC * T::kScales;
 
     for (int t0 = 0; t0 < cur.n; t0 += 16) {
-      // ---- S = Q K^T for positions t0 + 8t + (0..7): lane supplies position t0 + 8t + g
-      float sc[2][4];
+      // ---- S^T = K Q^T for positions t0 + g (rows g) and t0 + 8 + g (rows g + 8):
+      // this lane's K spans are the A fragments, the query the B fragment
+      float sc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      {
+        uint32_t ka[KR], kb[KR];
+        k_span<B, D>(sk + (t0 + g) * T::kStrideK, sks + (t0 + g) * T::kScales, j, ka);
+        k_span<B, D>(sk + (t0 + 8 + g) * T::kStrideK, sks + (t0 + 8 + g) * T::kScales, j, kb);
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const int i = t0 + 8 * t + g;
-        uint32_t kb[KR];
-        k_span<B, D>(sk + i * T::kStrideK, sks + i * T::kScales, j, kb);
-        sc[t][0] = sc[t][1] = sc[t][2] = sc[t][3] = 0.0f;
-#pragma unroll
-        for (int s = 0; s < KS; ++s) mma_16816(sc[t], qa0[s], 0u, qa2[s], 0u, kb[2 * s], kb[2 * s + 1]);
+        for (int s = 0; s < KS; ++s) mma_16816(sc, ka[2 * s], kb[2 * s], ka[2 * s + 1], kb[2 * s + 1], qb0[s], qb1[s]);
       }
-      // scores of head g at positions t0 + 8t + 2j + e (c0, c1); positions without data -inf
-      float p[2][2];
-      float mx = -INFINITY;
+      // x[e], x[2 + e]: scaled scores of column 2j + e at positions t0 + g and
+      // t0 + 8 + g; positions without data -inf (only a step with such
+      // positions pays for the mask)
+      float x[4];
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
+      for (int i = 0; i < 4; ++i) x[i] = sc[i] * a.scale_log2;
+      const uint32_t live16 = (mask_cur >> t0) & 0xFFFFu;
+      const bool full = live16 == 0xFFFFu;  // the same in every lane
+      if (!full) {
+        if (!((live16 >> g) & 1u)) x[0] = x[1] = -INFINITY;
+        if (!((live16 >> (g + 8)) & 1u)) x[2] = x[3] = -INFINITY;
+      }
+      // lazy rescale: the reference of a head moves only when the step's maximum
+      // exceeds it by more than the threshold; each lane tests its own scores and
+      // the warp takes the maximum only when one of them does
+      const bool grow = fmaxf(x[0], x[2]) > m_ref[0] + kAttnRescaleLog2 ||
+                        fmaxf(x[1], x[3]) > m_ref[1] + kAttnRescaleLog2;
+      if (__any_sync(0xFFFFFFFFu, grow)) {
+        float al[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int i = t0 + 8 * t + 2 * j + e;
-          const float v = ((mask_cur >> i) & 1u) ? sc[t][e] * a.scale_log2 : -INFINITY;
-          p[t][e] = v;
-          mx = fmaxf(mx, v);
+          float mx = fmaxf(x[e], x[2 + e]);
+          mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 16));
+          al[e] = 1.0f;
+          if (mx > m_ref[e] + kAttnRescaleLog2) {
+            al[e] = (m_ref[e] == -INFINITY) ? 0.0f : exp2_approx(m_ref[e] - mx);
+            m_ref[e] = mx;
+          }
+          l_part[e] *= al[e];
         }
-      }
-      mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 2));
-      // lazy rescale: move the reference only when a score exceeds it by more than the threshold
-      const bool grow = mx > m_ref + kAttnRescaleLog2;
-      if (__any_sync(0xFFFFFFFFu, grow)) {
-        const float m_new = grow ? mx : m_ref;
-        const float alpha = (m_ref == -INFINITY) ? 0.0f : exp2_approx(m_ref - m_new);
-        l_part *= alpha;
-        // accumulators hold heads 2j, 2j+1: their factors live in quads 2j, 2j+1
-        const float a0 = __shfl_sync(0xFFFFFFFFu, alpha, 8 * j);
-        const float a1 = __shfl_sync(0xFFFFFFFFu, alpha, 8 * j + 4);
+        // accumulator columns 2j, 2j + 1 belong to this lane's heads
 #pragma unroll
         for (int mt = 0; mt < KS; ++mt) {
-          acc[mt][0] *= a0;
-          acc[mt][1] *= a1;
-          acc[mt][2] *= a0;
-          acc[mt][3] *= a1;
-        }
-        m_ref = m_new;
-      }
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          p[t][e] = (p[t][e] == -INFINITY) ? 0.0f : exp2_approx(p[t][e] - m_ref);
-          l_part += p[t][e];
+          acc[mt][0] *= al[0];
+          acc[mt][1] *= al[1];
+          acc[mt][2] *= al[0];
+          acc[mt][3] *= al[1];
         }
       }
-      // ---- P^T B fragment: b0 = P[g][2j, 2j+1] (tile 0), b1 = P[g][8 + 2j, 8 + 2j + 1] (tile 1),
-      // as a binary16 high part and a binary16 residual
-      const uint32_t bh0 = pack_half2(p[0][0], p[0][1]), bh1 = pack_half2(p[1][0], p[1][1]);
-      const float2 f0 = __half22float2(as_h2(bh0)), f1 = __half22float2(as_h2(bh1));
-      const uint32_t bl0 = pack_half2(p[0][0] - f0.x, p[0][1] - f0.y);
-      const uint32_t bl1 = pack_half2(p[1][0] - f1.x, p[1][1] - f1.y);
+      float p[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) p[i] = exp2_approx(x[i] - m_ref[i & 1]);
+      if (!full) {
+        // a head with no data yet has reference -inf: its masked scores weigh 0
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (x[i] == -INFINITY) p[i] = 0.0f;
+      }
+      l_part[0] += p[0] + p[2];
+      l_part[1] += p[1] + p[3];
+      // ---- the weights as a binary16 high part and a binary16 residual; rows of
+      // the 8 x 8 blocks P[t0 + (0..7)][columns] and P[t0 + 8 + (0..7)][columns],
+      // transposed into the B fragments of P^T
+      const uint32_t h0 = pack_half2(p[0], p[1]), h1 = pack_half2(p[2], p[3]);
+      const float2 f0 = __half22float2(as_h2(h0)), f1 = __half22float2(as_h2(h1));
+      const uint32_t r0 = pack_half2(p[0] - f0.x, p[1] - f0.y), r1 = pack_half2(p[2] - f1.x, p[3] - f1.y);
 
       // ---- O^T += V^T P^T: row pairs (2j, 2j+1) and (2j+8, 2j+9) of the 16 positions
       uint32_t va[KR], vb[KR];
@@ -799,40 +953,65 @@ __global__ void __launch_bounds__(kAttnThreads, D > 128 ? 2 : 4)
         v_span_pair<B, D>(sv + i0 * T::kStrideV, sv + (i0 + 1) * T::kStrideV, s00, s01, g, va);
         v_span_pair<B, D>(sv + i1 * T::kStrideV, sv + (i1 + 1) * T::kStrideV, s10, s11, g, vb);
       }
+      if constexpr (kG4) {
+        // columns 0..3 the high parts, 4..7 (lanes j >= 2) the residuals
+        const uint32_t b0 = movmatrix_trans(j >= 2 ? r0 : h0), b1 = movmatrix_trans(j >= 2 ? r1 : h1);
 #pragma unroll
-      for (int mt = 0; mt < KS; ++mt) {
-        mma_16816(acc[mt], va[2 * mt], va[2 * mt + 1], vb[2 * mt], vb[2 * mt + 1], bh0, bh1);
-        mma_16816(acc[mt], va[2 * mt], va[2 * mt + 1], vb[2 * mt], vb[2 * mt + 1], bl0, bl1);
+        for (int mt = 0; mt < KS; ++mt) mma_16816(acc[mt], va[2 * mt], va[2 * mt + 1], vb[2 * mt], vb[2 * mt + 1], b0, b1);
+      } else {
+        const uint32_t bh0 = movmatrix_trans(h0), bh1 = movmatrix_trans(h1);
+        const uint32_t bl0 = movmatrix_trans(r0), bl1 = movmatrix_trans(r1);
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+          mma_16816(acc[mt], va[2 * mt], va[2 * mt + 1], vb[2 * mt], vb[2 * mt + 1], bh0, bh1);
+          mma_16816(acc[mt], va[2 * mt], va[2 * mt + 1], vb[2 * mt], vb[2 * mt + 1], bl0, bl1);
+        }
       }
     }
 
-    if (cur.last) {
-      // the item's partial result: (max, sum, accumulator) of every head of the group
-      float l_sum = l_part;
-      l_sum += __shfl_xor_sync(0xFFFFFFFFu, l_sum, 1);
-      l_sum += __shfl_xor_sync(0xFFFFFFFFu, l_sum, 2);
+    // the state is written when it ends: at the last sub-chunk of an item that the
+    // next one does not continue
+    if (cur.last && (nxt.item < 0 || nxt.fresh)) {
+      // the state's partial result: (max, sum, accumulator) of every head of the group
+      float l_sum[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float l = l_part[e];
+        l += __shfl_xor_sync(0xFFFFFFFFu, l, 4);
+        l += __shfl_xor_sync(0xFFFFFFFFu, l, 8);
+        l += __shfl_xor_sync(0xFFFFFFFFu, l, 16);
+        l_sum[e] = l;
+      }
+      if constexpr (kG4) {
+        // high part (lanes j < 2) plus residual (lanes j + 2)
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[mt][i] += __shfl_xor_sync(0xFFFFFFFFu, acc[mt][i], 2);
+      }
       const long long head0 = static_cast<long long>(cur.seq) * a.n_heads + static_cast<long long>(cur.kvh) * a.group;
-      float* const entry = a.ws + (head0 * a.max_chunks + cur.chunk) * (D + 2);
+      float* const entry = a.ws + (head0 * a.max_chunks + run_chunk) * (D + 2);
       const long long entry_stride = static_cast<long long>(a.max_chunks) * (D + 2);  // next head, same chunk
       // kSplit: the warp's quarter goes to its own buffer (free now: the next
       // sub-chunk streams into the other one), one (D + 2)-float row per head
       float* const ws = kSplit ? reinterpret_cast<float*>(wbuf + b * T::kBufBytes) : entry;
       const long long hstride = kSplit ? D + 2 : entry_stride;
       if (kSplit) __syncwarp();  // every lane is done reading the buffer
-      if (j == 0 && g < a.group) {
-        ws[g * hstride] = m_ref;
-        ws[g * hstride + 1] = l_sum;
-      }
+      if (!kG4 || j < 2) {
 #pragma unroll
-      for (int mt = 0; mt < KS; ++mt) {
-        const int da = T::VN * g + Codec::xrow_elem(2 * mt), db = T::VN * g + Codec::xrow_elem(2 * mt + 1);
-        if (2 * j < a.group) {
-          ws[(2 * j) * hstride + 2 + da] = acc[mt][0];
-          ws[(2 * j) * hstride + 2 + db] = acc[mt][2];
-        }
-        if (2 * j + 1 < a.group) {
-          ws[(2 * j + 1) * hstride + 2 + da] = acc[mt][1];
-          ws[(2 * j + 1) * hstride + 2 + db] = acc[mt][3];
+        for (int e = 0; e < 2; ++e) {
+          const int h = 2 * j + e;
+          if (h < a.group) {
+            if (g == 0) {
+              ws[h * hstride] = m_ref[e];
+              ws[h * hstride + 1] = l_sum[e];
+            }
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+              ws[h * hstride + 2 + T::VN * g + Codec::xrow_elem(2 * mt)] = acc[mt][e];
+              ws[h * hstride + 2 + T::VN * g + Codec::xrow_elem(2 * mt + 1)] = acc[mt][2 + e];
+            }
+          }
         }
       }
       if constexpr (kSplit) {
@@ -873,8 +1052,8 @@ __global__ void __launch_bounds__(kAttnThreads, D > 128 ? 2 : 4)
   }
 }
 
-// Merge the chunks of every (sequence, head): CTA (head, sequence) of four
-// warps.  Warp w takes chunks w, w + 4, ... in batches of kCombineBatch<D>
+// Merge the chunk entries of every (sequence, head): CTA (head, sequence) of
+// four warps.  Warp w takes chunks w, w + 4, ... in batches of kCombineBatch<D>
 // whose loads are all issued before any is used (lane l owns head_dim elements
 // l, l + 32, ...), and folds each batch into a running (max, sum, accumulator)
 // that it rescales when the maximum moves; the four warps' results meet in
@@ -909,9 +1088,16 @@ __global__ void __launch_bounds__(kCombineThreads, 8) attn_combine_kernel(const 
       const bool in = c < nch;
       const float* e = ws + (in ? c : 0) * (D + 2);
       mc[i] = in ? e[0] : -INFINITY;
-      lc[i] = in ? e[1] : 0.0f;
+    }
 #pragma unroll
-      for (int k = 0; k < DPL; ++k) x[i][k] = in ? e[2 + lane + 32 * k] : 0.0f;
+    for (int i = 0; i < NB; ++i) {
+      // an entry with a -inf maximum holds nothing (no data, or merged into an earlier entry)
+      const long long c = c0 + static_cast<long long>(i) * kWarps;
+      const bool live = mc[i] != -INFINITY;
+      const float* e = ws + (live ? c : 0) * (D + 2);
+      lc[i] = live ? e[1] : 0.0f;
+#pragma unroll
+      for (int k = 0; k < DPL; ++k) x[i][k] = live ? e[2 + lane + 32 * k] : 0.0f;
     }
     float mb = m_run;
 #pragma unroll

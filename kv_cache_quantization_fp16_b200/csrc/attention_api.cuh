@@ -75,14 +75,14 @@ long long attn_max_chunks(const kvq_cache_desc* d, int page_size, int chunk) {
 
 // Dynamic shared memory opt-in, once per device for each partial kernel
 // (static plus dynamic shared memory above 48 KB needs it).
-template <int B, int D, bool kCompact, bool kSplit>
+template <int B, int D, bool kCompact, bool kSplit, bool kG4>
 bool allow_attention_smem() {
   constexpr int kMaxDevices = 64;
   static std::atomic<bool> done[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
   if (done[dev].load()) return true;
-  if (cudaFuncSetAttribute(kvq::attn_partial_kernel<B, D, kCompact, kSplit>,
+  if (cudaFuncSetAttribute(kvq::attn_partial_kernel<B, D, kCompact, kSplit, kG4>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            kvq::AttnTile<B, D>::kSmemBytes) != cudaSuccess) {
     cudaGetLastError();
@@ -94,34 +94,44 @@ bool allow_attention_smem() {
 
 // CTAs of a partial kernel the device holds at once (occupancy cached per
 // device), 0 on failure.
-template <int B, int D, bool kCompact, bool kSplit>
+template <int B, int D, bool kCompact, bool kSplit, bool kG4>
 long long partial_ctas() {
-  if (!allow_attention_smem<B, D, kCompact, kSplit>()) return 0;
+  if (!allow_attention_smem<B, D, kCompact, kSplit, kG4>()) return 0;
   constexpr int kMaxDevices = 64;
   static std::atomic<long long> resident[kMaxDevices];
-  return first_wave_ctas(kvq::attn_partial_kernel<B, D, kCompact, kSplit>, kvq::kAttnThreads,
+  return first_wave_ctas(kvq::attn_partial_kernel<B, D, kCompact, kSplit, kG4>, kvq::kAttnThreads,
                          kvq::AttnTile<B, D>::kSmemBytes, resident, kMaxDevices);
 }
 
 // Persistent grid of the partial kernel: every (sequence, 256-position chunk,
 // kv head) work item goes to one warp (to one CTA with kSplit); as many CTAs
 // as the device holds at once, never more than there are item slots.
-template <int B, int D, bool kCompact, bool kSplit>
+template <int B, int D, bool kCompact, bool kSplit, bool kG4>
 kvq_status launch_partial(const kvq::AttnParams& a, long long items, long long ctas_max, void* stream) {
   using T = kvq::AttnTile<B, D>;
   if (ctas_max < 1) return KVQ_ERR_CUDA;
   const long long need = kSplit ? items : (items + kvq::kAttnWarps - 1) / kvq::kAttnWarps;
-  const unsigned grid = static_cast<unsigned>(need < ctas_max ? need : ctas_max);
-  return launch_pdl(kvq::attn_partial_kernel<B, D, kCompact, kSplit>, dim3(grid), kvq::kAttnThreads, T::kSmemBytes,
-                    stream, a);
+  const long long grid = need < ctas_max ? need : ctas_max;
+  return launch_pdl(kvq::attn_partial_kernel<B, D, kCompact, kSplit, kG4>, dim3(static_cast<unsigned>(grid)),
+                    kvq::kAttnThreads, T::kSmemBytes, stream, a);
 }
 
-// The partial kernel walks only the items that hold data when the batch fits
-// its shared-memory slots and every item count fits an int; otherwise it
-// visits every item slot.  When the cache geometry has no more item slots
+// The partial kernel for every walk: only the items that hold data when the
+// batch fits its shared-memory slots and every item count fits an int,
+// otherwise every item slot.  When the cache geometry has no more item slots
 // than the device holds CTAs (batches of one or two long sequences; head_dim
 // <= 128), the four warps of a CTA share each item (measured: 10% faster
-// there, slower from two items per CTA on).  Then the combine kernel.
+// there, slower from two items per CTA on).
+template <int B, int D, bool kG4>
+kvq_status launch_partial_walk(const kvq::AttnParams& a, long long items, bool compact, void* stream) {
+  if (!compact) return launch_partial<B, D, false, false, kG4>(a, items, partial_ctas<B, D, false, false, kG4>(), stream);
+  const long long ctas = partial_ctas<B, D, true, false, kG4>();
+  if (D <= 128 && items <= ctas)
+    return launch_partial<B, D, true, D <= 128, kG4>(a, items, partial_ctas<B, D, true, D <= 128, kG4>(), stream);
+  return launch_partial<B, D, true, false, kG4>(a, items, ctas, stream);
+}
+
+// The partial kernel (tcgen05 or mma.sync), then the combine kernel.
 template <int B, int D>
 kvq_status launch_attention(kvq::AttnParams a, const kvq_cache_desc* desc, void* stream) {
   using T = kvq::AttnTile<B, D>;
@@ -136,6 +146,9 @@ kvq_status launch_attention(kvq::AttnParams a, const kvq_cache_desc* desc, void*
   if constexpr (D == kvq::kTcD) {
     // the tcgen05 kernel: head_dim 128, batches its shared memory stages (<= 256 sequences)
     if (path == KVQ_ATTENTION_TCGEN05 && compact) {
+      // kTcItem-position entries: every one of them is written
+      a.chunk = kvq::kTcItem;
+      a.max_chunks = static_cast<int>(attn_max_chunks(desc, a.page_size, kvq::kTcItem));
       switch (a.group) {
         case 1: st = launch_tc<B, 1>(a, items, stream); break;
         case 2: st = launch_tc<B, 2>(a, items, stream); break;
@@ -150,15 +163,8 @@ kvq_status launch_attention(kvq::AttnParams a, const kvq_cache_desc* desc, void*
       return launch_pdl(kvq::attn_combine_kernel<D>, dim3(a.n_heads, a.batch), kvq::kCombineThreads, 0, stream, a);
     }
   }
-  if (!compact) {
-    st = launch_partial<B, D, false, false>(a, items, partial_ctas<B, D, false, false>(), stream);
-  } else {
-    const long long ctas = partial_ctas<B, D, true, false>();
-    if (D <= 128 && items <= ctas)
-      st = launch_partial<B, D, true, D <= 128>(a, items, partial_ctas<B, D, true, D <= 128>(), stream);
-    else
-      st = launch_partial<B, D, true, false>(a, items, ctas, stream);
-  }
+  st = a.group <= 4 ? launch_partial_walk<B, D, true>(a, items, compact, stream)
+                    : launch_partial_walk<B, D, false>(a, items, compact, stream);
   if (st != KVQ_OK) return st;
   return launch_pdl(kvq::attn_combine_kernel<D>, dim3(a.n_heads, a.batch), kvq::kCombineThreads, 0, stream, a);
 }
@@ -246,6 +252,9 @@ kvq_status decode_attention(const void* q, const void* k_codes, const void* k_sc
   a.group = n_heads / desc->kv_heads;
   a.page_size = page_size;
   a.bt_stride = desc->block_table_stride;
+  a.page_shift = -1;
+  for (int sh = 0; sh < 31; ++sh)
+    if (page_size == (1 << sh)) a.page_shift = sh;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
   if (format == 4) return launch_attention_b<4>(a, desc, stream);
   if (format == 6) return launch_attention_b<6>(a, desc, stream);

@@ -20,9 +20,10 @@ the kernels perform (csrc/attention.cuh):
   maxima that feed them (at most five levels, each below u times the score range);
 * the weights enter P . V as a binary16 high part plus a binary16 residual (relative
   2^-22, and an absolute 2^-25 of the item's largest weight once the residual is
-  subnormal: at most 2^-17 of the weight sum over a 256-position item), summed by the
-  tensor core in 2 steps per 16 positions (32 steps per item), and the weight sums
-  and merges in binary32;
+  subnormal: at most 2^-17 of the weight sum over one softmax state, which spans at
+  most 256 positions), summed by the tensor core in 2 steps per 16 positions (32 steps
+  per state), and the weight sums and the merges of up to ceil(n / 128) workspace
+  entries (one per 128-position chunk) in binary32;
 * the final binary32 division and the rounding to binary16 (half an ulp).
 
 Each weight the kernels use is w_p * (1 + r_p) up to a common factor, with
@@ -47,8 +48,9 @@ import numpy as np
 U = 2.0 ** -24                # binary32 unit roundoff
 EPS_EXP2 = 2.0 ** -21         # bound on the relative error of ex2.approx.ftz and of exp2f (self-check)
 MMA_STEP_ULPS = 18.0          # one mma.sync step: error below this many 2^-23 of its largest term (self-check)
-CHUNK = 256                   # positions per work item
-STEPS_PER_ITEM = CHUNK // 16  # softmax steps (and lazy-rescale opportunities) per item
+CHUNK = 256                   # positions one softmax state spans at most
+ENTRY = 128                   # positions per workspace entry (the entries merged per output)
+STEPS_PER_ITEM = CHUNK // 16  # softmax steps (and lazy-rescale opportunities) per state
 LOG2E = 1.4426950408889634
 
 
@@ -71,7 +73,7 @@ def attention_bound(q, K, V, group, scale):
     tol = np.zeros((NH, D))
     if n == 0:
         return o, tol
-    nch = math.ceil(n / CHUNK)
+    nch = math.ceil(n / ENTRY)
     n_b = math.ceil(math.ceil(nch / 4) / (1024 // D))  # batch rescales per warp in the chunk merge
     gamma_s = MMA_STEP_ULPS * 2.0 ** -23 * (D / 16)
     gamma_n = MMA_STEP_ULPS * 2.0 ** -23 * (2 * STEPS_PER_ITEM) * (1 + 2.0 ** -10)

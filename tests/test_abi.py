@@ -138,12 +138,12 @@ def test_decode_attention_validation(kvq):
     P = [FAKE] * 6  # q, k_codes, k_scales, v_codes, v_scales, out
     ws = kvq.attention_workspace_bytes((2, 16, 2, 64), 2, 4)
     assert ws == L.kvq_decode_attention_workspace_size(by(d), 2, 4, 0) > 0
-    # one (2 + head_dim)-float entry per (sequence, query head, 256-position chunk slot)
+    # one (2 + head_dim)-float entry per (sequence, query head, 128-position chunk slot)
     assert ws == 2 * 4 * 1 * (2 + 64) * 4
     big = _desc(kvq, d0=64, d1=16384, H=8, D=128)
-    assert L.kvq_decode_attention_workspace_size(by(big), 64, 32, 0) == 64 * 32 * 64 * 130 * 4
+    assert L.kvq_decode_attention_workspace_size(by(big), 64, 32, 0) == 64 * 32 * 128 * 130 * 4
     paged = _desc(kvq, d0=2048, d1=256, H=8, D=128, stride=65)
-    assert L.kvq_decode_attention_workspace_size(by(paged), 32, 32, 256) == 32 * 32 * 65 * 130 * 4
+    assert L.kvq_decode_attention_workspace_size(by(paged), 32, 32, 256) == 32 * 32 * 130 * 130 * 4
 
     def call(*args, desc=d, bs=2, nh=4, ps=0, lens=FAKE, bt=None, wbits=4, wsp=FAKE, wsb=ws):
         return L.kvq_decode_attention_q(*(args or P), by(desc) if desc else None, bs, nh, ps, lens, bt, wbits,
@@ -234,7 +234,7 @@ def test_scratch_size_matches_the_header(kvq):
     # the size check, one entry more is refused (host-side validation only)
     L = kvq.library()
     by = ctypes.byref
-    d = _desc(kvq, d0=1, d1=256, H=1, D=126)  # one 256-position chunk, 128 floats per entry
+    d = _desc(kvq, d0=1, d1=128, H=1, D=126)  # one 128-position chunk, 128 floats per entry
     per_head = L.kvq_decode_attention_workspace_size(by(d), 1, 1, 0)
     assert per_head == 128 * 4
     heads_fit = kvq.ATTENTION_SCRATCH_BYTES // per_head

@@ -80,7 +80,7 @@ def test_noalloc_rejects_geometry_beyond_the_scratch(kvq):
     dev = torch.device("cuda:0")
     q, kc, ks, vc, vs, lens, bt = _case(kvq, dev, 13, 4, 0)
     B, NH, D = q.shape
-    # 64 sequences x 64 query heads x 1M positions need far more than 16 MiB of workspace
+    # 64 sequences x 64 query heads x 1M positions need far more than 32 MiB of workspace
     desc = kvq._Desc(64, 1 << 20, 8, D, 0)
     assert kvq.library().kvq_decode_attention_workspace_size(ctypes.byref(desc), 64, 64, 0) > \
         kvq.ATTENTION_SCRATCH_BYTES

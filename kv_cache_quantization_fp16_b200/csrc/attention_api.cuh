@@ -118,15 +118,15 @@ kvq_status launch_partial(const kvq::AttnParams& a, long long items, long long c
 
 // The partial kernel for every walk: only the items that hold data when the
 // batch fits its shared-memory slots and every item count fits an int,
-// otherwise every item slot.  When the cache geometry has no more item slots
-// than the device holds CTAs (batches of one or two long sequences; head_dim
-// <= 128), the four warps of a CTA share each item (measured: 10% faster
-// there, slower from two items per CTA on).
+// otherwise every item slot.  When the cache geometry has no more 256-position
+// item slots than the device holds CTAs (batches of one or two long sequences;
+// head_dim <= 128), the four warps of a CTA share each item (measured: 10%
+// faster there, slower from two 256-position items per CTA on).
 template <int B, int D, bool kG4>
 kvq_status launch_partial_walk(const kvq::AttnParams& a, long long items, bool compact, void* stream) {
   if (!compact) return launch_partial<B, D, false, false, kG4>(a, items, partial_ctas<B, D, false, false, kG4>(), stream);
   const long long ctas = partial_ctas<B, D, true, false, kG4>();
-  if (D <= 128 && items <= ctas)
+  if (D <= 128 && items * kvq::AttnTile<B, D>::kChunk <= ctas * 256)
     return launch_partial<B, D, true, D <= 128, kG4>(a, items, partial_ctas<B, D, true, D <= 128, kG4>(), stream);
   return launch_partial<B, D, true, false, kG4>(a, items, ctas, stream);
 }

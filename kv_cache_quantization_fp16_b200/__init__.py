@@ -521,7 +521,7 @@ ATTENTION_SCRATCH_BYTES = 32 << 20  # KVQ_ATTENTION_SCRATCH_BYTES
 def decode_attention_q_noalloc(q, k_codes, k_scales, v_codes, v_scales, out, batch_size, cache_seqlens, wbits,
                                softmax_scale, page_size=0, block_table=None) -> None:
     """decode_attention_q for callers that cannot allocate device memory at the call
-    site: the workspace is the library's own 16 MiB array (one per device), so nothing is
+    site: the workspace is the library's own 32 MiB array (one per device), so nothing is
     allocated, by torch or by CUDA.  Geometries needing more workspace than
     ATTENTION_SCRATCH_BYTES are rejected.  Calls that overlap on the GPU share the array
     and race; make the first call on a device before any stream capture."""

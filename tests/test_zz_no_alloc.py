@@ -89,7 +89,7 @@ def test_noalloc_rejects_geometry_beyond_the_scratch(kvq):
                                             q.data_ptr(), ctypes.byref(desc), 64, 64, 0, lens.data_ptr(), None, 4,
                                             ctypes.c_float(1.0), None)
     assert st == 4  # KVQ_ERR_RANGE, nothing enqueued
-    # 64 sequences x 128 query heads x four 256-position chunk slots x 130 floats: 17.0 MB
+    # 64 sequences x 128 query heads x eight 128-position chunk slots x 130 floats: 34.1 MB
     big_q = torch.zeros(64, 128, D, dtype=torch.float16, device=dev)
     with pytest.raises(ValueError, match="scratch"):
         kvq.decode_attention_q_noalloc(big_q, kc, ks, vc, vs, torch.empty_like(big_q), 64,

@@ -263,6 +263,20 @@ def test_small_batches_long_sequences(kvq, oracle_mod, dev):
         check(kvq, oracle_mod, q, kc, ks, vc, vs, lens, 4, 1.0 / math.sqrt(D), dev)
 
 
+@pytest.mark.parametrize("wbits,NH", [(6, 64), (4, 64), (6, 16)])
+def test_split_items_pair_of_chunks(kvq, oracle_mod, dev, wbits, NH):
+    """Small batches take the CTA-shared split walk, whose items are 256 positions: for
+    4- and 6-bit codes a pair of 128-position chunks whose second entry is marked empty.
+    Lengths end inside an item's first chunk, exactly at its boundary, and inside its
+    second chunk; groups of 8 and of 2 query heads per kv head."""
+    B, S, H, D = 3, 1500, 8, 128
+    k, v = workloads.normal_kv((B, S, H, D), 71 + wbits + NH)
+    kc, ks, vc, vs = quantize_on_gpu(kvq, k, v, wbits, dev)
+    lens = torch.tensor([1290, 1280, 1201], dtype=torch.int32)  # 5 x 256 + 10, + 0, 4 x 256 + 177
+    q = torch.randn(B, NH, D, generator=torch.Generator().manual_seed(72)).half()
+    check(kvq, oracle_mod, q, kc, ks, vc, vs, lens, wbits, 1.0 / math.sqrt(D), dev)
+
+
 def test_bad_paging_reported(kvq, dev):
     ps, H, D = 16, 1, 64
     k, v = workloads.small(shape=(4, ps, H, D))

@@ -277,6 +277,20 @@ def test_split_items_pair_of_chunks(kvq, oracle_mod, dev, wbits, NH):
     check(kvq, oracle_mod, q, kc, ks, vc, vs, lens, wbits, 1.0 / math.sqrt(D), dev)
 
 
+@pytest.mark.parametrize("wbits", [4, 8])
+def test_all_sequences_empty(kvq, oracle_mod, dev, wbits):
+    """Every window empty, on each walk: a batch of 2 (the split walk), of 200 (the blocked
+    or round-robin walk) and of 300 (the slot walk, over 256 sequences).  Every output is
+    0, over a workspace of garbage that no kernel may read."""
+    for B in (2, 200, 300):
+        S, H, D, NH = 512, 8, 64, 16
+        k, v = workloads.normal_kv((B, S, H, D), 80 + B)
+        kc, ks, vc, vs = quantize_on_gpu(kvq, k, v, wbits, dev)
+        lens = torch.zeros(B, dtype=torch.int32)
+        q = torch.randn(B, NH, D, generator=torch.Generator().manual_seed(81)).half()
+        check(kvq, oracle_mod, q, kc, ks, vc, vs, lens, wbits, 1.0 / math.sqrt(D), dev)
+
+
 def test_bad_paging_reported(kvq, dev):
     ps, H, D = 16, 1, 64
     k, v = workloads.small(shape=(4, ps, H, D))

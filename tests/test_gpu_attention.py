@@ -172,7 +172,7 @@ def test_contiguous(kvq, oracle_mod, dev, wbits, D, H, NH):
 
 
 @pytest.mark.parametrize("wbits", [4, 6, 8])
-@pytest.mark.parametrize("ps", [256, 16, 7])
+@pytest.mark.parametrize("ps", [256, 96, 16, 7])
 def test_paged(kvq, oracle_mod, dev, wbits, ps):
     pool = workloads.paged_pool(num_pages=4000 // ps + 40, page_size=ps, heads=2, head_dim=128, batch=5,
                                 max_len=700)
@@ -352,7 +352,7 @@ def test_fp8_contiguous(kvq, oracle_mod, dev, D, H, NH):
     assert same > 0.9
 
 
-@pytest.mark.parametrize("ps", [256, 16, 7])
+@pytest.mark.parametrize("ps", [256, 96, 16, 7])
 def test_fp8_paged(kvq, oracle_mod, dev, ps):
     pool = workloads.paged_pool(num_pages=4000 // ps + 40, page_size=ps, heads=2, head_dim=128, batch=5,
                                 max_len=700)

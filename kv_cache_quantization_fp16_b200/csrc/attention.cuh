@@ -10,37 +10,39 @@
 // code 0), the E5M2 bytes decoded exactly as fp8_to_fp16 does.
 //
 // Split-K flash decoding.  Kernel 1 (attn_partial_kernel) is a persistent
-// grid (one wave of CTAs of four warps).  Every (sequence, 256-position chunk,
-// kv head) that holds data is a work item; warp w of W takes items w, w + W,
-// ... of a compact enumeration of them, so the warps' shares differ by at most
-// one item.  (When there are no more items than CTAs, the four warps of a CTA
-// take a quarter of each item instead and merge the quarters in shared
-// memory.)  A warp streams its part of an item through two shared-memory
-// buffers of 16 or 32 positions (cp.async copies of K and V codes, scales
-// and, with the first sub-chunk, the group's query rows), filling one while it
-// computes on the other, 16 positions at a time:
-//   * S = Q K^T on mma.sync m16n8k16 with the query heads as the M dimension
-//     (rows >= group are zero) and 8 positions per N tile: each lane
-//     dequantizes one contiguous span of D/4 elements of one position (a B
-//     fragment needs 4 head_dim elements per k-step, and the head_dim order
-//     inside the MMA is permuted so that a lane's elements over all k-steps
-//     are that span); the query fragments use the same permutation;
+// grid (one wave of CTAs of four warps).  Every (sequence, chunk, kv head)
+// that holds data is a work item (128-position chunks for 4- and 6-bit codes,
+// 256 for 8-bit codes and E5M2); warps take them from a compact enumeration,
+// in contiguous ranges or round-robin depending on the format (AttnWalk).
+// (When there are few items, the four warps of a CTA take a quarter of each
+// item instead and merge the quarters in shared memory.)  A warp streams its
+// items through two shared-memory buffers of 16 or 32 positions (cp.async
+// copies of K and V codes, scales and, with an item's first sub-chunk, the
+// group's query rows), filling one while it computes on the other, 16
+// positions at a time:
+//   * S^T = K Q^T on mma.sync m16n8k16 with the cache rows as the A operand
+//     (16 positions) and the query heads as the N columns: each lane
+//     dequantizes one contiguous span of D/4 elements of each of its two
+//     positions (the head_dim order inside the MMA is permuted so that a
+//     lane's elements over all k-steps are that span); the query fragments
+//     use the same permutation;
 //   * online softmax (base 2) per query head with lazy rescaling: the
 //     reference maximum only moves when a score exceeds it by more than
 //     kAttnRescaleLog2, so the accumulators are rarely touched and every
 //     weight stays below 2^kAttnRescaleLog2;
-//   * O^T += V^T P^T: the S accumulators of two N tiles are exactly the B
-//     fragment of P^T for a 16-position k-step (no data movement); P is split
-//     into a binary16 high part and a binary16 residual (two MMAs), so the
-//     weights keep about 22 significant bits; V^T A fragments pair two
-//     positions at one head_dim index, built by interleaving the bytes of two
-//     rows before the codes are unpacked.
+//   * O^T += V^T P^T: the weights, split into a binary16 high part and a
+//     binary16 residual (about 22 significant bits), are transposed into the
+//     B fragment of P^T with movmatrix; for groups of up to four query heads
+//     one MMA carries both parts (columns 0-3 and 4-7); V^T A fragments pair
+//     two positions at one head_dim index, built by interleaving the bytes of
+//     two rows before the codes are unpacked.
 // Code unpacking avoids per-code shifts: `(w & 0x000F000F) | 0x64006400` is
 // the binary16 pair (1024 + c0, 1024 + c4) of a Q4 word, and the high-nibble
 // pair is 16x that, brought back exactly with an FMA by 1/16.
-// At the end of an item the warp writes its (max, sum, accumulator) per query
-// head to the workspace entry of that chunk.  Kernel 2 (attn_combine_kernel)
-// merges the chunks of each (sequence, head) and writes binary16 outputs.
+// When a softmax state ends the warp writes its (max, sum, accumulator) per
+// query head to the workspace entry of the state's first chunk.  Kernel 2
+// (attn_combine_kernel) merges the entries of each (sequence, head) and writes
+// binary16 outputs.
 #pragma once
 
 #include <type_traits>
@@ -287,12 +289,14 @@ struct AttnCodec<6> {
 };
 
 // Per-warp shared-memory staging.  A work item is one (sequence, kv head,
-// 256-position chunk: 128 measured 3-16% slower from per-item costs, 512
-// 25% slower from load imbalance); a warp streams it through two buffers of kSub
-// positions each (K codes, V codes, K scales, V scales), filling one while it
-// computes on the other.  Row strides are padded where that removes bank
-// conflicts of the fragment reads (K: one span per lane of eight consecutive
-// rows; V: four rows per lane, byte-interleaved in pairs).
+// kChunk-position chunk): 128 positions for 4- and 6-bit codes, whose walk
+// carries one softmax state over pairs of chunks, and 256 for 8-bit codes and
+// E5M2 (512 measured 25% slower from load imbalance).  A warp streams it
+// through two buffers of kSub positions each (K codes, V codes, K scales, V
+// scales), filling one while it computes on the other.  Row strides are padded
+// where that removes bank conflicts of the fragment reads (K: one span per
+// lane of two rows eight apart; V: four rows per lane, byte-interleaved in
+// pairs).
 template <int B, int D>
 struct AttnTile {
   static constexpr int kBits = B == 0 ? 8 : B;  // bits per cached element (format 0: E5M2 bytes)

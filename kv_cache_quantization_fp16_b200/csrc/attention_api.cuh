@@ -103,9 +103,9 @@ long long partial_ctas() {
                          kvq::AttnTile<B, D>::kSmemBytes, resident, kMaxDevices);
 }
 
-// Persistent grid of the partial kernel: every (sequence, 256-position chunk,
-// kv head) work item goes to one warp (to one CTA with kSplit); as many CTAs
-// as the device holds at once, never more than there are item slots.
+// Persistent grid of the partial kernel: every (sequence, chunk, kv head) work
+// item goes to one warp (to one CTA with kSplit); as many CTAs as the device
+// holds at once, never more than there are item slots.
 template <int B, int D, bool kCompact, bool kSplit, bool kG4>
 kvq_status launch_partial(const kvq::AttnParams& a, long long items, long long ctas_max, void* stream) {
   using T = kvq::AttnTile<B, D>;
@@ -185,7 +185,7 @@ size_t kvq_decode_attention_workspace_size(const kvq_cache_desc* desc, int batch
   if (!desc || batch_size < 0 || n_heads < 0 || page_size < 0 || desc->head_dim < 0 || desc->dim1 < 0 ||
       desc->block_table_stride < 0)
     return 0;
-  // one entry per (sequence, query head, 256-position chunk slot); SIZE_MAX when that overflows
+  // one entry per (sequence, query head, 128-position chunk slot); SIZE_MAX when that overflows
   const long long chunks = attn_max_chunks(desc, page_size, kvq::kAttnMinChunk);
   size_t n = static_cast<size_t>(batch_size);
   if (__builtin_mul_overflow(n, static_cast<size_t>(n_heads), &n) ||

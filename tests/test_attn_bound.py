@@ -35,25 +35,29 @@ def _encode_fp8(oracle_mod, k, v):
     return k8, v8, ky.view(np.float16).astype(np.float64), vy.view(np.float16).astype(np.float64)
 
 
-def _emulate_fp32(q, K, V, group, scale):
-    """A binary32 computation with the kernels' structure: 256-position items of 16-position
-    steps, binary32 scores, lazy rescaling (threshold 2^8), 2^x in binary32, weights split
-    into a binary16 high part and residual for the value sum, binary32 sums; the items merged
-    in binary32; the result rounded to binary16."""
+def _emulate_fp32(q, K, V, group, scale, states=None, split_sums=False):
+    """A binary32 computation with the kernels' structure: softmax states over spans of
+    16-position steps (`states`: (first, end) position spans, 256-position items by
+    default), binary32 scores, lazy rescaling (threshold 2^8), 2^x in binary32, weights
+    split into a binary16 high part and residual for the value sum (`split_sums`: the two
+    parts summed apart and added when the state ends, as for groups of up to four query
+    heads), binary32 sums; the states merged in binary32; the result rounded to binary16."""
     f32 = np.float32
     NH, D = q.shape
     n = K.shape[0]
     out = np.zeros((NH, D), np.float64)
     c = f32(f32(scale) * f32(attn_bound.LOG2E))
+    if states is None:
+        states = [(c0, min(n, c0 + attn_bound.CHUNK)) for c0 in range(0, n, attn_bound.CHUNK)]
     for h in range(NH):
         kvh = h // group
         qh = q[h].astype(f32)
         parts = []
-        for c0 in range(0, n, attn_bound.CHUNK):
-            m, l, acc = f32(-np.inf), f32(0), np.zeros(D, f32)
-            for t0 in range(c0, min(n, c0 + attn_bound.CHUNK), 16):
-                kk = K[t0:t0 + 16, kvh].astype(f32)
-                vv = V[t0:t0 + 16, kvh].astype(f32)
+        for c0, c1 in states:
+            m, l, acc, acc_lo = f32(-np.inf), f32(0), np.zeros(D, f32), np.zeros(D, f32)
+            for t0 in range(c0, c1, 16):
+                kk = K[t0:min(t0 + 16, c1), kvh].astype(f32)
+                vv = V[t0:min(t0 + 16, c1), kvh].astype(f32)
                 s = np.array([np.sum(kk[i] * qh, dtype=f32) for i in range(kk.shape[0])], f32)
                 x = (s * c).astype(f32)
                 mx = x.max()
@@ -61,13 +65,18 @@ def _emulate_fp32(q, K, V, group, scale):
                     alpha = f32(0) if m == -np.inf else f32(np.exp2(f32(m - mx)))
                     l = f32(l * alpha)
                     acc = (acc * alpha).astype(f32)
+                    acc_lo = (acc_lo * alpha).astype(f32)
                     m = mx
                 p = np.exp2((x - m).astype(f32)).astype(f32)
                 hi = p.astype(np.float16).astype(f32)
                 lo = (p - hi).astype(np.float16).astype(f32)
                 l = f32(l + np.sum(p, dtype=f32))
-                acc = (acc + ((hi + lo)[:, None] * vv).sum(axis=0, dtype=f32)).astype(f32)
-            parts.append((m, l, acc))
+                if split_sums:
+                    acc = (acc + (hi[:, None] * vv).sum(axis=0, dtype=f32)).astype(f32)
+                    acc_lo = (acc_lo + (lo[:, None] * vv).sum(axis=0, dtype=f32)).astype(f32)
+                else:
+                    acc = (acc + ((hi + lo)[:, None] * vv).sum(axis=0, dtype=f32)).astype(f32)
+            parts.append((m, l, (acc + acc_lo).astype(f32)))
         mstar = max(pm for pm, _, _ in parts)
         L, O = f32(0), np.zeros(D, f32)
         for pm, pl, pa in parts:
@@ -103,6 +112,27 @@ def test_binary32_restatement_within_bound(oracle_mod, outliers, seed):
         qi = q[i].float().numpy().astype(np.float64)
         o, tol = attn_bound.attention_bound(qi, K[i], V[i], 8, scale)
         y = _emulate_fp32(qi, K[i], V[i], 8, scale)
+        err = np.abs(y - o)
+        assert np.all(err <= tol), f"worst error {err.max():.4g}, bound there {tol[np.argmax(err / tol)]:.4g}"
+
+
+@pytest.mark.parametrize("outliers", [False, True])
+@pytest.mark.parametrize("seed", range(2))
+def test_binary32_restatement_split_sums_within_bound(oracle_mod, outliers, seed):
+    """The arithmetic of groups of up to four query heads: the weights' high parts and
+    residuals summed apart; softmax states of one chunk or of an aligned pair of
+    128-position chunks (as warps' contiguous ranges of chunks give them), merged over up
+    to ceil(n / 128) workspace entries."""
+    q, k, v = _fp8_case(10 + seed, S=700, D=128, NH=4, outliers=outliers)
+    _, _, K, V = _encode_fp8(oracle_mod, k, v)
+    scale = 1.0 / math.sqrt(128)
+    # one warp's range ends after chunk 0, the next starts at chunk 1 (alone: its pair
+    # partner belongs to the other warp), then aligned pairs (2, 3) and (4, 5)
+    states = [(0, 128), (128, 256), (256, 512), (512, 700)]
+    for i in range(q.shape[0]):
+        qi = q[i].float().numpy().astype(np.float64)
+        o, tol = attn_bound.attention_bound(qi, K[i], V[i], 4, scale)
+        y = _emulate_fp32(qi, K[i], V[i], 4, scale, states=states, split_sums=True)
         err = np.abs(y - o)
         assert np.all(err <= tol), f"worst error {err.max():.4g}, bound there {tol[np.argmax(err / tol)]:.4g}"
 
